@@ -1,0 +1,204 @@
+"""fp64 CPU oracle of the Causal-RoPE SP Q/K preparation step -- TEST INFRASTRUCTURE.
+
+Only the test suite, the smoke check (``__graft_entry__.smoke``) and the benchmark's
+CPU-baseline and reference legs may import this package; the CUDA product path never
+does.  The arithmetic lives in ``rope3d_oracle.c`` (plain C, double precision); this
+module builds that file with gcc and exposes it through ctypes on numpy float64 arrays.
+It shares no code with the CUDA library.
+
+Paper: "Accelerating Video Generation Inference with Sequential-Parallel 3D
+Positional Encoding Using a Global Time Index" (Yuan & Li) -- Section 3.3.1 (complex
+rotation), Section 3.3.2 (global time index, localized formula), Algorithm 2 (per-axis
+tables, adjacent-pair complex view, fp64), Section 3.3.3 (local-to-global index decode)
+and Algorithms 1 and 3, step 5 (KV-cache update).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "rope3d_oracle.c")
+LIBRARY = os.path.join(_HERE, "librope3d_oracle.so")
+
+# Default split of a 128-wide head: 22 t pairs, 21 h pairs, 21 w pairs; theta 10000.
+N_T, N_H, N_W, THETA = 22, 21, 21, 10000.0
+
+
+def build(force: bool = False, source: str = SOURCE, library: str = LIBRARY) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction, OpenMP on)."""
+    if (not force and os.path.exists(library)
+            and os.path.getmtime(library) >= os.path.getmtime(source)):
+        return library
+    tmp = library + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra",
+           source, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, library)
+    return library
+
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_DBL = ctypes.c_double
+
+
+def _declare(lib):
+    sig = {
+        "rope3d_oracle_inv_freq": ([_INT, _INT, _INT, _DBL, _INT, _D], _INT),
+        "rope3d_oracle_decode": ([_I64, _I64, _I64, _I64, _I64, ctypes.POINTER(_I64),
+                                  ctypes.POINTER(_I64), ctypes.POINTER(_I64)], None),
+        "rope3d_oracle_cache_row": ([_I64, _I64, _I64], _I64),
+        "rope3d_oracle_angles": ([_I64, _I64, _I64, _INT, _INT, _INT, _D, _D], None),
+        "rope3d_oracle_rotate": ([_D, _I64, _I64, _D, _D], None),
+        "rope3d_oracle_rms_norm": ([_D, _D, _I64, _DBL, _D], None),
+        "rope3d_oracle_token": ([_D, _D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
+                                 _D, _D, _DBL, _I64, _I64, _INT, _INT, _INT, _D,
+                                 _D, _D, _D, ctypes.POINTER(_I64)], _INT),
+        "rope3d_oracle_qk_norm_rope_append": ([_D, _D, _D, _D, _I64, _I64, _I64, _I64, _I64,
+                                               _I64, _I64, _I64, _I64, _D, _D, _DBL, _D, _D,
+                                               _I64, _I64, _INT, _INT, _INT, _DBL, _INT,
+                                               _INT], _INT),
+        "rope3d_oracle_apply": ([_D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
+                                 _I64, _INT, _INT, _INT, _DBL, _INT], _INT),
+        "rope3d_oracle_max_threads": ([], _INT),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+class OracleError(ValueError):
+    pass
+
+
+def _f64(a, name):
+    if not (isinstance(a, np.ndarray) and a.dtype == np.float64 and a.flags.c_contiguous):
+        raise TypeError(f"{name} must be a C-contiguous float64 numpy array")
+    return a.ctypes.data_as(_D)
+
+
+def _check(rc):
+    if rc != 0:
+        raise OracleError(f"oracle rejected the arguments (status {rc})")
+
+
+class Oracle:
+    """The compiled oracle library behind numpy-friendly methods."""
+
+    def __init__(self, library: str | None = None):
+        if library is None:
+            library = build()
+        self.path = library
+        self.lib = _declare(ctypes.CDLL(library))
+
+    def inv_freq(self, n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0) -> np.ndarray:
+        out = np.zeros(max(1, n_t + n_h + n_w), dtype=np.float64)
+        _check(self.lib.rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule,
+                                               _f64(out, "out")))
+        return out[: n_t + n_h + n_w]
+
+    def decode(self, i, frame_offset, T, H, W):
+        t, h, w = _I64(), _I64(), _I64()
+        self.lib.rope3d_oracle_decode(i, frame_offset, T, H, W, ctypes.byref(t),
+                                      ctypes.byref(h), ctypes.byref(w))
+        return t.value, h.value, w.value
+
+    def cache_row(self, i, slot, cache_tokens):
+        return self.lib.rope3d_oracle_cache_row(i, slot, cache_tokens)
+
+    def angles(self, t_g, h, w, n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        inv = self.inv_freq(n_t, n_h, n_w, theta, schedule)
+        phi = np.zeros(n_t + n_h + n_w, dtype=np.float64)
+        self.lib.rope3d_oracle_angles(t_g, h, w, n_t, n_h, n_w, _f64(inv, "inv"),
+                                      _f64(phi, "phi"))
+        return phi
+
+    def rotate(self, x, phi):
+        """x: [n_heads, head_dim] float64 (one token row); phi: [head_dim/2]."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        n_heads, head_dim = x.shape[-2], x.shape[-1]
+        phi = np.ascontiguousarray(phi, dtype=np.float64)
+        assert phi.shape == (head_dim // 2,)
+        y = np.empty_like(x)
+        self.lib.rope3d_oracle_rotate(_f64(x, "x"), n_heads, head_dim, _f64(phi, "phi"),
+                                      _f64(y, "y"))
+        return y
+
+    def rms_norm(self, x, weight, eps):
+        x = np.ascontiguousarray(x, dtype=np.float64).ravel()
+        weight = np.ascontiguousarray(weight, dtype=np.float64).ravel()
+        assert weight.shape == x.shape
+        y = np.empty_like(x)
+        self.lib.rope3d_oracle_rms_norm(_f64(x, "x"), _f64(weight, "weight"), x.size, eps,
+                                        _f64(y, "y"))
+        return y
+
+    def token(self, q, k, v, i, frame_offset, T, H, W, q_norm_w, k_norm_w, eps, slot,
+              cache_tokens, n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        """One token row ([N, D] each): returns (q_out, k_row, v_row, (t_g, h, w, row))."""
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        k = np.ascontiguousarray(k, dtype=np.float64)
+        v = np.ascontiguousarray(v, dtype=np.float64)
+        N, D = q.shape[-2], q.shape[-1]
+        inv = self.inv_freq(n_t, n_h, n_w, theta, schedule)
+        qw = np.ascontiguousarray(q_norm_w, dtype=np.float64)
+        kw = np.ascontiguousarray(k_norm_w, dtype=np.float64)
+        qo, ko, vo = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+        pos = (_I64 * 4)()
+        _check(self.lib.rope3d_oracle_token(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), N, D, i, frame_offset, T, H, W,
+            _f64(qw, "q_norm_w"), _f64(kw, "k_norm_w"), eps, slot, cache_tokens,
+            n_t, n_h, n_w, _f64(inv, "inv"), _f64(qo, "q_out"), _f64(ko, "k_row"),
+            _f64(vo, "v_row"), pos))
+        return qo, ko, vo, tuple(pos)
+
+    def qk_norm_rope_append(self, q, k, v, token_begin, token_end, frame_offset, T, H, W,
+                            q_norm_w, k_norm_w, eps, k_cache, v_cache, slot,
+                            n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0, nthreads=0):
+        """Whole step.  q, k, v: [B, n_tok, N, D] float64; k_cache, v_cache:
+        [B, cache_tokens, N, D] float64, updated in place.  Returns q_out."""
+        B, n_tok, N, D = q.shape
+        assert k.shape == q.shape and v.shape == q.shape
+        assert k_cache.shape[0] == B and k_cache.shape[2:] == (N, D)
+        assert v_cache.shape == k_cache.shape
+        q_out = np.empty_like(q)
+        _check(self.lib.rope3d_oracle_qk_norm_rope_append(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), _f64(q_out, "q_out"), B, N, D,
+            token_begin, token_end, frame_offset, T, H, W,
+            _f64(np.ascontiguousarray(q_norm_w, dtype=np.float64), "q_norm_w"),
+            _f64(np.ascontiguousarray(k_norm_w, dtype=np.float64), "k_norm_w"), eps,
+            _f64(k_cache, "k_cache"), _f64(v_cache, "v_cache"), k_cache.shape[1], slot,
+            n_t, n_h, n_w, theta, schedule, nthreads))
+        return q_out
+
+    def apply(self, x, token_begin, token_end, frame_offset, T, H, W,
+              n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        """Rotation alone over [B, n_tok, N, D] float64."""
+        B, n_tok, N, D = x.shape
+        out = np.empty_like(x)
+        _check(self.lib.rope3d_oracle_apply(_f64(x, "x"), _f64(out, "out"), B, N, D,
+                                            token_begin, token_end, frame_offset, T, H, W,
+                                            n_t, n_h, n_w, theta, schedule))
+        return out
+
+    def max_threads(self) -> int:
+        return self.lib.rope3d_oracle_max_threads()
+
+
+_default = None
+
+
+def default() -> Oracle:
+    """The oracle built from ``rope3d_oracle.c`` beside this file (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

@@ -1,0 +1,296 @@
+/*
+ * rope3d_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+ *
+ * A plain, slow, fp64 CPU statement of the per-chunk Q/K preparation step of a
+ * causal autoregressive video DiT with Causal-RoPE SP ("Accelerating Video
+ * Generation Inference with Sequential-Parallel 3D Positional Encoding Using a
+ * Global Time Index", Yuan & Li): position decode from the global token index,
+ * QK-RMSNorm, 3D rotary embedding by complex multiplication, and the K/V cache
+ * append.  Only the test suite, the smoke check and the benchmark's CPU-baseline
+ * leg may load this library.  It shares no code, header, table or constant with
+ * the CUDA path; each side is written from the definitions on its own.
+ *
+ * Everything here is computed in double precision with libm cos/sin/pow/sqrt,
+ * one token at a time, in the order the definitions give.  The only concession to
+ * speed is an OpenMP loop over independent token rows in the whole-step entry
+ * point; every row is computed by the same sequential code either way.
+ *
+ * Readings of points the paper leaves open (each is also listed in the design
+ * notes of the repository):
+ *   - per-axis frequency schedule: each of the t, h, w axes is an ordinary
+ *     rotary embedding over its own sub-dimension d_a = 2 n_a, so pair j of axis
+ *     a turns at theta^(-2j/d_a) per unit of position (schedule 0).  Schedule 1
+ *     instead takes one head-wide schedule theta^(-2j/D) for pair j = 0..D/2-1 and
+ *     hands the first n_t pairs to t, the next n_h to h and the last n_w to w.
+ *     The paper names the three per-axis frequency sets but prints no formula, so
+ *     which schedule is meant is not pinned by it.
+ *   - h and w decode: the paper gives only the time index; h and w follow from
+ *     the row-major (F, H, W) expansion of the frequency tables in its
+ *     Algorithm 2, so h = floor(i / W) mod H and w = i mod W.
+ *   - QK-RMSNorm is not on the paper's pages: it normalises one token's q (and,
+ *     separately, its k) over the token's whole N*D feature vector,
+ *     y = x / sqrt(mean(x^2) + eps) * weight, and runs before the rotation.
+ *     V is neither normalised nor rotated.
+ *   - cache placement: cache row = (slot + i) mod cache_tokens, token-major
+ *     [B][cache_tokens][N][D]; rotated K is stored with its global position.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_EINVAL (-1)
+
+/*
+ * Frequency schedule ("RoPE frequencies theta" of Algorithms 1-3; the three
+ * per-axis frequency sets freqs[0], freqs[1], freqs[2] of Algorithm 2).
+ * Writes inv[0 .. n_t+n_h+n_w-1]: the angle per unit position of every complex
+ * pair of a head, t pairs first, then h, then w (the concatenation order of
+ * Algorithm 2).
+ */
+int rope3d_oracle_inv_freq(int n_t, int n_h, int n_w, double theta, int schedule,
+                           double* inv)
+{
+    if (n_t < 0 || n_h < 0 || n_w < 0 || !(theta > 1.0) || inv == NULL) return ORACLE_EINVAL;
+    if (schedule != 0 && schedule != 1) return ORACLE_EINVAL;
+    int n_axis[3] = {n_t, n_h, n_w};
+    int pairs = n_t + n_h + n_w;
+    int first = 0; /* index of the axis' first pair within the head */
+    for (int a = 0; a < 3; ++a) {
+        for (int j = 0; j < n_axis[a]; ++j) {
+            double exponent;
+            if (schedule == 0) {
+                /* the axis' own sub-dimension: d_a = 2 n_a real elements */
+                double d_a = 2.0 * n_axis[a];
+                exponent = (2.0 * j) / d_a;
+            } else {
+                /* one head-wide schedule over D = 2 * pairs real elements */
+                double d = 2.0 * pairs;
+                exponent = (2.0 * (first + j)) / d;
+            }
+            inv[first + j] = 1.0 / pow(theta, exponent);
+        }
+        first += n_axis[a];
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Position decode of Section 3.3.3: a token with global sequence index i of a
+ * chunk with grid (F, H, W) = (T, H, W) and start frame s sits at local frame
+ * t = floor(i / (H W)), global frame t_g = s + t (Section 3.3.2, item 1); its
+ * row h and column w follow the row-major expansion of Algorithm 2.
+ */
+void rope3d_oracle_decode(int64_t i, int64_t s, int64_t T, int64_t H, int64_t W,
+                          int64_t* t_g, int64_t* h, int64_t* w)
+{
+    (void)T;
+    int64_t hw = H * W;
+    *t_g = s + i / hw;
+    *h = (i / W) % H;
+    *w = i % W;
+}
+
+/* Rolling KV-cache row of global token index i (cache of cache_tokens rows). */
+int64_t rope3d_oracle_cache_row(int64_t i, int64_t slot, int64_t cache_tokens)
+{
+    return (slot + i) % cache_tokens;
+}
+
+/* Angle of every pair of a head at position (t_g, h, w): Section 3.3.2, item 2,
+ * phi = t_g theta_T + h theta_H + w theta_W, each axis on its own pairs. */
+void rope3d_oracle_angles(int64_t t_g, int64_t h, int64_t w, int n_t, int n_h, int n_w,
+                          const double* inv, double* phi)
+{
+    for (int j = 0; j < n_t; ++j) phi[j] = (double)t_g * inv[j];
+    for (int j = 0; j < n_h; ++j) phi[n_t + j] = (double)h * inv[n_t + j];
+    for (int j = 0; j < n_w; ++j) phi[n_t + n_h + j] = (double)w * inv[n_t + n_h + j];
+}
+
+/*
+ * RoPE(x, phi) = x * e^{i phi} (Section 3.3.1) on one token row of n heads of D
+ * reals each.  Elements (2j, 2j+1) of a head are the real and imaginary part of
+ * complex pair j (Algorithm 2 views the last dimension as (-1, 2) pairs).
+ * The same angles apply to every head.  x and y may be the same array.
+ */
+void rope3d_oracle_rotate(const double* x, int64_t n_heads, int64_t head_dim,
+                          const double* phi, double* y)
+{
+    int64_t pairs = head_dim / 2;
+    for (int64_t n = 0; n < n_heads; ++n) {
+        for (int64_t j = 0; j < pairs; ++j) {
+            double a = x[n * head_dim + 2 * j];     /* real part */
+            double b = x[n * head_dim + 2 * j + 1]; /* imaginary part */
+            double c = cos(phi[j]);
+            double s = sin(phi[j]);
+            /* (a + i b)(c + i s) = (a c - b s) + i (a s + b c) */
+            y[n * head_dim + 2 * j] = a * c - b * s;
+            y[n * head_dim + 2 * j + 1] = a * s + b * c;
+        }
+    }
+}
+
+/* RMSNorm over one token's whole feature vector of length dim:
+ * y = x / sqrt(mean(x^2) + eps) * weight.  x and y may be the same array. */
+void rope3d_oracle_rms_norm(const double* x, const double* weight, int64_t dim, double eps,
+                            double* y)
+{
+    double sum_sq = 0.0;
+    for (int64_t e = 0; e < dim; ++e) sum_sq += x[e] * x[e];
+    double mean_sq = sum_sq / (double)dim;
+    double inv_rms = 1.0 / sqrt(mean_sq + eps);
+    for (int64_t e = 0; e < dim; ++e) y[e] = x[e] * inv_rms * weight[e];
+}
+
+/* Rotate one token row at the position that global index i decodes to. */
+void rope3d_oracle_rotate_at(const double* x, int64_t n_heads, int64_t head_dim,
+                             int64_t i, int64_t s, int64_t T, int64_t H, int64_t W,
+                             int n_t, int n_h, int n_w, const double* inv, double* y)
+{
+    double phi[512];
+    int64_t t_g, h, w;
+    rope3d_oracle_decode(i, s, T, H, W, &t_g, &h, &w);
+    rope3d_oracle_angles(t_g, h, w, n_t, n_h, n_w, inv, phi);
+    rope3d_oracle_rotate(x, n_heads, head_dim, phi, y);
+}
+
+static int check_common(int64_t N, int64_t D, int n_t, int n_h, int n_w,
+                        int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                        int64_t T, int64_t H, int64_t W)
+{
+    if (N <= 0 || D <= 0 || D % 2 != 0 || D / 2 > 512) return ORACLE_EINVAL;
+    if (n_t < 0 || n_h < 0 || n_w < 0 || (int64_t)(n_t + n_h + n_w) * 2 != D) return ORACLE_EINVAL;
+    if (T <= 0 || H <= 0 || W <= 0 || frame_offset < 0) return ORACLE_EINVAL;
+    if (token_begin < 0 || token_end <= token_begin || token_end > T * H * W) return ORACLE_EINVAL;
+    return ORACLE_OK;
+}
+
+/*
+ * One token row of the fused step for one batch sample.  Inputs are that row's
+ * q, k, v (N*D reals each, heads outermost); outputs are the row of q_out and
+ * the rows that go to the K and V caches, plus the decoded position
+ * (t_g, h, w) and the cache row in pos_out[0..3].
+ *   q_out = RoPE(RMSNorm(q; q_norm_w)),  k_row = RoPE(RMSNorm(k; k_norm_w)),
+ *   v_row = v  (Algorithm 1/3 step 5: KVCache[key] <- rotated k, KVCache[value] <- v)
+ */
+int rope3d_oracle_token(const double* q, const double* k, const double* v,
+                        int64_t N, int64_t D, int64_t i, int64_t frame_offset,
+                        int64_t T, int64_t H, int64_t W,
+                        const double* q_norm_w, const double* k_norm_w, double eps,
+                        int64_t slot, int64_t cache_tokens,
+                        int n_t, int n_h, int n_w, const double* inv,
+                        double* q_out, double* k_row, double* v_row, int64_t* pos_out)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, i, i + 1, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (cache_tokens <= 0 || slot < 0) return ORACLE_EINVAL;
+    int64_t dim = N * D;
+    int64_t t_g, h, w;
+    double phi[512];
+    rope3d_oracle_decode(i, frame_offset, T, H, W, &t_g, &h, &w);
+    rope3d_oracle_angles(t_g, h, w, n_t, n_h, n_w, inv, phi);
+
+    rope3d_oracle_rms_norm(q, q_norm_w, dim, eps, q_out);
+    rope3d_oracle_rotate(q_out, N, D, phi, q_out);
+    rope3d_oracle_rms_norm(k, k_norm_w, dim, eps, k_row);
+    rope3d_oracle_rotate(k_row, N, D, phi, k_row);
+    memcpy(v_row, v, (size_t)dim * sizeof(double));
+
+    if (pos_out != NULL) {
+        pos_out[0] = t_g;
+        pos_out[1] = h;
+        pos_out[2] = w;
+        pos_out[3] = rope3d_oracle_cache_row(i, slot, cache_tokens);
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The whole step over the token range [token_begin, token_end) of a chunk
+ * (Algorithm 3 steps 2, 3 and 5 for one rank whose slice starts at
+ * Delta = token_begin): q, k, v and q_out are [B][n_tok][N][D] with
+ * n_tok = token_end - token_begin, row r holding global index token_begin + r;
+ * k_cache and v_cache are [B][cache_tokens][N][D] and only the rows this range
+ * maps to are written.  nthreads <= 0 uses the OpenMP default.
+ */
+int rope3d_oracle_qk_norm_rope_append(
+    const double* q, const double* k, const double* v, double* q_out,
+    int64_t B, int64_t N, int64_t D,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset,
+    int64_t T, int64_t H, int64_t W,
+    const double* q_norm_w, const double* k_norm_w, double eps,
+    double* k_cache, double* v_cache, int64_t cache_tokens, int64_t slot,
+    int n_t, int n_h, int n_w, double theta, int schedule, int nthreads)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0 || cache_tokens <= 0 || slot < 0) return ORACLE_EINVAL;
+    if (token_end - token_begin > cache_tokens) return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    int64_t rows = B * n_tok;
+#ifdef _OPENMP
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel for schedule(static) num_threads(nt)
+#endif
+    for (int64_t u = 0; u < rows; ++u) {
+        int64_t b = u / n_tok;
+        int64_t r = u % n_tok;
+        int64_t i = token_begin + r;
+        int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);
+        int64_t in_off = (b * n_tok + r) * dim;
+        int64_t cache_off = (b * cache_tokens + row) * dim;
+        rope3d_oracle_token(q + in_off, k + in_off, v + in_off, N, D, i, frame_offset, T, H, W,
+                            q_norm_w, k_norm_w, eps, slot, cache_tokens, n_t, n_h, n_w, inv,
+                            q_out + in_off, k_cache + cache_off, v_cache + cache_off, NULL);
+    }
+#ifndef _OPENMP
+    (void)nthreads;
+#endif
+    return ORACLE_OK;
+}
+
+/*
+ * Rotation alone (Algorithm 2, CausalRoPE of Algorithm 3 step 3) over the token
+ * range [token_begin, token_end): x and out are [B][n_tok][N][D].
+ */
+int rope3d_oracle_apply(const double* x, double* out, int64_t B, int64_t N, int64_t D,
+                        int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                        int64_t T, int64_t H, int64_t W,
+                        int n_t, int n_h, int n_w, double theta, int schedule)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0) return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t r = 0; r < n_tok; ++r) {
+            int64_t off = (b * n_tok + r) * dim;
+            rope3d_oracle_rotate_at(x + off, N, D, token_begin + r, frame_offset, T, H, W,
+                                    n_t, n_h, n_w, inv, out + off);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Threads the whole-step entry point would use with nthreads <= 0. */
+int rope3d_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,371 @@
+"""Checks that tie the fp64 oracle to what the paper and the mathematics fix.
+
+Every check takes an ``oracle.Oracle`` and raises AssertionError on a mismatch.  The
+same checks run against the real oracle (tests/test_oracle_pins.py) and against copies
+of its source with a planted mistake (tests/test_oracle_mutants.py), which must each fail
+at least one of them.
+
+Paper: "Accelerating Video Generation Inference with Sequential-Parallel 3D Positional
+Encoding Using a Global Time Index" (Yuan & Li).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+D = 128
+P = 64
+NT, NH, NW = 22, 21, 21
+
+
+def _rows(name):
+    out = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                out.append(line)
+    return out
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- frequency schedule
+
+def check_inv_freq_special_values(orc):
+    """Per-axis schedule: pair j of an axis with n_a pairs turns at theta^(-j/n_a).
+    Closed forms: the first pair of each axis is 1; t pair 11 is 10000^(-1/2) = 0.01;
+    h pair 7 is 10000^(-1/3); w pair 14 is 10000^(-2/3)."""
+    inv = orc.inv_freq(NT, NH, NW, 10000.0, 0)
+    assert inv.shape == (P,)
+    for first in (0, NT, NT + NH):
+        assert inv[first] == 1.0
+    assert abs(inv[11] - 0.01) < 1e-17
+    assert abs(inv[NT + 7] - 0.046415888336127795) < 1e-16
+    assert abs(inv[NT + NH + 14] - 0.0021544346900318843) < 1e-17
+    # strictly decreasing within each axis, equal ratios between neighbours
+    for lo, n in ((0, NT), (NT, NH), (NT + NH, NW)):
+        seg = inv[lo:lo + n]
+        assert np.all(np.diff(seg) < 0)
+        ratios = seg[1:] / seg[:-1]
+        assert np.allclose(ratios, ratios[0], rtol=1e-13, atol=0)
+
+
+def check_inv_freq_single_schedule(orc):
+    """Alternative reading: one head-wide schedule theta^(-2j/128) split 22/21/21.
+    Pair 32 is 10000^(-1/2) = 0.01, pair 22 is 10^(-11/8), pair 0 is 1."""
+    inv = orc.inv_freq(NT, NH, NW, 10000.0, 1)
+    assert inv[0] == 1.0
+    assert abs(inv[32] - 0.01) < 1e-17
+    assert abs(inv[22] - 0.042169650342858224) < 1e-16
+    assert np.all(np.diff(inv) < 0)
+
+
+# ---------------------------------------------------------------- position decode
+
+def check_decode_golden(orc):
+    """Hand-derived decode of a (2, 2, 3) grid at s = 3 split over 4 ranks."""
+    L_local = 3
+    for line in _rows("decode_F2_H2_W3_s3_P4.txt"):
+        r, i_local, i_global, t_g, h, w = map(int, line.split())
+        assert r * L_local + i_local == i_global
+        assert orc.decode(i_global, 3, 2, 2, 3) == (t_g, h, w)
+
+
+def check_decode_brute_force(orc):
+    """Row-major enumeration (t outermost, w innermost) of several grids and offsets."""
+    for (T, H, W) in ((3, 4, 6), (1, 1, 1), (2, 5, 1), (4, 1, 7), (3, 30, 52)):
+        for s in (0, 3, 6, 237):
+            i = 0
+            for t in range(T):
+                for h in range(H):
+                    for w in range(W):
+                        if (T, H, W) != (3, 30, 52) or i % 97 == 0:
+                            assert orc.decode(i, s, T, H, W) == (s + t, h, w), (T, H, W, s, i)
+                        i += 1
+
+
+def check_start_frames_golden(orc):
+    """tau = 3: block k starts at frame 3k, so local frame t of block k is global 3k + t."""
+    H, W = 4, 6
+    for line in _rows("start_frames_tau3.txt"):
+        k, s = map(int, line.split())
+        assert s == 3 * k
+        for t in range(3):
+            assert orc.decode(t * H * W, s, 3, H, W)[0] == s + t
+            assert orc.decode(t * H * W + H * W - 1, s, 3, H, W)[0] == s + t
+
+
+def check_cache_rows_rolling_window(orc):
+    """Frame-level simulation of a rolling window of `window` frames: the tokens of global
+    frame f sit in window frame f mod window, spatial order kept.  The oracle places token
+    i of the chunk starting at frame s, with slot = (s mod window) * HW, at
+    (slot + i) mod cache_tokens; both must agree, wrap-around included."""
+    H, W, window = 2, 3, 5
+    hw = H * W
+    cache_tokens = window * hw
+    for s in range(0, 40, 3):
+        slot = (s % window) * hw
+        for i in range(3 * hw):
+            f = s + i // hw
+            expect = (f % window) * hw + i % hw
+            assert orc.cache_row(i, slot, cache_tokens) == expect, (s, i)
+    # a slot that is not frame aligned still places the range contiguously modulo the cache
+    rows = [orc.cache_row(i, 7, 20) for i in range(20)]
+    assert sorted(rows) == list(range(20))
+    assert rows[0] == 7 and rows[12] == 19 and rows[13] == 0
+
+
+# ---------------------------------------------------------------- rotation
+
+def _one_token_rotate(orc, x, t_g, h, w, schedule=0):
+    phi = orc.angles(t_g, h, w, NT, NH, NW, 10000.0, schedule)
+    return orc.rotate(x, phi)
+
+
+def check_rotation_golden(orc):
+    """Closed-form rotations at whole-radian angles (golden file)."""
+    for line in _rows("rotation_unit_angles.txt"):
+        t_g, h, w, j, re_in, im_in, re_out, im_out = line.split()
+        x = np.zeros((1, D))
+        x[0, 2 * int(j)] = float(re_in)
+        x[0, 2 * int(j) + 1] = float(im_in)
+        y = _one_token_rotate(orc, x, int(t_g), int(h), int(w))
+        assert abs(y[0, 2 * int(j)] - float(re_out)) < 1e-14, line
+        assert abs(y[0, 2 * int(j) + 1] - float(im_out)) < 1e-14, line
+        others = np.delete(y[0], [2 * int(j), 2 * int(j) + 1])
+        assert np.all(others == 0.0)
+
+
+def check_position_zero_identity(orc):
+    x = _rng(1).standard_normal((3, D))
+    y = _one_token_rotate(orc, x, 0, 0, 0)
+    assert np.array_equal(x, y)
+
+
+def check_one_hot_axis_ownership(orc):
+    """e_{2j} rotates to (cos phi_j, sin phi_j); each pair moves only with its own axis."""
+    inv = orc.inv_freq()
+    for (t_g, h, w) in ((5, 0, 0), (0, 4, 0), (0, 0, 6), (9, 2, 11)):
+        for j in range(P):
+            x = np.zeros((1, D))
+            x[0, 2 * j] = 1.0
+            y = _one_token_rotate(orc, x, t_g, h, w)
+            pos = t_g if j < NT else (h if j < NT + NH else w)
+            phi = pos * inv[j]
+            assert abs(y[0, 2 * j] - math.cos(phi)) < 1e-14
+            assert abs(y[0, 2 * j + 1] - math.sin(phi)) < 1e-14
+
+
+def check_rotation_matches_complex_exp(orc):
+    """The rotation equals numpy's complex multiply by exp(i phi) on adjacent pairs."""
+    rng = _rng(2)
+    inv = orc.inv_freq()
+    for _ in range(10):
+        t_g, h, w = (int(v) for v in rng.integers(0, 240, size=3))
+        x = rng.standard_normal((4, D))
+        pos = np.array([t_g] * NT + [h] * NH + [w] * NW, dtype=np.float64)
+        z = x.reshape(4, P, 2)
+        zc = (z[..., 0] + 1j * z[..., 1]) * np.exp(1j * pos * inv)
+        expect = np.stack([zc.real, zc.imag], axis=-1).reshape(4, D)
+        y = _one_token_rotate(orc, x, t_g, h, w)
+        assert np.allclose(y, expect, rtol=0, atol=1e-13)
+
+
+def check_pair_norms_preserved(orc):
+    rng = _rng(3)
+    x = rng.standard_normal((5, D))
+    y = _one_token_rotate(orc, x, 17, 29, 51)
+    nx = np.hypot(x[:, 0::2], x[:, 1::2])
+    ny = np.hypot(y[:, 0::2], y[:, 1::2])
+    assert np.allclose(nx, ny, rtol=0, atol=1e-12)
+
+
+def check_relative_offset_brute_force(orc):
+    """<R(p_m) q, R(p_n) k> = <q, R(p_n - p_m) k> for every pair of tokens of the 3x4x6
+    grid at start frame 3 (all 72 x 72 pairs); so the score depends only on the 3D offset."""
+    rng = _rng(4)
+    T, H, W, s = 3, 4, 6, 3
+    n = T * H * W
+    q = rng.standard_normal((n, 2, D))
+    k = rng.standard_normal((n, 2, D))
+    pos = [orc.decode(i, s, T, H, W) for i in range(n)]
+    rq = [_one_token_rotate(orc, q[m], *pos[m]) for m in range(n)]
+    rk = [_one_token_rotate(orc, k[m], *pos[m]) for m in range(n)]
+    for m in range(n):
+        for nn in range(n):
+            lhs = float(np.sum(rq[m] * rk[nn]))
+            d = tuple(pos[nn][a] - pos[m][a] for a in range(3))
+            rhs = float(np.sum(q[m] * _one_token_rotate(orc, k[nn], *d)))
+            assert abs(lhs - rhs) < 1e-10, (m, nn)
+
+
+def check_rotation_group_property(orc):
+    """R(a) R(b) = R(a + b) and R(a) R(-a) = identity."""
+    rng = _rng(5)
+    x = rng.standard_normal((2, D))
+    a, b = (3, 7, 11), (40, -2, 5)
+    ab = tuple(a[i] + b[i] for i in range(3))
+    y1 = _one_token_rotate(orc, _one_token_rotate(orc, x, *a), *b)
+    y2 = _one_token_rotate(orc, x, *ab)
+    assert np.allclose(y1, y2, rtol=0, atol=1e-12)
+    y3 = _one_token_rotate(orc, _one_token_rotate(orc, x, *a), *(-v for v in a))
+    assert np.allclose(y3, x, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def check_rms_norm_golden(orc):
+    for line in _rows("rmsnorm_examples.txt"):
+        eps, xs, ws, ys = (part.split() for part in line.split("|"))
+        y = orc.rms_norm(np.array(xs, float), np.array(ws, float), float(eps[0]))
+        assert np.allclose(y, np.array(ys, float), rtol=0, atol=1e-14), line
+
+
+def check_rms_norm_closed_forms(orc):
+    rng = _rng(6)
+    dim = 256
+    w = rng.uniform(0.5, 1.5, dim)
+    for c, eps in ((2.0, 1e-6), (0.1, 1e-2), (-3.0, 0.5)):
+        y = orc.rms_norm(np.full(dim, c), w, eps)
+        assert np.allclose(y, c / math.sqrt(c * c + eps) * w, rtol=1e-14, atol=0)
+    x = rng.standard_normal(dim)
+    ones = np.ones(dim)
+    y = orc.rms_norm(x, ones, 0.0)
+    assert abs(float(np.sum(y * y)) - dim) < 1e-10
+    for alpha in (1e-3, 7.0, 1e4):
+        assert np.allclose(orc.rms_norm(alpha * x, w, 0.0), orc.rms_norm(x, w, 0.0),
+                           rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- fused token and step
+
+def check_token_norms_and_weights(orc):
+    """With eps = 0 and constant weights c_q, c_k: |q_out|^2 = c_q^2 dim and
+    |k_row|^2 = c_k^2 dim (RMSNorm fixes the mean square, rotation keeps it); v is copied
+    bit for bit; the returned position and cache row are the decode and the rolling row."""
+    rng = _rng(7)
+    N = 3
+    dim = N * D
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    qo, ko, vo, pos = orc.token(q, k, v, 29, 6, 3, 4, 6, np.full(dim, 1.0), np.full(dim, 2.0),
+                                0.0, 100, 144)
+    assert abs(float(np.sum(qo * qo)) - dim) < 1e-9
+    assert abs(float(np.sum(ko * ko)) - 4.0 * dim) < 1e-9
+    assert np.array_equal(vo, v)
+    assert pos == (6 + 1, (29 // 6) % 4, 29 % 6, (100 + 29) % 144)
+
+
+def check_token_is_norm_then_rotate(orc):
+    """q_out = RoPE(RMSNorm(q)) -- the norm of one row is taken before rotating, with the
+    q weights for q and the k weights for k.  Weights differ per element, so swapping the
+    order or the weights changes the result."""
+    rng = _rng(8)
+    N = 2
+    dim = N * D
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    wq, wk = rng.uniform(0.5, 1.5, dim), rng.uniform(0.5, 1.5, dim)
+    qo, ko, _, (t_g, h, w, _) = orc.token(q, k, v, 50, 3, 3, 4, 6, wq, wk, 1e-6, 0, 144)
+    phi = orc.angles(t_g, h, w)
+    expect_q = orc.rotate(orc.rms_norm(q, wq, 1e-6).reshape(N, D), phi)
+    expect_k = orc.rotate(orc.rms_norm(k, wk, 1e-6).reshape(N, D), phi)
+    assert np.allclose(qo, expect_q, rtol=0, atol=1e-13)
+    assert np.allclose(ko, expect_k, rtol=0, atol=1e-13)
+    # independent recomputation of the mean square for one element
+    rs = 1.0 / math.sqrt(np.mean(q.ravel() ** 2) + 1e-6)
+    a, b = q[1, 2 * 30] * rs * wq[D + 60], q[1, 2 * 30 + 1] * rs * wq[D + 61]
+    c, s = math.cos(phi[30]), math.sin(phi[30])
+    assert abs(qo[1, 60] - (a * c - b * s)) < 1e-13
+    assert abs(qo[1, 61] - (a * s + b * c)) < 1e-13
+
+
+def _step_inputs(seed, B, n_tok, N):
+    rng = _rng(seed)
+    q, k, v = (rng.standard_normal((B, n_tok, N, D)) for _ in range(3))
+    wq, wk = rng.uniform(0.5, 1.5, N * D), rng.uniform(0.5, 1.5, N * D)
+    return q, k, v, wq, wk
+
+
+def check_step_matches_tokens(orc):
+    """The whole step writes, for each (b, r), the token function's rows: q_out at row r,
+    K and V at (slot + i) mod cache_tokens of sample b; other cache rows stay untouched."""
+    B, N, T, H, W = 2, 2, 3, 4, 6
+    tb, te, s, slot, C = 10, 50, 3, 130, 144
+    q, k, v, wq, wk = _step_inputs(9, B, te - tb, N)
+    kc = np.full((B, C, N, D), 7.0)
+    vc = np.full((B, C, N, D), -7.0)
+    qo = orc.qk_norm_rope_append(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kc, vc, slot)
+    touched = set()
+    for b in range(B):
+        for r in range(te - tb):
+            i = tb + r
+            eq, ek, ev, pos = orc.token(q[b, r], k[b, r], v[b, r], i, s, T, H, W, wq, wk, 1e-6,
+                                        slot, C)
+            row = pos[3]
+            assert row == (slot + i) % C
+            assert np.array_equal(qo[b, r], eq)
+            assert np.array_equal(kc[b, row], ek)
+            assert np.array_equal(vc[b, row], ev)
+            touched.add((b, row))
+    for b in range(B):
+        for row in range(C):
+            if (b, row) not in touched:
+                assert np.all(kc[b, row] == 7.0) and np.all(vc[b, row] == -7.0)
+
+
+def check_slices_equal_whole(orc):
+    """Section 3.3.3: processing [r L/P, (r+1) L/P) on each of P ranks gives the whole-
+    sequence result.  Uneven slices cut through rows and frames."""
+    B, N, T, H, W, s, C = 1, 2, 3, 4, 6, 6, 144
+    n = T * H * W
+    q, k, v, wq, wk = _step_inputs(10, B, n, N)
+    kc0, vc0 = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    q0 = orc.qk_norm_rope_append(q, k, v, 0, n, s, T, H, W, wq, wk, 1e-6, kc0, vc0, 72)
+    kc1, vc1 = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    q1 = np.empty_like(q0)
+    for (a, e) in ((0, 5), (5, 29), (29, 30), (30, 72)):
+        q1[:, a:e] = orc.qk_norm_rope_append(q[:, a:e].copy(), k[:, a:e].copy(),
+                                             v[:, a:e].copy(), a, e, s, T, H, W, wq, wk,
+                                             1e-6, kc1, vc1, 72)
+    assert np.array_equal(q0, q1)
+    assert np.array_equal(kc0, kc1)
+    assert np.array_equal(vc0, vc1)
+
+
+def check_frame_shift_invariant(orc):
+    """Causal-RoPE SP on a chunk starting at frame s equals full-sequence RoPE on the
+    longer video: out(i, s) on grid (T, H, W) == out(i + s H W, 0) on grid (T + s, H, W)."""
+    B, N, T, H, W, s = 1, 2, 3, 4, 6, 6
+    hw = H * W
+    n = T * hw
+    q, k, v, wq, wk = _step_inputs(11, B, n, N)
+    C = (T + s) * hw
+    kc_a, vc_a = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    qa = orc.qk_norm_rope_append(q, k, v, 0, n, s, T, H, W, wq, wk, 1e-6, kc_a, vc_a, s * hw)
+    kc_b, vc_b = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    qb = orc.qk_norm_rope_append(q, k, v, s * hw, s * hw + n, 0, T + s, H, W, wq, wk, 1e-6,
+                                 kc_b, vc_b, 0)
+    assert np.array_equal(qa, qb)
+    assert np.array_equal(kc_a, kc_b)
+    assert np.array_equal(vc_a, vc_b)
+
+
+def check_apply_matches_rotation(orc):
+    """The rotation-only entry point rotates row r by the angles of index begin + r."""
+    B, N, T, H, W, s = 2, 2, 3, 4, 6, 9
+    rng = _rng(12)
+    x = rng.standard_normal((B, 40, N, D))
+    y = orc.apply(x, 20, 60, s, T, H, W)
+    for b in range(B):
+        for r in range(40):
+            t_g, h, w = orc.decode(20 + r, s, T, H, W)
+            assert (t_g, h, w) == (s + (20 + r) // 24, ((20 + r) // 6) % 4, (20 + r) % 6)
+            assert np.array_equal(y[b, r], _one_token_rotate(orc, x[b, r], t_g, h, w))
+
+
+ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

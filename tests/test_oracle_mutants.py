@@ -1,0 +1,70 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and require that the pins
+catch every one: a dropped term, a wrong sign, a swapped or transposed operand, an
+off-by-one.  The mistakes are planted on the CPU only, in a temporary build."""
+import os
+import shutil
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_CHECKS
+
+MUTANTS = {
+    "rotate_real_sign": ("y[n * head_dim + 2 * j] = a * c - b * s;",
+                         "y[n * head_dim + 2 * j] = a * c + b * s;"),
+    "rotate_imag_transposed": ("y[n * head_dim + 2 * j + 1] = a * s + b * c;",
+                               "y[n * head_dim + 2 * j + 1] = b * s + a * c;"),
+    "pair_layout_rotate_half": ("double a = x[n * head_dim + 2 * j];     /* real part */",
+                                "double a = x[n * head_dim + j];"),
+    "axis_subdim_off_by_one": ("double d_a = 2.0 * n_axis[a];",
+                               "double d_a = 2.0 * n_axis[a] + 2.0;"),
+    "single_schedule_wrong_offset": ("exponent = (2.0 * (first + j)) / d;",
+                                     "exponent = (2.0 * j) / d;"),
+    "decode_drops_start_frame": ("*t_g = s + i / hw;", "*t_g = i / hw;"),
+    "decode_h_w_swapped": ("*h = (i / W) % H;", "*h = (i / H) % W;"),
+    "angle_h_uses_w": ("phi[n_t + j] = (double)h * inv[n_t + j];",
+                       "phi[n_t + j] = (double)w * inv[n_t + j];"),
+    "rms_mean_wrong_count": ("double mean_sq = sum_sq / (double)dim;",
+                             "double mean_sq = sum_sq / (double)(dim - 1);"),
+    "rms_drops_eps": ("double inv_rms = 1.0 / sqrt(mean_sq + eps);",
+                      "double inv_rms = 1.0 / sqrt(mean_sq);"),
+    "rms_drops_weight": ("y[e] = x[e] * inv_rms * weight[e];", "y[e] = x[e] * inv_rms;"),
+    "k_uses_q_weights": ("rope3d_oracle_rms_norm(k, k_norm_w, dim, eps, k_row);",
+                         "rope3d_oracle_rms_norm(k, q_norm_w, dim, eps, k_row);"),
+    "rotate_before_norm": (
+        "    rope3d_oracle_rms_norm(q, q_norm_w, dim, eps, q_out);\n"
+        "    rope3d_oracle_rotate(q_out, N, D, phi, q_out);",
+        "    rope3d_oracle_rotate(q, N, D, phi, q_out);\n"
+        "    rope3d_oracle_rms_norm(q_out, q_norm_w, dim, eps, q_out);"),
+    "v_copies_k": ("memcpy(v_row, v, (size_t)dim * sizeof(double));",
+                   "memcpy(v_row, k, (size_t)dim * sizeof(double));"),
+    "cache_row_ignores_slot": ("return (slot + i) % cache_tokens;", "return i % cache_tokens;"),
+    "cache_offset_wrong_stride": ("int64_t cache_off = (b * cache_tokens + row) * dim;",
+                                  "int64_t cache_off = (b * n_tok + row) * dim;"),
+    "step_index_ignores_begin": ("int64_t i = token_begin + r;", "int64_t i = r;"),
+}
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(oracle.SOURCE).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    path = os.path.join(tmp_path, f"{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    return oracle.build(force=True, source=path, library=os.path.join(tmp_path, f"{name}.so"))
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    orc = oracle.Oracle(_build_mutant(str(tmp_path), name, old, new))
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check(orc)
+        except AssertionError:
+            caught.append(check.__name__)
+        except Exception as e:  # a crash also counts as caught, but say which
+            caught.append(f"{check.__name__} ({type(e).__name__})")
+    assert caught, f"no pin catches the planted mistake {name}"
