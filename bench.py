@@ -1,0 +1,542 @@
+#!/usr/bin/env python
+"""Benchmark of the fused QK-RMSNorm + causal 3D RoPE + KV-cache append step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload chunk720p|chunk480p|longhorizon] [--trig table|onthefly]
+
+One step is the whole 720P sequence of a Wan-14B-shaped backbone (21 latent frames of
+45x80, 40 heads of 128, bf16) in seven chunk calls of 10800 tokens, start frames 0, 3,
+..., 18, appended into a 75600-token KV cache -- the Self-Forcing chunk loop of
+"Accelerating Video Generation Inference with Sequential-Parallel 3D Positional Encoding
+Using a Global Time Index" (Section 3.3.2), at the 720P size.  Inputs are seeded
+synthetic tensors (N(0,1) rounded to bf16; RMSNorm weights U(0.5, 1.5)); every chunk has
+its own buffers and each launch streams 663.6 MB, well above the 126 MB L2, so no L2
+flush is needed between launches.
+
+Under torchrun every rank runs the same job on its own GPU with its own seed (weak
+scaling, no collective on the data path); the reported time is the maximum over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from rotary_position_encoding_b200 import workloads as wl  # noqa: E402
+
+WORKLOADS = {
+    "chunk720p": wl.chunk_720p,
+    "chunk480p": wl.chunk_480p,
+    "longhorizon": wl.long_horizon,
+}
+METRIC = "fused norm+3D-RoPE+KV-append tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
+KERNEL_SOURCES = [os.path.join(ROOT, "rotary_position_encoding_b200", "csrc", f)
+                  for f in ("rope3d_kernels.cuh", "rope3d.cu")]
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chunk720p")
+    ap.add_argument("--trig", choices=["table", "onthefly"], default="table")
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="use only the first CHUNKS chunk calls per step (profiling captures "
+                         "of a smaller case; 0 = the whole step)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="upper bound on the oracle's timed CPU work")
+    return ap.parse_args(argv)
+
+
+def workload_for(args) -> wl.Workload:
+    w = WORKLOADS[args.workload]()
+    if args.chunks:
+        w.chunks = w.chunks[: args.chunks]
+        w.name += f"_first{len(w.chunks)}chunks"
+    return w
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend: str):
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg is not None:
+            self.pg.barrier()
+
+    def max(self, x: float, device) -> float:
+        if self.pg is None:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------- inputs
+
+def make_inputs(w: wl.Workload, seed_offset: int):
+    """Host tensors of every chunk call of one step (bf16 bit patterns), generated in
+    parallel threads (each tensor has its own seeded generator)."""
+    n = w.tokens_per_chunk
+    shape = (w.B, n, w.N, wl.HEAD_DIM)
+    jobs = [(ci, t) for ci in range(len(w.chunks)) for t in range(3)]
+
+    def gen(job):
+        ci, t = job
+        rng = wl.rng_for(w.seed + seed_offset, ci, t)
+        return wl.normal_tensor(rng, shape, w.dtype)
+
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        arrays = list(ex.map(gen, jobs))
+    return [tuple(arrays[3 * ci + t] for t in range(3)) for ci in range(len(w.chunks))]
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons for one GPU."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+        self.t_start = self.t_end = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which: str):
+        setattr(self, "t_" + which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for rec in csv.reader(f):
+                if len(rec) >= 10:
+                    rows.append([x.strip() for x in rec])
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        # keep the samples taken inside the timed region when there are any
+        def stamp(r):
+            try:
+                return time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S")) + \
+                    float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+            except ValueError:
+                return None
+        if self.t_start is not None and self.t_end is not None:
+            inside = [r for r in rows if (stamp(r) is not None
+                                          and self.t_start - 0.06 <= stamp(r) <= self.t_end + 0.06)]
+            window = "timed region"
+            if not inside:
+                inside, window = rows, "whole run (timed region shorter than the sampling period)"
+            rows = inside
+        else:
+            window = "whole run"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        reasons = sorted({names[j] for r in rows for j in range(4)
+                          if r[6 + j].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "window": window}
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str, trig: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(f"{workload_name}/{trig}")
+    if not entry or entry.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0}, "fallback"
+
+
+def run_ours(args, dist: Dist):
+    import torch
+
+    from rotary_position_encoding_b200 import rope3d
+
+    torch.cuda.set_device(dist.local_rank)
+    device = torch.device("cuda", dist.local_rank)
+    dist.init("nccl")
+    w = workload_for(args)
+    trig = rope3d.ROPE3D_TRIG_TABLE if args.trig == "table" else rope3d.ROPE3D_TRIG_ONTHEFLY
+    n = w.tokens_per_chunk
+    tokens_per_step = w.B * n * len(w.chunks)
+    bytes_per_launch = w.algorithmic_bytes(n)
+
+    host = make_inputs(w, seed_offset=dist.rank)
+    wq, wk = wl.norm_weights(w.seed, w.dim)
+    wq_d = torch.from_numpy(wq).to(device)
+    wk_d = torch.from_numpy(wk).to(device)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev_tensor(a):
+        if w.dtype == "bf16":
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a).to(device)
+
+    inputs = [tuple(dev_tensor(a) for a in chunk) for chunk in host]
+    q_out = [torch.empty_like(c[0]) for c in inputs]
+    cache_shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    k_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
+    v_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
+    max_t = max(c.frame_offset for c in w.chunks) + w.T
+    tables = rope3d.rope3d_tables_init(max_t=max_t, max_h=w.H, max_w=w.W)
+    stream = torch.cuda.current_stream(device)
+
+    def step(events=None):
+        for ci, chunk in enumerate(w.chunks):
+            q, k, v = inputs[ci]
+            if events is not None:
+                events[2 * ci].record(stream)
+            rope3d.rope3d_qk_norm_rope_append(
+                q, k, v, q_out[ci], chunk.token_begin, chunk.token_end, chunk.frame_offset,
+                w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
+                stream)
+            if events is not None:
+                events[2 * ci + 1].record(stream)
+
+    clocks = ClockSampler(dist.local_rank) if dist.rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-launch events of every timed launch (the kernel's own duration) and the region
+    n_launch = len(w.chunks)
+    per_step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+                       for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark("start")
+    start.record(stream)
+    for s in range(args.steps):
+        step(per_step_events[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark("end")
+    dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    launch_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for ev in per_step_events
+                 for j in range(n_launch)]
+    clock_info = clocks.stop() if clocks else None
+
+    elapsed_ms = dist.max(elapsed_ms, device)
+    avg_launch_ms = dist.max(statistics.fmean(launch_ms), device)
+    total_tokens = tokens_per_step * args.steps * dist.world
+    value = total_tokens / (elapsed_ms / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
+
+    del per_step_events
+    tables.close()
+    dist.close()
+    if dist.rank != 0:
+        return None
+
+    peaks, peak_kind = measured_peaks()
+    achieved_gbs = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
+    roofline = {
+        "bound": "hbm",
+        "achieved": round(achieved_gbs, 1),
+        "peak": peaks["hbm_gbs"],
+        "unit": "GB/s",
+        "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+        "traffic": recorded_traffic(w.name, args.trig),
+        "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+        else "fallback 6.65 TB/s",
+        "kernel": "rope3d::qk_norm_rope_kernel",
+        "algorithmic_bytes_per_launch": bytes_per_launch,
+        "avg_launch_us": round(avg_launch_ms * 1e3, 2),
+    }
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, U(0.5,1.5) fp32 norm weights)",
+        "config": {
+            "workload": w.name,
+            "grid_per_chunk": [w.T, w.H, w.W],
+            "chunks_per_step": len(w.chunks),
+            "tokens_per_step": tokens_per_step,
+            "batch": w.B,
+            "heads": w.N,
+            "head_dim": wl.HEAD_DIM,
+            "cache_tokens": w.cache_tokens,
+            "trig": args.trig,
+            "l2": "no flush: inputs larger than L2 (each launch streams "
+                  f"{bytes_per_launch / 1e6:.1f} MB from its own buffers)",
+            "parallelism": f"replicas x{dist.world} (independent streams, no collective)",
+        },
+        "hbm_gbs": round(bytes_per_launch * n_launch * args.steps * dist.world
+                         / (elapsed_ms / 1e3) / 1e9, 1),
+        "roofline": roofline,
+        "gpu_launches": n_launch * args.steps,
+        "clocks": clock_info,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and dist.world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, host, args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch):
+    """Same workload through the public call with the step's inputs copied in from pinned
+    host memory and its results (q_out and the appended K/V rows) copied back, every step,
+    inside the timed region."""
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    n = w.tokens_per_chunk
+
+    def pinned_from(a):
+        t = torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a)
+        t = t.view(torch.bfloat16) if w.dtype == "bf16" else t
+        return t.pin_memory()
+
+    h_in = [tuple(pinned_from(a) for a in chunk) for chunk in host]
+    shape = (w.B, n, w.N, wl.HEAD_DIM)
+    h_out = [tuple(torch.empty(shape, dtype=tdt).pin_memory() for _ in range(3))
+             for _ in w.chunks]
+    d_in = [tuple(torch.empty(shape, dtype=tdt, device=device) for _ in range(3))]
+    d_qo = torch.empty(shape, dtype=tdt, device=device)
+    cache_shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    k_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
+    v_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
+    stream = torch.cuda.current_stream(device)
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        for ci, chunk in enumerate(w.chunks):
+            q, k, v = d_in[0]
+            for dst, src in zip((q, k, v), h_in[ci]):
+                dst.copy_(src, non_blocking=True)
+                h2d += src.numel() * src.element_size()
+            rope3d.rope3d_qk_norm_rope_append(
+                q, k, v, d_qo, chunk.token_begin, chunk.token_end, chunk.frame_offset,
+                w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
+                stream)
+            rows = slice(chunk.slot, chunk.slot + n)  # no wrap inside a chunk here
+            for dst, src in zip(h_out[ci], (d_qo, k_cache[:, rows], v_cache[:, rows])):
+                dst.copy_(src, non_blocking=True)
+                d2h += dst.numel() * dst.element_size()
+
+    steps = max(1, min(args.e2e_steps, args.steps))
+    step()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end), device)
+    tokens = w.B * n * len(w.chunks) * steps * dist.world
+    return {"value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3),
+            "path": "pinned host -> cudaMemcpyAsync -> rope3d_qk_norm_rope_append -> "
+                    "cudaMemcpyAsync -> pinned host, one stream"}
+
+
+# ---------------------------------------------------------------- the oracle on the host
+
+def oracle_sample(w, host, budget_s: float, max_tokens=None):
+    """Run the fp64 oracle over the step's chunks in 512-token sub-batches until the whole
+    step or the time budget is done; returns (tokens, seconds, threads)."""
+    import oracle
+    orc = oracle.default()
+    wq, wk = wl.norm_weights(w.seed, w.dim)
+    wq64, wk64 = wq.astype(np.float64), wk.astype(np.float64)
+    n = w.tokens_per_chunk
+    sub = 512
+    done, spent = 0, 0.0
+    for ci, chunk in enumerate(w.chunks):
+        for a in range(0, n, sub):
+            e = min(n, a + sub)
+            f = [wl.to_f64(x[:, a:e], w.dtype) for x in host[ci]]
+            m = e - a
+            # a cache of m rows placed so the sub-batch fills it exactly; the per-token
+            # work is that of the real cache placement
+            kc = np.zeros((w.B, m, w.N, wl.HEAD_DIM))
+            vc = np.zeros_like(kc)
+            t0 = time.perf_counter()
+            orc.qk_norm_rope_append(f[0], f[1], f[2], a, e, chunk.frame_offset, w.T, w.H, w.W,
+                                    wq64, wk64, w.eps, kc, vc, (-a) % m, nthreads=0)
+            spent += time.perf_counter() - t0
+            done += w.B * m
+            if spent >= budget_s or (max_tokens is not None and done >= max_tokens):
+                return done, spent, orc.max_threads()
+    return done, spent, orc.max_threads()
+
+
+def cpu_baseline(w, host, budget_s):
+    tokens, secs, threads = oracle_sample(w, host, budget_s)
+    return {"value": round(tokens / secs, 1), "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{tokens} tokens of the step ({w.name}) in 512-token sub-batches, "
+                      f"{secs:.2f} s of fp64 oracle time on {threads} OpenMP threads"}
+
+
+def run_reference(args, dist: Dist):
+    """The oracle as it stands on the host cores, on this benchmark's workload; each step
+    is a bounded sample sized so the whole run stays within a few minutes."""
+    if dist.rank != 0:
+        return None
+    w = workload_for(args)
+    host = make_inputs(w, seed_offset=0)
+    # calibrate: tokens per second of the oracle on this host
+    tok, secs, threads = oracle_sample(w, host, 1.0, max_tokens=1024)
+    rate = tok / secs
+    total_budget = 150.0
+    per_step = int(max(1, min(w.B * w.tokens_per_chunk * len(w.chunks),
+                              rate * total_budget / max(1, args.steps + args.warmup))))
+    for _ in range(args.warmup):
+        oracle_sample(w, host, 1e9, max_tokens=per_step)
+    total_tok, total_s = 0, 0.0
+    for _ in range(args.steps):
+        t, s, threads = oracle_sample(w, host, 1e9, max_tokens=per_step)
+        total_tok += t
+        total_s += s
+    value = total_tok / total_s
+    sample = (f"{per_step} tokens per step from the start of the {w.name} step, "
+              f"512-token sub-batches, fp64 oracle, {threads} OpenMP threads")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_s / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, U(0.5,1.5) fp32 norm weights)",
+        "config": {"workload": w.name, "tokens_per_step_sampled": per_step,
+                   "heads": w.N, "head_dim": wl.HEAD_DIM, "trig": "fp64 libm"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        line = run_reference(args, dist)
+    else:
+        line = run_ours(args, dist)
+    if line is not None and dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

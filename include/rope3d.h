@@ -1,0 +1,180 @@
+/*
+ * rope3d.h -- C ABI of the fused QK-RMSNorm + causal 3D RoPE + KV-cache append
+ * library for NVIDIA B200 (sm_100a), librope3d.so.
+ *
+ * The operation is the per-chunk Q/K preparation step of a causal autoregressive
+ * video DiT under "Causal-RoPE SP", from "Accelerating Video Generation Inference
+ * with Sequential-Parallel 3D Positional Encoding Using a Global Time Index"
+ * (Yuan & Li):
+ *   - every token's (t, h, w) comes from its global sequence index i and the
+ *     chunk's start frame s (Section 3.3.2 item 1; Section 3.3.3):
+ *       t_g = s + floor(i / (H W)),  h = floor(i / W) mod H,  w = i mod W;
+ *   - the rotation is a complex multiply x' = x * e^{i(t_g th_T + h th_H + w th_W)}
+ *     on adjacent element pairs (2j, 2j+1) = (re, im) of each head (Section 3.3.1,
+ *     Section 3.3.2 item 2, Algorithm 2), pairs 0..n_t-1 turning with t_g, the next
+ *     n_h with h and the last n_w with w;
+ *   - the rotated K and the raw V are written to the KV cache (Algorithm 1 and 3,
+ *     step 5), here at cache row (slot + i) mod cache_tokens of a rolling window.
+ * Before the rotation q and k each go through RMSNorm over the token's whole
+ * N*D feature vector, y = x / sqrt(mean(x^2) + eps) * weight (QK-RMSNorm of the
+ * Wan2.1-style backbone; the paper's pages do not state it).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers on the current CUDA device, contiguous,
+ *     16-byte aligned.  The caller owns them and the stream; the library owns only
+ *     what rope3d_tables_init allocates.
+ *   - Work is enqueued on cuda_stream (a cudaStream_t; NULL = the legacy default
+ *     stream) and returns without synchronising.  No allocation happens per call.
+ *   - Arguments are checked on the host before anything is enqueued; a negative
+ *     status means nothing was launched and no output was touched.  A launch
+ *     failure reports ROPE3D_ECUDA.  No exception crosses the ABI, nothing aborts,
+ *     no device code traps.  rope3d_last_error() gives the reason in words for the
+ *     calling thread's most recent failure.
+ *   - Layouts: activations [B][n_tok][N][D] with n_tok = token_end - token_begin,
+ *     input row r holding global index token_begin + r; caches [B][cache_tokens][N][D].
+ *     D must be 128 = 2 (n_t + n_h + n_w) for the tables it was built with.
+ *   - Results do not depend on how [0, T*H*W) is cut into token ranges: a range
+ *     processed alone is bit-identical to the same rows of a whole-sequence call.
+ */
+#ifndef ROPE3D_H
+#define ROPE3D_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define ROPE3D_API __attribute__((visibility("default")))
+#else
+#define ROPE3D_API
+#endif
+
+/* Status codes. */
+#define ROPE3D_OK 0
+#define ROPE3D_EINVAL (-1)   /* a size, count, enum or null pointer is invalid        */
+#define ROPE3D_ERANGE (-2)   /* an index range exceeds the grid, cache or tables      */
+#define ROPE3D_ECUDA (-3)    /* the CUDA runtime reported an error                    */
+#define ROPE3D_EDEVICE (-4)  /* no sm_100 device, or the tables live on another device */
+#define ROPE3D_EALIGN (-5)   /* a tensor pointer is not 16-byte aligned                */
+#define ROPE3D_EOVERLAP (-6) /* output buffers overlap each other or an input          */
+
+/* Element types of q, k, v, q_out and the caches (all the same type). */
+#define ROPE3D_F32 0
+#define ROPE3D_BF16 1
+
+/* Frequency schedules (the paper names per-axis frequencies theta_T, theta_H,
+ * theta_W and three frequency tables, Algorithm 2, but prints no formula):
+ *   PER_AXIS  -- pair j of an axis with n_a pairs turns at theta^(-2j / (2 n_a))
+ *                per unit position (each axis an ordinary RoPE over its own
+ *                sub-dimension; the default);
+ *   HEAD_WIDE -- one schedule theta^(-2j / D) over the head's pairs j = 0..D/2-1,
+ *                cut into n_t, n_h, n_w contiguous pieces. */
+#define ROPE3D_SCHEDULE_PER_AXIS 0
+#define ROPE3D_SCHEDULE_HEAD_WIDE 1
+
+/* How the kernels obtain cos/sin of each pair's angle. */
+#define ROPE3D_TRIG_TABLE 0     /* read the precomputed tables (fp64-built, fp32-stored) */
+#define ROPE3D_TRIG_ONTHEFLY 1  /* fp32 angle = position * fp32(inv_freq), then sincosf  */
+
+/* Opaque frequency configuration: split, theta, schedule, the fp32 inverse
+ * frequencies and, optionally, per-axis cos/sin tables in device memory. */
+typedef struct rope3d_tables rope3d_tables;
+
+/*
+ * Build the frequency configuration on the current device ("RoPE Frequency
+ * Precomputation", Section 3.4.1 item 2: contiguous precomputed tensors instead of
+ * a per-call cache).  For each axis a in (t, h, w) and each position p < max_a the
+ * table holds cos and sin of p * inv_a[j] computed in fp64 and stored as fp32,
+ * laid out [max_a][n_a] of (cos, sin) pairs.  max_t = max_h = max_w = 0 builds no
+ * tables: only ROPE3D_TRIG_ONTHEFLY can then be used.
+ *   out       : receives the handle (set to NULL on failure)
+ *   head_dim  : must equal 2 (n_t + n_h + n_w); the kernels support 128
+ *   theta     : base, > 1 (10000 for the Wan2.1-style backbone)
+ *   schedule  : ROPE3D_SCHEDULE_*
+ *   cuda_stream: stream for the table upload; the call synchronises it before
+ *               returning (this is set-up, not the per-chunk path)
+ * Errors: EINVAL for bad sizes, ECUDA if allocation or upload fails, EDEVICE if the
+ * current device is not compute capability 10.0.  Ownership: the library; release
+ * with rope3d_tables_destroy on the same device.
+ */
+ROPE3D_API int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int n_w,
+                       double theta, int max_t, int max_h, int max_w, int schedule,
+                       void* cuda_stream);
+
+/* Free the tables (NULL is accepted).  Synchronises the device that holds them. */
+ROPE3D_API void rope3d_tables_destroy(rope3d_tables* tables);
+
+/*
+ * The fused step for one token range of one chunk (Algorithm 3 steps 2, 3 and 5 on
+ * a rank whose slice begins at Delta = token_begin, Section 3.3.3), for all B
+ * samples, which share grid, start frame and slot:
+ *   q_out[b][r]           = RoPE(RMSNorm(q[b][r]; q_norm_w, eps), pos(i))
+ *   k_cache[b][row(i)]    = RoPE(RMSNorm(k[b][r]; k_norm_w, eps), pos(i))
+ *   v_cache[b][row(i)]    = v[b][r]                       (bit copy)
+ * with i = token_begin + r, pos(i) the decode above with s = frame_offset, and
+ * row(i) = (slot + i) mod cache_tokens.  Arithmetic is fp32; bf16 results are
+ * rounded once, to nearest even, when stored.
+ *   q, k, v   : [B][n_tok][N][D] of dtype (device, read only)
+ *   q_out     : [B][n_tok][N][D]; may be q itself (in place), must not overlap k, v
+ *               or the caches otherwise
+ *   B, N, D   : batch, heads, head size (D = 128)
+ *   dtype     : ROPE3D_F32 or ROPE3D_BF16
+ *   token_begin, token_end : 0 <= begin < end <= T*H*W; end - begin <= cache_tokens
+ *   frame_offset : start frame s >= 0 of the chunk (Self-Forcing's start_frame)
+ *   T, H, W   : the chunk's latent grid (frames, rows, columns), each >= 1
+ *   q_norm_w, k_norm_w : [N*D] fp32 RMSNorm weights (device)
+ *   eps       : >= 0, added to the mean square
+ *   k_cache, v_cache : [B][cache_tokens][N][D] of dtype; only the rows of this range
+ *               are written; they must not overlap each other or any input
+ *   cache_tokens, slot : cache rows (>= 1) and slot >= 0 of global index 0
+ *   tables    : from rope3d_tables_init on this device, with D = its head_dim
+ *   trig      : ROPE3D_TRIG_TABLE (needs s + floor((token_end-1)/(H W)) < max_t,
+ *               H <= max_h, W <= max_w) or ROPE3D_TRIG_ONTHEFLY
+ * Errors: EINVAL, ERANGE, EALIGN, EOVERLAP, EDEVICE, ECUDA as above.
+ */
+ROPE3D_API int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void* q_out,
+                               int64_t B, int64_t N, int D, int dtype,
+                               int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                               int T, int H, int W,
+                               const float* q_norm_w, const float* k_norm_w, float eps,
+                               void* k_cache, void* v_cache, int64_t cache_tokens,
+                               int64_t slot, const rope3d_tables* tables, int trig,
+                               void* cuda_stream);
+
+/*
+ * The rotation alone -- CausalRoPE of Algorithm 3 step 3 / Algorithm 2 -- on one
+ * token range: out[b][r] = RoPE(x[b][r], pos(token_begin + r)).  x and out are
+ * [B][n_tok][N][D] of dtype; out may be x (in place) or must not overlap it.  Other
+ * arguments as for rope3d_qk_norm_rope_append.
+ */
+ROPE3D_API int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
+                 int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                 int T, int H, int W, const rope3d_tables* tables, int trig,
+                 void* cuda_stream);
+
+/*
+ * Integer part of the step, for inspection: for each index i of [token_begin,
+ * token_end) writes out[4 (i - token_begin) + {0,1,2,3}] = t_g, h, w and the cache
+ * row (slot + i) mod cache_tokens, as int64 into the device array out
+ * ([n_tok][4], 8-byte aligned).  Section 3.3.3; Algorithm 3, step 3.
+ */
+ROPE3D_API int rope3d_decode_positions(int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                            int T, int H, int W, int64_t cache_tokens, int64_t slot,
+                            int64_t* out, void* cuda_stream);
+
+/* Fixed text for a status code (never NULL). */
+ROPE3D_API const char* rope3d_strerror(int status);
+
+/* Details of the calling thread's most recent failure ("" if none). */
+ROPE3D_API const char* rope3d_last_error(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+ROPE3D_API int rope3d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROPE3D_H */

@@ -1,0 +1,535 @@
+// rope3d.cu -- host side of librope3d.so: argument checks, frequency tables and
+// kernel launches behind the C ABI of include/rope3d.h.
+//
+// Paper: "Accelerating Video Generation Inference with Sequential-Parallel 3D
+// Positional Encoding Using a Global Time Index" (Yuan & Li).  The tables follow
+// Section 3.4.1 item 2 (precomputed contiguous cos/sin tensors instead of a per-call
+// cache) and Algorithm 2 (one table per axis, concatenated t | h | w).
+#include "rope3d.h"
+#include "rope3d_kernels.cuh"
+
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#ifndef ROPE3D_VPT_TARGET
+#define ROPE3D_VPT_TARGET 4  // vectors per thread per tensor the team size aims for
+#endif
+#ifndef ROPE3D_BLOCK_TARGET
+#define ROPE3D_BLOCK_TARGET 512  // threads per block the team count aims for
+#endif
+
+struct rope3d_tables {
+    int device;
+    int head_dim;
+    int n_t, n_h, n_w;
+    double theta;
+    int schedule;
+    int max_t, max_h, max_w;
+    float2* d_tab;  // one allocation: t table, then h, then w
+    float2* tab_t;
+    float2* tab_h;
+    float2* tab_w;
+    float inv_freq[rope3d::kPairs];
+};
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int ok() {
+    g_last_error[0] = '\0';
+    return ROPE3D_OK;
+}
+
+// ---- per-device facts, looked up once
+struct DeviceInfo {
+    bool known = false;
+    bool supported = false;
+    int sms = 0;
+    int max_smem_optin = 0;
+};
+std::mutex g_mutex;
+std::vector<DeviceInfo> g_devices;
+
+int device_info(DeviceInfo* out, int* device) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if ((int)g_devices.size() <= dev) g_devices.resize(dev + 1);
+    DeviceInfo& d = g_devices[dev];
+    if (!d.known) {
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) ||
+            (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) ||
+            (e = cudaDeviceGetAttribute(&d.max_smem_optin,
+                                        cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)))
+            return fail(ROPE3D_ECUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        d.supported = (major == 10 && minor == 0);
+        d.known = true;
+    }
+    if (!d.supported)
+        return fail(ROPE3D_EDEVICE, "device %d is not compute capability 10.0 (sm_100a)", dev);
+    *out = d;
+    *device = dev;
+    return ROPE3D_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// Checks shared by the fused and apply entry points.
+int check_common(int64_t B, int64_t N, int D, int dtype, int64_t token_begin,
+                 int64_t token_end, int64_t frame_offset, int T, int H, int W,
+                 const rope3d_tables* tables, int trig) {
+    if (tables == nullptr) return fail(ROPE3D_EINVAL, "tables is NULL");
+    if (dtype != ROPE3D_F32 && dtype != ROPE3D_BF16)
+        return fail(ROPE3D_EINVAL, "dtype %d is neither ROPE3D_F32 nor ROPE3D_BF16", dtype);
+    if (D != rope3d::kHeadDim || D != tables->head_dim)
+        return fail(ROPE3D_EINVAL, "head size D=%d: the kernels and these tables need %d", D,
+                    tables->head_dim);
+    if (B < 1 || N < 1) return fail(ROPE3D_EINVAL, "B=%lld and N=%lld must be >= 1",
+                                    (long long)B, (long long)N);
+    if (T < 1 || H < 1 || W < 1)
+        return fail(ROPE3D_EINVAL, "grid T=%d H=%d W=%d must be >= 1", T, H, W);
+    if (frame_offset < 0) return fail(ROPE3D_EINVAL, "frame_offset %lld < 0",
+                                      (long long)frame_offset);
+    const int64_t L = (int64_t)T * H * W;
+    if (token_begin < 0 || token_end <= token_begin)
+        return fail(ROPE3D_ERANGE, "token range [%lld, %lld) is empty or negative",
+                    (long long)token_begin, (long long)token_end);
+    if (token_end > L)
+        return fail(ROPE3D_ERANGE, "token_end %lld exceeds T*H*W = %lld", (long long)token_end,
+                    (long long)L);
+    if (trig != ROPE3D_TRIG_TABLE && trig != ROPE3D_TRIG_ONTHEFLY)
+        return fail(ROPE3D_EINVAL, "trig %d is not a ROPE3D_TRIG_* value", trig);
+    if (trig == ROPE3D_TRIG_TABLE) {
+        const int64_t t_last = frame_offset + (token_end - 1) / ((int64_t)H * W);
+        if (tables->d_tab == nullptr)
+            return fail(ROPE3D_ERANGE, "these tables hold no cos/sin rows; use ROPE3D_TRIG_ONTHEFLY");
+        if (t_last >= tables->max_t || H > tables->max_h || W > tables->max_w)
+            return fail(ROPE3D_ERANGE,
+                        "positions exceed the tables: frame %lld (max_t %d), H %d (max_h %d), "
+                        "W %d (max_w %d)", (long long)t_last, tables->max_t, H, tables->max_h,
+                        W, tables->max_w);
+    }
+    return ROPE3D_OK;
+}
+
+// Team geometry, a function of (N, dtype) only -- it fixes the reduction order, so it
+// must not depend on the token range or the grid.
+struct Geometry {
+    int dim_vecs;
+    int tpr;
+    int vpt;
+};
+
+Geometry geometry(int64_t N, int dtype) {
+    const int elems_per_vec = dtype == ROPE3D_BF16 ? 8 : 4;
+    Geometry g;
+    g.dim_vecs = (int)(N * rope3d::kHeadDim / elems_per_vec);
+    const int per_warp = 32 * ROPE3D_VPT_TARGET;
+    g.tpr = 32 * ((g.dim_vecs + per_warp - 1) / per_warp);
+    g.vpt = (g.dim_vecs + g.tpr - 1) / g.tpr;
+    return g;
+}
+
+using KernelFn = void (*)(const rope3d::Params);
+
+template <typename T, int TRIG, int MODE>
+KernelFn pick_vpt(int vpt) {
+    switch (vpt) {
+        case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE>;
+        case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE>;
+        case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE>;
+        case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE>;
+        default: return nullptr;
+    }
+}
+
+template <int MODE>
+KernelFn pick_kernel(int dtype, int trig, int vpt) {
+    if (dtype == ROPE3D_BF16)
+        return trig == ROPE3D_TRIG_TABLE ? pick_vpt<__nv_bfloat16, rope3d::kTrigTable, MODE>(vpt)
+                                         : pick_vpt<__nv_bfloat16, rope3d::kTrigOnTheFly, MODE>(vpt);
+    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<float, rope3d::kTrigTable, MODE>(vpt)
+                                     : pick_vpt<float, rope3d::kTrigOnTheFly, MODE>(vpt);
+}
+
+// Resident blocks per SM for a kernel at a block size and shared-memory size; also
+// raises the kernel's dynamic shared-memory limit when needed.  Cached per device.
+struct OccKey {
+    int dev;
+    KernelFn fn;
+    int threads;
+    size_t smem;
+    int blocks;
+};
+std::vector<OccKey> g_occ;
+
+int occupancy(int dev, KernelFn fn, int threads, size_t smem, int* blocks) {
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        for (const OccKey& k : g_occ)
+            if (k.dev == dev && k.fn == fn && k.threads == threads && k.smem == smem) {
+                *blocks = k.blocks;
+                return ROPE3D_OK;
+            }
+    }
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return fail(ROPE3D_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(fn),
+                                                      threads, smem);
+    if (e != cudaSuccess)
+        return fail(ROPE3D_ECUDA, "cudaOccupancyMaxActiveBlocksPerMultiprocessor: %s",
+                    cudaGetErrorString(e));
+    if (n < 1) return fail(ROPE3D_EINVAL, "a block of %d threads with %zu bytes of shared "
+                                          "memory does not fit on an SM", threads, smem);
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_occ.push_back(OccKey{dev, fn, threads, smem, n});
+    *blocks = n;
+    return ROPE3D_OK;
+}
+
+template <int MODE>
+int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const DeviceInfo& info,
+           cudaStream_t stream) {
+    const Geometry g = geometry(N, dtype);
+    if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4)
+        return fail(ROPE3D_EINVAL, "N=%lld heads is more than one row team can hold",
+                    (long long)N);
+    int teams = (ROPE3D_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_BLOCK_TARGET
+                                                                : rope3d::kMaxBlockThreads) / g.tpr;
+    if (teams < 1) teams = 1;
+    if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
+    if ((int64_t)teams > p.units) teams = (int)p.units;
+    const int threads = teams * g.tpr;
+    const int warps_per_team = g.tpr / 32;
+    size_t smem = 0;
+    if (MODE == rope3d::kModeFused) {
+        smem = (size_t)2 * p.dim * sizeof(float);
+        if (warps_per_team > 1) smem += (size_t)2 * teams * warps_per_team * sizeof(float2);
+    }
+    if (smem > (size_t)info.max_smem_optin)
+        return fail(ROPE3D_EINVAL, "N=%lld needs %zu bytes of shared memory (limit %d)",
+                    (long long)N, smem, info.max_smem_optin);
+    KernelFn fn = pick_kernel<MODE>(dtype, trig, g.vpt);
+    if (fn == nullptr) return fail(ROPE3D_EINVAL, "no kernel for vpt=%d", g.vpt);
+    int per_sm = 0;
+    int rc = occupancy(dev, fn, threads, smem, &per_sm);
+    if (rc != ROPE3D_OK) return rc;
+    const int64_t needed = (p.units + teams - 1) / teams;
+    int64_t grid = (int64_t)info.sms * per_sm;
+    if (grid > needed) grid = needed;
+    p.dim_vecs = g.dim_vecs;
+    p.tpr = g.tpr;
+    p.teams = teams;
+    fn<<<(unsigned)grid, threads, smem, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+void fill_common(rope3d::Params& p, int64_t B, int64_t N, int64_t token_begin, int64_t token_end,
+                 int64_t frame_offset, int H, int W, const rope3d_tables* tables) {
+    p.n_tok = token_end - token_begin;
+    p.units = B * p.n_tok;
+    p.token_begin = token_begin;
+    p.frame_offset = frame_offset;
+    p.hw = (int64_t)H * W;
+    p.H = H;
+    p.W = W;
+    p.dim = (int)(N * rope3d::kHeadDim);
+    p.inv_dim = 1.0f / (float)p.dim;
+    p.n_t = tables->n_t;
+    p.n_h = tables->n_h;
+    p.n_w = tables->n_w;
+    p.tab_t = tables->tab_t;
+    p.tab_h = tables->tab_h;
+    p.tab_w = tables->tab_w;
+    std::memcpy(p.inv_freq, tables->inv_freq, sizeof(p.inv_freq));
+}
+
+int check_tables_device(const rope3d_tables* tables, int dev) {
+    if (tables->device != dev)
+        return fail(ROPE3D_EDEVICE, "tables were built on device %d, current device is %d",
+                    tables->device, dev);
+    return ROPE3D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rope3d_version(void) { return 10000; }
+
+const char* rope3d_strerror(int status) {
+    switch (status) {
+        case ROPE3D_OK: return "success";
+        case ROPE3D_EINVAL: return "invalid argument";
+        case ROPE3D_ERANGE: return "index range out of bounds";
+        case ROPE3D_ECUDA: return "CUDA runtime error";
+        case ROPE3D_EDEVICE: return "unsupported or mismatched device";
+        case ROPE3D_EALIGN: return "tensor pointer not 16-byte aligned";
+        case ROPE3D_EOVERLAP: return "output buffers overlap";
+        default: return "unknown status";
+    }
+}
+
+const char* rope3d_last_error(void) { return g_last_error; }
+
+int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int n_w,
+                       double theta, int max_t, int max_h, int max_w, int schedule,
+                       void* cuda_stream) {
+    if (out == nullptr) return fail(ROPE3D_EINVAL, "out is NULL");
+    *out = nullptr;
+    if (n_t < 0 || n_h < 0 || n_w < 0 || head_dim != 2 * (n_t + n_h + n_w))
+        return fail(ROPE3D_EINVAL, "head_dim %d != 2 (n_t + n_h + n_w) = 2 (%d + %d + %d)",
+                    head_dim, n_t, n_h, n_w);
+    if (head_dim != rope3d::kHeadDim)
+        return fail(ROPE3D_EINVAL, "head_dim %d: the kernels support %d", head_dim,
+                    rope3d::kHeadDim);
+    if (!(theta > 1.0) || !std::isfinite(theta))
+        return fail(ROPE3D_EINVAL, "theta must be finite and > 1");
+    if (schedule != ROPE3D_SCHEDULE_PER_AXIS && schedule != ROPE3D_SCHEDULE_HEAD_WIDE)
+        return fail(ROPE3D_EINVAL, "schedule %d is not a ROPE3D_SCHEDULE_* value", schedule);
+    if (max_t < 0 || max_h < 0 || max_w < 0)
+        return fail(ROPE3D_EINVAL, "table sizes must be >= 0");
+    const bool with_tables = max_t > 0 || max_h > 0 || max_w > 0;
+    if (with_tables && (max_t == 0 || max_h == 0 || max_w == 0))
+        return fail(ROPE3D_EINVAL, "max_t, max_h, max_w must be all zero or all positive");
+    if ((int64_t)max_t * n_t + (int64_t)max_h * n_h + (int64_t)max_w * n_w > (int64_t)1 << 28)
+        return fail(ROPE3D_EINVAL, "tables too large");
+    DeviceInfo info;
+    int dev = 0;
+    int rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+
+    rope3d_tables* tb = new rope3d_tables();
+    tb->device = dev;
+    tb->head_dim = head_dim;
+    tb->n_t = n_t;
+    tb->n_h = n_h;
+    tb->n_w = n_w;
+    tb->theta = theta;
+    tb->schedule = schedule;
+    tb->max_t = max_t;
+    tb->max_h = max_h;
+    tb->max_w = max_w;
+    tb->d_tab = nullptr;
+
+    // Inverse frequency of every pair, in double, then the fp32 copy the on-the-fly
+    // path multiplies positions by.
+    const int n_axis[3] = {n_t, n_h, n_w};
+    const int pairs = n_t + n_h + n_w;
+    double inv[rope3d::kPairs];
+    int first = 0;
+    for (int a = 0; a < 3; ++a) {
+        for (int j = 0; j < n_axis[a]; ++j) {
+            const double e = schedule == ROPE3D_SCHEDULE_PER_AXIS
+                                 ? (double)(2 * j) / (double)(2 * n_axis[a])
+                                 : (double)(2 * (first + j)) / (double)(2 * pairs);
+            inv[first + j] = std::pow(theta, -e);
+            tb->inv_freq[first + j] = (float)inv[first + j];
+        }
+        first += n_axis[a];
+    }
+
+    if (with_tables) {
+        const int max_pos[3] = {max_t, max_h, max_w};
+        size_t count = 0;
+        for (int a = 0; a < 3; ++a) count += (size_t)max_pos[a] * n_axis[a];
+        std::vector<float2> host(count);
+        size_t off = 0;
+        size_t axis_off[3];
+        first = 0;
+        for (int a = 0; a < 3; ++a) {
+            axis_off[a] = off;
+            for (int p = 0; p < max_pos[a]; ++p)
+                for (int j = 0; j < n_axis[a]; ++j) {
+                    const double phi = (double)p * inv[first + j];
+                    host[off++] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+                }
+            first += n_axis[a];
+        }
+        cudaError_t e = cudaMalloc(&tb->d_tab, count * sizeof(float2));
+        if (e != cudaSuccess) {
+            delete tb;
+            return fail(ROPE3D_ECUDA, "cudaMalloc(%zu): %s", count * sizeof(float2),
+                        cudaGetErrorString(e));
+        }
+        cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+        e = cudaMemcpyAsync(tb->d_tab, host.data(), count * sizeof(float2),
+                            cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+        if (e != cudaSuccess) {
+            cudaFree(tb->d_tab);
+            delete tb;
+            return fail(ROPE3D_ECUDA, "table upload: %s", cudaGetErrorString(e));
+        }
+        tb->tab_t = tb->d_tab + axis_off[0];
+        tb->tab_h = tb->d_tab + axis_off[1];
+        tb->tab_w = tb->d_tab + axis_off[2];
+    } else {
+        tb->tab_t = tb->tab_h = tb->tab_w = nullptr;
+    }
+    *out = tb;
+    return ok();
+}
+
+void rope3d_tables_destroy(rope3d_tables* tables) {
+    if (tables == nullptr) return;
+    if (tables->d_tab != nullptr) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        if (cur != tables->device) cudaSetDevice(tables->device);
+        cudaDeviceSynchronize();
+        cudaFree(tables->d_tab);
+        if (cur != tables->device) cudaSetDevice(cur);
+    }
+    delete tables;
+}
+
+int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void* q_out,
+                               int64_t B, int64_t N, int D, int dtype,
+                               int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                               int T, int H, int W,
+                               const float* q_norm_w, const float* k_norm_w, float eps,
+                               void* k_cache, void* v_cache, int64_t cache_tokens,
+                               int64_t slot, const rope3d_tables* tables, int trig,
+                               void* cuda_stream) {
+    int rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
+                          trig);
+    if (rc != ROPE3D_OK) return rc;
+    if (!q || !k || !v || !q_out || !k_cache || !v_cache || !q_norm_w || !k_norm_w)
+        return fail(ROPE3D_EINVAL, "a tensor pointer is NULL");
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(ROPE3D_EINVAL, "eps must be >= 0");
+    if (cache_tokens < 1) return fail(ROPE3D_EINVAL, "cache_tokens must be >= 1");
+    if (slot < 0) return fail(ROPE3D_EINVAL, "slot must be >= 0");
+    if (token_end - token_begin > cache_tokens)
+        return fail(ROPE3D_ERANGE, "%lld tokens do not fit a cache of %lld rows",
+                    (long long)(token_end - token_begin), (long long)cache_tokens);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_out) ||
+        !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q_norm_w) ||
+        !aligned16(k_norm_w))
+        return fail(ROPE3D_EALIGN, "every tensor pointer must be 16-byte aligned");
+    const size_t esz = dtype == ROPE3D_BF16 ? 2 : 4;
+    const size_t row = (size_t)N * D * esz;
+    const size_t act = (size_t)B * (size_t)(token_end - token_begin) * row;
+    const size_t cache = (size_t)B * (size_t)cache_tokens * row;
+    if (q_out != q && overlap(q_out, act, q, act))
+        return fail(ROPE3D_EOVERLAP, "q_out partly overlaps q (only exact in-place is allowed)");
+    if (overlap(q_out, act, k, act) || overlap(q_out, act, v, act) ||
+        overlap(q_out, act, k_cache, cache) || overlap(q_out, act, v_cache, cache))
+        return fail(ROPE3D_EOVERLAP, "q_out overlaps k, v or a cache");
+    if (overlap(k_cache, cache, v_cache, cache) || overlap(k_cache, cache, q, act) ||
+        overlap(k_cache, cache, k, act) || overlap(k_cache, cache, v, act) ||
+        overlap(v_cache, cache, q, act) || overlap(v_cache, cache, k, act) ||
+        overlap(v_cache, cache, v, act))
+        return fail(ROPE3D_EOVERLAP, "a cache overlaps the other cache or an input");
+
+    DeviceInfo info;
+    int dev = 0;
+    rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_tables_device(tables, dev);
+    if (rc != ROPE3D_OK) return rc;
+
+    rope3d::Params p{};
+    fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.q_out = q_out;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.q_w = q_norm_w;
+    p.k_w = k_norm_w;
+    p.cache_tokens = cache_tokens;
+    p.slot = slot;
+    p.eps = eps;
+    return launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info,
+                                      static_cast<cudaStream_t>(cuda_stream));
+}
+
+int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
+                 int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                 int T, int H, int W, const rope3d_tables* tables, int trig,
+                 void* cuda_stream) {
+    int rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
+                          trig);
+    if (rc != ROPE3D_OK) return rc;
+    if (!x || !out) return fail(ROPE3D_EINVAL, "a tensor pointer is NULL");
+    if (!aligned16(x) || !aligned16(out))
+        return fail(ROPE3D_EALIGN, "every tensor pointer must be 16-byte aligned");
+    const size_t esz = dtype == ROPE3D_BF16 ? 2 : 4;
+    const size_t act = (size_t)B * (size_t)(token_end - token_begin) * (size_t)N * D * esz;
+    if (out != x && overlap(out, act, x, act))
+        return fail(ROPE3D_EOVERLAP, "out partly overlaps x (only exact in-place is allowed)");
+    DeviceInfo info;
+    int dev = 0;
+    rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_tables_device(tables, dev);
+    if (rc != ROPE3D_OK) return rc;
+    rope3d::Params p{};
+    fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
+    p.q = x;
+    p.q_out = out;
+    return launch<rope3d::kModeApply>(p, N, dtype, trig, dev, info,
+                                      static_cast<cudaStream_t>(cuda_stream));
+}
+
+int rope3d_decode_positions(int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                            int T, int H, int W, int64_t cache_tokens, int64_t slot,
+                            int64_t* out, void* cuda_stream) {
+    if (T < 1 || H < 1 || W < 1)
+        return fail(ROPE3D_EINVAL, "grid T=%d H=%d W=%d must be >= 1", T, H, W);
+    if (frame_offset < 0 || cache_tokens < 1 || slot < 0)
+        return fail(ROPE3D_EINVAL, "frame_offset, slot must be >= 0 and cache_tokens >= 1");
+    if (token_begin < 0 || token_end <= token_begin)
+        return fail(ROPE3D_ERANGE, "token range [%lld, %lld) is empty or negative",
+                    (long long)token_begin, (long long)token_end);
+    if (token_end > (int64_t)T * H * W)
+        return fail(ROPE3D_ERANGE, "token_end exceeds T*H*W");
+    if (out == nullptr) return fail(ROPE3D_EINVAL, "out is NULL");
+    if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0)
+        return fail(ROPE3D_EALIGN, "out must be 8-byte aligned");
+    DeviceInfo info;
+    int dev = 0;
+    int rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    const int64_t n = token_end - token_begin;
+    const int threads = 256;
+    const int64_t blocks = (n + threads - 1) / threads;
+    rope3d::decode_positions_kernel<<<(unsigned)blocks, threads, 0,
+                                      static_cast<cudaStream_t>(cuda_stream)>>>(
+        token_begin, n, frame_offset, (int64_t)H * W, W, H, cache_tokens, slot, out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,213 @@
+"""ctypes binding of librope3d.so (include/rope3d.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does nothing but
+turn torch tensors into device pointers and sizes, call the library on the current
+CUDA stream, and turn a negative status into an exception.  All the work runs in the
+library's CUDA kernels; there is no CPU path.  If the library has not been built,
+the first call raises ``RuntimeError`` naming the build command.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "librope3d.so")
+
+ROPE3D_OK = 0
+ROPE3D_EINVAL = -1
+ROPE3D_ERANGE = -2
+ROPE3D_ECUDA = -3
+ROPE3D_EDEVICE = -4
+ROPE3D_EALIGN = -5
+ROPE3D_EOVERLAP = -6
+
+ROPE3D_F32 = 0
+ROPE3D_BF16 = 1
+
+ROPE3D_SCHEDULE_PER_AXIS = 0
+ROPE3D_SCHEDULE_HEAD_WIDE = 1
+
+ROPE3D_TRIG_TABLE = 0
+ROPE3D_TRIG_ONTHEFLY = 1
+
+_VP = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+
+# name -> (argtypes, restype), in the order of include/rope3d.h
+SIGNATURES = {
+    "rope3d_tables_init": ([ctypes.POINTER(_VP), _INT, _INT, _INT, _INT, ctypes.c_double,
+                            _INT, _INT, _INT, _INT, _VP], _INT),
+    "rope3d_tables_destroy": ([_VP], None),
+    "rope3d_qk_norm_rope_append": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64,
+                                    _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP, _VP, _I64,
+                                    _I64, _VP, _INT, _VP], _INT),
+    "rope3d_apply": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT, _VP,
+                      _INT, _VP], _INT),
+    "rope3d_decode_positions": ([_I64, _I64, _I64, _INT, _INT, _INT, _I64, _I64, _VP, _VP], _INT),
+    "rope3d_strerror": ([_INT], ctypes.c_char_p),
+    "rope3d_last_error": ([], ctypes.c_char_p),
+    "rope3d_version": ([], _INT),
+}
+
+_lib = None
+
+
+def load_library(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load librope3d.so and declare its entry points (no CUDA call is made)."""
+    global _lib
+    if _lib is not None and path == LIBRARY:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m rotary_position_encoding_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    if path == LIBRARY:
+        _lib = lib
+    return lib
+
+
+class Rope3dError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"rope3d status {status}: {detail}")
+
+
+def _check(status: int) -> None:
+    if status != ROPE3D_OK:
+        lib = load_library()
+        msg = lib.rope3d_last_error().decode() or lib.rope3d_strerror(status).decode()
+        raise Rope3dError(status, msg)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ROPE3D_BF16
+    if t.dtype == torch.float32:
+        return ROPE3D_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _dev_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class Tables:
+    """Owns a ``rope3d_tables*``; frees it when garbage-collected or on ``close()``."""
+
+    def __init__(self, handle: int, head_dim, n_t, n_h, n_w, theta, max_t, max_h, max_w,
+                 schedule):
+        self.handle = handle
+        self.head_dim, self.n_t, self.n_h, self.n_w = head_dim, n_t, n_h, n_w
+        self.theta, self.schedule = theta, schedule
+        self.max_t, self.max_h, self.max_w = max_t, max_h, max_w
+
+    def close(self) -> None:
+        if self.handle:
+            load_library().rope3d_tables_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def rope3d_tables_init(head_dim: int = 128, n_t: int = 22, n_h: int = 21, n_w: int = 21,
+                       theta: float = 10000.0, max_t: int = 0, max_h: int = 0, max_w: int = 0,
+                       schedule: int = ROPE3D_SCHEDULE_PER_AXIS, stream=None) -> Tables:
+    lib = load_library()
+    handle = _VP()
+    _check(lib.rope3d_tables_init(ctypes.byref(handle), head_dim, n_t, n_h, n_w, theta, max_t,
+                                  max_h, max_w, schedule, _stream(stream)))
+    return Tables(handle.value, head_dim, n_t, n_h, n_w, theta, max_t, max_h, max_w, schedule)
+
+
+def rope3d_tables_destroy(tables: Tables) -> None:
+    tables.close()
+
+
+def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
+                               frame_offset: int, T: int, H: int, W: int, q_norm_w, k_norm_w,
+                               eps: float, k_cache, v_cache, slot: int, tables: Tables,
+                               trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
+    """q, k, v, q_out: [B, n_tok, N, 128]; k_cache, v_cache: [B, cache_tokens, N, 128];
+    q_norm_w, k_norm_w: [N*128] float32.  Enqueued on ``stream`` (default: current)."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or q_out.shape != q.shape:
+        raise ValueError("q, k, v and q_out must all be [B, n_tok, N, D]")
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must both be [B, cache_tokens, N, D]")
+    B, n_tok, N, D = q.shape
+    if k_cache.shape[0] != B or k_cache.shape[2:] != q.shape[2:]:
+        raise ValueError("cache shape does not match q")
+    if n_tok != token_end - token_begin:
+        raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
+    code = _dtype_code(q)
+    for name, t in (("k", k), ("v", v), ("q_out", q_out), ("k_cache", k_cache),
+                    ("v_cache", v_cache)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have q's dtype {q.dtype}")
+    for name, t in (("q_norm_w", q_norm_w), ("k_norm_w", k_norm_w)):
+        if t.dtype != torch.float32 or t.numel() != N * D:
+            raise ValueError(f"{name} must be float32 with N*D elements")
+    _check(load_library().rope3d_qk_norm_rope_append(
+        _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
+        B, N, D, code, token_begin, token_end, frame_offset, T, H, W,
+        _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), k_cache.shape[1], slot,
+        tables.handle, trig, _stream(stream)))
+
+
+def rope3d_apply(x, out, token_begin: int, token_end: int, frame_offset: int, T: int, H: int,
+                 W: int, tables: Tables, trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
+    """x, out: [B, n_tok, N, 128] (out may be x)."""
+    if x.dim() != 4 or out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("x and out must be [B, n_tok, N, D] of one dtype")
+    B, n_tok, N, D = x.shape
+    if n_tok != token_end - token_begin:
+        raise ValueError("x has n_tok rows but the range holds token_end - token_begin")
+    _check(load_library().rope3d_apply(
+        _dev_ptr(x, "x"), _dev_ptr(out, "out"), B, N, D, _dtype_code(x), token_begin,
+        token_end, frame_offset, T, H, W, tables.handle, trig, _stream(stream)))
+
+
+def rope3d_decode_positions(token_begin: int, token_end: int, frame_offset: int, T: int,
+                            H: int, W: int, cache_tokens: int, slot: int, out,
+                            stream=None) -> None:
+    """out: int64 CUDA tensor [n_tok, 4] receiving (t_g, h, w, cache row)."""
+    if out.dtype != torch.int64 or out.shape != (token_end - token_begin, 4):
+        raise ValueError("out must be int64 [token_end - token_begin, 4]")
+    _check(load_library().rope3d_decode_positions(
+        token_begin, token_end, frame_offset, T, H, W, cache_tokens, slot,
+        _dev_ptr(out, "out"), _stream(stream)))
+
+
+def rope3d_strerror(status: int) -> str:
+    return load_library().rope3d_strerror(status).decode()
+
+
+def rope3d_last_error() -> str:
+    return load_library().rope3d_last_error().decode()
+
+
+def rope3d_version() -> int:
+    return load_library().rope3d_version()

@@ -1,0 +1,93 @@
+"""The C ABI library without a GPU: it loads, exports every entry point that
+include/rope3d.h declares, and rejects bad arguments with a status (never a crash).
+Compute calls need a GPU and live in the gpu-marked tests."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rotary_position_encoding_b200 import build as native_build
+from rotary_position_encoding_b200 import rope3d
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rope3d.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    native_build.build()
+    return rope3d.load_library()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return re.findall(r"ROPE3D_API\s+[\w\s\*]+?\b(rope3d_\w+)\s*\(", text)
+
+
+def header_constants():
+    text = open(HEADER).read()
+    return {m[0]: int(m[1]) for m in re.findall(r"#define\s+(ROPE3D_[A-Z0-9_]+)\s+\(?(-?\d+)\)?",
+                                                  text)}
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for required in ("rope3d_tables_init", "rope3d_tables_destroy",
+                     "rope3d_qk_norm_rope_append", "rope3d_apply", "rope3d_decode_positions",
+                     "rope3d_strerror"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(rope3d.SIGNATURES), "binding and header disagree"
+
+
+def test_binding_constants_match_header():
+    for name, value in header_constants().items():
+        if hasattr(rope3d, name):
+            assert getattr(rope3d, name) == value, name
+
+
+def test_strerror_and_version(lib):
+    for status in (0, -1, -2, -3, -4, -5, -6, -99):
+        assert lib.rope3d_strerror(status)
+    assert rope3d.rope3d_version() >= 10000
+
+
+def test_null_and_bad_arguments_rejected_without_device(lib):
+    handle = ctypes.c_void_p(12345)
+    # head_dim must equal 2 (n_t + n_h + n_w): rejected before any CUDA call
+    assert lib.rope3d_tables_init(ctypes.byref(handle), 128, 22, 21, 20, 1e4, 0, 0, 0, 0,
+                                  None) == rope3d.ROPE3D_EINVAL
+    assert handle.value is None
+    assert lib.rope3d_tables_init(None, 128, 22, 21, 21, 1e4, 0, 0, 0, 0, None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_tables_init(ctypes.byref(handle), 128, 22, 21, 21, 0.5, 0, 0, 0, 0,
+                                  None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_tables_init(ctypes.byref(handle), 128, 22, 21, 21, 1e4, 0, 0, 0, 7,
+                                  None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_tables_init(ctypes.byref(handle), 128, 22, 21, 21, 1e4, 10, 0, 5, 0,
+                                  None) == rope3d.ROPE3D_EINVAL
+    assert "head_dim" in rope3d.rope3d_last_error() or rope3d.rope3d_last_error()
+    # the fused step and the rotation with NULL tables
+    p = ctypes.c_void_p(0x10000)
+    assert lib.rope3d_qk_norm_rope_append(p, p, p, p, 1, 2, 128, 1, 0, 72, 0, 3, 4, 6, p, p,
+                                          1e-6, p, p, 144, 0, None, 0, None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_apply(p, p, 1, 2, 128, 1, 0, 72, 0, 3, 4, 6, None, 0, None) == rope3d.ROPE3D_EINVAL
+    # decode: empty range, range past the grid, bad grid, misaligned output
+    assert lib.rope3d_decode_positions(5, 5, 0, 3, 4, 6, 144, 0, p, None) == rope3d.ROPE3D_ERANGE
+    assert lib.rope3d_decode_positions(0, 73, 0, 3, 4, 6, 144, 0, p, None) == rope3d.ROPE3D_ERANGE
+    assert lib.rope3d_decode_positions(0, 10, 0, 0, 4, 6, 144, 0, p, None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_decode_positions(0, 10, 0, 3, 4, 6, 0, 0, p, None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_decode_positions(0, 10, 0, 3, 4, 6, 144, 0, ctypes.c_void_p(0x10004),
+                                       None) == rope3d.ROPE3D_EALIGN
+    assert lib.rope3d_decode_positions(0, 10, -1, 3, 4, 6, 144, 0, p, None) == rope3d.ROPE3D_EINVAL
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        rope3d.load_library(str(tmp_path / "librope3d.so"))
