@@ -15,6 +15,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #ifndef ROPE3D_VPT_TARGET
@@ -175,8 +176,10 @@ KernelFn pick_kernel(int dtype, int trig, int vpt) {
                                      : pick_vpt<float, rope3d::kTrigOnTheFly, MODE>(vpt);
 }
 
-// Resident blocks per SM for a kernel at a block size and shared-memory size; also
-// raises the kernel's dynamic shared-memory limit when needed.  Cached per device.
+// Resident blocks per SM for a kernel at a block size and shared-memory size.  The
+// first use of a kernel on a device raises its dynamic shared-memory limit to the
+// device's opt-in maximum (a per-kernel setting, so it is set once and never lowered).
+// Both are cached per device.
 struct OccKey {
     int dev;
     KernelFn fn;
@@ -185,8 +188,10 @@ struct OccKey {
     int blocks;
 };
 std::vector<OccKey> g_occ;
+std::vector<std::pair<int, KernelFn>> g_smem_raised;
 
-int occupancy(int dev, KernelFn fn, int threads, size_t smem, int* blocks) {
+int occupancy(int dev, KernelFn fn, int threads, size_t smem, int max_smem, int* blocks) {
+    bool raised = false;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         for (const OccKey& k : g_occ)
@@ -194,11 +199,18 @@ int occupancy(int dev, KernelFn fn, int threads, size_t smem, int* blocks) {
                 *blocks = k.blocks;
                 return ROPE3D_OK;
             }
+        for (const auto& r : g_smem_raised)
+            if (r.first == dev && r.second == fn) raised = true;
     }
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess)
-        return fail(ROPE3D_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    cudaError_t e;
+    if (!raised) {
+        e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+        if (e != cudaSuccess)
+            return fail(ROPE3D_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        std::lock_guard<std::mutex> lock(g_mutex);
+        g_smem_raised.emplace_back(dev, fn);
+    }
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(fn),
                                                       threads, smem);
@@ -238,7 +250,7 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const Dev
     KernelFn fn = pick_kernel<MODE>(dtype, trig, g.vpt);
     if (fn == nullptr) return fail(ROPE3D_EINVAL, "no kernel for vpt=%d", g.vpt);
     int per_sm = 0;
-    int rc = occupancy(dev, fn, threads, smem, &per_sm);
+    int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
     if (rc != ROPE3D_OK) return rc;
     const int64_t needed = (p.units + teams - 1) / teams;
     int64_t grid = (int64_t)info.sms * per_sm;
@@ -246,8 +258,9 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const Dev
     p.dim_vecs = g.dim_vecs;
     p.tpr = g.tpr;
     p.teams = teams;
-    fn<<<(unsigned)grid, threads, smem, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+    void* args[] = {&p};
+    const cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn),
+                                           dim3((unsigned)grid), dim3(threads), args, smem, stream);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -524,10 +537,12 @@ int rope3d_decode_positions(int64_t token_begin, int64_t token_end, int64_t fram
     const int64_t n = token_end - token_begin;
     const int threads = 256;
     const int64_t blocks = (n + threads - 1) / threads;
-    rope3d::decode_positions_kernel<<<(unsigned)blocks, threads, 0,
-                                      static_cast<cudaStream_t>(cuda_stream)>>>(
-        token_begin, n, frame_offset, (int64_t)H * W, W, H, cache_tokens, slot, out);
-    cudaError_t e = cudaGetLastError();
+    int64_t hw = (int64_t)H * W;
+    void* args[] = {&token_begin, const_cast<int64_t*>(&n), &frame_offset, &hw, &W, &H,
+                    &cache_tokens, &slot, &out};
+    const cudaError_t e = cudaLaunchKernel(
+        reinterpret_cast<const void*>(&rope3d::decode_positions_kernel), dim3((unsigned)blocks),
+        dim3(threads), args, 0, static_cast<cudaStream_t>(cuda_stream));
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }

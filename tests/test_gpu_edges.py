@@ -102,7 +102,7 @@ def test_degenerate_grids(grid, schedule):
     T, H, W = grid
     n = T * H * W
     s, C, slot = 237, n, 0
-    raw, dev, wq, wk, kc, vc, tables = _setup(1, n, 2, "f32", 9, C, 240, H, W, schedule)
+    raw, dev, wq, wk, kc, vc, tables = _setup(1, n, 2, "f32", 9, C, s + T, H, W, schedule)
     qo = torch.empty_like(dev[0])
     rope3d.rope3d_qk_norm_rope_append(dev[0], dev[1], dev[2], qo, 0, n, s, T, H, W,
                                       torch.from_numpy(wq).cuda(), torch.from_numpy(wk).cuda(),
