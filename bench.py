@@ -57,6 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chunk720p")
     ap.add_argument("--trig", choices=["table", "onthefly"], default="table")
+    ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
+                    help="kernel path of the fused step (auto: the bulk-copy ring when it "
+                         "fits in shared memory)")
     ap.add_argument("--chunks", type=int, default=0,
                     help="use only the first CHUNKS chunk calls per step (profiling captures "
                          "of a smaller case; 0 = the whole step)")
@@ -266,6 +269,9 @@ def run_ours(args, dist: Dist):
     max_t = max(c.frame_offset for c in w.chunks) + w.T
     tables = rope3d.rope3d_tables_init(max_t=max_t, max_h=w.H, max_w=w.W)
     stream = torch.cuda.current_stream(device)
+    rope3d.rope3d_testing_force_path({"auto": rope3d.ROPE3D_PATH_AUTO,
+                                      "registers": rope3d.ROPE3D_PATH_REGISTERS,
+                                      "tma": rope3d.ROPE3D_PATH_TMA}[args.path])
 
     def step(events=None):
         for ci, chunk in enumerate(w.chunks):
@@ -315,6 +321,9 @@ def run_ours(args, dist: Dist):
     total_tokens = tokens_per_step * args.steps * dist.world
     value = total_tokens / (elapsed_ms / 1e3)
 
+    device_status = rope3d.rope3d_check_device_status(tables)
+    if device_status != rope3d.ROPE3D_OK:
+        raise RuntimeError("a kernel wait timed out during the benchmark")
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
@@ -336,7 +345,8 @@ def run_ours(args, dist: Dist):
         "traffic": recorded_traffic(w.name, args.trig),
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
         else "fallback 6.65 TB/s",
-        "kernel": "rope3d::qk_norm_rope_kernel",
+        "kernel": "rope3d::qk_norm_rope_tma_kernel" if args.path != "registers"
+        else "rope3d::qk_norm_rope_kernel",
         "algorithmic_bytes_per_launch": bytes_per_launch,
         "avg_launch_us": round(avg_launch_ms * 1e3, 2),
     }
@@ -363,6 +373,7 @@ def run_ours(args, dist: Dist):
             "head_dim": wl.HEAD_DIM,
             "cache_tokens": w.cache_tokens,
             "trig": args.trig,
+            "kernel_path": args.path,
             "l2": "no flush: inputs larger than L2 (each launch streams "
                   f"{bytes_per_launch / 1e6:.1f} MB from its own buffers)",
             "parallelism": f"replicas x{dist.world} (independent streams, no collective)",

@@ -59,6 +59,7 @@ extern "C" {
 #define ROPE3D_EDEVICE (-4)  /* no sm_100 device, or the tables live on another device */
 #define ROPE3D_EALIGN (-5)   /* a tensor pointer is not 16-byte aligned                */
 #define ROPE3D_EOVERLAP (-6) /* output buffers overlap each other or an input          */
+#define ROPE3D_ETIMEOUT (-7) /* a kernel gave up a bounded wait (see check_device_status) */
 
 /* Element types of q, k, v, q_out and the caches (all the same type). */
 #define ROPE3D_F32 0
@@ -163,6 +164,17 @@ ROPE3D_API int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int 
 ROPE3D_API int rope3d_decode_positions(int64_t token_begin, int64_t token_end, int64_t frame_offset,
                             int T, int H, int W, int64_t cache_tokens, int64_t slot,
                             int64_t* out, void* cuda_stream);
+
+/*
+ * Device-side status of the kernels launched with these tables.  The fused kernel that
+ * streams rows through shared memory waits on each stage with a time limit (2 s); if a
+ * stage never fills, the kernel stops, its output rows are incomplete, and it records
+ * the event in a device word that belongs to the tables.  This call synchronises
+ * cuda_stream, reads and clears that word, and returns ROPE3D_ETIMEOUT if any launch
+ * since the last check gave up, else ROPE3D_OK (ECUDA / EDEVICE / EINVAL on failure to
+ * read it).  Not needed on the normal path; intended for health checks.
+ */
+ROPE3D_API int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream);
 
 /* Fixed text for a status code (never NULL). */
 ROPE3D_API const char* rope3d_strerror(int status);

@@ -1,0 +1,37 @@
+/*
+ * rope3d_testing.h -- test hooks of librope3d.so.  Not for production use: they change
+ * process-wide settings of the library for every later launch on every thread.
+ */
+#ifndef ROPE3D_TESTING_H
+#define ROPE3D_TESTING_H
+
+#include <stdint.h>
+
+#include "rope3d.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Kernel path of rope3d_qk_norm_rope_append. */
+#define ROPE3D_PATH_AUTO 0       /* bulk-copy ring when it fits in shared memory, else registers */
+#define ROPE3D_PATH_REGISTERS 1  /* rows loaded straight into registers                        */
+#define ROPE3D_PATH_TMA 2        /* rows streamed through shared memory (EINVAL if it does not fit) */
+
+/*
+ * Bounded-wait settings of the bulk-copy ring kernel for later launches:
+ * wait_limit_ns replaces the 2 s limit (0 restores it); tx_extra_bytes makes every
+ * stage wait for that many bytes more than its copies deliver, so its wait runs out
+ * and the kernel reports ROPE3D_ETIMEOUT through rope3d_check_device_status (0 is the
+ * normal setting).  No fault is involved: the copies land, the wait simply expires.
+ */
+ROPE3D_API void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes);
+
+/* Choose the kernel path for later launches (ROPE3D_PATH_*).  EINVAL for other values. */
+ROPE3D_API int rope3d_testing_force_path(int path);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROPE3D_TESTING_H */

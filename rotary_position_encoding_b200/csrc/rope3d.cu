@@ -6,7 +6,9 @@
 // Section 3.4.1 item 2 (precomputed contiguous cos/sin tensors instead of a per-call
 // cache) and Algorithm 2 (one table per axis, concatenated t | h | w).
 #include "rope3d.h"
+#include "rope3d_testing.h"
 #include "rope3d_kernels.cuh"
+#include "rope3d_tma.cuh"
 
 #include <cuda_runtime.h>
 
@@ -14,6 +16,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -36,12 +39,19 @@ struct rope3d_tables {
     float2* tab_t;
     float2* tab_h;
     float2* tab_w;
+    int* d_status;  // device word the bounded waits of the TMA kernel report into
     float inv_freq[rope3d::kPairs];
 };
 
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// Settings that tests use to exercise the bounded waits and both kernel paths.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<uint32_t> g_tx_extra{0};
+std::atomic<int> g_force_path{ROPE3D_PATH_AUTO};
 
 int fail(int status, const char* fmt, ...) {
     va_list ap;
@@ -176,6 +186,27 @@ KernelFn pick_kernel(int dtype, int trig, int vpt) {
                                      : pick_vpt<float, rope3d::kTrigOnTheFly, MODE>(vpt);
 }
 
+using TmaKernelFn = void (*)(const rope3d::Params);
+
+template <typename T, int TRIG>
+TmaKernelFn pick_tma_vpt(int vpt) {
+    switch (vpt) {
+        case 1: return rope3d::qk_norm_rope_tma_kernel<T, 1, TRIG>;
+        case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG>;
+        case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG>;
+        case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG>;
+        default: return nullptr;
+    }
+}
+
+TmaKernelFn pick_tma_kernel(int dtype, int trig, int vpt) {
+    if (dtype == ROPE3D_BF16)
+        return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<__nv_bfloat16, rope3d::kTrigTable>(vpt)
+                                         : pick_tma_vpt<__nv_bfloat16, rope3d::kTrigOnTheFly>(vpt);
+    return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<float, rope3d::kTrigTable>(vpt)
+                                     : pick_tma_vpt<float, rope3d::kTrigOnTheFly>(vpt);
+}
+
 // Resident blocks per SM for a kernel at a block size and shared-memory size.  The
 // first use of a kernel on a device raises its dynamic shared-memory limit to the
 // device's opt-in maximum (a per-kernel setting, so it is set once and never lowered).
@@ -223,6 +254,81 @@ int occupancy(int dev, KernelFn fn, int threads, size_t smem, int max_smem, int*
     g_occ.push_back(OccKey{dev, fn, threads, smem, n});
     *blocks = n;
     return ROPE3D_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shared-memory plan of the TMA kernel for `teams` teams of `stages` stages each;
+// returns the total dynamic shared memory and fills the offsets.
+size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) {
+    size_t off = 0;
+    p.off_bars = (uint32_t)off;
+    off += (size_t)teams * stages * sizeof(uint64_t);
+    off = align_up(off, 16);
+    p.off_fail = (uint32_t)off;
+    off += (size_t)teams * sizeof(int);
+    off = align_up(off, 16);
+    p.off_part = (uint32_t)off;
+    off += (size_t)2 * teams * warps_per_team * sizeof(float2);
+    off = align_up(off, 16);
+    p.off_w = (uint32_t)off;
+    off += (size_t)2 * p.dim * sizeof(float);
+    off = align_up(off, 128);
+    p.off_stage = (uint32_t)off;
+    off += (size_t)teams * stages * 3 * p.row_bytes;
+    return off;
+}
+
+#ifndef ROPE3D_TMA_MAX_STAGES
+#define ROPE3D_TMA_MAX_STAGES 4
+#endif
+
+// The fused step through the bulk-copy ring, when a ring of at least two stages per
+// team fits in shared memory; returns 1 if it launched nothing (caller falls back).
+int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
+                     const DeviceInfo& info, cudaStream_t stream, bool* launched) {
+    *launched = false;
+    const Geometry g = geometry(N, dtype);
+    if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
+    const int warps_per_team = g.tpr / 32;
+    p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
+    int teams = (ROPE3D_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_BLOCK_TARGET
+                                                                : rope3d::kMaxBlockThreads) / g.tpr;
+    if (teams < 1) teams = 1;
+    if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
+    if ((int64_t)teams > p.units) teams = (int)p.units;
+    int stages = 0;
+    size_t smem = 0;
+    for (; teams >= 1; --teams) {
+        for (stages = ROPE3D_TMA_MAX_STAGES; stages >= 2; --stages) {
+            smem = tma_layout(p, teams, stages, warps_per_team);
+            if (smem <= (size_t)info.max_smem_optin) break;
+        }
+        if (stages >= 2) break;
+    }
+    if (teams < 1 || stages < 2) return ROPE3D_OK;  // does not fit: register kernel
+    smem = tma_layout(p, teams, stages, warps_per_team);
+    TmaKernelFn fn = pick_tma_kernel(dtype, trig, g.vpt);
+    if (fn == nullptr) return ROPE3D_OK;
+    const int threads = teams * g.tpr;
+    int per_sm = 0;
+    int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
+    if (rc != ROPE3D_OK) return rc;
+    const int64_t needed = (p.units + teams - 1) / teams;
+    int64_t grid = (int64_t)info.sms * per_sm;
+    if (grid > needed) grid = needed;
+    p.dim_vecs = g.dim_vecs;
+    p.tpr = g.tpr;
+    p.teams = teams;
+    p.stages = stages;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.tx_extra = g_tx_extra.load();
+    void* args[] = {&p};
+    const cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn),
+                                           dim3((unsigned)grid), dim3(threads), args, smem, stream);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
+    *launched = true;
+    return ok();
 }
 
 template <int MODE>
@@ -283,6 +389,15 @@ void fill_common(rope3d::Params& p, int64_t B, int64_t N, int64_t token_begin, i
     p.tab_h = tables->tab_h;
     p.tab_w = tables->tab_w;
     std::memcpy(p.inv_freq, tables->inv_freq, sizeof(p.inv_freq));
+    p.status = tables->d_status;
+    p.cache_tokens = 1;  // the fused entry point overwrites these two
+    p.slot = 0;
+}
+
+void set_small_idx(rope3d::Params& p) {
+    const int64_t lim = (int64_t)1 << 31;
+    p.small_idx = (p.units < lim && p.token_begin + p.n_tok + p.slot < lim &&
+                   p.cache_tokens < lim && p.hw < lim) ? 1 : 0;
 }
 
 int check_tables_device(const rope3d_tables* tables, int dev) {
@@ -307,6 +422,7 @@ const char* rope3d_strerror(int status) {
         case ROPE3D_EDEVICE: return "unsupported or mismatched device";
         case ROPE3D_EALIGN: return "tensor pointer not 16-byte aligned";
         case ROPE3D_EOVERLAP: return "output buffers overlap";
+        case ROPE3D_ETIMEOUT: return "a kernel wait timed out";
         default: return "unknown status";
     }
 }
@@ -352,6 +468,16 @@ int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int 
     tb->max_h = max_h;
     tb->max_w = max_w;
     tb->d_tab = nullptr;
+    tb->d_status = nullptr;
+    {
+        cudaError_t e = cudaMalloc(&tb->d_status, 16);
+        if (e == cudaSuccess) e = cudaMemset(tb->d_status, 0, 16);
+        if (e != cudaSuccess) {
+            if (tb->d_status) cudaFree(tb->d_status);
+            delete tb;
+            return fail(ROPE3D_ECUDA, "status word allocation: %s", cudaGetErrorString(e));
+        }
+    }
 
     // Inverse frequency of every pair, in double, then the fp32 copy the on-the-fly
     // path multiplies positions by.
@@ -389,6 +515,7 @@ int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int 
         }
         cudaError_t e = cudaMalloc(&tb->d_tab, count * sizeof(float2));
         if (e != cudaSuccess) {
+            cudaFree(tb->d_status);
             delete tb;
             return fail(ROPE3D_ECUDA, "cudaMalloc(%zu): %s", count * sizeof(float2),
                         cudaGetErrorString(e));
@@ -399,6 +526,7 @@ int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int 
         if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
         if (e != cudaSuccess) {
             cudaFree(tb->d_tab);
+            cudaFree(tb->d_status);
             delete tb;
             return fail(ROPE3D_ECUDA, "table upload: %s", cudaGetErrorString(e));
         }
@@ -414,15 +542,47 @@ int rope3d_tables_init(rope3d_tables** out, int head_dim, int n_t, int n_h, int 
 
 void rope3d_tables_destroy(rope3d_tables* tables) {
     if (tables == nullptr) return;
-    if (tables->d_tab != nullptr) {
-        int cur = 0;
-        cudaGetDevice(&cur);
-        if (cur != tables->device) cudaSetDevice(tables->device);
-        cudaDeviceSynchronize();
-        cudaFree(tables->d_tab);
-        if (cur != tables->device) cudaSetDevice(cur);
-    }
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != tables->device) cudaSetDevice(tables->device);
+    cudaDeviceSynchronize();
+    if (tables->d_tab != nullptr) cudaFree(tables->d_tab);
+    if (tables->d_status != nullptr) cudaFree(tables->d_status);
+    if (cur != tables->device) cudaSetDevice(cur);
     delete tables;
+}
+
+int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream) {
+    if (tables == nullptr) return fail(ROPE3D_EINVAL, "tables is NULL");
+    int cur = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (cur != tables->device)
+        return fail(ROPE3D_EDEVICE, "tables were built on device %d, current device is %d",
+                    tables->device, cur);
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    int word = 0;
+    e = cudaMemcpyAsync(&word, tables->d_status, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && word != 0)
+        e = cudaMemsetAsync(tables->d_status, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "status read: %s", cudaGetErrorString(e));
+    if (word & rope3d::kStatusWaitTimeout)
+        return fail(ROPE3D_ETIMEOUT, "a kernel gave up waiting for a shared-memory stage to fill");
+    return ok();
+}
+
+void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes) {
+    g_wait_limit_ns.store(wait_limit_ns ? wait_limit_ns : kDefaultWaitLimitNs);
+    g_tx_extra.store(tx_extra_bytes);
+}
+
+int rope3d_testing_force_path(int path) {
+    if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA)
+        return fail(ROPE3D_EINVAL, "path %d is not a ROPE3D_PATH_* value", path);
+    g_force_path.store(path);
+    return ok();
 }
 
 int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void* q_out,
@@ -483,8 +643,17 @@ int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void
     p.cache_tokens = cache_tokens;
     p.slot = slot;
     p.eps = eps;
-    return launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info,
-                                      static_cast<cudaStream_t>(cuda_stream));
+    set_small_idx(p);
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const int path = g_force_path.load();
+    if (path != ROPE3D_PATH_REGISTERS) {
+        bool launched = false;
+        rc = launch_fused_tma(p, N, dtype, trig, dev, info, stream, &launched);
+        if (rc != ROPE3D_OK || launched) return rc;
+        if (path == ROPE3D_PATH_TMA)
+            return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);
+    }
+    return launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info, stream);
 }
 
 int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
@@ -511,6 +680,7 @@ int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtyp
     fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
     p.q = x;
     p.q_out = out;
+    set_small_idx(p);
     return launch<rope3d::kModeApply>(p, N, dtype, trig, dev, info,
                                       static_cast<cudaStream_t>(cuda_stream));
 }

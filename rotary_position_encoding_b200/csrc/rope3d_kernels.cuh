@@ -5,23 +5,26 @@
 //
 // The step moves 6 * N * 128 elements per token and does ~15 flops per element of
 // q and k, so it is bound by HBM bandwidth, not by arithmetic: no tensor cores.
-// Design:
+//
+// Shared design of both fused kernels:
 //   * A "team" of TPR threads (a multiple of 32) owns one token row at a time.
 //     Thread t of a team holds the 16-byte vectors t, t + TPR, t + 2 TPR, ... of the
-//     row (coalesced 128-bit accesses).  TPR is a multiple of the vectors per head,
-//     so a thread always sees the same position inside a head, hence the same few
-//     complex pairs: its cos/sin are computed once per row and reused for every head
-//     it holds and for both q and k.
+//     row.  TPR is a multiple of the vectors per head, so a thread always sees the
+//     same position inside a head, hence the same few complex pairs: its cos/sin are
+//     computed once per row and reused for every head it holds and for q and k.
 //   * RMSNorm needs the sum of squares of the whole N*128 row before any output, so
-//     a thread keeps its vectors of q, k and v in registers; the sum is a fixed
-//     warp butterfly followed, for multi-warp teams, by a fixed-order sum of the
-//     warps' partials (one named barrier per row, double-buffered partials).  The
-//     reduction order depends only on N and the dtype, never on the token range or
-//     the grid, so any slice of a sequence is bit-identical to the whole.
-//   * Blocks are persistent (grid = SMs x resident blocks); each block stages the
-//     two RMSNorm weight vectors in shared memory once and its teams stride over
-//     the (batch, token) rows.  Inputs are read with evict-first loads; the V row is
-//     stored as soon as it arrives, K and Q once normalised and rotated.
+//     a thread keeps its vectors of the row in registers; the sum is a fixed warp
+//     butterfly followed, for multi-warp teams, by a fixed-order sum of the warps'
+//     partials (one named barrier per row, double-buffered partials).  The reduction
+//     order depends only on N and the dtype, never on the token range or the grid,
+//     so any slice of a sequence is bit-identical to the whole.
+//   * Blocks are persistent; each block stages the two RMSNorm weight vectors in
+//     shared memory once, and its teams stride over the (batch, token) rows.
+//
+// qk_norm_rope_kernel reads the rows straight into registers (coalesced 128-bit
+// loads), so the bytes in flight per SM are bounded by the register file.
+// qk_norm_rope_tma_kernel (rope3d_tma.cuh) streams rows into a ring of shared-memory
+// stages with bulk asynchronous copies, decoupling bytes in flight from registers.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -50,6 +53,7 @@ struct Params {
     const float2* tab_t;  // [max_t][n_t] (cos, sin)
     const float2* tab_h;  // [max_h][n_h]
     const float2* tab_w;  // [max_w][n_w]
+    int* status;          // device status word of the bounded waits (TMA kernel)
     int64_t n_tok;        // rows per batch sample
     int64_t units;        // B * n_tok rows in total
     int64_t token_begin;
@@ -57,15 +61,22 @@ struct Params {
     int64_t cache_tokens;
     int64_t slot;
     int64_t hw;           // H * W
+    uint64_t wait_limit_ns;  // TMA kernel: give up on a stage after this long
     int H;
     int W;
     int dim;              // N * 128 elements per row
     int dim_vecs;         // 16-byte vectors per row
     int tpr;              // threads per team (multiple of 32)
     int teams;            // teams per block
+    int small_idx;        // all index arithmetic fits in 32 bits
     float eps;
     float inv_dim;        // 1 / dim
     int n_t, n_h, n_w;
+    // TMA kernel shared-memory layout (byte offsets into dynamic shared memory)
+    int stages;           // ring stages per team
+    uint32_t row_bytes;   // bytes of one token row of one tensor
+    uint32_t tx_extra;    // extra bytes each stage waits for (0; tests use it to time out)
+    uint32_t off_bars, off_fail, off_part, off_w, off_stage;
     float inv_freq[kPairs];  // fp32 angle per unit position of every pair
 };
 
@@ -121,7 +132,187 @@ __device__ __forceinline__ float warp_allreduce_sum(float x) {
     return x;
 }
 
-// ---------------------------------------------------------------- the kernel
+// ---------------------------------------------------------------- per-row pieces
+
+// Position of token row u (Section 3.3.3: i = token_begin + r, t_g = s + floor(i/HW),
+// h = floor(i/W) mod H, w = i mod W) and its rolling-cache row (slot + i) mod C.
+struct RowPos {
+    int64_t b, r, i, t_g, crow;
+    int h, w;
+};
+
+__device__ __forceinline__ RowPos decode_row(const Params& p, int64_t u) {
+    RowPos q;
+    if (p.small_idx) {
+        const uint32_t uu = (uint32_t)u, ntok = (uint32_t)p.n_tok;
+        const uint32_t b = uu / ntok;
+        const uint32_t r = uu - b * ntok;
+        const uint32_t i = (uint32_t)p.token_begin + r;
+        const uint32_t hw = (uint32_t)p.hw, W = (uint32_t)p.W;
+        const uint32_t tl = i / hw;
+        const uint32_t rem = i - tl * hw;
+        const uint32_t h = rem / W;
+        q.b = b;
+        q.r = r;
+        q.i = i;
+        q.t_g = p.frame_offset + tl;
+        q.h = (int)h;
+        q.w = (int)(rem - h * W);
+        q.crow = ((uint32_t)p.slot + i) % (uint32_t)p.cache_tokens;
+    } else {
+        q.b = u / p.n_tok;
+        q.r = u - q.b * p.n_tok;
+        q.i = p.token_begin + q.r;
+        const int64_t tl = q.i / p.hw;
+        const int64_t rem = q.i - tl * p.hw;
+        q.h = (int)(rem / p.W);
+        q.w = (int)(rem - (int64_t)q.h * p.W);
+        q.t_g = p.frame_offset + tl;
+        q.crow = (p.slot + q.i) % p.cache_tokens;
+    }
+    return q;
+}
+
+// The complex pairs a thread rotates (fixed for the thread's whole life).
+template <int PPV>
+struct PairInfo {
+    float inv[PPV];             // angle per unit position
+    int axis[PPV];              // 0 = t, 1 = h, 2 = w
+    const float2* tab[PPV];     // table column of the pair (row 0)
+    int stride[PPV];            // table row length of the pair's axis
+};
+
+template <int PPV>
+__device__ __forceinline__ PairInfo<PPV> pair_info(const Params& p, int pair0) {
+    PairInfo<PPV> pi;
+#pragma unroll
+    for (int m = 0; m < PPV; ++m) {
+        const int j = pair0 + m;
+        pi.inv[m] = p.inv_freq[j];
+        if (j < p.n_t) {
+            pi.axis[m] = 0; pi.tab[m] = p.tab_t + j; pi.stride[m] = p.n_t;
+        } else if (j < p.n_t + p.n_h) {
+            pi.axis[m] = 1; pi.tab[m] = p.tab_h + (j - p.n_t); pi.stride[m] = p.n_h;
+        } else {
+            pi.axis[m] = 2; pi.tab[m] = p.tab_w + (j - p.n_t - p.n_h); pi.stride[m] = p.n_w;
+        }
+    }
+    return pi;
+}
+
+// cos and sin of each of the thread's pairs at (t_g, h, w): Section 3.3.2 item 2,
+// phi_j = t_g theta_T,j | h theta_H,j | w theta_W,j on the pair's own axis.
+template <int TRIG, int PPV>
+__device__ __forceinline__ void pair_trig(const PairInfo<PPV>& pi, const RowPos& pos,
+                                          float (&cs)[PPV], float (&sn)[PPV]) {
+#pragma unroll
+    for (int m = 0; m < PPV; ++m) {
+        const int64_t x = pi.axis[m] == 0 ? pos.t_g : (pi.axis[m] == 1 ? (int64_t)pos.h
+                                                                        : (int64_t)pos.w);
+        if (TRIG == kTrigTable) {
+            const float2 e = __ldg(pi.tab[m] + x * pi.stride[m]);
+            cs[m] = e.x;
+            sn[m] = e.y;
+        } else {
+            const float phi = (float)x * pi.inv[m];
+            sincosf(phi, &sn[m], &cs[m]);
+        }
+    }
+}
+
+// Sum of squares of this thread's share of one row of q and of k (fixed order).
+template <typename T, int VPT>
+__device__ __forceinline__ void partial_sum_squares(const typename VecTraits<T>::Vec (&xq)[VPT],
+                                                    const typename VecTraits<T>::Vec (&xk)[VPT],
+                                                    int t, int tpr, int dim_vecs, float& sq,
+                                                    float& sk) {
+    using Tr = VecTraits<T>;
+    sq = 0.f;
+    sk = 0.f;
+#pragma unroll
+    for (int s = 0; s < VPT; ++s) {
+        if (t + s * tpr < dim_vecs) {
+#pragma unroll
+            for (int m = 0; m < Tr::kPairsPerVec; ++m) {
+                float a, c;
+                Tr::pair(xq[s], m, a, c);
+                sq = fmaf(a, a, sq);
+                sq = fmaf(c, c, sq);
+                Tr::pair(xk[s], m, a, c);
+                sk = fmaf(a, a, sk);
+                sk = fmaf(c, c, sk);
+            }
+        }
+    }
+}
+
+// Team-wide totals of (sq, sk): warp butterfly, then the warps' partials in warp order.
+// For multi-warp teams this is the row's one named barrier; it also orders every read
+// of the row made before it ahead of everything after it.
+__device__ __forceinline__ float2 team_sum(float sq, float sk, float2* s_part, int team,
+                                           int teams, int warp_in_team, int warps_per_team,
+                                           int lane, int tpr, int& parity) {
+    sq = warp_allreduce_sum(sq);
+    sk = warp_allreduce_sum(sk);
+    if (warps_per_team > 1) {
+        float2* part = s_part + (parity * teams + team) * warps_per_team;
+        if (lane == 0) part[warp_in_team] = make_float2(sq, sk);
+        team_barrier(1 + team, tpr);
+        sq = 0.f;
+        sk = 0.f;
+        for (int wi = 0; wi < warps_per_team; ++wi) {
+            const float2 pp = part[wi];
+            sq += pp.x;
+            sk += pp.y;
+        }
+        parity ^= 1;
+    }
+    return make_float2(sq, sk);
+}
+
+// y = x * rs * w (RMSNorm), then (y_re + i y_im) * (cos + i sin) (RoPE), for the
+// pairs of one vector; weights come from shared memory.
+template <typename T, bool NORM>
+__device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
+    const typename VecTraits<T>::Vec& x, float rs, const float* s_w, int e0,
+    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec]) {
+    using Tr = VecTraits<T>;
+    constexpr int PPV = Tr::kPairsPerVec;
+    float w[2 * PPV];
+    if (NORM) {
+#pragma unroll
+        for (int c = 0; c < 2 * PPV / 4; ++c) {
+            const float4 a = *reinterpret_cast<const float4*>(s_w + e0 + 4 * c);
+            w[4 * c] = a.x; w[4 * c + 1] = a.y; w[4 * c + 2] = a.z; w[4 * c + 3] = a.w;
+        }
+    }
+    typename Tr::Vec out;
+#pragma unroll
+    for (int m = 0; m < PPV; ++m) {
+        float a, c;
+        Tr::pair(x, m, a, c);
+        if (NORM) {
+            a = a * rs * w[2 * m];
+            c = c * rs * w[2 * m + 1];
+        }
+        Tr::set_pair(out, m, a * cs[m] - c * sn[m], a * sn[m] + c * cs[m]);
+    }
+    return out;
+}
+
+__device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, float* s_wk) {
+    // dim is a multiple of 128, so float4 copies cover it
+    const float4* gq = reinterpret_cast<const float4*>(p.q_w);
+    const float4* gk = reinterpret_cast<const float4*>(p.k_w);
+    float4* sq4 = reinterpret_cast<float4*>(s_wq);
+    float4* sk4 = reinterpret_cast<float4*>(s_wk);
+    for (int e = threadIdx.x; e < p.dim / 4; e += blockDim.x) {
+        sq4[e] = __ldg(gq + e);
+        sk4[e] = __ldg(gk + e);
+    }
+}
+
+// ---------------------------------------------------------------- register kernel
 
 template <typename T, int VPT, int TRIG, int MODE>
 __global__ void __launch_bounds__(kMaxBlockThreads)
@@ -144,30 +335,10 @@ qk_norm_rope_kernel(const Params p) {
     const int warps_per_team = p.tpr >> 5;
 
     if (MODE == kModeFused) {
-        // Stage both weight vectors (dim is a multiple of 128, so float4 copies).
-        const float4* gq = reinterpret_cast<const float4*>(p.q_w);
-        const float4* gk = reinterpret_cast<const float4*>(p.k_w);
-        float4* sq4 = reinterpret_cast<float4*>(s_wq);
-        float4* sk4 = reinterpret_cast<float4*>(s_wk);
-        for (int e = tid; e < p.dim / 4; e += blockDim.x) {
-            sq4[e] = __ldg(gq + e);
-            sk4[e] = __ldg(gk + e);
-        }
+        stage_weights(p, s_wq, s_wk);
         __syncthreads();
     }
-
-    // The pairs this thread rotates: positions inside a head are fixed per thread.
-    const int pair0 = (t % Tr::kVecsPerHead) * PPV;
-    float inv[PPV];
-    int axis[PPV];
-    int tab_col[PPV];
-#pragma unroll
-    for (int m = 0; m < PPV; ++m) {
-        const int j = pair0 + m;
-        inv[m] = p.inv_freq[j];
-        axis[m] = j < p.n_t ? 0 : (j < p.n_t + p.n_h ? 1 : 2);
-        tab_col[m] = axis[m] == 0 ? j : (axis[m] == 1 ? j - p.n_t : j - p.n_t - p.n_h);
-    }
+    const PairInfo<PPV> pi = pair_info<PPV>(p, (t % Tr::kVecsPerHead) * PPV);
 
     const Vec* qg = reinterpret_cast<const Vec*>(p.q);
     const Vec* kg = reinterpret_cast<const Vec*>(p.k);
@@ -179,17 +350,7 @@ qk_norm_rope_kernel(const Params p) {
     const int64_t stride = (int64_t)gridDim.x * p.teams;
     int parity = 0;
     for (int64_t u = (int64_t)blockIdx.x * p.teams + team; u < p.units; u += stride) {
-        // ---- integer part: position decode (Section 3.3.3) and cache row
-        const int64_t b = u / p.n_tok;
-        const int64_t r = u - b * p.n_tok;
-        const int64_t i = p.token_begin + r;
-        const int64_t t_local = i / p.hw;
-        const int64_t rem = i - t_local * p.hw;
-        const int h = (int)(rem / p.W);
-        const int w = (int)(rem - (int64_t)h * p.W);
-        const int64_t t_g = p.frame_offset + t_local;
-
-        // ---- loads (issued first, to keep many bytes in flight)
+        const RowPos pos = decode_row(p, u);
         const int64_t row_vec = u * p.dim_vecs;
         Vec xq[VPT], xk[VPT], xv[VPT];
 #pragma unroll
@@ -203,100 +364,35 @@ qk_norm_rope_kernel(const Params p) {
                 }
             }
         }
-
-        // ---- cos / sin of this thread's pairs at (t_g, h, w)
         float cs[PPV], sn[PPV];
-#pragma unroll
-        for (int m = 0; m < PPV; ++m) {
-            const int64_t pos = axis[m] == 0 ? t_g : (axis[m] == 1 ? (int64_t)h : (int64_t)w);
-            if (TRIG == kTrigTable) {
-                const float2* tab = axis[m] == 0 ? p.tab_t : (axis[m] == 1 ? p.tab_h : p.tab_w);
-                const int ncol = axis[m] == 0 ? p.n_t : (axis[m] == 1 ? p.n_h : p.n_w);
-                const float2 e = __ldg(tab + pos * ncol + tab_col[m]);
-                cs[m] = e.x;
-                sn[m] = e.y;
-            } else {
-                const float phi = (float)pos * inv[m];
-                sincosf(phi, &sn[m], &cs[m]);
-            }
-        }
+        pair_trig<TRIG>(pi, pos, cs, sn);
 
         float rq = 1.0f, rk = 1.0f;
         int64_t cache_vec = 0;
         if (MODE == kModeFused) {
-            const int64_t crow = (p.slot + i) % p.cache_tokens;
-            cache_vec = (b * p.cache_tokens + crow) * p.dim_vecs;
-            // V goes to the cache untouched.
+            cache_vec = (pos.b * p.cache_tokens + pos.crow) * p.dim_vecs;
 #pragma unroll
             for (int s = 0; s < VPT; ++s) {
                 const int idx = t + s * p.tpr;
                 if (idx < p.dim_vecs) store_out(vc + cache_vec + idx, xv[s]);
             }
-            // Sum of squares of q and of k over the whole row, in a fixed order.
-            float sq = 0.f, sk = 0.f;
-#pragma unroll
-            for (int s = 0; s < VPT; ++s) {
-                const int idx = t + s * p.tpr;
-                if (idx < p.dim_vecs) {
-#pragma unroll
-                    for (int m = 0; m < PPV; ++m) {
-                        float a, c;
-                        Tr::pair(xq[s], m, a, c);
-                        sq = fmaf(a, a, sq);
-                        sq = fmaf(c, c, sq);
-                        Tr::pair(xk[s], m, a, c);
-                        sk = fmaf(a, a, sk);
-                        sk = fmaf(c, c, sk);
-                    }
-                }
-            }
-            sq = warp_allreduce_sum(sq);
-            sk = warp_allreduce_sum(sk);
-            if (warps_per_team > 1) {
-                float2* part = s_part + (parity * p.teams + team) * warps_per_team;
-                if (lane == 0) part[warp_in_team] = make_float2(sq, sk);
-                team_barrier(1 + team, p.tpr);
-                sq = 0.f;
-                sk = 0.f;
-                for (int wi = 0; wi < warps_per_team; ++wi) {
-                    const float2 pp = part[wi];
-                    sq += pp.x;
-                    sk += pp.y;
-                }
-                parity ^= 1;
-            }
-            rq = rsqrtf(fmaf(sq, p.inv_dim, p.eps));
-            rk = rsqrtf(fmaf(sk, p.inv_dim, p.eps));
+            float sq, sk;
+            partial_sum_squares<T, VPT>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
+            const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
+                                        warps_per_team, lane, p.tpr, parity);
+            rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
+            rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
-
-        // ---- normalise, rotate, store
 #pragma unroll
         for (int s = 0; s < VPT; ++s) {
             const int idx = t + s * p.tpr;
             if (idx < p.dim_vecs) {
                 const int e0 = idx * EPV;
-                Vec oq, ok;
-#pragma unroll
-                for (int m = 0; m < PPV; ++m) {
-                    float a, c;
-                    Tr::pair(xq[s], m, a, c);
-                    if (MODE == kModeFused) {
-                        const float2 wq = *reinterpret_cast<const float2*>(s_wq + e0 + 2 * m);
-                        a = a * rq * wq.x;
-                        c = c * rq * wq.y;
-                    }
-                    Tr::set_pair(oq, m, a * cs[m] - c * sn[m], a * sn[m] + c * cs[m]);
-                    if (MODE == kModeFused) {
-                        float ka, kb;
-                        Tr::pair(xk[s], m, ka, kb);
-                        const float2 wk = *reinterpret_cast<const float2*>(s_wk + e0 + 2 * m);
-                        ka = ka * rk * wk.x;
-                        kb = kb * rk * wk.y;
-                        Tr::set_pair(ok, m, ka * cs[m] - kb * sn[m], ka * sn[m] + kb * cs[m]);
-                    }
-                }
-                store_out(qo + row_vec + idx, oq);
-                if (MODE == kModeFused) store_out(kc + cache_vec + idx, ok);
+                store_out(qo + row_vec + idx,
+                          norm_rotate<T, MODE == kModeFused>(xq[s], rq, s_wq, e0, cs, sn));
+                if (MODE == kModeFused)
+                    store_out(kc + cache_vec + idx,
+                              norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
             }
         }
     }

@@ -23,6 +23,7 @@ ROPE3D_ECUDA = -3
 ROPE3D_EDEVICE = -4
 ROPE3D_EALIGN = -5
 ROPE3D_EOVERLAP = -6
+ROPE3D_ETIMEOUT = -7
 
 ROPE3D_F32 = 0
 ROPE3D_BF16 = 1
@@ -33,11 +34,16 @@ ROPE3D_SCHEDULE_HEAD_WIDE = 1
 ROPE3D_TRIG_TABLE = 0
 ROPE3D_TRIG_ONTHEFLY = 1
 
+# include/rope3d_testing.h
+ROPE3D_PATH_AUTO = 0
+ROPE3D_PATH_REGISTERS = 1
+ROPE3D_PATH_TMA = 2
+
 _VP = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _INT = ctypes.c_int
 
-# name -> (argtypes, restype), in the order of include/rope3d.h
+# name -> (argtypes, restype), in the order of include/rope3d.h and include/rope3d_testing.h
 SIGNATURES = {
     "rope3d_tables_init": ([ctypes.POINTER(_VP), _INT, _INT, _INT, _INT, ctypes.c_double,
                             _INT, _INT, _INT, _INT, _VP], _INT),
@@ -48,9 +54,12 @@ SIGNATURES = {
     "rope3d_apply": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT, _VP,
                       _INT, _VP], _INT),
     "rope3d_decode_positions": ([_I64, _I64, _I64, _INT, _INT, _INT, _I64, _I64, _VP, _VP], _INT),
+    "rope3d_check_device_status": ([_VP, _VP], _INT),
     "rope3d_strerror": ([_INT], ctypes.c_char_p),
     "rope3d_last_error": ([], ctypes.c_char_p),
     "rope3d_version": ([], _INT),
+    "rope3d_testing_set_waits": ([ctypes.c_uint64, ctypes.c_uint32], None),
+    "rope3d_testing_force_path": ([_INT], _INT),
 }
 
 _lib = None
@@ -199,6 +208,23 @@ def rope3d_decode_positions(token_begin: int, token_end: int, frame_offset: int,
     _check(load_library().rope3d_decode_positions(
         token_begin, token_end, frame_offset, T, H, W, cache_tokens, slot,
         _dev_ptr(out, "out"), _stream(stream)))
+
+
+def rope3d_check_device_status(tables: Tables, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status of kernels launched
+    with these tables: ROPE3D_OK or ROPE3D_ETIMEOUT.  Raises on a failure to read it."""
+    status = load_library().rope3d_check_device_status(tables.handle, _stream(stream))
+    if status not in (ROPE3D_OK, ROPE3D_ETIMEOUT):
+        _check(status)
+    return status
+
+
+def rope3d_testing_set_waits(wait_limit_ns: int = 0, tx_extra_bytes: int = 0) -> None:
+    load_library().rope3d_testing_set_waits(wait_limit_ns, tx_extra_bytes)
+
+
+def rope3d_testing_force_path(path: int = ROPE3D_PATH_AUTO) -> None:
+    _check(load_library().rope3d_testing_force_path(path))
 
 
 def rope3d_strerror(status: int) -> str:

@@ -2,6 +2,8 @@
 run the CUDA path through the C ABI binding, and compare with the fp64 oracle."""
 from __future__ import annotations
 
+import contextlib
+
 import numpy as np
 import torch
 
@@ -104,3 +106,16 @@ def oracle_rows(w: wl.Workload, case: Case, q, k, v, chunk: wl.Chunk, rows,
                                     w.cache_tokens, schedule=case.schedule)
         out.append((b, r, qo, ko, vo, pos))
     return out
+
+
+@contextlib.contextmanager
+def kernel_path(path: int):
+    """Run the block with the fused step forced onto one kernel path."""
+    rope3d.rope3d_testing_force_path(path)
+    try:
+        yield
+    finally:
+        rope3d.rope3d_testing_force_path(rope3d.ROPE3D_PATH_AUTO)
+
+
+PATHS = {"tma": rope3d.ROPE3D_PATH_TMA, "registers": rope3d.ROPE3D_PATH_REGISTERS}

@@ -11,7 +11,7 @@ from rotary_position_encoding_b200 import build as native_build
 from rotary_position_encoding_b200 import rope3d
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "rope3d.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("rope3d.h", "rope3d_testing.h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,13 +20,16 @@ def lib():
     return rope3d.load_library()
 
 
+def _header_text():
+    return "\n".join(open(h).read() for h in HEADERS)
+
+
 def header_functions():
-    text = open(HEADER).read()
-    return re.findall(r"ROPE3D_API\s+[\w\s\*]+?\b(rope3d_\w+)\s*\(", text)
+    return re.findall(r"ROPE3D_API\s+[\w\s\*]+?\b(rope3d_\w+)\s*\(", _header_text())
 
 
 def header_constants():
-    text = open(HEADER).read()
+    text = _header_text()
     return {m[0]: int(m[1]) for m in re.findall(r"#define\s+(ROPE3D_[A-Z0-9_]+)\s+\(?(-?\d+)\)?",
                                                   text)}
 
@@ -54,7 +57,7 @@ def test_binding_constants_match_header():
 
 
 def test_strerror_and_version(lib):
-    for status in (0, -1, -2, -3, -4, -5, -6, -99):
+    for status in (0, -1, -2, -3, -4, -5, -6, -7, -99):
         assert lib.rope3d_strerror(status)
     assert rope3d.rope3d_version() >= 10000
 
@@ -86,6 +89,13 @@ def test_null_and_bad_arguments_rejected_without_device(lib):
     assert lib.rope3d_decode_positions(0, 10, 0, 3, 4, 6, 144, 0, ctypes.c_void_p(0x10004),
                                        None) == rope3d.ROPE3D_EALIGN
     assert lib.rope3d_decode_positions(0, 10, -1, 3, 4, 6, 144, 0, p, None) == rope3d.ROPE3D_EINVAL
+
+
+def test_testing_hooks_validate_without_device(lib):
+    assert lib.rope3d_testing_force_path(7) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_testing_force_path(rope3d.ROPE3D_PATH_AUTO) == rope3d.ROPE3D_OK
+    lib.rope3d_testing_set_waits(0, 0)
+    assert lib.rope3d_check_device_status(None, None) == rope3d.ROPE3D_EINVAL
 
 
 def test_missing_library_fails_loudly(tmp_path):

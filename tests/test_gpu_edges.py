@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_support import assert_close, to_bits, to_device, to_f64, torch_dtype
+from gpu_support import PATHS, assert_close, kernel_path, to_bits, to_device, to_f64, torch_dtype
 from rotary_position_encoding_b200 import rope3d, workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -42,45 +42,53 @@ def _check_against_oracle(raw, dtype, wq, wk, qo, kc, vc, tb, te, s, T, H, W, C,
     assert np.array_equal(to_f64(vc), vc_ref), "v_cache"
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("rng_", [(0, 1), (71, 72), (5, 42), (23, 25), (0, 72), (17, 71)])
-def test_ragged_and_single_token_ranges(dtype, rng_):
+def test_ragged_and_single_token_ranges(dtype, rng_, path):
     tb, te = rng_
     T, H, W, s, C, slot = 3, 4, 6, 6, 144, 100
     raw, dev, wq, wk, kc, vc, tables = _setup(2, te - tb, 2, dtype, 7, C, 9, H, W)
     qo = torch.empty_like(dev[0])
-    rope3d.rope3d_qk_norm_rope_append(dev[0], dev[1], dev[2], qo, tb, te, s, T, H, W,
-                                      torch.from_numpy(wq).cuda(), torch.from_numpy(wk).cuda(),
-                                      EPS, kc, vc, slot, tables)
+    with kernel_path(PATHS[path]):
+        rope3d.rope3d_qk_norm_rope_append(dev[0], dev[1], dev[2], qo, tb, te, s, T, H, W,
+                                          torch.from_numpy(wq).cuda(),
+                                          torch.from_numpy(wk).cuda(), EPS, kc, vc, slot, tables)
     torch.cuda.synchronize()
     _check_against_oracle(raw, dtype, wq, wk, qo, kc, vc, tb, te, s, T, H, W, C, slot)
 
 
+@pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("trig", [rope3d.ROPE3D_TRIG_TABLE, rope3d.ROPE3D_TRIG_ONTHEFLY])
-def test_in_place_q_and_cache_wrap(trig):
+def test_in_place_q_and_cache_wrap(trig, path):
     T, H, W, s, C = 3, 30, 52, 12, 5000
     n = T * H * W
     slot = C - 777  # the range wraps around the end of the cache
     raw, dev, wq, wk, kc, vc, tables = _setup(1, n, 12, "bf16", 8, C, 15, H, W)
     q_inplace = dev[0].clone()
-    rope3d.rope3d_qk_norm_rope_append(q_inplace, dev[1], dev[2], q_inplace, 0, n, s, T, H, W,
-                                      torch.from_numpy(wq).cuda(), torch.from_numpy(wk).cuda(),
-                                      EPS, kc, vc, slot, tables, trig)
+    with kernel_path(PATHS[path]):
+        rope3d.rope3d_qk_norm_rope_append(q_inplace, dev[1], dev[2], q_inplace, 0, n, s, T, H,
+                                          W, torch.from_numpy(wq).cuda(),
+                                          torch.from_numpy(wk).cuda(), EPS, kc, vc, slot, tables,
+                                          trig)
     torch.cuda.synchronize()
     _check_against_oracle(raw, "bf16", wq, wk, q_inplace, kc, vc, 0, n, s, T, H, W, C, slot)
 
 
+@pytest.mark.parametrize("path", ["auto", "registers"])
 @pytest.mark.parametrize("dtype,N", [("bf16", 1), ("bf16", 3), ("bf16", 5), ("bf16", 12),
                                      ("bf16", 40), ("bf16", 64), ("bf16", 128), ("f32", 1),
                                      ("f32", 3), ("f32", 12), ("f32", 64)])
-def test_head_counts_up_to_maximum(dtype, N):
+def test_head_counts_up_to_maximum(dtype, N, path):
     T, H, W, s, C, slot = 2, 3, 5, 4, 64, 7
     n = T * H * W
     raw, dev, wq, wk, kc, vc, tables = _setup(2, n, N, dtype, 100 + N, C, 6, H, W)
     qo = torch.empty_like(dev[0])
-    rope3d.rope3d_qk_norm_rope_append(dev[0], dev[1], dev[2], qo, 0, n, s, T, H, W,
-                                      torch.from_numpy(wq).cuda(), torch.from_numpy(wk).cuda(),
-                                      EPS, kc, vc, slot, tables)
+    forced = rope3d.ROPE3D_PATH_AUTO if path == "auto" else rope3d.ROPE3D_PATH_REGISTERS
+    with kernel_path(forced):
+        rope3d.rope3d_qk_norm_rope_append(dev[0], dev[1], dev[2], qo, 0, n, s, T, H, W,
+                                          torch.from_numpy(wq).cuda(),
+                                          torch.from_numpy(wk).cuda(), EPS, kc, vc, slot, tables)
     torch.cuda.synchronize()
     _check_against_oracle(raw, dtype, wq, wk, qo, kc, vc, 0, n, s, T, H, W, C, slot)
 

@@ -10,12 +10,21 @@ import pytest
 import torch
 
 import oracle
-from gpu_support import (Case, assert_close, oracle_rows, to_bits, to_device, to_f64)
+from gpu_support import (PATHS, Case, assert_close, kernel_path, oracle_rows, to_bits, to_device,
+                         to_f64)
 from rotary_position_encoding_b200 import rope3d, workloads as wl
 
 pytestmark = pytest.mark.gpu
 
 TABLE, ONTHEFLY = rope3d.ROPE3D_TRIG_TABLE, rope3d.ROPE3D_TRIG_ONTHEFLY
+
+
+@pytest.fixture(params=sorted(PATHS))
+def path(request):
+    """Both kernel paths of the fused step: the shared-memory bulk-copy ring and the
+    register kernel."""
+    with kernel_path(PATHS[request.param]):
+        yield request.param
 
 
 def _inputs(w, chunk_index, n_tok=None):
@@ -48,7 +57,7 @@ def _cache_rows(chunk, w, token_begin, token_end):
 
 @pytest.mark.parametrize("trig", [TABLE, ONTHEFLY])
 @pytest.mark.parametrize("schedule", [0, 1])
-def test_tiny_fp32_every_element(trig, schedule):
+def test_tiny_fp32_every_element(trig, schedule, path):
     w = wl.tiny()
     case = Case(w, schedule=schedule)
     expect_k = np.zeros((w.B, w.cache_tokens, w.N, wl.HEAD_DIM))
@@ -69,7 +78,7 @@ def test_tiny_fp32_every_element(trig, schedule):
 # ---------------------------------------------------------------- 480p chunk, every element
 
 @pytest.mark.slow
-def test_chunk_480p_every_element_all_offsets():
+def test_chunk_480p_every_element_all_offsets(path):
     w = wl.chunk_480p()
     case = Case(w)
     written = np.zeros(w.cache_tokens, dtype=bool)
@@ -90,7 +99,7 @@ def test_chunk_480p_every_element_all_offsets():
 # ---------------------------------------------------------------- full 480p: slices vs whole
 
 @pytest.mark.slow
-def test_full_480p_slices_bit_identical_to_whole():
+def test_full_480p_slices_bit_identical_to_whole(path):
     w = wl.full_480p()
     n = w.tokens_per_chunk
     chunk = w.chunks[0]
@@ -121,7 +130,7 @@ def test_full_480p_slices_bit_identical_to_whole():
 # ---------------------------------------------------------------- 720p, sampled rows
 
 @pytest.mark.slow
-def test_chunk_720p_sampled_rows_all_chunks():
+def test_chunk_720p_sampled_rows_all_chunks(path):
     w = wl.chunk_720p()
     case = Case(w)
     rng = np.random.default_rng(44)
@@ -150,7 +159,7 @@ def test_chunk_720p_sampled_rows_all_chunks():
 # ---------------------------------------------------------------- long horizon, rolling window
 
 @pytest.mark.slow
-def test_long_horizon_rolling_window_table_and_onthefly():
+def test_long_horizon_rolling_window_table_and_onthefly(path):
     w = wl.long_horizon()
     tab = Case(w, max_t=240)
     fly = Case(w, max_t=240)
@@ -190,3 +199,25 @@ def test_long_horizon_rolling_window_table_and_onthefly():
         (b, rr, q_ref, k_ref, v_ref, pos) = oracle_rows(w, tab, *raw, chunk, [(1, r)], 0)[0]
         assert pos[3] == row
         assert_close(to_f64(tab.k_cache[1, row]), k_ref, "bf16", f"final window row {row}")
+
+
+# ---------------------------------------------------------------- the two kernel paths agree
+
+@pytest.mark.slow
+@pytest.mark.parametrize("make", [wl.chunk_480p, wl.chunk_720p, wl.long_horizon, wl.tiny])
+def test_kernel_paths_bit_identical(make):
+    """The register kernel and the bulk-copy ring kernel run the same per-row arithmetic
+    in the same order, so their outputs agree bit for bit."""
+    w = make()
+    chunk = w.chunks[1]
+    dev, raw = _inputs(w, 1)
+    outs = {}
+    for name in sorted(PATHS):
+        case = Case(w)
+        with kernel_path(PATHS[name]):
+            q = case.run(*dev, chunk)
+        torch.cuda.synchronize()
+        outs[name] = (q, case.k_cache, case.v_cache)
+    for a, b in zip(outs["registers"], outs["tma"]):
+        assert torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                           b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
