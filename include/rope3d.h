@@ -176,6 +176,40 @@ ROPE3D_API int rope3d_decode_positions(int64_t token_begin, int64_t token_end, i
  */
 ROPE3D_API int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream);
 
+/*
+ * The fused step without any device allocation.  The paper has no counterpart; this
+ * entry point exists for callers that cannot call cudaMalloc: a host framework that owns
+ * all device memory through its own allocator and forbids direct allocations, a process
+ * whose caching allocator already holds the free device memory, or a latency-critical
+ * loop that cannot afford cudaMalloc's implicit synchronisation.  rope3d_tables_init
+ * allocates (its cos/sin tables and a status word), so those callers cannot use it.
+ *
+ * Here the frequency configuration is passed directly (n_t + n_h + n_w = 64, theta,
+ * schedule), and everything the step needs beyond the caller's inputs and outputs sits
+ * in one file-scope device array of 65,792 bytes that every GPU loading this library
+ * holds until the process exits: a status word and room for 8192 (cos, sin) entries.
+ * With trig = ROPE3D_TRIG_TABLE each call computes, in fp64 on the host, the cos/sin rows
+ * of its own positions -- (frames touched) * n_t + H * n_h + W * n_w entries -- and
+ * copies them into that array on cuda_stream (a copy from pageable host memory, so the
+ * call waits for the stream to drain before it returns); a call needing more than 8192
+ * entries returns ROPE3D_ERANGE and launches nothing.  With ROPE3D_TRIG_ONTHEFLY nothing
+ * is copied.  Each call first clears the status word.  Outputs are bit-identical to
+ * rope3d_qk_norm_rope_append with tables built from the same configuration.
+ *
+ * Every call shares the array and it keeps the last call's contents; calls that overlap
+ * on the GPU (on different streams or from different host threads) race on it and must
+ * be serialised by the caller.  The status word of the bounded waits is not reported
+ * back.  The first call on a device looks up the array's device address (one-time set-up
+ * with that device current); make that first call before any stream capture.  Other
+ * arguments, layouts and errors are those of rope3d_qk_norm_rope_append.
+ */
+ROPE3D_API int rope3d_qk_norm_rope_append_noalloc(
+    const void* q, const void* k, const void* v, void* q_out, int64_t B, int64_t N, int D,
+    int dtype, int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
+    const float* q_norm_w, const float* k_norm_w, float eps, void* k_cache, void* v_cache,
+    int64_t cache_tokens, int64_t slot, int n_t, int n_h, int n_w, double theta, int schedule,
+    int trig, void* cuda_stream);
+
 /* Fixed text for a status code (never NULL). */
 ROPE3D_API const char* rope3d_strerror(int status);
 

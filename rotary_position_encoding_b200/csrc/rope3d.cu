@@ -718,3 +718,156 @@ int rope3d_decode_positions(int64_t token_begin, int64_t token_end, int64_t fram
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- no-allocation entry point
+//
+// rope3d_qk_norm_rope_append_noalloc serves callers that cannot call cudaMalloc (see
+// include/rope3d.h).  Everything the fused step needs beyond the caller's inputs and
+// outputs -- the cos/sin rows of this call's positions and the status word of the
+// bounded waits -- lives in one file-scope device array instead of a rope3d_tables
+// allocation.  The array exists on every GPU that loads this library until the process
+// exits.  Every call shares it and it keeps the last call's contents; each call writes
+// its own table rows and clears the status word first.  Calls that overlap on the GPU
+// (different streams, or different host threads) race on it.
+
+namespace {
+
+constexpr int kNoAllocStatusBytes = 256;       // status word, padded to the array's alignment
+constexpr int kNoAllocTableEntries = 8192;     // (cos, sin) pairs: 64 KiB
+constexpr size_t kNoAllocScratchBytes = kNoAllocStatusBytes + kNoAllocTableEntries * sizeof(float2);
+
+std::mutex g_noalloc_mutex;
+std::vector<void*> g_noalloc_addr;            // per device: device address of the array
+float2 g_noalloc_host[kNoAllocTableEntries];  // host staging of one call's rows (under the mutex)
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of the array on the current device.  Host code sees only a host-side
+// stand-in under the array's name, so the real address is asked for once per device,
+// with that device current, and remembered.
+int noalloc_scratch_address(int dev, unsigned char** out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if ((int)g_noalloc_addr.size() <= dev) g_noalloc_addr.resize(dev + 1, nullptr);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr)
+            return fail(ROPE3D_ECUDA, "cudaGetSymbolAddress of the scratch array: %s",
+                        cudaGetErrorString(e));
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = static_cast<unsigned char*>(g_noalloc_addr[dev]);
+    return ROPE3D_OK;
+}
+
+}  // namespace
+
+extern "C" int rope3d_qk_norm_rope_append_noalloc(
+    const void* q, const void* k, const void* v, void* q_out, int64_t B, int64_t N, int D,
+    int dtype, int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
+    const float* q_norm_w, const float* k_norm_w, float eps, void* k_cache, void* v_cache,
+    int64_t cache_tokens, int64_t slot, int n_t, int n_h, int n_w, double theta, int schedule,
+    int trig, void* cuda_stream) {
+    if (n_t < 0 || n_h < 0 || n_w < 0 || 2 * (n_t + n_h + n_w) != rope3d::kHeadDim)
+        return fail(ROPE3D_EINVAL, "n_t + n_h + n_w must be %d", rope3d::kHeadDim / 2);
+    if (!(theta > 1.0) || !std::isfinite(theta))
+        return fail(ROPE3D_EINVAL, "theta must be finite and > 1");
+    if (schedule != ROPE3D_SCHEDULE_PER_AXIS && schedule != ROPE3D_SCHEDULE_HEAD_WIDE)
+        return fail(ROPE3D_EINVAL, "schedule %d is not a ROPE3D_SCHEDULE_* value", schedule);
+    if (trig != ROPE3D_TRIG_TABLE && trig != ROPE3D_TRIG_ONTHEFLY)
+        return fail(ROPE3D_EINVAL, "trig %d is not a ROPE3D_TRIG_* value", trig);
+    if (T < 1 || H < 1 || W < 1 || frame_offset < 0 || token_begin < 0 ||
+        token_end <= token_begin || token_end > (int64_t)T * H * W)
+        return fail(ROPE3D_ERANGE, "grid or token range invalid");
+
+    // Rows of the three tables this call reads: frames [t_first, t_last], all H rows and
+    // all W columns.  They must fit the array.
+    const int64_t hw = (int64_t)H * W;
+    const int64_t t_first = frame_offset + token_begin / hw;
+    const int64_t t_last = frame_offset + (token_end - 1) / hw;
+    const int64_t entries = (t_last - t_first + 1) * n_t + (int64_t)H * n_h + (int64_t)W * n_w;
+    if (trig == ROPE3D_TRIG_TABLE && entries > kNoAllocTableEntries)
+        return fail(ROPE3D_ERANGE,
+                    "this call needs %lld cos/sin entries; the no-allocation scratch holds %d "
+                    "(use ROPE3D_TRIG_ONTHEFLY or the rope3d_tables entry points)",
+                    (long long)entries, kNoAllocTableEntries);
+
+    DeviceInfo info;
+    int dev = 0;
+    int rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    unsigned char* scratch = nullptr;
+    rc = noalloc_scratch_address(dev, &scratch);
+    if (rc != ROPE3D_OK) return rc;
+
+    // A frequency configuration on the stack that points into the scratch array.
+    rope3d_tables tb{};
+    tb.device = dev;
+    tb.head_dim = rope3d::kHeadDim;
+    tb.n_t = n_t;
+    tb.n_h = n_h;
+    tb.n_w = n_w;
+    tb.theta = theta;
+    tb.schedule = schedule;
+    tb.d_status = reinterpret_cast<int*>(scratch);
+    const int n_axis[3] = {n_t, n_h, n_w};
+    const int pairs = n_t + n_h + n_w;
+    double inv[rope3d::kPairs];
+    int first = 0;
+    for (int a = 0; a < 3; ++a) {
+        for (int j = 0; j < n_axis[a]; ++j) {
+            const double e = schedule == ROPE3D_SCHEDULE_PER_AXIS
+                                 ? (double)(2 * j) / (double)(2 * n_axis[a])
+                                 : (double)(2 * (first + j)) / (double)(2 * pairs);
+            inv[first + j] = std::pow(theta, -e);
+            tb.inv_freq[first + j] = (float)inv[first + j];
+        }
+        first += n_axis[a];
+    }
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "status clear: %s", cudaGetErrorString(e));
+    if (trig == ROPE3D_TRIG_TABLE) {
+        // fp64 cos/sin of position * inv_freq stored as fp32, as rope3d_tables_init does
+        float2* h = g_noalloc_host;
+        size_t off = 0;
+        for (int64_t p = t_first; p <= t_last; ++p)
+            for (int j = 0; j < n_t; ++j) {
+                const double phi = (double)p * inv[j];
+                h[off++] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+            }
+        const size_t off_h = off;
+        for (int p = 0; p < H; ++p)
+            for (int j = 0; j < n_h; ++j) {
+                const double phi = (double)p * inv[n_t + j];
+                h[off++] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+            }
+        const size_t off_w = off;
+        for (int p = 0; p < W; ++p)
+            for (int j = 0; j < n_w; ++j) {
+                const double phi = (double)p * inv[n_t + n_h + j];
+                h[off++] = make_float2((float)std::cos(phi), (float)std::sin(phi));
+            }
+        float2* d_tab = reinterpret_cast<float2*>(scratch + kNoAllocStatusBytes);
+        // From pageable memory the copy has consumed the host rows when it returns.
+        e = cudaMemcpyAsync(d_tab, h, off * sizeof(float2), cudaMemcpyHostToDevice, stream);
+        if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "table upload: %s", cudaGetErrorString(e));
+        tb.d_tab = d_tab;
+        // the t rows start at frame t_first; the kernel indexes them by global frame
+        tb.tab_t = reinterpret_cast<float2*>(reinterpret_cast<uintptr_t>(d_tab) -
+                                             (uintptr_t)(t_first * n_t) * sizeof(float2));
+        tb.tab_h = d_tab + off_h;
+        tb.tab_w = d_tab + off_w;
+        tb.max_t = (int)(t_last + 1);
+        tb.max_h = H;
+        tb.max_w = W;
+    }
+    return rope3d_qk_norm_rope_append(q, k, v, q_out, B, N, D, dtype, token_begin, token_end,
+                                      frame_offset, T, H, W, q_norm_w, k_norm_w, eps, k_cache,
+                                      v_cache, cache_tokens, slot, &tb, trig, cuda_stream);
+}

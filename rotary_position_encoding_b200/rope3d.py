@@ -55,6 +55,10 @@ SIGNATURES = {
                       _INT, _VP], _INT),
     "rope3d_decode_positions": ([_I64, _I64, _I64, _INT, _INT, _INT, _I64, _I64, _VP, _VP], _INT),
     "rope3d_check_device_status": ([_VP, _VP], _INT),
+    "rope3d_qk_norm_rope_append_noalloc": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64,
+                                            _I64, _I64, _INT, _INT, _INT, _VP, _VP,
+                                            ctypes.c_float, _VP, _VP, _I64, _I64, _INT, _INT,
+                                            _INT, ctypes.c_double, _INT, _INT, _VP], _INT),
     "rope3d_strerror": ([_INT], ctypes.c_char_p),
     "rope3d_last_error": ([], ctypes.c_char_p),
     "rope3d_version": ([], _INT),
@@ -184,6 +188,24 @@ def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
         _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), k_cache.shape[1], slot,
         tables.handle, trig, _stream(stream)))
+
+
+def rope3d_qk_norm_rope_append_noalloc(q, k, v, q_out, token_begin: int, token_end: int,
+                                       frame_offset: int, T: int, H: int, W: int, q_norm_w,
+                                       k_norm_w, eps: float, k_cache, v_cache, slot: int,
+                                       n_t: int = 22, n_h: int = 21, n_w: int = 21,
+                                       theta: float = 10000.0,
+                                       schedule: int = ROPE3D_SCHEDULE_PER_AXIS,
+                                       trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
+    """The fused step with no device allocation (frequency configuration passed directly;
+    its cos/sin rows and status word live in the library's fixed scratch array)."""
+    B, n_tok, N, D = q.shape
+    _check(load_library().rope3d_qk_norm_rope_append_noalloc(
+        _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
+        B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,
+        _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), k_cache.shape[1], slot,
+        n_t, n_h, n_w, theta, schedule, trig, _stream(stream)))
 
 
 def rope3d_apply(x, out, token_begin: int, token_end: int, frame_offset: int, T: int, H: int,
