@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
                          "fits in shared memory)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step (all chunk calls) in a CUDA graph and replay it; "
+                         "the per-launch time is then the step time over its launches")
     ap.add_argument("--chunks", type=int, default=0,
                     help="use only the first CHUNKS chunk calls per step (profiling captures "
                          "of a smaller case; 0 = the whole step)")
@@ -295,8 +298,22 @@ def run_ours(args, dist: Dist):
 
     # per-launch events of every timed launch (the kernel's own duration) and the region
     n_launch = len(w.chunks)
-    per_step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
-                       for _ in range(args.steps)]
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                stream = torch.cuda.current_stream(device)
+                step()
+        stream = torch.cuda.current_stream(device)
+        graph.replay()
+        torch.cuda.synchronize()
+        per_step_events = []
+    else:
+        per_step_events = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+                           for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     dist.barrier()
@@ -305,15 +322,21 @@ def run_ours(args, dist: Dist):
         clocks.mark("start")
     start.record(stream)
     for s in range(args.steps):
-        step(per_step_events[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            step(per_step_events[s])
     end.record(stream)
     torch.cuda.synchronize()
     if clocks:
         clocks.mark("end")
     dist.barrier()
     elapsed_ms = start.elapsed_time(end)
-    launch_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for ev in per_step_events
-                 for j in range(n_launch)]
+    if graph is not None:
+        launch_ms = [elapsed_ms / (args.steps * n_launch)]
+    else:
+        launch_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for ev in per_step_events
+                     for j in range(n_launch)]
     clock_info = clocks.stop() if clocks else None
 
     elapsed_ms = dist.max(elapsed_ms, device)
@@ -329,6 +352,7 @@ def run_ours(args, dist: Dist):
         e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
 
     del per_step_events
+    graph = None
     tables.close()
     dist.close()
     if dist.rank != 0:
@@ -349,6 +373,8 @@ def run_ours(args, dist: Dist):
         else "rope3d::qk_norm_rope_kernel",
         "algorithmic_bytes_per_launch": bytes_per_launch,
         "avg_launch_us": round(avg_launch_ms * 1e3, 2),
+        "launch_timing": "step time / launches (graph replay)" if args.graph
+        else "CUDA event pair around every timed launch",
     }
     line = {
         "metric": METRIC,
@@ -374,6 +400,8 @@ def run_ours(args, dist: Dist):
             "cache_tokens": w.cache_tokens,
             "trig": args.trig,
             "kernel_path": args.path,
+            "launch": "CUDA graph of one step, replayed" if args.graph
+            else "eager, one C-ABI call per chunk",
             "l2": "no flush: inputs larger than L2 (each launch streams "
                   f"{bytes_per_launch / 1e6:.1f} MB from its own buffers)",
             "parallelism": f"replicas x{dist.world} (independent streams, no collective)",

@@ -24,8 +24,14 @@
 #ifndef ROPE3D_VPT_TARGET
 #define ROPE3D_VPT_TARGET 4  // vectors per thread per tensor the team size aims for
 #endif
-#ifndef ROPE3D_BLOCK_TARGET
-#define ROPE3D_BLOCK_TARGET 512  // threads per block the team count aims for
+// Threads per block the team count aims for, per kernel path.  Measured on B200 at the
+// 720P shape (40 heads, TPR 160): the register kernel is fastest with one team per
+// block (several blocks per SM); the bulk-copy ring with two teams of three stages.
+#ifndef ROPE3D_REG_BLOCK_TARGET
+#define ROPE3D_REG_BLOCK_TARGET 256
+#endif
+#ifndef ROPE3D_TMA_BLOCK_TARGET
+#define ROPE3D_TMA_BLOCK_TARGET 320
 #endif
 
 struct rope3d_tables {
@@ -258,6 +264,25 @@ int occupancy(int dev, KernelFn fn, int threads, size_t smem, int max_smem, int*
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Launch with programmatic stream serialisation: the kernel may start while the
+// previous kernel on the stream drains, and waits for it (griddepcontrol.wait) before
+// it touches global memory.
+cudaError_t launch_pdl(const void* fn, int64_t grid, int threads, size_t smem,
+                       cudaStream_t stream, rope3d::Params* p) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {p};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 // Shared-memory plan of the TMA kernel for `teams` teams of `stages` stages each;
 // returns the total dynamic shared memory and fills the offsets.
 size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) {
@@ -280,7 +305,7 @@ size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) 
 }
 
 #ifndef ROPE3D_TMA_MAX_STAGES
-#define ROPE3D_TMA_MAX_STAGES 4
+#define ROPE3D_TMA_MAX_STAGES 3
 #endif
 
 // The fused step through the bulk-copy ring, when a ring of at least two stages per
@@ -292,8 +317,8 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
     if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
     const int warps_per_team = g.tpr / 32;
     p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
-    int teams = (ROPE3D_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_BLOCK_TARGET
-                                                                : rope3d::kMaxBlockThreads) / g.tpr;
+    int teams = (ROPE3D_TMA_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_TMA_BLOCK_TARGET
+                                                                    : rope3d::kMaxBlockThreads) / g.tpr;
     if (teams < 1) teams = 1;
     if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
     if ((int64_t)teams > p.units) teams = (int)p.units;
@@ -323,9 +348,8 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
     p.stages = stages;
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.tx_extra = g_tx_extra.load();
-    void* args[] = {&p};
-    const cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn),
-                                           dim3((unsigned)grid), dim3(threads), args, smem, stream);
+    const cudaError_t e =
+        launch_pdl(reinterpret_cast<const void*>(fn), grid, threads, smem, stream, &p);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     *launched = true;
     return ok();
@@ -338,8 +362,8 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const Dev
     if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4)
         return fail(ROPE3D_EINVAL, "N=%lld heads is more than one row team can hold",
                     (long long)N);
-    int teams = (ROPE3D_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_BLOCK_TARGET
-                                                                : rope3d::kMaxBlockThreads) / g.tpr;
+    int teams = (ROPE3D_REG_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_REG_BLOCK_TARGET
+                                                                    : rope3d::kMaxBlockThreads) / g.tpr;
     if (teams < 1) teams = 1;
     if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
     if ((int64_t)teams > p.units) teams = (int)p.units;
@@ -364,9 +388,8 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const Dev
     p.dim_vecs = g.dim_vecs;
     p.tpr = g.tpr;
     p.teams = teams;
-    void* args[] = {&p};
-    const cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn),
-                                           dim3((unsigned)grid), dim3(threads), args, smem, stream);
+    const cudaError_t e =
+        launch_pdl(reinterpret_cast<const void*>(fn), grid, threads, smem, stream, &p);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }

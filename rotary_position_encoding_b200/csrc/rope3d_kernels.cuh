@@ -120,6 +120,16 @@ __device__ __forceinline__ float4 load_stream(const float4* p) { return __ldcs(p
 __device__ __forceinline__ void store_out(uint4* p, const uint4& v) { *p = v; }
 __device__ __forceinline__ void store_out(float4* p, const float4& v) { *p = v; }
 
+// Programmatic dependent launch: let the next kernel on the stream start its prologue
+// while this grid drains, and wait for the previous grid (and its memory) before this
+// grid reads anything from global memory.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_previous_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void team_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
@@ -334,6 +344,8 @@ qk_norm_rope_kernel(const Params p) {
     const int warp_in_team = t >> 5;
     const int warps_per_team = p.tpr >> 5;
 
+    pdl_launch_dependents();
+    pdl_wait_previous_grid();
     if (MODE == kModeFused) {
         stage_weights(p, s_wq, s_wk);
         __syncthreads();

@@ -13,8 +13,8 @@
 //
 // Waits are bounded: a stage that has not filled after p.wait_limit_ns makes the
 // whole team (by a vote at the reduction barrier) leave its loop, record
-// ROPE3D_STATUS_WAIT_TIMEOUT in *p.status, wait (bounded again) for its copies still in
-// flight, and return.  No bulk copy uses cluster multicast.
+// kStatusWaitTimeout in *p.status (read back as ROPE3D_ETIMEOUT), wait (bounded again)
+// for its copies still in flight, and return.  No bulk copy uses cluster multicast.
 #pragma once
 
 #include "rope3d_kernels.cuh"
@@ -120,12 +120,14 @@ qk_norm_rope_tma_kernel(const Params p) {
         bulk_load(dst + 2 * rb, static_cast<const char*>(p.v) + off, rb, bar);
     };
 
+    pdl_launch_dependents();
     if (t == 0) {
         for (int s = 0; s < S; ++s) mbar_init(bar0 + 8u * s, 1);
         s_fail[team] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
+    pdl_wait_previous_grid();
     stage_weights(p, s_wq, s_wk);
     __syncthreads();
     if (t == 0)
