@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload chunk720p|chunk480p|longhorizon] [--trig table|onthefly]
+                    [--eager] [--path auto|registers|tma]
 
 One step is the whole 720P sequence of a Wan-14B-shaped backbone (21 latent frames of
 45x80, 40 heads of 128, bf16) in seven chunk calls of 10800 tokens, start frames 0, 3,
@@ -12,6 +13,9 @@ Using a Global Time Index" (Section 3.3.2), at the 720P size.  Inputs are seeded
 synthetic tensors (N(0,1) rounded to bf16; RMSNorm weights U(0.5, 1.5)); every chunk has
 its own buffers and each launch streams 663.6 MB, well above the 126 MB L2, so no L2
 flush is needed between launches.
+
+One step's seven launches are captured once in a CUDA graph and replayed (the chunk loop
+of an inference server); --eager launches them one by one instead.
 
 Under torchrun every rank runs the same job on its own GPU with its own seed (weak
 scaling, no collective on the data path); the reported time is the maximum over ranks.
@@ -60,9 +64,11 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
                          "fits in shared memory)")
-    ap.add_argument("--graph", action="store_true",
-                    help="capture one step (all chunk calls) in a CUDA graph and replay it; "
-                         "the per-launch time is then the step time over its launches")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every chunk call from Python and time each launch with its "
+                         "own CUDA event pair (default: capture one step -- all its chunk "
+                         "calls -- in a CUDA graph and replay it; the per-launch time is then "
+                         "the step time over its launches)")
     ap.add_argument("--chunks", type=int, default=0,
                     help="use only the first CHUNKS chunk calls per step (profiling captures "
                          "of a smaller case; 0 = the whole step)")
@@ -299,7 +305,7 @@ def run_ours(args, dist: Dist):
     # per-launch events of every timed launch (the kernel's own duration) and the region
     n_launch = len(w.chunks)
     graph = None
-    if args.graph:
+    if (not args.eager):
         side = torch.cuda.Stream(device)
         side.wait_stream(stream)
         graph = torch.cuda.CUDAGraph()
@@ -373,7 +379,7 @@ def run_ours(args, dist: Dist):
         else "rope3d::qk_norm_rope_kernel",
         "algorithmic_bytes_per_launch": bytes_per_launch,
         "avg_launch_us": round(avg_launch_ms * 1e3, 2),
-        "launch_timing": "step time / launches (graph replay)" if args.graph
+        "launch_timing": "step time / launches (graph replay)" if (not args.eager)
         else "CUDA event pair around every timed launch",
     }
     line = {
@@ -400,7 +406,7 @@ def run_ours(args, dist: Dist):
             "cache_tokens": w.cache_tokens,
             "trig": args.trig,
             "kernel_path": args.path,
-            "launch": "CUDA graph of one step, replayed" if args.graph
+            "launch": "CUDA graph of one step, replayed" if (not args.eager)
             else "eager, one C-ABI call per chunk",
             "l2": "no flush: inputs larger than L2 (each launch streams "
                   f"{bytes_per_launch / 1e6:.1f} MB from its own buffers)",

@@ -14,7 +14,7 @@ extern "C" {
 #endif
 
 /* Kernel path of rope3d_qk_norm_rope_append. */
-#define ROPE3D_PATH_AUTO 0       /* bulk-copy ring when it fits in shared memory, else registers */
+#define ROPE3D_PATH_AUTO 0       /* the path measured faster for the shape (see rope3d.cu)     */
 #define ROPE3D_PATH_REGISTERS 1  /* rows loaded straight into registers                        */
 #define ROPE3D_PATH_TMA 2        /* rows streamed through shared memory (EINVAL if it does not fit) */
 

@@ -309,9 +309,13 @@ size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) 
 #endif
 
 // The fused step through the bulk-copy ring, when a ring of at least two stages per
-// team fits in shared memory; returns 1 if it launched nothing (caller falls back).
+// team fits in shared memory; *launched stays false if it launched nothing (the caller
+// falls back to the register kernel).  Unless `forced`, the ring is also declined where
+// the register kernel measured faster on B200 (graph-replayed launches, 2 to 64 heads,
+// 1560 to 32760 tokens): teams under 96 threads, a single team per block, or fewer
+// than 16 rows per team.  The ring won by 2-5% at 24 to 40 heads and >= 10800 tokens.
 int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
-                     const DeviceInfo& info, cudaStream_t stream, bool* launched) {
+                     const DeviceInfo& info, cudaStream_t stream, bool forced, bool* launched) {
     *launched = false;
     const Geometry g = geometry(N, dtype);
     if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
@@ -332,6 +336,9 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
         if (stages >= 2) break;
     }
     if (teams < 1 || stages < 2) return ROPE3D_OK;  // does not fit: register kernel
+    if (!forced && (g.tpr < 96 || teams < 2 ||
+                    p.units < (int64_t)16 * info.sms * teams))
+        return ROPE3D_OK;
     smem = tma_layout(p, teams, stages, warps_per_team);
     TmaKernelFn fn = pick_tma_kernel(dtype, trig, g.vpt);
     if (fn == nullptr) return ROPE3D_OK;
@@ -671,7 +678,8 @@ int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void
     const int path = g_force_path.load();
     if (path != ROPE3D_PATH_REGISTERS) {
         bool launched = false;
-        rc = launch_fused_tma(p, N, dtype, trig, dev, info, stream, &launched);
+        rc = launch_fused_tma(p, N, dtype, trig, dev, info, stream, path == ROPE3D_PATH_TMA,
+                              &launched);
         if (rc != ROPE3D_OK || launched) return rc;
         if (path == ROPE3D_PATH_TMA)
             return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);

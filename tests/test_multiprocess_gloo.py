@@ -1,0 +1,105 @@
+"""Multi-process host logic on CPU with the gloo backend, world size 2.
+
+The step shards with no exchange: the paper's Causal-RoPE SP lets each rank compute its
+own token slice [r L/P, (r+1) L/P) with the global index offset Delta = r L_local and no
+communication ("Accelerating Video Generation Inference with Sequential-Parallel 3D
+Positional Encoding Using a Global Time Index", Section 3.3.3; Algorithm 3 steps 2-3).
+These tests run ranks as processes: (1) each rank computes its slice with the oracle
+and rank 0 checks the gathered result against the whole sequence; (2) the benchmark's
+timing reduction takes the maximum over ranks and scales the token count by the ranks."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _init(rank, world, port):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+
+
+def _sp_rank(rank, world, port, q_path):
+    _init(rank, world, port)
+    import datetime
+
+    import oracle
+    from rotary_position_encoding_b200 import workloads as wl
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        w = wl.tiny()
+        chunk = w.chunks[1]  # start frame 3, slot 72
+        n = w.tokens_per_chunk
+        q, k, v = (wl.to_f64(x, w.dtype) for x in wl.chunk_inputs(w, 1))
+        wq, wk = (x.astype(np.float64) for x in wl.norm_weights(w.seed, w.dim))
+        L_local = n // world
+        delta = rank * L_local  # Algorithm 3 step 2
+        a, e = delta, delta + L_local
+        kc = np.zeros((w.B, w.cache_tokens, w.N, wl.HEAD_DIM))
+        vc = np.zeros_like(kc)
+        q_loc = oracle.default().qk_norm_rope_append(
+            q[:, a:e].copy(), k[:, a:e].copy(), v[:, a:e].copy(), a, e, chunk.frame_offset,
+            w.T, w.H, w.W, wq, wk, w.eps, kc, vc, chunk.slot)
+        gathered = [torch.zeros(q_loc.shape, dtype=torch.float64) for _ in range(world)]
+        dist.all_gather(gathered, torch.from_numpy(q_loc))
+        kc_t = torch.from_numpy(kc)
+        dist.all_reduce(kc_t)  # each cache row is written by exactly one rank
+        if rank == 0:
+            q_sp = torch.cat(gathered, dim=1).numpy()
+            kc0 = np.zeros_like(kc)
+            vc0 = np.zeros_like(kc)
+            q_whole = oracle.default().qk_norm_rope_append(
+                q, k, v, 0, n, chunk.frame_offset, w.T, w.H, w.W, wq, wk, w.eps, kc0, vc0,
+                chunk.slot)
+            ok = np.array_equal(q_sp, q_whole) and np.array_equal(kc_t.numpy(), kc0)
+            with open(q_path, "w") as f:
+                f.write("ok" if ok else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
+def _timing_rank(rank, world, port, out_path):
+    _init(rank, world, port)
+    import bench
+    d = bench.Dist()
+    d.init("gloo")
+    try:
+        worst = d.max(10.0 * (rank + 1), torch.device("cpu"))
+        d.barrier()
+        if rank == 0:
+            tokens = 75600 * 3 * d.world  # every rank processed its own full job
+            with open(out_path, "w") as f:
+                f.write(f"{d.world} {worst} {tokens / (worst / 1e3)}")
+    finally:
+        d.close()
+
+
+def test_sequence_parallel_slices_on_two_ranks(tmp_path):
+    out = str(tmp_path / "sp.txt")
+    mp.start_processes(_sp_rank, args=(2, _free_port(), out), nprocs=2, start_method="spawn",
+                       join=True)
+    assert open(out).read() == "ok"
+
+
+def test_bench_timing_is_max_over_ranks(tmp_path):
+    out = str(tmp_path / "timing.txt")
+    mp.start_processes(_timing_rank, args=(2, _free_port(), out), nprocs=2,
+                       start_method="spawn", join=True)
+    world, worst, value = open(out).read().split()
+    assert int(world) == 2
+    assert float(worst) == 20.0
+    assert float(value) == pytest.approx(75600 * 3 * 2 / 0.020)
