@@ -318,11 +318,11 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
                      const DeviceInfo& info, cudaStream_t stream, bool forced, bool* launched) {
     *launched = false;
     const Geometry g = geometry(N, dtype);
-    if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
+    if (g.tpr > rope3d::kTmaMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
     const int warps_per_team = g.tpr / 32;
     p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
-    int teams = (ROPE3D_TMA_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_TMA_BLOCK_TARGET
-                                                                    : rope3d::kMaxBlockThreads) / g.tpr;
+    int teams = (ROPE3D_TMA_BLOCK_TARGET < rope3d::kTmaMaxBlockThreads
+                     ? ROPE3D_TMA_BLOCK_TARGET : rope3d::kTmaMaxBlockThreads) / g.tpr;
     if (teams < 1) teams = 1;
     if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
     if ((int64_t)teams > p.units) teams = (int)p.units;

@@ -37,6 +37,7 @@ constexpr int kHeadDim = 128;
 constexpr int kPairs = kHeadDim / 2;
 constexpr int kMaxTeamsPerBlock = 15;  // named barriers 1..15 (0 is __syncthreads)
 constexpr int kMaxBlockThreads = 512;  // leaves up to 128 registers per thread
+constexpr int kTmaMaxBlockThreads = 320;  // ring kernel: one block per SM, up to 204 registers
 
 enum Mode : int { kModeFused = 0, kModeApply = 1 };
 enum Trig : int { kTrigTable = 0, kTrigOnTheFly = 1 };
@@ -117,8 +118,10 @@ template <> struct VecTraits<float> {
 
 __device__ __forceinline__ uint4 load_stream(const uint4* p) { return __ldcs(p); }
 __device__ __forceinline__ float4 load_stream(const float4* p) { return __ldcs(p); }
-__device__ __forceinline__ void store_out(uint4* p, const uint4& v) { *p = v; }
-__device__ __forceinline__ void store_out(float4* p, const float4& v) { *p = v; }
+// Outputs are written once and not read again by this kernel: streaming (evict-first)
+// stores keep them from displacing lines still in use (measured 1-2% faster on B200).
+__device__ __forceinline__ void store_out(uint4* p, const uint4& v) { __stcs(p, v); }
+__device__ __forceinline__ void store_out(float4* p, const float4& v) { __stcs(p, v); }
 
 // Programmatic dependent launch: let the next kernel on the stream start its prologue
 // while this grid drains, and wait for the previous grid (and its memory) before this

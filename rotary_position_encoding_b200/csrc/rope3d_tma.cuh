@@ -77,7 +77,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 }
 
 template <typename T, int VPT, int TRIG>
-__global__ void __launch_bounds__(kMaxBlockThreads)
+__global__ void __launch_bounds__(kTmaMaxBlockThreads, 1)
 qk_norm_rope_tma_kernel(const Params p) {
     using Tr = VecTraits<T>;
     using Vec = typename Tr::Vec;
