@@ -58,6 +58,7 @@ constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<uint32_t> g_tx_extra{0};
 std::atomic<int> g_force_path{ROPE3D_PATH_AUTO};
+thread_local int g_last_path = ROPE3D_PATH_AUTO;  // path of this thread's last fused launch
 
 int fail(int status, const char* fmt, ...) {
     va_list ap;
@@ -608,6 +609,8 @@ void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes) {
     g_tx_extra.store(tx_extra_bytes);
 }
 
+int rope3d_testing_last_path(void) { return g_last_path; }
+
 int rope3d_testing_force_path(int path) {
     if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA)
         return fail(ROPE3D_EINVAL, "path %d is not a ROPE3D_PATH_* value", path);
@@ -680,11 +683,14 @@ int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void
         bool launched = false;
         rc = launch_fused_tma(p, N, dtype, trig, dev, info, stream, path == ROPE3D_PATH_TMA,
                               &launched);
+        if (launched) g_last_path = ROPE3D_PATH_TMA;
         if (rc != ROPE3D_OK || launched) return rc;
         if (path == ROPE3D_PATH_TMA)
             return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);
     }
-    return launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info, stream);
+    rc = launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info, stream);
+    if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
+    return rc;
 }
 
 int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
