@@ -96,18 +96,28 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.backend = None
 
     def init(self, backend: str):
+        self.backend = backend
         if self.world > 1:
             import datetime
 
             import torch.distributed as dist
-            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+            kw = {}
+            if backend == "nccl":
+                import torch
+                kw["device_id"] = torch.device("cuda", self.local_rank)
+            dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120),
+                                    **kw)
             self.pg = dist
 
     def barrier(self):
         if self.pg is not None:
-            self.pg.barrier()
+            if self.backend == "nccl":
+                self.pg.barrier(device_ids=[self.local_rank])
+            else:
+                self.pg.barrier()
 
     def max(self, x: float, device) -> float:
         if self.pg is None:
@@ -427,9 +437,12 @@ def run_ours(args, dist: Dist):
 
 
 def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch):
-    """Same workload through the public call with the step's inputs copied in from pinned
-    host memory and its results (q_out and the appended K/V rows) copied back, every step,
-    inside the timed region."""
+    """Same workload through the public call, with the step's inputs copied in from pinned
+    host memory and its results (q_out and the appended K/V rows) copied back every step,
+    inside the timed region.  The copies run on two side streams, one per direction, so
+    chunk c+1's upload and chunk c-1's download overlap chunk c's kernel.  Two device
+    slots double-buffer the inputs and q_out; events order each slot's reuse and keep
+    the download of a cache range ahead of its next overwrite."""
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     n = w.tokens_per_chunk
 
@@ -442,30 +455,55 @@ def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch
     shape = (w.B, n, w.N, wl.HEAD_DIM)
     h_out = [tuple(torch.empty(shape, dtype=tdt).pin_memory() for _ in range(3))
              for _ in w.chunks]
-    d_in = [tuple(torch.empty(shape, dtype=tdt, device=device) for _ in range(3))]
-    d_qo = torch.empty(shape, dtype=tdt, device=device)
+    slots = 2
+    d_in = [tuple(torch.empty(shape, dtype=tdt, device=device) for _ in range(3))
+            for _ in range(slots)]
+    d_qo = [torch.empty(shape, dtype=tdt, device=device) for _ in range(slots)]
     cache_shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
     k_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
     v_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
-    stream = torch.cuda.current_stream(device)
+    comp = torch.cuda.current_stream(device)
+    up = torch.cuda.Stream(device)
+    down = torch.cuda.Stream(device)
+    ev_comp, ev_out = {}, {}
+    counter = [0]
     h2d = d2h = 0
 
     def step():
         nonlocal h2d, d2h
         h2d = d2h = 0
         for ci, chunk in enumerate(w.chunks):
-            q, k, v = d_in[0]
-            for dst, src in zip((q, k, v), h_in[ci]):
-                dst.copy_(src, non_blocking=True)
-                h2d += src.numel() * src.element_size()
+            g = counter[0]
+            j = g % slots
+            with torch.cuda.stream(up):
+                if g - slots in ev_comp:            # the slot's last reader is done
+                    up.wait_event(ev_comp[g - slots])
+                for dst, src in zip(d_in[j], h_in[ci]):
+                    dst.copy_(src, non_blocking=True)
+                    h2d += src.numel() * src.element_size()
+                ev_in = torch.cuda.Event()
+                ev_in.record(up)
+            comp.wait_event(ev_in)
+            if g - slots in ev_out:                 # q_out slot and cache rows downloaded
+                comp.wait_event(ev_out[g - slots])
+            q, k, v = d_in[j]
             rope3d.rope3d_qk_norm_rope_append(
-                q, k, v, d_qo, chunk.token_begin, chunk.token_end, chunk.frame_offset,
+                q, k, v, d_qo[j], chunk.token_begin, chunk.token_end, chunk.frame_offset,
                 w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
-                stream)
-            rows = slice(chunk.slot, chunk.slot + n)  # no wrap inside a chunk here
-            for dst, src in zip(h_out[ci], (d_qo, k_cache[:, rows], v_cache[:, rows])):
-                dst.copy_(src, non_blocking=True)
-                d2h += dst.numel() * dst.element_size()
+                comp)
+            ev_comp[g] = torch.cuda.Event()
+            ev_comp[g].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_comp[g])
+                rows = slice(chunk.slot, chunk.slot + n)  # no wrap inside a chunk here
+                for dst, src in zip(h_out[ci], (d_qo[j], k_cache[:, rows], v_cache[:, rows])):
+                    dst.copy_(src, non_blocking=True)
+                    d2h += dst.numel() * dst.element_size()
+                ev_out[g] = torch.cuda.Event()
+                ev_out[g].record(down)
+            ev_comp.pop(g - slots, None)
+            ev_out.pop(g - slots, None)
+            counter[0] += 1
 
     steps = max(1, min(args.e2e_steps, args.steps))
     step()
@@ -474,10 +512,14 @@ def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch
     end = torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize()
-    start.record(stream)
+    start.record(comp)
+    up.wait_stream(comp)
+    down.wait_stream(comp)
     for _ in range(steps):
         step()
-    end.record(stream)
+    comp.wait_stream(up)
+    comp.wait_stream(down)
+    end.record(comp)
     torch.cuda.synchronize()
     dist.barrier()
     ms = dist.max(start.elapsed_time(end), device)
@@ -485,8 +527,9 @@ def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch
     return {"value": round(tokens / (ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3),
-            "path": "pinned host -> cudaMemcpyAsync -> rope3d_qk_norm_rope_append -> "
-                    "cudaMemcpyAsync -> pinned host, one stream"}
+            "path": "pinned host -> cudaMemcpyAsync (upload stream) -> "
+                    "rope3d_qk_norm_rope_append -> cudaMemcpyAsync (download stream) -> "
+                    "pinned host, double-buffered, copies overlapping kernels"}
 
 
 # ---------------------------------------------------------------- the oracle on the host
