@@ -27,6 +27,10 @@ LIBRARY = os.path.join(_HERE, "librope3d_oracle.so")
 # Default split of a 128-wide head: 22 t pairs, 21 h pairs, 21 w pairs; theta 10000.
 N_T, N_H, N_W, THETA = 22, 21, 21, 10000.0
 
+# Pairing of a head's elements and KV-cache layouts (the layout-variant functions).
+PAIRING_ADJACENT, PAIRING_HALF = 0, 1
+CACHE_TOKEN_MAJOR, CACHE_HEAD_MAJOR = 0, 1
+
 
 def build(force: bool = False, source: str = SOURCE, library: str = LIBRARY) -> str:
     """Compile the oracle with gcc (no fast-math, no FMA contraction, OpenMP on)."""
@@ -67,6 +71,17 @@ def _declare(lib):
         "rope3d_oracle_apply": ([_D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
                                  _I64, _INT, _INT, _INT, _DBL, _INT], _INT),
         "rope3d_oracle_max_threads": ([], _INT),
+        "rope3d_oracle_rotate_half": ([_D, _I64, _I64, _D, _D], None),
+        "rope3d_oracle_rotate_pairing": ([_D, _I64, _I64, _D, _INT, _D], _INT),
+        "rope3d_oracle_token_pairing": ([_D, _D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
+                                         _D, _D, _DBL, _I64, _I64, _INT, _INT, _INT, _D, _INT,
+                                         _D, _D, _D, ctypes.POINTER(_I64)], _INT),
+        "rope3d_oracle_qk_norm_rope_append_layout": ([_D, _D, _D, _D, _I64, _I64, _I64, _I64,
+                                                      _I64, _I64, _I64, _I64, _I64, _D, _D,
+                                                      _DBL, _D, _D, _I64, _I64, _INT, _INT,
+                                                      _INT, _DBL, _INT, _INT, _INT, _INT], _INT),
+        "rope3d_oracle_apply_pairing": ([_D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
+                                         _I64, _I64, _INT, _INT, _INT, _DBL, _INT, _INT], _INT),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +206,64 @@ class Oracle:
 
     def max_threads(self) -> int:
         return self.lib.rope3d_oracle_max_threads()
+
+    # ---- layout variants: rotate_half pairing, head-major cache
+
+    def rotate_pairing(self, x, phi, pairing):
+        """x: [n_heads, head_dim] float64 (one token row); phi: [head_dim/2]."""
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        n_heads, head_dim = x.shape[-2], x.shape[-1]
+        phi = np.ascontiguousarray(phi, dtype=np.float64)
+        y = np.empty_like(x)
+        _check(self.lib.rope3d_oracle_rotate_pairing(_f64(x, "x"), n_heads, head_dim,
+                                                     _f64(phi, "phi"), pairing, _f64(y, "y")))
+        return y
+
+    def token_pairing(self, q, k, v, i, frame_offset, T, H, W, q_norm_w, k_norm_w, eps, slot,
+                      cache_tokens, pairing, n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA,
+                      schedule=0):
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        k = np.ascontiguousarray(k, dtype=np.float64)
+        v = np.ascontiguousarray(v, dtype=np.float64)
+        N, D = q.shape[-2], q.shape[-1]
+        inv = self.inv_freq(n_t, n_h, n_w, theta, schedule)
+        qw = np.ascontiguousarray(q_norm_w, dtype=np.float64)
+        kw = np.ascontiguousarray(k_norm_w, dtype=np.float64)
+        qo, ko, vo = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+        pos = (_I64 * 4)()
+        _check(self.lib.rope3d_oracle_token_pairing(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), N, D, i, frame_offset, T, H, W,
+            _f64(qw, "q_norm_w"), _f64(kw, "k_norm_w"), eps, slot, cache_tokens,
+            n_t, n_h, n_w, _f64(inv, "inv"), pairing, _f64(qo, "q_out"), _f64(ko, "k_row"),
+            _f64(vo, "v_row"), pos))
+        return qo, ko, vo, tuple(pos)
+
+    def qk_norm_rope_append_layout(self, q, k, v, token_begin, token_end, frame_offset, T,
+                                   H, W, q_norm_w, k_norm_w, eps, k_cache, v_cache, slot,
+                                   pairing=PAIRING_ADJACENT, cache_layout=CACHE_TOKEN_MAJOR,
+                                   n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0,
+                                   nthreads=0):
+        """Whole step; caches are [B, C, N, D] (token-major) or [B, N, C, D] (head-major)."""
+        B, n_tok, N, D = q.shape
+        C = k_cache.shape[1] if cache_layout == CACHE_TOKEN_MAJOR else k_cache.shape[2]
+        q_out = np.empty_like(q)
+        _check(self.lib.rope3d_oracle_qk_norm_rope_append_layout(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), _f64(q_out, "q_out"), B, N, D,
+            token_begin, token_end, frame_offset, T, H, W,
+            _f64(np.ascontiguousarray(q_norm_w, dtype=np.float64), "q_norm_w"),
+            _f64(np.ascontiguousarray(k_norm_w, dtype=np.float64), "k_norm_w"), eps,
+            _f64(k_cache, "k_cache"), _f64(v_cache, "v_cache"), C, slot,
+            n_t, n_h, n_w, theta, schedule, pairing, cache_layout, nthreads))
+        return q_out
+
+    def apply_pairing(self, x, token_begin, token_end, frame_offset, T, H, W, pairing,
+                      n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        B, n_tok, N, D = x.shape
+        out = np.empty_like(x)
+        _check(self.lib.rope3d_oracle_apply_pairing(
+            _f64(x, "x"), _f64(out, "out"), B, N, D, token_begin, token_end, frame_offset,
+            T, H, W, n_t, n_h, n_w, theta, schedule, pairing))
+        return out
 
 
 _default = None

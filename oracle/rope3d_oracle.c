@@ -37,6 +37,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -280,6 +281,192 @@ int rope3d_oracle_apply(const double* x, double* out, int64_t B, int64_t N, int6
             int64_t off = (b * n_tok + r) * dim;
             rope3d_oracle_rotate_at(x + off, N, D, token_begin + r, frame_offset, T, H, W,
                                     n_t, n_h, n_w, inv, out + off);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ layout variants
+ *
+ * Section 3.3.1 of the paper contrasts two ways of writing the same rotation: Wan2.1's
+ * complex multiply on adjacent pairs (Algorithm 2's view, used above) and Qwen2.5-VL's
+ * cos/sin form with rotate_half, where element j of a head pairs with element
+ * j + D/2.  The functions below add that second pairing and a head-major KV cache
+ * ([B][N][cache_tokens][D], each head's rows contiguous).  Everything else -- decode,
+ * angles, RMSNorm, cache row -- is the same as above.
+ */
+#define ORACLE_PAIRING_ADJACENT 0
+#define ORACLE_PAIRING_HALF 1
+#define ORACLE_CACHE_TOKEN_MAJOR 0
+#define ORACLE_CACHE_HEAD_MAJOR 1
+
+/* RoPE with the rotate_half pairing: pair j of a head is (x[j], x[j + D/2]) as
+ * (re, im); x * e^{i phi_j} on it.  x and y may be the same array. */
+void rope3d_oracle_rotate_half(const double* x, int64_t n_heads, int64_t head_dim,
+                               const double* phi, double* y)
+{
+    int64_t pairs = head_dim / 2;
+    for (int64_t n = 0; n < n_heads; ++n) {
+        for (int64_t j = 0; j < pairs; ++j) {
+            double a = x[n * head_dim + j];          /* real part: first half */
+            double b = x[n * head_dim + pairs + j];  /* imaginary part: second half */
+            double c = cos(phi[j]);
+            double s = sin(phi[j]);
+            y[n * head_dim + j] = a * c - b * s;
+            y[n * head_dim + pairs + j] = a * s + b * c;
+        }
+    }
+}
+
+int rope3d_oracle_rotate_pairing(const double* x, int64_t n_heads, int64_t head_dim,
+                                 const double* phi, int pairing, double* y)
+{
+    if (pairing == ORACLE_PAIRING_ADJACENT) {
+        rope3d_oracle_rotate(x, n_heads, head_dim, phi, y);
+        return ORACLE_OK;
+    }
+    if (pairing == ORACLE_PAIRING_HALF) {
+        rope3d_oracle_rotate_half(x, n_heads, head_dim, phi, y);
+        return ORACLE_OK;
+    }
+    return ORACLE_EINVAL;
+}
+
+/* rope3d_oracle_token with a choice of pairing. */
+int rope3d_oracle_token_pairing(const double* q, const double* k, const double* v,
+                                int64_t N, int64_t D, int64_t i, int64_t frame_offset,
+                                int64_t T, int64_t H, int64_t W,
+                                const double* q_norm_w, const double* k_norm_w, double eps,
+                                int64_t slot, int64_t cache_tokens,
+                                int n_t, int n_h, int n_w, const double* inv, int pairing,
+                                double* q_out, double* k_row, double* v_row, int64_t* pos_out)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, i, i + 1, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (cache_tokens <= 0 || slot < 0) return ORACLE_EINVAL;
+    if (pairing != ORACLE_PAIRING_ADJACENT && pairing != ORACLE_PAIRING_HALF)
+        return ORACLE_EINVAL;
+    int64_t dim = N * D;
+    int64_t t_g, h, w;
+    double phi[512];
+    rope3d_oracle_decode(i, frame_offset, T, H, W, &t_g, &h, &w);
+    rope3d_oracle_angles(t_g, h, w, n_t, n_h, n_w, inv, phi);
+
+    rope3d_oracle_rms_norm(q, q_norm_w, dim, eps, q_out);
+    rope3d_oracle_rotate_pairing(q_out, N, D, phi, pairing, q_out);
+    rope3d_oracle_rms_norm(k, k_norm_w, dim, eps, k_row);
+    rope3d_oracle_rotate_pairing(k_row, N, D, phi, pairing, k_row);
+    memcpy(v_row, v, (size_t)dim * sizeof(double));
+
+    if (pos_out != NULL) {
+        pos_out[0] = t_g;
+        pos_out[1] = h;
+        pos_out[2] = w;
+        pos_out[3] = rope3d_oracle_cache_row(i, slot, cache_tokens);
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * The whole step with a choice of pairing and of cache layout.  Token-major caches are
+ * [B][cache_tokens][N][D]; head-major caches are [B][N][cache_tokens][D].  Head n of
+ * the token's K and V rows goes to cache row `row` of head n.
+ */
+int rope3d_oracle_qk_norm_rope_append_layout(
+    const double* q, const double* k, const double* v, double* q_out,
+    int64_t B, int64_t N, int64_t D,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset,
+    int64_t T, int64_t H, int64_t W,
+    const double* q_norm_w, const double* k_norm_w, double eps,
+    double* k_cache, double* v_cache, int64_t cache_tokens, int64_t slot,
+    int n_t, int n_h, int n_w, double theta, int schedule, int pairing, int cache_layout,
+    int nthreads)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0 || cache_tokens <= 0 || slot < 0) return ORACLE_EINVAL;
+    if (token_end - token_begin > cache_tokens) return ORACLE_EINVAL;
+    if (pairing != ORACLE_PAIRING_ADJACENT && pairing != ORACLE_PAIRING_HALF)
+        return ORACLE_EINVAL;
+    if (cache_layout != ORACLE_CACHE_TOKEN_MAJOR && cache_layout != ORACLE_CACHE_HEAD_MAJOR)
+        return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    int64_t rows = B * n_tok;
+    int failed = 0;
+#ifdef _OPENMP
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+#pragma omp parallel num_threads(nt)
+#endif
+    {
+        double* k_row = (double*)malloc((size_t)dim * sizeof(double));
+        double* v_row = (double*)malloc((size_t)dim * sizeof(double));
+        if (k_row == NULL || v_row == NULL) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            failed = 1;
+        } else {
+#ifdef _OPENMP
+#pragma omp for schedule(static)
+#endif
+            for (int64_t u = 0; u < rows; ++u) {
+                int64_t b = u / n_tok;
+                int64_t r = u % n_tok;
+                int64_t i = token_begin + r;
+                int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);
+                int64_t in_off = (b * n_tok + r) * dim;
+                rope3d_oracle_token_pairing(q + in_off, k + in_off, v + in_off, N, D, i,
+                                            frame_offset, T, H, W, q_norm_w, k_norm_w, eps,
+                                            slot, cache_tokens, n_t, n_h, n_w, inv, pairing,
+                                            q_out + in_off, k_row, v_row, NULL);
+                for (int64_t n = 0; n < N; ++n) {
+                    int64_t cache_off = cache_layout == ORACLE_CACHE_TOKEN_MAJOR
+                                            ? ((b * cache_tokens + row) * N + n) * D
+                                            : ((b * N + n) * cache_tokens + row) * D;
+                    memcpy(k_cache + cache_off, k_row + n * D, (size_t)D * sizeof(double));
+                    memcpy(v_cache + cache_off, v_row + n * D, (size_t)D * sizeof(double));
+                }
+            }
+        }
+        free(k_row);
+        free(v_row);
+    }
+#ifndef _OPENMP
+    (void)nthreads;
+#endif
+    return failed ? ORACLE_EINVAL : ORACLE_OK;
+}
+
+/* The rotation alone with a choice of pairing, over [B][n_tok][N][D]. */
+int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t N, int64_t D,
+                                int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                                int64_t T, int64_t H, int64_t W,
+                                int n_t, int n_h, int n_w, double theta, int schedule,
+                                int pairing)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0) return ORACLE_EINVAL;
+    if (pairing != ORACLE_PAIRING_ADJACENT && pairing != ORACLE_PAIRING_HALF)
+        return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    double phi[512];
+    for (int64_t b = 0; b < B; ++b) {
+        for (int64_t r = 0; r < n_tok; ++r) {
+            int64_t off = (b * n_tok + r) * dim;
+            int64_t t_g, h, w;
+            rope3d_oracle_decode(token_begin + r, frame_offset, T, H, W, &t_g, &h, &w);
+            rope3d_oracle_angles(t_g, h, w, n_t, n_h, n_w, inv, phi);
+            rope3d_oracle_rotate_pairing(x + off, N, D, phi, pairing, out + off);
         }
     }
     return ORACLE_OK;

@@ -368,4 +368,159 @@ def check_apply_matches_rotation(orc):
             assert np.array_equal(y[b, r], _one_token_rotate(orc, x[b, r], t_g, h, w))
 
 
+# ---------------------------------------------------------------- layout variants
+
+def _half_to_adjacent_perm(D=128):
+    """Index map: element j (j < D/2) -> 2j and element D/2 + j -> 2j + 1."""
+    perm = np.empty(D, dtype=np.int64)
+    half = D // 2
+    for j in range(half):
+        perm[2 * j] = j
+        perm[2 * j + 1] = half + j
+    return perm
+
+
+def check_half_pairing_golden(orc):
+    """Closed-form rotate_half rotations at whole-radian angles (golden file), on the
+    16/24/24 head-wide split of M-RoPE."""
+    for line in _rows("rotation_half_unit_angles.txt"):
+        t_g, h, w, j, re_in, im_in, re_out, im_out = line.split()
+        j = int(j)
+        x = np.zeros((1, D))
+        x[0, j] = float(re_in)
+        x[0, 64 + j] = float(im_in)
+        phi = orc.angles(int(t_g), int(h), int(w), 16, 24, 24, 10000.0, 1)
+        y = orc.rotate_pairing(x, phi, 1)
+        assert abs(y[0, j] - float(re_out)) < 1e-14, line
+        assert abs(y[0, 64 + j] - float(im_out)) < 1e-14, line
+        others = np.delete(y[0], [j, 64 + j])
+        assert np.all(others == 0.0)
+
+
+def check_half_pairing_is_permuted_adjacent(orc):
+    """rotate_half on x equals the adjacent-pair rotation on x with each pair's two
+    elements brought next to each other, mapped back."""
+    rng = _rng(20)
+    perm = _half_to_adjacent_perm()
+    for (t_g, h, w) in ((0, 0, 0), (3, 7, 11), (239, 44, 79)):
+        x = rng.standard_normal((3, D))
+        phi = orc.angles(t_g, h, w)
+        y_half = orc.rotate_pairing(x, phi, 1)
+        y_adj = orc.rotate(x[:, perm], phi)
+        back = np.empty_like(y_adj)
+        back[:, perm] = y_adj
+        assert np.array_equal(y_half, back)
+
+
+def check_half_pairing_matches_complex_exp(orc):
+    rng = _rng(21)
+    inv = orc.inv_freq(16, 24, 24, 10000.0, 1)
+    for _ in range(5):
+        t_g, h, w = (int(v) for v in rng.integers(0, 100, size=3))
+        x = rng.standard_normal((2, D))
+        pos = np.array([t_g] * 16 + [h] * 24 + [w] * 24, dtype=np.float64)
+        z = (x[:, :64] + 1j * x[:, 64:]) * np.exp(1j * pos * inv)
+        expect = np.concatenate([z.real, z.imag], axis=1)
+        phi = orc.angles(t_g, h, w, 16, 24, 24, 10000.0, 1)
+        assert np.allclose(orc.rotate_pairing(x, phi, 1), expect, rtol=0, atol=1e-13)
+
+
+def check_half_pairing_relative_offset(orc):
+    """<R(p_m) q, R(p_n) k> = <q, R(p_n - p_m) k> with the rotate_half pairing, all pairs
+    of 24 tokens of a 2x3x4 grid."""
+    rng = _rng(22)
+    T, H, W, s = 2, 3, 4, 5
+    n = T * H * W
+    q = rng.standard_normal((n, 2, D))
+    k = rng.standard_normal((n, 2, D))
+    pos = [orc.decode(i, s, T, H, W) for i in range(n)]
+
+    def rot(x, p):
+        return orc.rotate_pairing(x, orc.angles(*p), 1)
+    rq = [rot(q[m], pos[m]) for m in range(n)]
+    rk = [rot(k[m], pos[m]) for m in range(n)]
+    for m in range(n):
+        for nn in range(n):
+            d = tuple(pos[nn][a] - pos[m][a] for a in range(3))
+            assert abs(float(np.sum(rq[m] * rk[nn])) - float(np.sum(q[m] * rot(k[nn], d)))) < 1e-10
+
+
+def check_layout_step_default_equals_base_step(orc):
+    """Adjacent pairing with a token-major cache is the base step, bit for bit."""
+    B, N, T, H, W, s, slot, C = 2, 2, 3, 4, 6, 3, 50, 144
+    q, k, v, wq, wk = _step_inputs(23, B, 72, N)
+    kc0, vc0 = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    q0 = orc.qk_norm_rope_append(q, k, v, 0, 72, s, T, H, W, wq, wk, 1e-6, kc0, vc0, slot)
+    kc1, vc1 = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    q1 = orc.qk_norm_rope_append_layout(q, k, v, 0, 72, s, T, H, W, wq, wk, 1e-6, kc1, vc1, slot,
+                                        0, 0)
+    assert np.array_equal(q0, q1) and np.array_equal(kc0, kc1) and np.array_equal(vc0, vc1)
+
+
+def check_head_major_cache_is_transpose(orc):
+    """A head-major cache holds exactly the token-major cache with heads moved forward."""
+    B, N, T, H, W, s, slot, C = 2, 3, 3, 4, 6, 6, 100, 144
+    q, k, v, wq, wk = _step_inputs(24, B, 72, N)
+    for pairing in (0, 1):
+        kt, vt = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+        qt = orc.qk_norm_rope_append_layout(q, k, v, 0, 72, s, T, H, W, wq, wk, 1e-6, kt, vt,
+                                            slot, pairing, 0)
+        kh, vh = np.zeros((B, N, C, D)), np.zeros((B, N, C, D))
+        qh = orc.qk_norm_rope_append_layout(q, k, v, 0, 72, s, T, H, W, wq, wk, 1e-6, kh, vh,
+                                            slot, pairing, 1)
+        assert np.array_equal(qt, qh)
+        assert np.array_equal(kh, kt.transpose(0, 2, 1, 3))
+        assert np.array_equal(vh, vt.transpose(0, 2, 1, 3))
+
+
+def check_layout_step_slices_and_rows(orc):
+    """A token range that starts mid-chunk, in either pairing and layout, writes row r of
+    q_out from global index begin + r and cache row (slot + begin + r) mod C, exactly as
+    the per-token function computes them."""
+    B, N, T, H, W, s, slot, C = 1, 2, 3, 4, 6, 3, 130, 144
+    tb, te = 13, 60
+    q, k, v, wq, wk = _step_inputs(27, B, te - tb, N)
+    for pairing in (0, 1):
+        for layout in (0, 1):
+            shape = (B, C, N, D) if layout == 0 else (B, N, C, D)
+            kc, vc = np.zeros(shape), np.zeros(shape)
+            qo = orc.qk_norm_rope_append_layout(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kc,
+                                                vc, slot, pairing, layout)
+            for r in (0, 11, te - tb - 1):
+                eq, ek, ev, pos = orc.token_pairing(q[0, r], k[0, r], v[0, r], tb + r, s, T, H,
+                                                    W, wq, wk, 1e-6, slot, C, pairing)
+                assert pos[3] == (slot + tb + r) % C
+                assert np.array_equal(qo[0, r], eq)
+                got_k = kc[0, pos[3]] if layout == 0 else kc[0, :, pos[3]]
+                got_v = vc[0, pos[3]] if layout == 0 else vc[0, :, pos[3]]
+                assert np.array_equal(got_k, ek) and np.array_equal(got_v, ev)
+
+
+def check_half_step_is_norm_then_rotate_half(orc):
+    """With the rotate_half pairing the step's q and K rows are rotate_half(RMSNorm(x))
+    built from the separately pinned pieces; V is copied."""
+    B, N, T, H, W, s, slot, C = 1, 2, 3, 4, 6, 3, 0, 72
+    q, k, v, wq, wk = _step_inputs(25, B, 72, N)
+    kc, vc = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    qo = orc.qk_norm_rope_append_layout(q, k, v, 0, 72, s, T, H, W, wq, wk, 1e-6, kc, vc, slot,
+                                        1, 0)
+    for r in (0, 17, 71):
+        phi = orc.angles(*orc.decode(r, s, T, H, W))
+        eq = orc.rotate_pairing(orc.rms_norm(q[0, r], wq, 1e-6).reshape(N, D), phi, 1)
+        ek = orc.rotate_pairing(orc.rms_norm(k[0, r], wk, 1e-6).reshape(N, D), phi, 1)
+        assert np.allclose(qo[0, r], eq, rtol=0, atol=1e-13)
+        assert np.allclose(kc[0, r], ek, rtol=0, atol=1e-13)
+        assert np.array_equal(vc[0, r], v[0, r])
+
+
+def check_apply_half_matches_rotation(orc):
+    B, N, T, H, W, s = 1, 2, 3, 4, 6, 9
+    rng = _rng(26)
+    x = rng.standard_normal((B, 30, N, D))
+    y = orc.apply_pairing(x, 10, 40, s, T, H, W, 1)
+    for r in range(30):
+        phi = orc.angles(*orc.decode(10 + r, s, T, H, W))
+        assert np.array_equal(y[0, r], orc.rotate_pairing(x[0, r], phi, 1))
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -42,23 +42,52 @@ MUTANTS = {
     "cache_offset_wrong_stride": ("int64_t cache_off = (b * cache_tokens + row) * dim;",
                                   "int64_t cache_off = (b * n_tok + row) * dim;"),
     "step_index_ignores_begin": ("int64_t i = token_begin + r;", "int64_t i = r;"),
+    "half_pairs_reversed": ("double b = x[n * head_dim + pairs + j];  /* imaginary part: second half */",
+                            "double b = x[n * head_dim + 2 * pairs - 1 - j];"),
+    "half_real_sign": ("y[n * head_dim + j] = a * c - b * s;",
+                       "y[n * head_dim + j] = a * c + b * s;"),
+    "half_k_not_rotated_half": ("rope3d_oracle_rotate_pairing(k_row, N, D, phi, pairing, k_row);",
+                                "rope3d_oracle_rotate(k_row, N, D, phi, k_row);"),
+    "head_major_offset_is_token_major": (": ((b * N + n) * cache_tokens + row) * D;",
+                                         ": ((b * cache_tokens + row) * N + n) * D;"),
+    # the same mistakes made only in the layout-variant functions (second occurrence)
+    "k_uses_q_weights_in_pairing_token": ("rope3d_oracle_rms_norm(k, k_norm_w, dim, eps, k_row);",
+                                          "rope3d_oracle_rms_norm(k, q_norm_w, dim, eps, k_row);",
+                                          1),
+    "v_copies_k_in_pairing_token": ("memcpy(v_row, v, (size_t)dim * sizeof(double));",
+                                    "memcpy(v_row, k, (size_t)dim * sizeof(double));", 1),
+    "layout_step_ignores_begin": ("int64_t i = token_begin + r;", "int64_t i = r;", 1),
+    "layout_step_row_ignores_slot": ("int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);",
+                                     "int64_t row = rope3d_oracle_cache_row(i, 0, cache_tokens);",
+                                     1),
 }
 
 
-def _build_mutant(tmp_path, name, old, new):
+def _build_mutant(tmp_path, name, old, new, occurrence=None):
+    """Plant the mistake at every occurrence of `old`, or only at the given one (0-based)."""
     src = open(oracle.SOURCE).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    count = src.count(old)
+    assert count >= 1, f"mutation site for {name} not found"
+    if occurrence is None:
+        mutated = src.replace(old, new)
+    else:
+        assert occurrence < count, f"{name}: only {count} occurrences"
+        at = -1
+        for _ in range(occurrence + 1):
+            at = src.index(old, at + 1)
+        mutated = src[:at] + new + src[at + len(old):]
     path = os.path.join(tmp_path, f"{name}.c")
     with open(path, "w") as f:
-        f.write(src.replace(old, new))
+        f.write(mutated)
     return oracle.build(force=True, source=path, library=os.path.join(tmp_path, f"{name}.so"))
 
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(tmp_path, name):
-    old, new = MUTANTS[name]
-    orc = oracle.Oracle(_build_mutant(str(tmp_path), name, old, new))
+    old, new, *occurrence = MUTANTS[name]
+    orc = oracle.Oracle(_build_mutant(str(tmp_path), name, old, new,
+                                      occurrence[0] if occurrence else None))
     caught = []
     for check in ALL_CHECKS:
         try:
