@@ -61,6 +61,10 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="chunk720p")
     ap.add_argument("--trig", choices=["table", "onthefly"], default="table")
+    ap.add_argument("--pairing", choices=["adjacent", "half"], default="adjacent",
+                    help="pairing of a head's elements (half: rotate_half, as in M-RoPE)")
+    ap.add_argument("--cache-layout", choices=["token", "head"], default="token",
+                    help="KV cache [B][C][N][D] (token) or [B][N][C][D] (head)")
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
                          "fits in shared memory)")
@@ -282,7 +286,10 @@ def run_ours(args, dist: Dist):
 
     inputs = [tuple(dev_tensor(a) for a in chunk) for chunk in host]
     q_out = [torch.empty_like(c[0]) for c in inputs]
-    cache_shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    pairing = rope3d.ROPE3D_PAIRING_HALF if args.pairing == "half" else rope3d.ROPE3D_PAIRING_ADJACENT
+    layout = rope3d.ROPE3D_CACHE_HEAD_MAJOR if args.cache_layout == "head" else rope3d.ROPE3D_CACHE_TOKEN_MAJOR
+    cache_shape = ((w.B, w.cache_tokens, w.N, wl.HEAD_DIM) if args.cache_layout == "token"
+                   else (w.B, w.N, w.cache_tokens, wl.HEAD_DIM))
     k_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
     v_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
     max_t = max(c.frame_offset for c in w.chunks) + w.T
@@ -297,10 +304,10 @@ def run_ours(args, dist: Dist):
             q, k, v = inputs[ci]
             if events is not None:
                 events[2 * ci].record(stream)
-            rope3d.rope3d_qk_norm_rope_append(
+            rope3d.rope3d_qk_norm_rope_append_ex(
                 q, k, v, q_out[ci], chunk.token_begin, chunk.token_end, chunk.frame_offset,
                 w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
-                stream)
+                pairing, layout, stream)
             if events is not None:
                 events[2 * ci + 1].record(stream)
 
@@ -367,6 +374,8 @@ def run_ours(args, dist: Dist):
     if device_status != rope3d.ROPE3D_OK:
         raise RuntimeError("a kernel wait timed out during the benchmark")
     e2e = None
+    if not args.no_e2e and (args.pairing, args.cache_layout) != ("adjacent", "token"):
+        args.no_e2e = True  # the e2e leg runs the default layout only
     if not args.no_e2e:
         e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
 
@@ -418,6 +427,8 @@ def run_ours(args, dist: Dist):
             "cache_tokens": w.cache_tokens,
             "trig": args.trig,
             "kernel_path": args.path,
+            "pairing": args.pairing,
+            "cache_layout": args.cache_layout,
             "launch": "CUDA graph of one step, replayed" if (not args.eager)
             else "eager, one C-ABI call per chunk",
             "l2": "no flush: inputs larger than L2 (each launch streams "

@@ -79,6 +79,30 @@ extern "C" {
 #define ROPE3D_TRIG_TABLE 0     /* read the precomputed tables (fp64-built, fp32-stored) */
 #define ROPE3D_TRIG_ONTHEFLY 1  /* fp32 angle = position * fp32(inv_freq), then sincosf  */
 
+/* Pairing of a head's 128 elements into 64 complex pairs (Section 3.3.1 sets the two
+ * forms side by side):
+ *   ADJACENT -- pair j = (x[2j], x[2j+1]) as (re, im): the complex view of Algorithm 2
+ *               (Wan2.1); the default;
+ *   HALF     -- pair j = (x[j], x[j+64]): the cos/sin "rotate_half" form of Qwen2.5-VL's
+ *               M-RoPE (with ROPE3D_SCHEDULE_HEAD_WIDE and a 16/24/24 split it is that
+ *               layout).  Pair j keeps its axis and frequency either way. */
+#define ROPE3D_PAIRING_ADJACENT 0
+#define ROPE3D_PAIRING_HALF 1
+
+/* KV-cache layouts: TOKEN_MAJOR [B][cache_tokens][N][D] (default; one appended token is
+ * one contiguous row) or HEAD_MAJOR [B][N][cache_tokens][D] (each head's keys and values
+ * contiguous, as attention kernels read them). */
+#define ROPE3D_CACHE_TOKEN_MAJOR 0
+#define ROPE3D_CACHE_HEAD_MAJOR 1
+
+/* Options of the _ex entry points; a NULL pointer or a zeroed struct gives the defaults
+ * (adjacent pairing, token-major cache), i.e. the plain entry points' behaviour. */
+typedef struct rope3d_options {
+    int pairing;       /* ROPE3D_PAIRING_*                                         */
+    int cache_layout;  /* ROPE3D_CACHE_* (fused step only; must be 0 for apply)     */
+    int reserved[6];   /* must be zero                                             */
+} rope3d_options;
+
 /* Opaque frequency configuration: split, theta, schedule, the fp32 inverse
  * frequencies and, optionally, per-axis cos/sin tables in device memory. */
 typedef struct rope3d_tables rope3d_tables;
@@ -145,6 +169,19 @@ ROPE3D_API int rope3d_qk_norm_rope_append(const void* q, const void* k, const vo
                                void* cuda_stream);
 
 /*
+ * rope3d_qk_norm_rope_append with options (pairing and cache layout; see
+ * rope3d_options).  With ROPE3D_CACHE_HEAD_MAJOR the caches are [B][N][cache_tokens][D]
+ * and head n of token i goes to k_cache[b][n][(slot + i) mod cache_tokens].  Errors as
+ * for rope3d_qk_norm_rope_append, plus EINVAL for unknown option values.
+ */
+ROPE3D_API int rope3d_qk_norm_rope_append_ex(
+    const void* q, const void* k, const void* v, void* q_out, int64_t B, int64_t N, int D,
+    int dtype, int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
+    const float* q_norm_w, const float* k_norm_w, float eps, void* k_cache, void* v_cache,
+    int64_t cache_tokens, int64_t slot, const rope3d_tables* tables, int trig,
+    const rope3d_options* options, void* cuda_stream);
+
+/*
  * The rotation alone -- CausalRoPE of Algorithm 3 step 3 / Algorithm 2 -- on one
  * token range: out[b][r] = RoPE(x[b][r], pos(token_begin + r)).  x and out are
  * [B][n_tok][N][D] of dtype; out may be x (in place) or must not overlap it.  Other
@@ -154,6 +191,12 @@ ROPE3D_API int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int 
                  int64_t token_begin, int64_t token_end, int64_t frame_offset,
                  int T, int H, int W, const rope3d_tables* tables, int trig,
                  void* cuda_stream);
+
+/* rope3d_apply with options (only the pairing applies). */
+ROPE3D_API int rope3d_apply_ex(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
+                               int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                               int T, int H, int W, const rope3d_tables* tables, int trig,
+                               const rope3d_options* options, void* cuda_stream);
 
 /*
  * Integer part of the step, for inspection: for each index i of [token_begin,

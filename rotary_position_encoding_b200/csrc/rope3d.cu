@@ -153,18 +153,26 @@ int check_common(int64_t B, int64_t N, int D, int dtype, int64_t token_begin,
     return ROPE3D_OK;
 }
 
-// Team geometry, a function of (N, dtype) only -- it fixes the reduction order, so it
-// must not depend on the token range or the grid.
+// Team geometry, a function of (N, dtype, pairing) only -- it fixes the reduction order,
+// so it must not depend on the token range or the grid.
 struct Geometry {
     int dim_vecs;
     int tpr;
     int vpt;
 };
 
-Geometry geometry(int64_t N, int dtype) {
+Geometry geometry(int64_t N, int dtype, int pairing) {
     const int elems_per_vec = dtype == ROPE3D_BF16 ? 8 : 4;
     Geometry g;
     g.dim_vecs = (int)(N * rope3d::kHeadDim / elems_per_vec);
+    if (pairing == ROPE3D_PAIRING_HALF) {
+        // slots come in twos (a head's two halves at one position): count half units
+        const int units = g.dim_vecs / 2;
+        const int per_warp = 32 * (ROPE3D_VPT_TARGET / 2);
+        g.tpr = 32 * ((units + per_warp - 1) / per_warp);
+        g.vpt = 2 * ((units + g.tpr - 1) / g.tpr);
+        return g;
+    }
     const int per_warp = 32 * ROPE3D_VPT_TARGET;
     g.tpr = 32 * ((g.dim_vecs + per_warp - 1) / per_warp);
     g.vpt = (g.dim_vecs + g.tpr - 1) / g.tpr;
@@ -173,45 +181,75 @@ Geometry geometry(int64_t N, int dtype) {
 
 using KernelFn = void (*)(const rope3d::Params);
 
-template <typename T, int TRIG, int MODE>
+template <typename T, int TRIG, int MODE, int PAIR>
 KernelFn pick_vpt(int vpt) {
-    switch (vpt) {
-        case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE>;
-        case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE>;
-        case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE>;
-        case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE>;
-        default: return nullptr;
+    if constexpr (PAIR == rope3d::kPairHalf) {  // slots come in twos
+        switch (vpt) {
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR>;
+            default: return nullptr;
+        }
+    } else {
+        switch (vpt) {
+            case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE, PAIR>;
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR>;
+            case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR>;
+            default: return nullptr;
+        }
     }
 }
 
+template <typename T, int MODE, int PAIR>
+KernelFn pick_trig(int trig, int vpt) {
+    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<T, rope3d::kTrigTable, MODE, PAIR>(vpt)
+                                     : pick_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR>(vpt);
+}
+
 template <int MODE>
-KernelFn pick_kernel(int dtype, int trig, int vpt) {
+KernelFn pick_kernel(int dtype, int trig, int pairing, int vpt) {
     if (dtype == ROPE3D_BF16)
-        return trig == ROPE3D_TRIG_TABLE ? pick_vpt<__nv_bfloat16, rope3d::kTrigTable, MODE>(vpt)
-                                         : pick_vpt<__nv_bfloat16, rope3d::kTrigOnTheFly, MODE>(vpt);
-    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<float, rope3d::kTrigTable, MODE>(vpt)
-                                     : pick_vpt<float, rope3d::kTrigOnTheFly, MODE>(vpt);
+        return pairing == ROPE3D_PAIRING_HALF
+                   ? pick_trig<__nv_bfloat16, MODE, rope3d::kPairHalf>(trig, vpt)
+                   : pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent>(trig, vpt);
+    return pairing == ROPE3D_PAIRING_HALF ? pick_trig<float, MODE, rope3d::kPairHalf>(trig, vpt)
+                                          : pick_trig<float, MODE, rope3d::kPairAdjacent>(trig, vpt);
 }
 
 using TmaKernelFn = void (*)(const rope3d::Params);
 
-template <typename T, int TRIG>
+template <typename T, int TRIG, int PAIR>
 TmaKernelFn pick_tma_vpt(int vpt) {
-    switch (vpt) {
-        case 1: return rope3d::qk_norm_rope_tma_kernel<T, 1, TRIG>;
-        case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG>;
-        case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG>;
-        case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG>;
-        default: return nullptr;
+    if constexpr (PAIR == rope3d::kPairHalf) {
+        switch (vpt) {
+            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR>;
+            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR>;
+            default: return nullptr;
+        }
+    } else {
+        switch (vpt) {
+            case 1: return rope3d::qk_norm_rope_tma_kernel<T, 1, TRIG, PAIR>;
+            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR>;
+            case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG, PAIR>;
+            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR>;
+            default: return nullptr;
+        }
     }
 }
 
-TmaKernelFn pick_tma_kernel(int dtype, int trig, int vpt) {
+template <typename T, int PAIR>
+TmaKernelFn pick_tma_trig(int trig, int vpt) {
+    return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<T, rope3d::kTrigTable, PAIR>(vpt)
+                                     : pick_tma_vpt<T, rope3d::kTrigOnTheFly, PAIR>(vpt);
+}
+
+TmaKernelFn pick_tma_kernel(int dtype, int trig, int pairing, int vpt) {
     if (dtype == ROPE3D_BF16)
-        return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<__nv_bfloat16, rope3d::kTrigTable>(vpt)
-                                         : pick_tma_vpt<__nv_bfloat16, rope3d::kTrigOnTheFly>(vpt);
-    return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<float, rope3d::kTrigTable>(vpt)
-                                     : pick_tma_vpt<float, rope3d::kTrigOnTheFly>(vpt);
+        return pairing == ROPE3D_PAIRING_HALF
+                   ? pick_tma_trig<__nv_bfloat16, rope3d::kPairHalf>(trig, vpt)
+                   : pick_tma_trig<__nv_bfloat16, rope3d::kPairAdjacent>(trig, vpt);
+    return pairing == ROPE3D_PAIRING_HALF ? pick_tma_trig<float, rope3d::kPairHalf>(trig, vpt)
+                                          : pick_tma_trig<float, rope3d::kPairAdjacent>(trig, vpt);
 }
 
 // Resident blocks per SM for a kernel at a block size and shared-memory size.  The
@@ -315,10 +353,10 @@ size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) 
 // the register kernel measured faster on B200 (graph-replayed launches, 2 to 64 heads,
 // 1560 to 32760 tokens): teams under 96 threads, a single team per block, or fewer
 // than 16 rows per team.  The ring won by 2-5% at 24 to 40 heads and >= 10800 tokens.
-int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
+int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int dev,
                      const DeviceInfo& info, cudaStream_t stream, bool forced, bool* launched) {
     *launched = false;
-    const Geometry g = geometry(N, dtype);
+    const Geometry g = geometry(N, dtype, pairing);
     if (g.tpr > rope3d::kTmaMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
     const int warps_per_team = g.tpr / 32;
     p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
@@ -341,7 +379,7 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
                     p.units < (int64_t)16 * info.sms * teams))
         return ROPE3D_OK;
     smem = tma_layout(p, teams, stages, warps_per_team);
-    TmaKernelFn fn = pick_tma_kernel(dtype, trig, g.vpt);
+    TmaKernelFn fn = pick_tma_kernel(dtype, trig, pairing, g.vpt);
     if (fn == nullptr) return ROPE3D_OK;
     const int threads = teams * g.tpr;
     int per_sm = 0;
@@ -364,9 +402,9 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int dev,
 }
 
 template <int MODE>
-int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const DeviceInfo& info,
-           cudaStream_t stream) {
-    const Geometry g = geometry(N, dtype);
+int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int dev,
+           const DeviceInfo& info, cudaStream_t stream) {
+    const Geometry g = geometry(N, dtype, pairing);
     if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4)
         return fail(ROPE3D_EINVAL, "N=%lld heads is more than one row team can hold",
                     (long long)N);
@@ -385,7 +423,7 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int dev, const Dev
     if (smem > (size_t)info.max_smem_optin)
         return fail(ROPE3D_EINVAL, "N=%lld needs %zu bytes of shared memory (limit %d)",
                     (long long)N, smem, info.max_smem_optin);
-    KernelFn fn = pick_kernel<MODE>(dtype, trig, g.vpt);
+    KernelFn fn = pick_kernel<MODE>(dtype, trig, pairing, g.vpt);
     if (fn == nullptr) return fail(ROPE3D_EINVAL, "no kernel for vpt=%d", g.vpt);
     int per_sm = 0;
     int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
@@ -429,6 +467,31 @@ void set_small_idx(rope3d::Params& p) {
     const int64_t lim = (int64_t)1 << 31;
     p.small_idx = (p.units < lim && p.token_begin + p.n_tok + p.slot < lim &&
                    p.cache_tokens < lim && p.hw < lim) ? 1 : 0;
+}
+
+// The options of a call (NULL = all defaults), checked.
+int read_options(const rope3d_options* options, rope3d_options* out, bool with_cache) {
+    rope3d_options o{};
+    if (options != nullptr) o = *options;
+    if (o.pairing != ROPE3D_PAIRING_ADJACENT && o.pairing != ROPE3D_PAIRING_HALF)
+        return fail(ROPE3D_EINVAL, "options.pairing %d is not a ROPE3D_PAIRING_* value",
+                    o.pairing);
+    if (o.cache_layout != ROPE3D_CACHE_TOKEN_MAJOR && o.cache_layout != ROPE3D_CACHE_HEAD_MAJOR)
+        return fail(ROPE3D_EINVAL, "options.cache_layout %d is not a ROPE3D_CACHE_* value",
+                    o.cache_layout);
+    if (!with_cache && o.cache_layout != ROPE3D_CACHE_TOKEN_MAJOR)
+        return fail(ROPE3D_EINVAL, "options.cache_layout applies to the fused step only");
+    for (int r : o.reserved)
+        if (r != 0) return fail(ROPE3D_EINVAL, "options.reserved must be zero");
+    *out = o;
+    return ROPE3D_OK;
+}
+
+void fill_layout(rope3d::Params& p, int64_t N, int dtype, const rope3d_options& o) {
+    const int vph = rope3d::kHeadDim / (dtype == ROPE3D_BF16 ? 8 : 4);
+    p.cache_head_major = o.cache_layout == ROPE3D_CACHE_HEAD_MAJOR ? 1 : 0;
+    p.n_heads = (int)N;
+    p.vph_log2 = vph == 16 ? 4 : 5;
 }
 
 int check_tables_device(const rope3d_tables* tables, int dev) {
@@ -626,7 +689,24 @@ int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void
                                void* k_cache, void* v_cache, int64_t cache_tokens,
                                int64_t slot, const rope3d_tables* tables, int trig,
                                void* cuda_stream) {
-    int rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
+    return rope3d_qk_norm_rope_append_ex(q, k, v, q_out, B, N, D, dtype, token_begin, token_end,
+                                         frame_offset, T, H, W, q_norm_w, k_norm_w, eps, k_cache,
+                                         v_cache, cache_tokens, slot, tables, trig, nullptr,
+                                         cuda_stream);
+}
+
+int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, void* q_out,
+                                  int64_t B, int64_t N, int D, int dtype,
+                                  int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                                  int T, int H, int W,
+                                  const float* q_norm_w, const float* k_norm_w, float eps,
+                                  void* k_cache, void* v_cache, int64_t cache_tokens,
+                                  int64_t slot, const rope3d_tables* tables, int trig,
+                                  const rope3d_options* options, void* cuda_stream) {
+    rope3d_options opt;
+    int rc = read_options(options, &opt, true);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
                           trig);
     if (rc != ROPE3D_OK) return rc;
     if (!q || !k || !v || !q_out || !k_cache || !v_cache || !q_norm_w || !k_norm_w)
@@ -676,19 +756,20 @@ int rope3d_qk_norm_rope_append(const void* q, const void* k, const void* v, void
     p.cache_tokens = cache_tokens;
     p.slot = slot;
     p.eps = eps;
+    fill_layout(p, N, dtype, opt);
     set_small_idx(p);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     const int path = g_force_path.load();
     if (path != ROPE3D_PATH_REGISTERS) {
         bool launched = false;
-        rc = launch_fused_tma(p, N, dtype, trig, dev, info, stream, path == ROPE3D_PATH_TMA,
-                              &launched);
+        rc = launch_fused_tma(p, N, dtype, trig, opt.pairing, dev, info, stream,
+                              path == ROPE3D_PATH_TMA, &launched);
         if (launched) g_last_path = ROPE3D_PATH_TMA;
         if (rc != ROPE3D_OK || launched) return rc;
         if (path == ROPE3D_PATH_TMA)
             return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);
     }
-    rc = launch<rope3d::kModeFused>(p, N, dtype, trig, dev, info, stream);
+    rc = launch<rope3d::kModeFused>(p, N, dtype, trig, opt.pairing, dev, info, stream);
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
     return rc;
 }
@@ -697,7 +778,18 @@ int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtyp
                  int64_t token_begin, int64_t token_end, int64_t frame_offset,
                  int T, int H, int W, const rope3d_tables* tables, int trig,
                  void* cuda_stream) {
-    int rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
+    return rope3d_apply_ex(x, out, B, N, D, dtype, token_begin, token_end, frame_offset, T, H,
+                           W, tables, trig, nullptr, cuda_stream);
+}
+
+int rope3d_apply_ex(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,
+                    int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                    int T, int H, int W, const rope3d_tables* tables, int trig,
+                    const rope3d_options* options, void* cuda_stream) {
+    rope3d_options opt;
+    int rc = read_options(options, &opt, false);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
                           trig);
     if (rc != ROPE3D_OK) return rc;
     if (!x || !out) return fail(ROPE3D_EINVAL, "a tensor pointer is NULL");
@@ -717,8 +809,9 @@ int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtyp
     fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
     p.q = x;
     p.q_out = out;
+    fill_layout(p, N, dtype, opt);
     set_small_idx(p);
-    return launch<rope3d::kModeApply>(p, N, dtype, trig, dev, info,
+    return launch<rope3d::kModeApply>(p, N, dtype, trig, opt.pairing, dev, info,
                                       static_cast<cudaStream_t>(cuda_stream));
 }
 

@@ -41,6 +41,9 @@ constexpr int kTmaMaxBlockThreads = 320;  // ring kernel: one block per SM, up t
 
 enum Mode : int { kModeFused = 0, kModeApply = 1 };
 enum Trig : int { kTrigTable = 0, kTrigOnTheFly = 1 };
+// Pairing of a head's elements into complex pairs: adjacent (2j, 2j+1) -- the complex
+// view of Wan2.1 -- or rotate_half (j, j + 64), the cos/sin form of M-RoPE.
+enum Pairing : int { kPairAdjacent = 0, kPairHalf = 1 };
 
 struct Params {
     const void* q;        // fused: q;  apply: x
@@ -78,6 +81,10 @@ struct Params {
     uint32_t row_bytes;   // bytes of one token row of one tensor
     uint32_t tx_extra;    // extra bytes each stage waits for (0; tests use it to time out)
     uint32_t off_bars, off_fail, off_part, off_w, off_stage;
+    // layout options
+    int cache_head_major;  // caches are [B][N][cache_tokens][D] instead of [B][cache_tokens][N][D]
+    int n_heads;           // N
+    int vph_log2;          // log2 of the 16-byte vectors per head
     float inv_freq[kPairs];  // fp32 angle per unit position of every pair
 };
 
@@ -99,6 +106,17 @@ template <> struct VecTraits<__nv_bfloat16> {
         uint32_t u = *reinterpret_cast<uint32_t*>(&h);
         if (m == 0) x.x = u; else if (m == 1) x.y = u; else if (m == 2) x.z = u; else x.w = u;
     }
+    static constexpr int kElems = 8;
+    __device__ static inline float elem(const Vec& x, int m) {
+        const uint32_t u = (m >> 1) == 0 ? x.x : (m >> 1) == 1 ? x.y : (m >> 1) == 2 ? x.z : x.w;
+        return (m & 1) ? __uint_as_float(u & 0xffff0000u) : __uint_as_float(u << 16);
+    }
+    __device__ static inline Vec pack_elems(const float (&v)[8]) {
+        Vec o;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) set_pair(o, w, v[2 * w], v[2 * w + 1]);
+        return o;
+    }
 };
 
 template <> struct VecTraits<float> {
@@ -112,7 +130,49 @@ template <> struct VecTraits<float> {
     __device__ static inline void set_pair(Vec& x, int m, float re, float im) {
         if (m == 0) { x.x = re; x.y = im; } else { x.z = re; x.w = im; }
     }
+    static constexpr int kElems = 4;
+    __device__ static inline float elem(const Vec& x, int m) {
+        return m == 0 ? x.x : m == 1 ? x.y : m == 2 ? x.z : x.w;
+    }
+    __device__ static inline Vec pack_elems(const float (&v)[4]) {
+        return make_float4(v[0], v[1], v[2], v[3]);
+    }
 };
+
+// Pairs a thread rotates: with adjacent pairing the kPairsPerVec pairs of its vector;
+// with rotate_half the kElems pairs whose real (first half of the head) or imaginary
+// (second half) parts its vector holds.
+template <typename T, int PAIR>
+struct PairCount {
+    static constexpr int value =
+        PAIR == kPairAdjacent ? VecTraits<T>::kPairsPerVec : VecTraits<T>::kElems;
+};
+
+// Vector (16-byte unit of the row) that slot s of thread t holds.
+//  adjacent pairing: t + s * TPR -- coalesced, and a thread's position inside a head
+//                    is t mod (vectors per head);
+//  rotate_half:      slots come in twos over "half units" u = t + (s/2) * TPR; unit u
+//                    is position u mod HALF of head u / HALF, and its even slot holds
+//                    the head's first-half vector there, its odd slot the second-half
+//                    vector HALF further on -- the real and imaginary parts of the same
+//                    pairs, so no data crosses lanes.
+// In both, a vector index >= dim_vecs marks an empty slot.
+template <typename T, int PAIR>
+__device__ __forceinline__ int slot_vec(int t, int s, int tpr) {
+    using Tr = VecTraits<T>;
+    if (PAIR == kPairAdjacent) return t + s * tpr;
+    constexpr int HALF = Tr::kVecsPerHead / 2;
+    const int u = t + (s >> 1) * tpr;
+    return (u / HALF) * Tr::kVecsPerHead + (u % HALF) + (s & 1) * HALF;
+}
+
+// First pair of a thread whose vectors sit at position `pos_in_head` of their heads.
+template <typename T, int PAIR>
+__device__ __forceinline__ int first_pair(int pos_in_head) {
+    using Tr = VecTraits<T>;
+    return PAIR == kPairAdjacent ? pos_in_head * Tr::kPairsPerVec
+                                 : (pos_in_head % (Tr::kVecsPerHead / 2)) * Tr::kElems;
+}
 
 // ---------------------------------------------------------------- memory helpers
 
@@ -186,6 +246,15 @@ __device__ __forceinline__ RowPos decode_row(const Params& p, int64_t u) {
     return q;
 }
 
+// Index (in 16-byte vectors) of vector idx of a row's K/V in the cache, for the row's
+// cache row: token-major [B][C][N][D] or head-major [B][N][C][D].
+__device__ __forceinline__ int64_t cache_vec_index(const Params& p, const RowPos& pos, int idx) {
+    if (!p.cache_head_major) return (pos.b * p.cache_tokens + pos.crow) * p.dim_vecs + idx;
+    const int n = idx >> p.vph_log2;
+    const int v = idx & ((1 << p.vph_log2) - 1);
+    return (((pos.b * p.n_heads + n) * p.cache_tokens + pos.crow) << p.vph_log2) + v;
+}
+
 // The complex pairs a thread rotates (fixed for the thread's whole life).
 template <int PPV>
 struct PairInfo {
@@ -234,7 +303,7 @@ __device__ __forceinline__ void pair_trig(const PairInfo<PPV>& pi, const RowPos&
 }
 
 // Sum of squares of this thread's share of one row of q and of k (fixed order).
-template <typename T, int VPT>
+template <typename T, int VPT, int PAIR>
 __device__ __forceinline__ void partial_sum_squares(const typename VecTraits<T>::Vec (&xq)[VPT],
                                                     const typename VecTraits<T>::Vec (&xk)[VPT],
                                                     int t, int tpr, int dim_vecs, float& sq,
@@ -244,7 +313,7 @@ __device__ __forceinline__ void partial_sum_squares(const typename VecTraits<T>:
     sk = 0.f;
 #pragma unroll
     for (int s = 0; s < VPT; ++s) {
-        if (t + s * tpr < dim_vecs) {
+        if (slot_vec<T, PAIR>(t, s, tpr) < dim_vecs) {
 #pragma unroll
             for (int m = 0; m < Tr::kPairsPerVec; ++m) {
                 float a, c;
@@ -313,6 +382,44 @@ __device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
     return out;
 }
 
+// rotate_half pairing: `re_v` is a head's first-half vector at some position and
+// `im_v` its second-half vector at the same position -- the real and imaginary parts of
+// kElems pairs.  Both are normalised with their own weights, y = x * rs * w, and
+// (y_re + i y_im) * (cos + i sin) is returned as the two vectors of the result.
+template <typename T, bool NORM>
+__device__ __forceinline__ void norm_rotate_half(
+    const typename VecTraits<T>::Vec& re_v, const typename VecTraits<T>::Vec& im_v, float rs,
+    const float* s_w, int e_re, int e_im,
+    const float (&cs)[VecTraits<T>::kElems], const float (&sn)[VecTraits<T>::kElems],
+    typename VecTraits<T>::Vec& out_re, typename VecTraits<T>::Vec& out_im) {
+    using Tr = VecTraits<T>;
+    constexpr int E = Tr::kElems;
+    float wr[E], wi[E];
+    if (NORM) {
+#pragma unroll
+        for (int c = 0; c < E / 4; ++c) {
+            const float4 a = *reinterpret_cast<const float4*>(s_w + e_re + 4 * c);
+            const float4 b = *reinterpret_cast<const float4*>(s_w + e_im + 4 * c);
+            wr[4 * c] = a.x; wr[4 * c + 1] = a.y; wr[4 * c + 2] = a.z; wr[4 * c + 3] = a.w;
+            wi[4 * c] = b.x; wi[4 * c + 1] = b.y; wi[4 * c + 2] = b.z; wi[4 * c + 3] = b.w;
+        }
+    }
+    float o_re[E], o_im[E];
+#pragma unroll
+    for (int m = 0; m < E; ++m) {
+        float a = Tr::elem(re_v, m);
+        float c = Tr::elem(im_v, m);
+        if (NORM) {
+            a = a * rs * wr[m];
+            c = c * rs * wi[m];
+        }
+        o_re[m] = a * cs[m] - c * sn[m];
+        o_im[m] = a * sn[m] + c * cs[m];
+    }
+    out_re = Tr::pack_elems(o_re);
+    out_im = Tr::pack_elems(o_im);
+}
+
 __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, float* s_wk) {
     // dim is a multiple of 128, so float4 copies cover it
     const float4* gq = reinterpret_cast<const float4*>(p.q_w);
@@ -325,15 +432,65 @@ __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, floa
     }
 }
 
+// ---------------------------------------------------------------- per-row output
+
+// Normalise, rotate and store this thread's vectors of one row: q_out, and in the fused
+// mode the K row into the cache (V is stored by the caller).  With rotate_half pairing
+// slots 2m and 2m+1 hold the two halves of the same pairs (see slot_vec).
+template <typename T, int VPT, int PAIR, int MODE>
+__device__ __forceinline__ void emit_row(
+    const Params& p, int t, const RowPos& pos, int64_t row_vec,
+    const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
+    float rq, float rk, const float* s_wq, const float* s_wk,
+    const float (&cs)[PairCount<T, PAIR>::value], const float (&sn)[PairCount<T, PAIR>::value],
+    typename VecTraits<T>::Vec* qo, typename VecTraits<T>::Vec* kc) {
+    using Tr = VecTraits<T>;
+    using Vec = typename Tr::Vec;
+    constexpr int EPV = Tr::kElems;
+    constexpr bool NORM = MODE == kModeFused;
+    if constexpr (PAIR == kPairAdjacent) {
+#pragma unroll
+        for (int s = 0; s < VPT; ++s) {
+            const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+            if (idx < p.dim_vecs) {
+                const int e0 = idx * EPV;
+                store_out(qo + row_vec + idx, norm_rotate<T, NORM>(xq[s], rq, s_wq, e0, cs, sn));
+                if (MODE == kModeFused)
+                    store_out(kc + cache_vec_index(p, pos, idx),
+                              norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
+            }
+        }
+    } else {
+        static_assert(VPT % 2 == 0, "rotate_half slots come in twos");
+#pragma unroll
+        for (int s = 0; s < VPT; s += 2) {
+            const int i_re = slot_vec<T, PAIR>(t, s, p.tpr);
+            const int i_im = slot_vec<T, PAIR>(t, s + 1, p.tpr);
+            if (i_re < p.dim_vecs) {
+                Vec o_re, o_im;
+                norm_rotate_half<T, NORM>(xq[s], xq[s + 1], rq, s_wq, i_re * EPV, i_im * EPV, cs,
+                                          sn, o_re, o_im);
+                store_out(qo + row_vec + i_re, o_re);
+                store_out(qo + row_vec + i_im, o_im);
+                if (MODE == kModeFused) {
+                    norm_rotate_half<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV, i_im * EPV,
+                                              cs, sn, o_re, o_im);
+                    store_out(kc + cache_vec_index(p, pos, i_re), o_re);
+                    store_out(kc + cache_vec_index(p, pos, i_im), o_im);
+                }
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- register kernel
 
-template <typename T, int VPT, int TRIG, int MODE>
+template <typename T, int VPT, int TRIG, int MODE, int PAIR>
 __global__ void __launch_bounds__(kMaxBlockThreads)
 qk_norm_rope_kernel(const Params p) {
     using Tr = VecTraits<T>;
     using Vec = typename Tr::Vec;
-    constexpr int PPV = Tr::kPairsPerVec;
-    constexpr int EPV = 2 * PPV;  // elements per vector
+    constexpr int NP = PairCount<T, PAIR>::value;
 
     extern __shared__ float4 smem4[];
     float* s_wq = reinterpret_cast<float*>(smem4);
@@ -353,7 +510,7 @@ qk_norm_rope_kernel(const Params p) {
         stage_weights(p, s_wq, s_wk);
         __syncthreads();
     }
-    const PairInfo<PPV> pi = pair_info<PPV>(p, (t % Tr::kVecsPerHead) * PPV);
+    const PairInfo<NP> pi = pair_info<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
 
     const Vec* qg = reinterpret_cast<const Vec*>(p.q);
     const Vec* kg = reinterpret_cast<const Vec*>(p.k);
@@ -370,7 +527,7 @@ qk_norm_rope_kernel(const Params p) {
         Vec xq[VPT], xk[VPT], xv[VPT];
 #pragma unroll
         for (int s = 0; s < VPT; ++s) {
-            const int idx = t + s * p.tpr;
+            const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
             if (idx < p.dim_vecs) {
                 xq[s] = load_stream(qg + row_vec + idx);
                 if (MODE == kModeFused) {
@@ -379,37 +536,25 @@ qk_norm_rope_kernel(const Params p) {
                 }
             }
         }
-        float cs[PPV], sn[PPV];
+        float cs[NP], sn[NP];
         pair_trig<TRIG>(pi, pos, cs, sn);
 
         float rq = 1.0f, rk = 1.0f;
-        int64_t cache_vec = 0;
         if (MODE == kModeFused) {
-            cache_vec = (pos.b * p.cache_tokens + pos.crow) * p.dim_vecs;
 #pragma unroll
             for (int s = 0; s < VPT; ++s) {
-                const int idx = t + s * p.tpr;
-                if (idx < p.dim_vecs) store_out(vc + cache_vec + idx, xv[s]);
+                const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+                if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[s]);
             }
             float sq, sk;
-            partial_sum_squares<T, VPT>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
+            partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
                                         warps_per_team, lane, p.tpr, parity);
             rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
-#pragma unroll
-        for (int s = 0; s < VPT; ++s) {
-            const int idx = t + s * p.tpr;
-            if (idx < p.dim_vecs) {
-                const int e0 = idx * EPV;
-                store_out(qo + row_vec + idx,
-                          norm_rotate<T, MODE == kModeFused>(xq[s], rq, s_wq, e0, cs, sn));
-                if (MODE == kModeFused)
-                    store_out(kc + cache_vec + idx,
-                              norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
-            }
-        }
+        emit_row<T, VPT, PAIR, MODE>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs, sn, qo,
+                                     kc);
     }
 }
 

@@ -76,13 +76,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-template <typename T, int VPT, int TRIG>
+template <typename T, int VPT, int TRIG, int PAIR>
 __global__ void __launch_bounds__(kTmaMaxBlockThreads, 1)
 qk_norm_rope_tma_kernel(const Params p) {
     using Tr = VecTraits<T>;
     using Vec = typename Tr::Vec;
-    constexpr int PPV = Tr::kPairsPerVec;
-    constexpr int EPV = 2 * PPV;
+    constexpr int NP = PairCount<T, PAIR>::value;
 
     extern __shared__ __align__(128) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bars);
@@ -133,7 +132,7 @@ qk_norm_rope_tma_kernel(const Params p) {
     if (t == 0)
         for (int kk = 0; kk < S; ++kk) issue(kk);
 
-    const PairInfo<PPV> pi = pair_info<PPV>(p, (t % Tr::kVecsPerHead) * PPV);
+    const PairInfo<NP> pi = pair_info<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
     Vec* qo = reinterpret_cast<Vec*>(p.q_out);
     Vec* kc = reinterpret_cast<Vec*>(p.k_cache);
     Vec* vc = reinterpret_cast<Vec*>(p.v_cache);
@@ -151,7 +150,7 @@ qk_norm_rope_tma_kernel(const Params p) {
         Vec xq[VPT], xk[VPT], xv[VPT];
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int idx = t + j * p.tpr;
+            const int idx = slot_vec<T, PAIR>(t, j, p.tpr);
             if (idx < p.dim_vecs) {
                 xq[j] = sq[idx];
                 xk[j] = sk[idx];
@@ -159,7 +158,7 @@ qk_norm_rope_tma_kernel(const Params p) {
             }
         }
         float psq, psk;
-        partial_sum_squares<T, VPT>(xq, xk, t, p.tpr, p.dim_vecs, psq, psk);
+        partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, psq, psk);
         // The reduction barrier doubles as the team's "stage consumed" point and its
         // vote on a timed-out wait.
         if (!ok) s_fail[team] = 1;
@@ -184,22 +183,18 @@ qk_norm_rope_tma_kernel(const Params p) {
         }
 
         const RowPos pos = decode_row(p, u);
-        float cs[PPV], sn[PPV];
+        float cs[NP], sn[NP];
         pair_trig<TRIG>(pi, pos, cs, sn);
         const float rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
         const float rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         const int64_t row_vec = u * p.dim_vecs;
-        const int64_t cache_vec = (pos.b * p.cache_tokens + pos.crow) * p.dim_vecs;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
-            const int idx = t + j * p.tpr;
-            if (idx < p.dim_vecs) {
-                const int e0 = idx * EPV;
-                store_out(vc + cache_vec + idx, xv[j]);
-                store_out(qo + row_vec + idx, norm_rotate<T, true>(xq[j], rq, s_wq, e0, cs, sn));
-                store_out(kc + cache_vec + idx, norm_rotate<T, true>(xk[j], rk, s_wk, e0, cs, sn));
-            }
+            const int idx = slot_vec<T, PAIR>(t, j, p.tpr);
+            if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[j]);
         }
+        emit_row<T, VPT, PAIR, kModeFused>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs,
+                                           sn, qo, kc);
     }
 
     if (failed && t == 0) {

@@ -34,6 +34,17 @@ ROPE3D_SCHEDULE_HEAD_WIDE = 1
 ROPE3D_TRIG_TABLE = 0
 ROPE3D_TRIG_ONTHEFLY = 1
 
+ROPE3D_PAIRING_ADJACENT = 0
+ROPE3D_PAIRING_HALF = 1
+ROPE3D_CACHE_TOKEN_MAJOR = 0
+ROPE3D_CACHE_HEAD_MAJOR = 1
+
+
+class rope3d_options(ctypes.Structure):
+    """struct rope3d_options of include/rope3d.h."""
+    _fields_ = [("pairing", ctypes.c_int), ("cache_layout", ctypes.c_int),
+                ("reserved", ctypes.c_int * 6)]
+
 # include/rope3d_testing.h
 ROPE3D_PATH_AUTO = 0
 ROPE3D_PATH_REGISTERS = 1
@@ -51,8 +62,14 @@ SIGNATURES = {
     "rope3d_qk_norm_rope_append": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64,
                                     _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP, _VP, _I64,
                                     _I64, _VP, _INT, _VP], _INT),
+    "rope3d_qk_norm_rope_append_ex": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64,
+                                       _I64, _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP,
+                                       _VP, _I64, _I64, _VP, _INT,
+                                       ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_apply": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT, _VP,
                       _INT, _VP], _INT),
+    "rope3d_apply_ex": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT,
+                         _VP, _INT, ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_decode_positions": ([_I64, _I64, _I64, _INT, _INT, _INT, _I64, _I64, _VP, _VP], _INT),
     "rope3d_check_device_status": ([_VP, _VP], _INT),
     "rope3d_qk_norm_rope_append_noalloc": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64,
@@ -207,6 +224,55 @@ def rope3d_qk_norm_rope_append_noalloc(q, k, v, q_out, token_begin: int, token_e
         _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), k_cache.shape[1], slot,
         n_t, n_h, n_w, theta, schedule, trig, _stream(stream)))
+
+
+def rope3d_qk_norm_rope_append_ex(q, k, v, q_out, token_begin: int, token_end: int,
+                                  frame_offset: int, T: int, H: int, W: int, q_norm_w, k_norm_w,
+                                  eps: float, k_cache, v_cache, slot: int, tables: Tables,
+                                  trig: int = ROPE3D_TRIG_TABLE,
+                                  pairing: int = ROPE3D_PAIRING_ADJACENT,
+                                  cache_layout: int = ROPE3D_CACHE_TOKEN_MAJOR,
+                                  stream=None) -> None:
+    """rope3d_qk_norm_rope_append with options; head-major caches are [B, N, C, 128]."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or q_out.shape != q.shape:
+        raise ValueError("q, k, v and q_out must all be [B, n_tok, N, D]")
+    B, n_tok, N, D = q.shape
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must have one 4-d shape")
+    if cache_layout == ROPE3D_CACHE_HEAD_MAJOR:
+        C = k_cache.shape[2]
+        ok = k_cache.shape[0] == B and k_cache.shape[1] == N and k_cache.shape[3] == D
+    else:
+        C = k_cache.shape[1]
+        ok = k_cache.shape[0] == B and k_cache.shape[2:] == q.shape[2:]
+    if not ok:
+        raise ValueError("cache shape does not match q and the cache layout")
+    if n_tok != token_end - token_begin:
+        raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
+    for name, t in (("k", k), ("v", v), ("q_out", q_out), ("k_cache", k_cache),
+                    ("v_cache", v_cache)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have q's dtype {q.dtype}")
+    opts = rope3d_options(pairing, cache_layout)
+    _check(load_library().rope3d_qk_norm_rope_append_ex(
+        _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
+        B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,
+        _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
+        _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), C, slot,
+        tables.handle, trig, ctypes.byref(opts), _stream(stream)))
+
+
+def rope3d_apply_ex(x, out, token_begin: int, token_end: int, frame_offset: int, T: int, H: int,
+                    W: int, tables: Tables, trig: int = ROPE3D_TRIG_TABLE,
+                    pairing: int = ROPE3D_PAIRING_ADJACENT, stream=None) -> None:
+    if x.dim() != 4 or out.shape != x.shape or out.dtype != x.dtype:
+        raise ValueError("x and out must be [B, n_tok, N, D] of one dtype")
+    B, n_tok, N, D = x.shape
+    opts = rope3d_options(pairing, 0)
+    _check(load_library().rope3d_apply_ex(
+        _dev_ptr(x, "x"), _dev_ptr(out, "out"), B, N, D, _dtype_code(x), token_begin,
+        token_end, frame_offset, T, H, W, tables.handle, trig, ctypes.byref(opts),
+        _stream(stream)))
 
 
 def rope3d_apply(x, out, token_begin: int, token_end: int, frame_offset: int, T: int, H: int,

@@ -101,3 +101,25 @@ def test_testing_hooks_validate_without_device(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         rope3d.load_library(str(tmp_path / "librope3d.so"))
+
+
+def test_options_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of rope3d_options has the C struct's size and field offsets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "rope3d.h"\n'
+                   'int main(void){printf("%zu %zu %zu %zu", sizeof(rope3d_options),'
+                   ' offsetof(rope3d_options, pairing), offsetof(rope3d_options, cache_layout),'
+                   ' offsetof(rope3d_options, reserved)); return 0;}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    size, o_pair, o_layout, o_res = map(int, subprocess.run([str(exe)], capture_output=True,
+                                                             text=True).stdout.split())
+    S = rope3d.rope3d_options
+    assert size == ctypes.sizeof(S)
+    assert (o_pair, o_layout, o_res) == (S.pairing.offset, S.cache_layout.offset,
+                                         S.reserved.offset)
