@@ -50,6 +50,8 @@ _D = ctypes.POINTER(ctypes.c_double)
 _I64 = ctypes.c_int64
 _INT = ctypes.c_int
 _DBL = ctypes.c_double
+_F = ctypes.POINTER(ctypes.c_float)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
 
 
 def _declare(lib):
@@ -82,6 +84,13 @@ def _declare(lib):
                                                       _INT, _DBL, _INT, _INT, _INT, _INT], _INT),
         "rope3d_oracle_apply_pairing": ([_D, _D, _I64, _I64, _I64, _I64, _I64, _I64, _I64,
                                          _I64, _I64, _INT, _INT, _INT, _DBL, _INT, _INT], _INT),
+        "rope3d_oracle_e4m3_value": ([_INT], _DBL),
+        "rope3d_oracle_e4m3_encode": ([ctypes.c_float], _INT),
+        "rope3d_oracle_quantize_head_e4m3": ([_F, _I64, _U8, _F], None),
+        "rope3d_oracle_qk_norm_rope_append_fp8": ([_D, _D, _D, _D, _I64, _I64, _I64, _I64, _I64,
+                                                   _I64, _I64, _I64, _I64, _D, _D, _DBL, _U8,
+                                                   _U8, _F, _F, _I64, _I64, _INT, _INT, _INT,
+                                                   _DBL, _INT, _INT, _INT], _INT),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -98,6 +107,18 @@ def _f64(a, name):
     if not (isinstance(a, np.ndarray) and a.dtype == np.float64 and a.flags.c_contiguous):
         raise TypeError(f"{name} must be a C-contiguous float64 numpy array")
     return a.ctypes.data_as(_D)
+
+
+def _f32(a, name):
+    if not (isinstance(a, np.ndarray) and a.dtype == np.float32 and a.flags.c_contiguous):
+        raise TypeError(f"{name} must be a C-contiguous float32 numpy array")
+    return a.ctypes.data_as(_F)
+
+
+def _u8(a, name):
+    if not (isinstance(a, np.ndarray) and a.dtype == np.uint8 and a.flags.c_contiguous):
+        raise TypeError(f"{name} must be a C-contiguous uint8 numpy array")
+    return a.ctypes.data_as(_U8)
 
 
 def _check(rc):
@@ -203,6 +224,41 @@ class Oracle:
                                             token_begin, token_end, frame_offset, T, H, W,
                                             n_t, n_h, n_w, theta, schedule))
         return out
+
+    # ---- FP8 E4M3 KV cache
+
+    def e4m3_value(self, code: int) -> float:
+        return self.lib.rope3d_oracle_e4m3_value(code)
+
+    def e4m3_encode(self, x: float) -> int:
+        return self.lib.rope3d_oracle_e4m3_encode(x)
+
+    def quantize_head_e4m3(self, x):
+        x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+        codes = np.empty(x.size, dtype=np.uint8)
+        scale = np.zeros(1, dtype=np.float32)
+        self.lib.rope3d_oracle_quantize_head_e4m3(_f32(x, "x"), x.size, _u8(codes, "codes"),
+                                                  _f32(scale, "scale"))
+        return codes, float(scale[0])
+
+    def qk_norm_rope_append_fp8(self, q, k, v, token_begin, token_end, frame_offset, T, H, W,
+                                q_norm_w, k_norm_w, eps, k_codes, v_codes, k_scale, v_scale,
+                                slot, pairing=PAIRING_ADJACENT, cache_layout=CACHE_TOKEN_MAJOR,
+                                n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        """Whole step with an FP8 cache: codes uint8 [B,C,N,D] / [B,N,C,D], scales float32
+        [B,C,N] / [B,N,C], updated in place.  Returns q_out (fp64)."""
+        B, n_tok, N, D = q.shape
+        C = k_codes.shape[1] if cache_layout == CACHE_TOKEN_MAJOR else k_codes.shape[2]
+        q_out = np.empty_like(q)
+        _check(self.lib.rope3d_oracle_qk_norm_rope_append_fp8(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), _f64(q_out, "q_out"), B, N, D,
+            token_begin, token_end, frame_offset, T, H, W,
+            _f64(np.ascontiguousarray(q_norm_w, dtype=np.float64), "q_norm_w"),
+            _f64(np.ascontiguousarray(k_norm_w, dtype=np.float64), "k_norm_w"), eps,
+            _u8(k_codes, "k_codes"), _u8(v_codes, "v_codes"), _f32(k_scale, "k_scale"),
+            _f32(v_scale, "v_scale"), C, slot, n_t, n_h, n_w, theta, schedule, pairing,
+            cache_layout))
+        return q_out
 
     def max_threads(self) -> int:
         return self.lib.rope3d_oracle_max_threads()

@@ -472,6 +472,132 @@ int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t
     return ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ FP8 KV cache
+ *
+ * Quantize-on-append: K and V rows go to the cache as FP8 E4M3 codes with one fp32
+ * scale per (token, head), scale = amax(|x|) / 448 over the head's D values (1 when the
+ * head is all zero), code = E4M3(x / scale) rounded to nearest, ties to the even code,
+ * saturating at +-448.  A reader recovers x ~ value(code) * scale.  The pages name
+ * NVFP4 KV-cache quantization for Blackwell (the LongLive-2.0 abstract) but give no
+ * format details; E4M3 with per-head scales is this build's reading.  The decision
+ * runs in fp32 (the precision the kernel computes the rows in): the oracle rounds its
+ * fp64 K row to fp32 first; V is exact.
+ *
+ * E4M3 (the OCP 8-bit float "E4M3"): sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent field 0 is subnormal (m/8 * 2^-6); the all-ones exponent with all-ones
+ * mantissa is NaN; there is no infinity; the largest finite value is 448.
+ */
+double rope3d_oracle_e4m3_value(int code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 15;
+    int m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code of x (finite), ties to the even code, saturating at +-448; found by
+ * scanning the 127 non-negative finite codes in increasing order. */
+int rope3d_oracle_e4m3_encode(float x)
+{
+    int sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    int best = 0;
+    for (int c = 0; c < 0x7E; ++c) {
+        double lo = rope3d_oracle_e4m3_value(c);
+        double hi = rope3d_oracle_e4m3_value(c + 1);
+        if (a >= lo && a <= hi) {
+            double dlo = a - lo, dhi = hi - a;
+            if (dlo < dhi) best = c;
+            else if (dhi < dlo) best = c + 1;
+            else best = (c % 2 == 0) ? c : c + 1;  /* tie: even mantissa */
+            break;
+        }
+    }
+    return sign | best;
+}
+
+/* One head of n fp32 values -> codes and its scale. */
+void rope3d_oracle_quantize_head_e4m3(const float* x, int64_t n, unsigned char* codes,
+                                      float* scale)
+{
+    float amax = 0.0f;
+    for (int64_t e = 0; e < n; ++e) {
+        float a = fabsf(x[e]);
+        if (a > amax) amax = a;
+    }
+    float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int64_t e = 0; e < n; ++e) codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(x[e] / s);
+    *scale = s;
+}
+
+/*
+ * The whole step with an FP8 E4M3 cache.  q_out is returned in fp64 as above; the
+ * caches are codes [B][cache_tokens][N][D] (token-major) or [B][N][cache_tokens][D]
+ * (head-major) and the scales [B][cache_tokens][N] or [B][N][cache_tokens].
+ */
+int rope3d_oracle_qk_norm_rope_append_fp8(
+    const double* q, const double* k, const double* v, double* q_out,
+    int64_t B, int64_t N, int64_t D,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset,
+    int64_t T, int64_t H, int64_t W,
+    const double* q_norm_w, const double* k_norm_w, double eps,
+    unsigned char* k_codes, unsigned char* v_codes, float* k_scale, float* v_scale,
+    int64_t cache_tokens, int64_t slot,
+    int n_t, int n_h, int n_w, double theta, int schedule, int pairing, int cache_layout)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0 || cache_tokens <= 0 || slot < 0) return ORACLE_EINVAL;
+    if (token_end - token_begin > cache_tokens) return ORACLE_EINVAL;
+    if (cache_layout != ORACLE_CACHE_TOKEN_MAJOR && cache_layout != ORACLE_CACHE_HEAD_MAJOR)
+        return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    double* k_row = (double*)malloc((size_t)dim * sizeof(double));
+    double* v_row = (double*)malloc((size_t)dim * sizeof(double));
+    float* head = (float*)malloc((size_t)D * sizeof(float));
+    if (k_row == NULL || v_row == NULL || head == NULL) {
+        free(k_row); free(v_row); free(head);
+        return ORACLE_EINVAL;
+    }
+    for (int64_t b = 0; b < B && rc == ORACLE_OK; ++b) {
+        for (int64_t r = 0; r < n_tok; ++r) {
+            int64_t i = token_begin + r;
+            int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);
+            int64_t in_off = (b * n_tok + r) * dim;
+            rc = rope3d_oracle_token_pairing(q + in_off, k + in_off, v + in_off, N, D, i,
+                                             frame_offset, T, H, W, q_norm_w, k_norm_w, eps,
+                                             slot, cache_tokens, n_t, n_h, n_w, inv, pairing,
+                                             q_out + in_off, k_row, v_row, NULL);
+            if (rc != ORACLE_OK) break;
+            for (int64_t n = 0; n < N; ++n) {
+                int64_t code_off = cache_layout == ORACLE_CACHE_TOKEN_MAJOR
+                                       ? ((b * cache_tokens + row) * N + n) * D
+                                       : ((b * N + n) * cache_tokens + row) * D;
+                int64_t scale_off = cache_layout == ORACLE_CACHE_TOKEN_MAJOR
+                                        ? (b * cache_tokens + row) * N + n
+                                        : (b * N + n) * cache_tokens + row;
+                for (int64_t e = 0; e < D; ++e) head[e] = (float)k_row[n * D + e];
+                rope3d_oracle_quantize_head_e4m3(head, D, k_codes + code_off, k_scale + scale_off);
+                for (int64_t e = 0; e < D; ++e) head[e] = (float)v_row[n * D + e];
+                rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, v_scale + scale_off);
+            }
+        }
+    }
+    free(k_row);
+    free(v_row);
+    free(head);
+    return rc;
+}
+
 /* Threads the whole-step entry point would use with nthreads <= 0. */
 int rope3d_oracle_max_threads(void)
 {

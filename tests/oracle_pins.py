@@ -523,4 +523,92 @@ def check_apply_half_matches_rotation(orc):
         assert np.array_equal(y[0, r], orc.rotate_pairing(x[0, r], phi, 1))
 
 
+# ---------------------------------------------------------------- FP8 E4M3 KV cache
+
+def check_e4m3_closed_form_values(orc):
+    """E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals, max 448, NaN at
+    the all-ones code."""
+    expect = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+              0x39: 1.125, 0x3C: 1.5, 0x40: 2.0, 0x77: 240.0, 0x7E: 448.0, 0xB8: -1.0,
+              0xFE: -448.0}
+    for code, value in expect.items():
+        assert orc.e4m3_value(code) == value, hex(code)
+    assert math.isnan(orc.e4m3_value(0x7F)) and math.isnan(orc.e4m3_value(0xFF))
+    assert math.copysign(1.0, orc.e4m3_value(0x80)) == -1.0
+
+
+def check_e4m3_encode_round_trip_ties_saturation(orc):
+    vals = [orc.e4m3_value(c) for c in range(0x7F)]
+    assert all(b > a for a, b in zip(vals, vals[1:]))        # strictly increasing
+    for c in range(0x7F):
+        assert orc.e4m3_encode(vals[c]) == c
+        assert orc.e4m3_encode(-vals[c]) == 0x80 | c
+    for c in range(0x7E):                                     # midpoints go to the even code
+        mid = (vals[c] + vals[c + 1]) / 2
+        if np.float32(mid) == mid:
+            assert orc.e4m3_encode(mid) == (c if c % 2 == 0 else c + 1), hex(c)
+    assert orc.e4m3_encode(1000.0) == 0x7E and orc.e4m3_encode(-1e9) == 0xFE
+    assert orc.e4m3_encode(448.0) == 0x7E and orc.e4m3_encode(463.99) == 0x7E
+
+
+def check_e4m3_encode_matches_torch(orc):
+    """In range, the encoder equals torch's float32 -> float8_e4m3fn conversion."""
+    import torch
+    rng = _rng(30)
+    xs = np.concatenate([rng.uniform(-447, 447, 300), rng.standard_normal(300),
+                         rng.standard_normal(200) * 1e-3,
+                         np.array([orc.e4m3_value(c) for c in range(0x7E)]) * 1.0625])
+    xs = xs.astype(np.float32)
+    got = np.array([orc.e4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+def check_e4m3_head_quantizer(orc):
+    """scale = amax / 448; the largest magnitude maps to +-448; every value is recovered
+    within half an E4M3 step; an all-zero head has scale 1 and zero codes."""
+    rng = _rng(31)
+    for _ in range(5):
+        x = (rng.standard_normal(128) * rng.uniform(0.1, 5)).astype(np.float32)
+        codes, scale = orc.quantize_head_e4m3(x)
+        assert scale == np.float32(np.max(np.abs(x))) / np.float32(448.0)
+        assert (codes[np.argmax(np.abs(x))] & 0x7F) == 0x7E
+        deq = np.array([orc.e4m3_value(int(c)) for c in codes]) * scale
+        y = np.abs(x.astype(np.float64) / scale)
+        step = np.where(y >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(y, 2.0 ** -6))) - 3),
+                        2.0 ** -9)
+        assert np.all(np.abs(deq - x) <= 0.5 * step * scale * (1 + 1e-6))
+    codes, scale = orc.quantize_head_e4m3(np.zeros(128, dtype=np.float32))
+    assert scale == 1.0 and np.all((codes & 0x7F) == 0)
+
+
+def check_fp8_step_matches_layout_step(orc):
+    """The FP8-cache step leaves q_out as the plain step does and stores, per (token,
+    head), the quantization of the plain step's K and V rows (rounded to fp32)."""
+    B, N, T, H, W, s, slot, C = 1, 2, 3, 4, 6, 3, 100, 144
+    tb, te = 5, 60
+    q, k, v, wq, wk = _step_inputs(32, B, te - tb, N)
+    for pairing in (0, 1):
+        for layout in (0, 1):
+            shape = (B, C, N, D) if layout == 0 else (B, N, C, D)
+            kf, vf = np.zeros(shape), np.zeros(shape)
+            q0 = orc.qk_norm_rope_append_layout(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kf, vf,
+                                                slot, pairing, layout)
+            kc = np.zeros(shape, dtype=np.uint8)
+            vc = np.zeros(shape, dtype=np.uint8)
+            ks = np.zeros(shape[:3], dtype=np.float32)
+            vs = np.zeros(shape[:3], dtype=np.float32)
+            q1 = orc.qk_norm_rope_append_fp8(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kc, vc,
+                                             ks, vs, slot, pairing, layout)
+            assert np.array_equal(q0, q1)
+            for r in (0, 20, te - tb - 1):
+                row = (slot + tb + r) % C
+                for n in range(N):
+                    idx = (0, row, n) if layout == 0 else (0, n, row)
+                    ek, esk = orc.quantize_head_e4m3(kf[idx])
+                    ev, esv = orc.quantize_head_e4m3(vf[idx])
+                    assert np.array_equal(kc[idx], ek) and ks[idx] == esk
+                    assert np.array_equal(vc[idx], ev) and vs[idx] == esv
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

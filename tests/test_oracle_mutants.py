@@ -60,6 +60,16 @@ MUTANTS = {
     "layout_step_row_ignores_slot": ("int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);",
                                      "int64_t row = rope3d_oracle_cache_row(i, 0, cache_tokens);",
                                      1),
+    # FP8 E4M3 quantizer
+    "e4m3_ties_to_odd": ("else best = (c % 2 == 0) ? c : c + 1;  /* tie: even mantissa */",
+                         "else best = (c % 2 == 0) ? c + 1 : c;"),
+    "e4m3_bias_8": ("else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                    "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 464.0) return sign | 0x7F;"),
+    "fp8_scale_240": ("float s = amax > 0.0f ? amax / 448.0f : 1.0f;",
+                      "float s = amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "fp8_v_scale_from_k": ("rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, v_scale + scale_off);",
+                           "rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, k_scale + scale_off);"),
 }
 
 
