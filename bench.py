@@ -65,6 +65,8 @@ def parse_args(argv=None):
                     help="pairing of a head's elements (half: rotate_half, as in M-RoPE)")
     ap.add_argument("--cache-layout", choices=["token", "head"], default="token",
                     help="KV cache [B][C][N][D] (token) or [B][N][C][D] (head)")
+    ap.add_argument("--cache-dtype", choices=["same", "fp8"], default="same",
+                    help="KV cache in the input dtype or FP8 E4M3 codes with per-head scales")
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
                          "fits in shared memory)")
@@ -272,6 +274,11 @@ def run_ours(args, dist: Dist):
     n = w.tokens_per_chunk
     tokens_per_step = w.B * n * len(w.chunks)
     bytes_per_launch = w.algorithmic_bytes(n)
+    if args.cache_dtype == "fp8":
+        # q, k, v read and q_out written in the input dtype; K and V cache rows one byte per
+        # element plus one fp32 scale per head each
+        e = w.elem_bytes
+        bytes_per_launch = w.B * n * (w.dim * (4 * e + 2) + 2 * 4 * w.N)
 
     host = make_inputs(w, seed_offset=dist.rank)
     wq, wk = wl.norm_weights(w.seed, w.dim)
@@ -290,8 +297,11 @@ def run_ours(args, dist: Dist):
     layout = rope3d.ROPE3D_CACHE_HEAD_MAJOR if args.cache_layout == "head" else rope3d.ROPE3D_CACHE_TOKEN_MAJOR
     cache_shape = ((w.B, w.cache_tokens, w.N, wl.HEAD_DIM) if args.cache_layout == "token"
                    else (w.B, w.N, w.cache_tokens, wl.HEAD_DIM))
-    k_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
-    v_cache = torch.zeros(cache_shape, dtype=tdt, device=device)
+    fp8 = args.cache_dtype == "fp8"
+    k_cache = torch.zeros(cache_shape, dtype=torch.uint8 if fp8 else tdt, device=device)
+    v_cache = torch.zeros(cache_shape, dtype=torch.uint8 if fp8 else tdt, device=device)
+    k_scale = torch.zeros(cache_shape[:3], dtype=torch.float32, device=device) if fp8 else None
+    v_scale = torch.zeros(cache_shape[:3], dtype=torch.float32, device=device) if fp8 else None
     max_t = max(c.frame_offset for c in w.chunks) + w.T
     tables = rope3d.rope3d_tables_init(max_t=max_t, max_h=w.H, max_w=w.W)
     stream = torch.cuda.current_stream(device)
@@ -307,7 +317,7 @@ def run_ours(args, dist: Dist):
             rope3d.rope3d_qk_norm_rope_append_ex(
                 q, k, v, q_out[ci], chunk.token_begin, chunk.token_end, chunk.frame_offset,
                 w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
-                pairing, layout, stream)
+                pairing, layout, k_scale, v_scale, stream)
             if events is not None:
                 events[2 * ci + 1].record(stream)
 
@@ -374,7 +384,8 @@ def run_ours(args, dist: Dist):
     if device_status != rope3d.ROPE3D_OK:
         raise RuntimeError("a kernel wait timed out during the benchmark")
     e2e = None
-    if not args.no_e2e and (args.pairing, args.cache_layout) != ("adjacent", "token"):
+    if not args.no_e2e and (args.pairing, args.cache_layout, args.cache_dtype) != (
+            "adjacent", "token", "same"):
         args.no_e2e = True  # the e2e leg runs the default layout only
     if not args.no_e2e:
         e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
@@ -429,6 +440,7 @@ def run_ours(args, dist: Dist):
             "kernel_path": args.path,
             "pairing": args.pairing,
             "cache_layout": args.cache_layout,
+            "cache_dtype": args.cache_dtype,
             "launch": "CUDA graph of one step, replayed" if (not args.eager)
             else "eager, one C-ABI call per chunk",
             "l2": "no flush: inputs larger than L2 (each launch streams "

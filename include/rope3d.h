@@ -95,12 +95,32 @@ extern "C" {
 #define ROPE3D_CACHE_TOKEN_MAJOR 0
 #define ROPE3D_CACHE_HEAD_MAJOR 1
 
+/* KV-cache element formats:
+ *   SAME     -- the caches have the dtype of q, k, v (default);
+ *   FP8_E4M3 -- quantize-on-append: each head of an appended K or V row is stored as
+ *               128 FP8 E4M3 codes (1 byte each; the OCP E4M3 format, max 448) with one
+ *               fp32 scale, scale = amax(|x|) / 448 over the head (1 if all zero);
+ *               code = E4M3(x * (448 / amax)) in fp32 (x * 1 for a zero head), rounded
+ *               to nearest even, saturating.  K is
+ *               quantized from its fp32 value after RMSNorm and RoPE.  A reader recovers
+ *               x ~ value(code) * scale.  Scales are laid out like the cache rows:
+ *               [B][cache_tokens][N] (token-major) or [B][N][cache_tokens] (head-major).
+ *               (The pages mention NVFP4 KV-cache quantization on Blackwell without a
+ *               format; E4M3 with per-head scales is this library's choice.) */
+#define ROPE3D_CACHE_SAME 0
+#define ROPE3D_CACHE_FP8_E4M3 1
+
 /* Options of the _ex entry points; a NULL pointer or a zeroed struct gives the defaults
- * (adjacent pairing, token-major cache), i.e. the plain entry points' behaviour. */
+ * (adjacent pairing, token-major cache of the input dtype), i.e. the plain entry points'
+ * behaviour. */
 typedef struct rope3d_options {
-    int pairing;       /* ROPE3D_PAIRING_*                                         */
-    int cache_layout;  /* ROPE3D_CACHE_* (fused step only; must be 0 for apply)     */
-    int reserved[6];   /* must be zero                                             */
+    int pairing;       /* ROPE3D_PAIRING_*                                          */
+    int cache_layout;  /* ROPE3D_CACHE_TOKEN_MAJOR / _HEAD_MAJOR (fused step only)   */
+    int cache_dtype;   /* ROPE3D_CACHE_SAME / _FP8_E4M3 (fused step only)            */
+    int reserved0;     /* must be zero                                              */
+    float* k_scale;    /* FP8 cache: device fp32 scales of K (NULL otherwise)        */
+    float* v_scale;    /* FP8 cache: device fp32 scales of V (NULL otherwise)        */
+    int reserved[4];   /* must be zero                                              */
 } rope3d_options;
 
 /* Opaque frequency configuration: split, theta, schedule, the fp32 inverse

@@ -476,8 +476,10 @@ int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t
  *
  * Quantize-on-append: K and V rows go to the cache as FP8 E4M3 codes with one fp32
  * scale per (token, head), scale = amax(|x|) / 448 over the head's D values (1 when the
- * head is all zero), code = E4M3(x / scale) rounded to nearest, ties to the even code,
- * saturating at +-448.  A reader recovers x ~ value(code) * scale.  The pages name
+ * head is all zero).  Codes are E4M3(x * inv) with inv = 448 / amax (1 for a zero
+ * head) -- one fp32 division per head, one multiply per element -- rounded to
+ * nearest, ties to the even code, saturating at +-448.  A reader recovers
+ * x ~ value(code) * scale.  The pages name
  * NVFP4 KV-cache quantization for Blackwell (the LongLive-2.0 abstract) but give no
  * format details; E4M3 with per-head scales is this build's reading.  The decision
  * runs in fp32 (the precision the kernel computes the rows in): the oracle rounds its
@@ -531,7 +533,8 @@ void rope3d_oracle_quantize_head_e4m3(const float* x, int64_t n, unsigned char* 
         if (a > amax) amax = a;
     }
     float s = amax > 0.0f ? amax / 448.0f : 1.0f;
-    for (int64_t e = 0; e < n; ++e) codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(x[e] / s);
+    float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+    for (int64_t e = 0; e < n; ++e) codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(x[e] * inv);
     *scale = s;
 }
 

@@ -181,75 +181,94 @@ Geometry geometry(int64_t N, int dtype, int pairing) {
 
 using KernelFn = void (*)(const rope3d::Params);
 
-template <typename T, int TRIG, int MODE, int PAIR>
+// Kernel instantiation for the launch's element type, trig mode, pairing, cache format
+// and vectors per thread.  Pairing rotate_half uses even VPT only (slots come in twos);
+// the rotation-only mode writes no cache.
+
+template <typename T, int TRIG, int MODE, int PAIR, bool CFP8>
 KernelFn pick_vpt(int vpt) {
-    if constexpr (PAIR == rope3d::kPairHalf) {  // slots come in twos
+    if constexpr (PAIR == rope3d::kPairHalf) {
         switch (vpt) {
-            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR>;
-            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR>;
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CFP8>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CFP8>;
             default: return nullptr;
         }
     } else {
         switch (vpt) {
-            case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE, PAIR>;
-            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR>;
-            case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR>;
-            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR>;
+            case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE, PAIR, CFP8>;
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CFP8>;
+            case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR, CFP8>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CFP8>;
             default: return nullptr;
         }
     }
 }
 
-template <typename T, int MODE, int PAIR>
+template <typename T, int MODE, int PAIR, bool CFP8>
 KernelFn pick_trig(int trig, int vpt) {
-    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<T, rope3d::kTrigTable, MODE, PAIR>(vpt)
-                                     : pick_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR>(vpt);
+    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<T, rope3d::kTrigTable, MODE, PAIR, CFP8>(vpt)
+                                     : pick_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR, CFP8>(vpt);
+}
+
+template <typename T, int MODE, bool CFP8>
+KernelFn pick_pairing(int pairing, int trig, int vpt) {
+    return pairing == ROPE3D_PAIRING_HALF ? pick_trig<T, MODE, rope3d::kPairHalf, CFP8>(trig, vpt)
+                                          : pick_trig<T, MODE, rope3d::kPairAdjacent, CFP8>(trig, vpt);
 }
 
 template <int MODE>
-KernelFn pick_kernel(int dtype, int trig, int pairing, int vpt) {
-    if (dtype == ROPE3D_BF16)
-        return pairing == ROPE3D_PAIRING_HALF
-                   ? pick_trig<__nv_bfloat16, MODE, rope3d::kPairHalf>(trig, vpt)
-                   : pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent>(trig, vpt);
-    return pairing == ROPE3D_PAIRING_HALF ? pick_trig<float, MODE, rope3d::kPairHalf>(trig, vpt)
-                                          : pick_trig<float, MODE, rope3d::kPairAdjacent>(trig, vpt);
+KernelFn pick_kernel(int dtype, int trig, int pairing, bool fp8, int vpt) {
+    if constexpr (MODE == rope3d::kModeApply) {
+        return dtype == ROPE3D_BF16 ? pick_pairing<__nv_bfloat16, MODE, false>(pairing, trig, vpt)
+                                    : pick_pairing<float, MODE, false>(pairing, trig, vpt);
+    } else {
+        if (dtype == ROPE3D_BF16)
+            return fp8 ? pick_pairing<__nv_bfloat16, MODE, true>(pairing, trig, vpt)
+                       : pick_pairing<__nv_bfloat16, MODE, false>(pairing, trig, vpt);
+        return fp8 ? pick_pairing<float, MODE, true>(pairing, trig, vpt)
+                   : pick_pairing<float, MODE, false>(pairing, trig, vpt);
+    }
 }
 
 using TmaKernelFn = void (*)(const rope3d::Params);
 
-template <typename T, int TRIG, int PAIR>
+template <typename T, int TRIG, int PAIR, bool CFP8>
 TmaKernelFn pick_tma_vpt(int vpt) {
     if constexpr (PAIR == rope3d::kPairHalf) {
         switch (vpt) {
-            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR>;
-            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR>;
+            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR, CFP8>;
+            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR, CFP8>;
             default: return nullptr;
         }
     } else {
         switch (vpt) {
-            case 1: return rope3d::qk_norm_rope_tma_kernel<T, 1, TRIG, PAIR>;
-            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR>;
-            case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG, PAIR>;
-            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR>;
+            case 1: return rope3d::qk_norm_rope_tma_kernel<T, 1, TRIG, PAIR, CFP8>;
+            case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR, CFP8>;
+            case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG, PAIR, CFP8>;
+            case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR, CFP8>;
             default: return nullptr;
         }
     }
 }
 
-template <typename T, int PAIR>
+template <typename T, int PAIR, bool CFP8>
 TmaKernelFn pick_tma_trig(int trig, int vpt) {
-    return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<T, rope3d::kTrigTable, PAIR>(vpt)
-                                     : pick_tma_vpt<T, rope3d::kTrigOnTheFly, PAIR>(vpt);
+    return trig == ROPE3D_TRIG_TABLE ? pick_tma_vpt<T, rope3d::kTrigTable, PAIR, CFP8>(vpt)
+                                     : pick_tma_vpt<T, rope3d::kTrigOnTheFly, PAIR, CFP8>(vpt);
 }
 
-TmaKernelFn pick_tma_kernel(int dtype, int trig, int pairing, int vpt) {
+template <typename T, bool CFP8>
+TmaKernelFn pick_tma_pairing(int pairing, int trig, int vpt) {
+    return pairing == ROPE3D_PAIRING_HALF ? pick_tma_trig<T, rope3d::kPairHalf, CFP8>(trig, vpt)
+                                          : pick_tma_trig<T, rope3d::kPairAdjacent, CFP8>(trig, vpt);
+}
+
+TmaKernelFn pick_tma_kernel(int dtype, int trig, int pairing, bool fp8, int vpt) {
     if (dtype == ROPE3D_BF16)
-        return pairing == ROPE3D_PAIRING_HALF
-                   ? pick_tma_trig<__nv_bfloat16, rope3d::kPairHalf>(trig, vpt)
-                   : pick_tma_trig<__nv_bfloat16, rope3d::kPairAdjacent>(trig, vpt);
-    return pairing == ROPE3D_PAIRING_HALF ? pick_tma_trig<float, rope3d::kPairHalf>(trig, vpt)
-                                          : pick_tma_trig<float, rope3d::kPairAdjacent>(trig, vpt);
+        return fp8 ? pick_tma_pairing<__nv_bfloat16, true>(pairing, trig, vpt)
+                   : pick_tma_pairing<__nv_bfloat16, false>(pairing, trig, vpt);
+    return fp8 ? pick_tma_pairing<float, true>(pairing, trig, vpt)
+               : pick_tma_pairing<float, false>(pairing, trig, vpt);
 }
 
 // Resident blocks per SM for a kernel at a block size and shared-memory size.  The
@@ -379,7 +398,7 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pair
                     p.units < (int64_t)16 * info.sms * teams))
         return ROPE3D_OK;
     smem = tma_layout(p, teams, stages, warps_per_team);
-    TmaKernelFn fn = pick_tma_kernel(dtype, trig, pairing, g.vpt);
+    TmaKernelFn fn = pick_tma_kernel(dtype, trig, pairing, p.k_scale != nullptr, g.vpt);
     if (fn == nullptr) return ROPE3D_OK;
     const int threads = teams * g.tpr;
     int per_sm = 0;
@@ -423,7 +442,7 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int d
     if (smem > (size_t)info.max_smem_optin)
         return fail(ROPE3D_EINVAL, "N=%lld needs %zu bytes of shared memory (limit %d)",
                     (long long)N, smem, info.max_smem_optin);
-    KernelFn fn = pick_kernel<MODE>(dtype, trig, pairing, g.vpt);
+    KernelFn fn = pick_kernel<MODE>(dtype, trig, pairing, p.k_scale != nullptr, g.vpt);
     if (fn == nullptr) return fail(ROPE3D_EINVAL, "no kernel for vpt=%d", g.vpt);
     int per_sm = 0;
     int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
@@ -481,6 +500,20 @@ int read_options(const rope3d_options* options, rope3d_options* out, bool with_c
                     o.cache_layout);
     if (!with_cache && o.cache_layout != ROPE3D_CACHE_TOKEN_MAJOR)
         return fail(ROPE3D_EINVAL, "options.cache_layout applies to the fused step only");
+    if (o.cache_dtype != ROPE3D_CACHE_SAME && o.cache_dtype != ROPE3D_CACHE_FP8_E4M3)
+        return fail(ROPE3D_EINVAL, "options.cache_dtype %d is not a ROPE3D_CACHE_* value",
+                    o.cache_dtype);
+    if (!with_cache && (o.cache_dtype != ROPE3D_CACHE_SAME || o.k_scale || o.v_scale))
+        return fail(ROPE3D_EINVAL, "options.cache_dtype and scales apply to the fused step only");
+    if (o.cache_dtype == ROPE3D_CACHE_FP8_E4M3) {
+        if (o.k_scale == nullptr || o.v_scale == nullptr)
+            return fail(ROPE3D_EINVAL, "an FP8 cache needs k_scale and v_scale");
+        if ((reinterpret_cast<uintptr_t>(o.k_scale) & 3u) || (reinterpret_cast<uintptr_t>(o.v_scale) & 3u))
+            return fail(ROPE3D_EALIGN, "k_scale and v_scale must be 4-byte aligned");
+    } else if (o.k_scale != nullptr || o.v_scale != nullptr) {
+        return fail(ROPE3D_EINVAL, "k_scale / v_scale are only for an FP8 cache");
+    }
+    if (o.reserved0 != 0) return fail(ROPE3D_EINVAL, "options.reserved0 must be zero");
     for (int r : o.reserved)
         if (r != 0) return fail(ROPE3D_EINVAL, "options.reserved must be zero");
     *out = o;
@@ -492,6 +525,8 @@ void fill_layout(rope3d::Params& p, int64_t N, int dtype, const rope3d_options& 
     p.cache_head_major = o.cache_layout == ROPE3D_CACHE_HEAD_MAJOR ? 1 : 0;
     p.n_heads = (int)N;
     p.vph_log2 = vph == 16 ? 4 : 5;
+    p.k_scale = o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 ? o.k_scale : nullptr;
+    p.v_scale = o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 ? o.v_scale : nullptr;
 }
 
 int check_tables_device(const rope3d_tables* tables, int dev) {
@@ -724,7 +759,19 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
     const size_t esz = dtype == ROPE3D_BF16 ? 2 : 4;
     const size_t row = (size_t)N * D * esz;
     const size_t act = (size_t)B * (size_t)(token_end - token_begin) * row;
-    const size_t cache = (size_t)B * (size_t)cache_tokens * row;
+    const bool fp8 = opt.cache_dtype == ROPE3D_CACHE_FP8_E4M3;
+    const size_t cache = (size_t)B * (size_t)cache_tokens * (size_t)N * D * (fp8 ? 1 : esz);
+    if (fp8) {
+        const size_t sc = (size_t)B * (size_t)cache_tokens * (size_t)N * sizeof(float);
+        const void* bufs[6] = {q, k, v, q_out, k_cache, v_cache};
+        const size_t sizes[6] = {act, act, act, act, cache, cache};
+        for (int b2 = 0; b2 < 6; ++b2)
+            if (overlap(opt.k_scale, sc, bufs[b2], sizes[b2]) ||
+                overlap(opt.v_scale, sc, bufs[b2], sizes[b2]))
+                return fail(ROPE3D_EOVERLAP, "a scale array overlaps a tensor");
+        if (overlap(opt.k_scale, sc, opt.v_scale, sc))
+            return fail(ROPE3D_EOVERLAP, "k_scale overlaps v_scale");
+    }
     if (q_out != q && overlap(q_out, act, q, act))
         return fail(ROPE3D_EOVERLAP, "q_out partly overlaps q (only exact in-place is allowed)");
     if (overlap(q_out, act, k, act) || overlap(q_out, act, v, act) ||

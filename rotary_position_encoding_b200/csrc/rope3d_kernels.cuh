@@ -28,6 +28,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -85,6 +86,8 @@ struct Params {
     int cache_head_major;  // caches are [B][N][cache_tokens][D] instead of [B][cache_tokens][N][D]
     int n_heads;           // N
     int vph_log2;          // log2 of the 16-byte vectors per head
+    float* k_scale;        // FP8 caches: per (token, head) scales, laid out like the cache rows
+    float* v_scale;
     float inv_freq[kPairs];  // fp32 angle per unit position of every pair
 };
 
@@ -255,6 +258,13 @@ __device__ __forceinline__ int64_t cache_vec_index(const Params& p, const RowPos
     return (((pos.b * p.n_heads + n) * p.cache_tokens + pos.crow) << p.vph_log2) + v;
 }
 
+// Index of the scale of head n of a row's K/V in an FP8 cache's scale array:
+// [B][C][N] (token-major) or [B][N][C] (head-major).
+__device__ __forceinline__ int64_t cache_scale_index(const Params& p, const RowPos& pos, int n) {
+    return p.cache_head_major ? (pos.b * p.n_heads + n) * p.cache_tokens + pos.crow
+                              : (pos.b * p.cache_tokens + pos.crow) * p.n_heads + n;
+}
+
 // The complex pairs a thread rotates (fixed for the thread's whole life).
 template <int PPV>
 struct PairInfo {
@@ -353,11 +363,12 @@ __device__ __forceinline__ float2 team_sum(float sq, float sk, float2* s_part, i
 }
 
 // y = x * rs * w (RMSNorm), then (y_re + i y_im) * (cos + i sin) (RoPE), for the
-// pairs of one vector; weights come from shared memory.
+// pairs of one vector, as fp32 in element order; weights come from shared memory.
 template <typename T, bool NORM>
-__device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
+__device__ __forceinline__ void norm_rotate_f(
     const typename VecTraits<T>::Vec& x, float rs, const float* s_w, int e0,
-    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec]) {
+    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec],
+    float (&out)[VecTraits<T>::kElems]) {
     using Tr = VecTraits<T>;
     constexpr int PPV = Tr::kPairsPerVec;
     float w[2 * PPV];
@@ -368,7 +379,6 @@ __device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
             w[4 * c] = a.x; w[4 * c + 1] = a.y; w[4 * c + 2] = a.z; w[4 * c + 3] = a.w;
         }
     }
-    typename Tr::Vec out;
 #pragma unroll
     for (int m = 0; m < PPV; ++m) {
         float a, c;
@@ -377,21 +387,31 @@ __device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
             a = a * rs * w[2 * m];
             c = c * rs * w[2 * m + 1];
         }
-        Tr::set_pair(out, m, a * cs[m] - c * sn[m], a * sn[m] + c * cs[m]);
+        out[2 * m] = a * cs[m] - c * sn[m];
+        out[2 * m + 1] = a * sn[m] + c * cs[m];
     }
-    return out;
+}
+
+// The same, rounded once to the element type.
+template <typename T, bool NORM>
+__device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
+    const typename VecTraits<T>::Vec& x, float rs, const float* s_w, int e0,
+    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec]) {
+    float out[VecTraits<T>::kElems];
+    norm_rotate_f<T, NORM>(x, rs, s_w, e0, cs, sn, out);
+    return VecTraits<T>::pack_elems(out);
 }
 
 // rotate_half pairing: `re_v` is a head's first-half vector at some position and
 // `im_v` its second-half vector at the same position -- the real and imaginary parts of
 // kElems pairs.  Both are normalised with their own weights, y = x * rs * w, and
-// (y_re + i y_im) * (cos + i sin) is returned as the two vectors of the result.
+// (y_re + i y_im) * (cos + i sin) is returned as fp32 in the two vectors' element order.
 template <typename T, bool NORM>
-__device__ __forceinline__ void norm_rotate_half(
+__device__ __forceinline__ void norm_rotate_half_f(
     const typename VecTraits<T>::Vec& re_v, const typename VecTraits<T>::Vec& im_v, float rs,
     const float* s_w, int e_re, int e_im,
     const float (&cs)[VecTraits<T>::kElems], const float (&sn)[VecTraits<T>::kElems],
-    typename VecTraits<T>::Vec& out_re, typename VecTraits<T>::Vec& out_im) {
+    float (&o_re)[VecTraits<T>::kElems], float (&o_im)[VecTraits<T>::kElems]) {
     using Tr = VecTraits<T>;
     constexpr int E = Tr::kElems;
     float wr[E], wi[E];
@@ -404,7 +424,6 @@ __device__ __forceinline__ void norm_rotate_half(
             wi[4 * c] = b.x; wi[4 * c + 1] = b.y; wi[4 * c + 2] = b.z; wi[4 * c + 3] = b.w;
         }
     }
-    float o_re[E], o_im[E];
 #pragma unroll
     for (int m = 0; m < E; ++m) {
         float a = Tr::elem(re_v, m);
@@ -416,8 +435,60 @@ __device__ __forceinline__ void norm_rotate_half(
         o_re[m] = a * cs[m] - c * sn[m];
         o_im[m] = a * sn[m] + c * cs[m];
     }
-    out_re = Tr::pack_elems(o_re);
-    out_im = Tr::pack_elems(o_im);
+}
+
+// ---------------------------------------------------------------- FP8 E4M3 cache rows
+//
+// Quantize-on-append: a head's K or V row goes to the cache as E4M3 codes with one fp32
+// scale, scale = amax / 448 (1 for an all-zero head); codes are E4M3(x * inv) with
+// inv = 448 / amax (1 for a zero head), rounded to nearest even with saturation -- one
+// division per head, one multiply per element.  The lanes holding a head (at one slot)
+// find its amax with a butterfly max; the head's first lane writes the scale.
+
+__device__ __forceinline__ float group_max(float x, int lanes) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        if (off < lanes) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+    return x;
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    // element a in the low byte (lower address)
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+struct Fp8Scale {
+    float scale;  // stored for the reader: x ~ value(code) * scale
+    float inv;    // codes are E4M3(x * inv)
+};
+
+__device__ __forceinline__ Fp8Scale fp8_scale(float amax) {
+    Fp8Scale s;
+    s.scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    s.inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+    return s;
+}
+
+// Store E codes of one vector at vector index vi of an FP8 cache (E bytes per vector).
+__device__ __forceinline__ void store_fp8(void* cache, int64_t vi, const float (&v)[8],
+                                          float inv) {
+    uint2 c;
+    c.x = e4m3x2(v[0] * inv, v[1] * inv) | (e4m3x2(v[2] * inv, v[3] * inv) << 16);
+    c.y = e4m3x2(v[4] * inv, v[5] * inv) | (e4m3x2(v[6] * inv, v[7] * inv) << 16);
+    __stcs(reinterpret_cast<uint2*>(cache) + vi, c);
+}
+__device__ __forceinline__ void store_fp8(void* cache, int64_t vi, const float (&v)[4],
+                                          float inv) {
+    const uint32_t c = e4m3x2(v[0] * inv, v[1] * inv) | (e4m3x2(v[2] * inv, v[3] * inv) << 16);
+    __stcs(reinterpret_cast<unsigned int*>(cache) + vi, c);
+}
+
+template <int E>
+__device__ __forceinline__ float abs_max(const float (&v)[E]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(v[e]));
+    return m;
 }
 
 __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, float* s_wk) {
@@ -435,9 +506,11 @@ __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, floa
 // ---------------------------------------------------------------- per-row output
 
 // Normalise, rotate and store this thread's vectors of one row: q_out, and in the fused
-// mode the K row into the cache (V is stored by the caller).  With rotate_half pairing
-// slots 2m and 2m+1 hold the two halves of the same pairs (see slot_vec).
-template <typename T, int VPT, int PAIR, int MODE>
+// mode the K row into the cache (V is stored by store_v_row).  With rotate_half pairing
+// slots 2m and 2m+1 hold the two halves of the same pairs (see slot_vec).  With an FP8
+// cache (CFP8) the K values stay fp32 until they are quantized; every lane of the warp
+// takes part in the head-wise maximum, whether its slot holds a vector or not.
+template <typename T, int VPT, int PAIR, int MODE, bool CFP8>
 __device__ __forceinline__ void emit_row(
     const Params& p, int t, const RowPos& pos, int64_t row_vec,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -448,16 +521,29 @@ __device__ __forceinline__ void emit_row(
     using Vec = typename Tr::Vec;
     constexpr int EPV = Tr::kElems;
     constexpr bool NORM = MODE == kModeFused;
+    constexpr int VPH = Tr::kVecsPerHead;
     if constexpr (PAIR == kPairAdjacent) {
 #pragma unroll
         for (int s = 0; s < VPT; ++s) {
             const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
-            if (idx < p.dim_vecs) {
-                const int e0 = idx * EPV;
+            const bool valid = idx < p.dim_vecs;
+            const int e0 = idx * EPV;
+            if (valid)
                 store_out(qo + row_vec + idx, norm_rotate<T, NORM>(xq[s], rq, s_wq, e0, cs, sn));
-                if (MODE == kModeFused)
+            if constexpr (MODE == kModeFused) {
+                if constexpr (CFP8) {
+                    float o[EPV];
+                    if (valid) norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
+                    const Fp8Scale sc = fp8_scale(group_max(valid ? abs_max<EPV>(o) : 0.0f, VPH));
+                    if (valid) {
+                        store_fp8(kc, cache_vec_index(p, pos, idx), o, sc.inv);
+                        if ((idx & (VPH - 1)) == 0)
+                            __stcs(p.k_scale + cache_scale_index(p, pos, idx / VPH), sc.scale);
+                    }
+                } else if (valid) {
                     store_out(kc + cache_vec_index(p, pos, idx),
                               norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
+                }
             }
         }
     } else {
@@ -466,18 +552,74 @@ __device__ __forceinline__ void emit_row(
         for (int s = 0; s < VPT; s += 2) {
             const int i_re = slot_vec<T, PAIR>(t, s, p.tpr);
             const int i_im = slot_vec<T, PAIR>(t, s + 1, p.tpr);
-            if (i_re < p.dim_vecs) {
-                Vec o_re, o_im;
-                norm_rotate_half<T, NORM>(xq[s], xq[s + 1], rq, s_wq, i_re * EPV, i_im * EPV, cs,
-                                          sn, o_re, o_im);
-                store_out(qo + row_vec + i_re, o_re);
-                store_out(qo + row_vec + i_im, o_im);
-                if (MODE == kModeFused) {
-                    norm_rotate_half<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV, i_im * EPV,
-                                              cs, sn, o_re, o_im);
-                    store_out(kc + cache_vec_index(p, pos, i_re), o_re);
-                    store_out(kc + cache_vec_index(p, pos, i_im), o_im);
+            const bool valid = i_re < p.dim_vecs;
+            float o_re[EPV], o_im[EPV];
+            if (valid) {
+                norm_rotate_half_f<T, NORM>(xq[s], xq[s + 1], rq, s_wq, i_re * EPV, i_im * EPV,
+                                            cs, sn, o_re, o_im);
+                store_out(qo + row_vec + i_re, Tr::pack_elems(o_re));
+                store_out(qo + row_vec + i_im, Tr::pack_elems(o_im));
+            }
+            if constexpr (MODE == kModeFused) {
+                if (valid)
+                    norm_rotate_half_f<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV,
+                                                i_im * EPV, cs, sn, o_re, o_im);
+                if constexpr (CFP8) {
+                    const float local = valid ? fmaxf(abs_max<EPV>(o_re), abs_max<EPV>(o_im)) : 0.0f;
+                    const Fp8Scale sc = fp8_scale(group_max(local, VPH / 2));
+                    if (valid) {
+                        store_fp8(kc, cache_vec_index(p, pos, i_re), o_re, sc.inv);
+                        store_fp8(kc, cache_vec_index(p, pos, i_im), o_im, sc.inv);
+                        if ((i_re & (VPH - 1)) == 0)
+                            __stcs(p.k_scale + cache_scale_index(p, pos, i_re / VPH), sc.scale);
+                    }
+                } else if (valid) {
+                    store_out(kc + cache_vec_index(p, pos, i_re), Tr::pack_elems(o_re));
+                    store_out(kc + cache_vec_index(p, pos, i_im), Tr::pack_elems(o_im));
                 }
+            }
+        }
+    }
+}
+
+// Store this thread's vectors of one row of V to the cache: a bit copy, or FP8 codes
+// with a per-head scale (every lane of the warp takes part in the head-wise maximum).
+template <typename T, int VPT, int PAIR, bool CFP8>
+__device__ __forceinline__ void store_v_row(const Params& p, int t, const RowPos& pos,
+                                            const typename VecTraits<T>::Vec (&xv)[VPT],
+                                            typename VecTraits<T>::Vec* vc) {
+    using Tr = VecTraits<T>;
+    constexpr int EPV = Tr::kElems;
+    constexpr int VPH = Tr::kVecsPerHead;
+    if constexpr (!CFP8) {
+#pragma unroll
+        for (int s = 0; s < VPT; ++s) {
+            const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+            if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[s]);
+        }
+    } else {
+        constexpr int STEP = PAIR == kPairAdjacent ? 1 : 2;  // slots that share one head
+        constexpr int LANES = PAIR == kPairAdjacent ? VPH : VPH / 2;
+#pragma unroll
+        for (int s = 0; s < VPT; s += STEP) {
+            const int idx0 = slot_vec<T, PAIR>(t, s, p.tpr);
+            const bool valid = idx0 < p.dim_vecs;
+            float v[STEP][EPV];
+            float local = 0.0f;
+#pragma unroll
+            for (int j = 0; j < STEP; ++j) {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) v[j][e] = valid ? Tr::elem(xv[s + j], e) : 0.0f;
+                local = fmaxf(local, abs_max<EPV>(v[j]));
+            }
+            const Fp8Scale sc = fp8_scale(group_max(local, LANES));
+            if (valid) {
+#pragma unroll
+                for (int j = 0; j < STEP; ++j)
+                    store_fp8(vc, cache_vec_index(p, pos, slot_vec<T, PAIR>(t, s + j, p.tpr)),
+                              v[j], sc.inv);
+                if ((idx0 & (VPH - 1)) == 0)
+                    __stcs(p.v_scale + cache_scale_index(p, pos, idx0 / VPH), sc.scale);
             }
         }
     }
@@ -485,7 +627,7 @@ __device__ __forceinline__ void emit_row(
 
 // ---------------------------------------------------------------- register kernel
 
-template <typename T, int VPT, int TRIG, int MODE, int PAIR>
+template <typename T, int VPT, int TRIG, int MODE, int PAIR, bool CFP8>
 __global__ void __launch_bounds__(kMaxBlockThreads)
 qk_norm_rope_kernel(const Params p) {
     using Tr = VecTraits<T>;
@@ -541,11 +683,7 @@ qk_norm_rope_kernel(const Params p) {
 
         float rq = 1.0f, rk = 1.0f;
         if (MODE == kModeFused) {
-#pragma unroll
-            for (int s = 0; s < VPT; ++s) {
-                const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
-                if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[s]);
-            }
+            store_v_row<T, VPT, PAIR, CFP8>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -553,8 +691,8 @@ qk_norm_rope_kernel(const Params p) {
             rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
-        emit_row<T, VPT, PAIR, MODE>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs, sn, qo,
-                                     kc);
+        emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs, sn,
+                                           qo, kc);
     }
 }
 

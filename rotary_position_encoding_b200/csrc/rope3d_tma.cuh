@@ -76,7 +76,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-template <typename T, int VPT, int TRIG, int PAIR>
+template <typename T, int VPT, int TRIG, int PAIR, bool CFP8>
 __global__ void __launch_bounds__(kTmaMaxBlockThreads, 1)
 qk_norm_rope_tma_kernel(const Params p) {
     using Tr = VecTraits<T>;
@@ -188,13 +188,9 @@ qk_norm_rope_tma_kernel(const Params p) {
         const float rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
         const float rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         const int64_t row_vec = u * p.dim_vecs;
-#pragma unroll
-        for (int j = 0; j < VPT; ++j) {
-            const int idx = slot_vec<T, PAIR>(t, j, p.tpr);
-            if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[j]);
-        }
-        emit_row<T, VPT, PAIR, kModeFused>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs,
-                                           sn, qo, kc);
+        store_v_row<T, VPT, PAIR, CFP8>(p, t, pos, xv, vc);
+        emit_row<T, VPT, PAIR, kModeFused, CFP8>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk,
+                                                 cs, sn, qo, kc);
     }
 
     if (failed && t == 0) {

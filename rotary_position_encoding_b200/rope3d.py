@@ -38,12 +38,16 @@ ROPE3D_PAIRING_ADJACENT = 0
 ROPE3D_PAIRING_HALF = 1
 ROPE3D_CACHE_TOKEN_MAJOR = 0
 ROPE3D_CACHE_HEAD_MAJOR = 1
+ROPE3D_CACHE_SAME = 0
+ROPE3D_CACHE_FP8_E4M3 = 1
 
 
 class rope3d_options(ctypes.Structure):
     """struct rope3d_options of include/rope3d.h."""
     _fields_ = [("pairing", ctypes.c_int), ("cache_layout", ctypes.c_int),
-                ("reserved", ctypes.c_int * 6)]
+                ("cache_dtype", ctypes.c_int), ("reserved0", ctypes.c_int),
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+                ("reserved", ctypes.c_int * 4)]
 
 # include/rope3d_testing.h
 ROPE3D_PATH_AUTO = 0
@@ -232,8 +236,10 @@ def rope3d_qk_norm_rope_append_ex(q, k, v, q_out, token_begin: int, token_end: i
                                   trig: int = ROPE3D_TRIG_TABLE,
                                   pairing: int = ROPE3D_PAIRING_ADJACENT,
                                   cache_layout: int = ROPE3D_CACHE_TOKEN_MAJOR,
-                                  stream=None) -> None:
-    """rope3d_qk_norm_rope_append with options; head-major caches are [B, N, C, 128]."""
+                                  k_scale=None, v_scale=None, stream=None) -> None:
+    """rope3d_qk_norm_rope_append with options; head-major caches are [B, N, C, 128].
+    Passing k_scale and v_scale (float32, [B, C, N] or [B, N, C]) selects the FP8 E4M3
+    cache: k_cache and v_cache are then uint8 code tensors."""
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or q_out.shape != q.shape:
         raise ValueError("q, k, v and q_out must all be [B, n_tok, N, D]")
     B, n_tok, N, D = q.shape
@@ -249,11 +255,22 @@ def rope3d_qk_norm_rope_append_ex(q, k, v, q_out, token_begin: int, token_end: i
         raise ValueError("cache shape does not match q and the cache layout")
     if n_tok != token_end - token_begin:
         raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
-    for name, t in (("k", k), ("v", v), ("q_out", q_out), ("k_cache", k_cache),
-                    ("v_cache", v_cache)):
+    fp8 = k_scale is not None or v_scale is not None
+    for name, t in (("k", k), ("v", v), ("q_out", q_out)) + (
+            () if fp8 else (("k_cache", k_cache), ("v_cache", v_cache))):
         if t.dtype != q.dtype:
             raise TypeError(f"{name} must have q's dtype {q.dtype}")
     opts = rope3d_options(pairing, cache_layout)
+    if fp8:
+        if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
+            raise TypeError("an FP8 cache is uint8 codes")
+        sshape = (B, C, N) if cache_layout == ROPE3D_CACHE_TOKEN_MAJOR else (B, N, C)
+        for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+            if t is None or t.dtype != torch.float32 or tuple(t.shape) != sshape:
+                raise ValueError(f"{name} must be float32 of shape {sshape}")
+        opts.cache_dtype = ROPE3D_CACHE_FP8_E4M3
+        opts.k_scale = _dev_ptr(k_scale, "k_scale")
+        opts.v_scale = _dev_ptr(v_scale, "v_scale")
     _check(load_library().rope3d_qk_norm_rope_append_ex(
         _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
         B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,

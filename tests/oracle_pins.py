@@ -565,19 +565,23 @@ def check_e4m3_encode_matches_torch(orc):
 
 
 def check_e4m3_head_quantizer(orc):
-    """scale = amax / 448; the largest magnitude maps to +-448; every value is recovered
-    within half an E4M3 step; an all-zero head has scale 1 and zero codes."""
+    """scale = amax / 448; codes are E4M3(x * (448 / amax)) in fp32; the largest magnitude
+    maps to +-448; every value is recovered within half an E4M3 step (plus the fp32
+    rounding of the multiply); an all-zero head has scale 1 and zero codes."""
     rng = _rng(31)
     for _ in range(5):
         x = (rng.standard_normal(128) * rng.uniform(0.1, 5)).astype(np.float32)
         codes, scale = orc.quantize_head_e4m3(x)
-        assert scale == np.float32(np.max(np.abs(x))) / np.float32(448.0)
+        amax = np.float32(np.max(np.abs(x)))
+        assert scale == amax / np.float32(448.0)
+        inv = np.float32(448.0) / amax
+        assert np.array_equal(codes, [orc.e4m3_encode(float(np.float32(v) * inv)) for v in x])
         assert (codes[np.argmax(np.abs(x))] & 0x7F) == 0x7E
         deq = np.array([orc.e4m3_value(int(c)) for c in codes]) * scale
         y = np.abs(x.astype(np.float64) / scale)
         step = np.where(y >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(y, 2.0 ** -6))) - 3),
                         2.0 ** -9)
-        assert np.all(np.abs(deq - x) <= 0.5 * step * scale * (1 + 1e-6))
+        assert np.all(np.abs(deq - x) <= (0.5 * step + 1e-6 * y) * scale * (1 + 1e-6))
     codes, scale = orc.quantize_head_e4m3(np.zeros(128, dtype=np.float32))
     assert scale == 1.0 and np.all((codes & 0x7F) == 0)
 

@@ -190,8 +190,11 @@ def test_invalid_options_rejected():
     kc = torch.zeros((1, 144, 2, D), device="cuda")
     wq = torch.ones(256, device="cuda")
     tables = rope3d.rope3d_tables_init(max_t=6, max_h=4, max_w=6)
+    reserved_set = rope3d.rope3d_options()
+    reserved_set.reserved[2] = 1
     for opts in (rope3d.rope3d_options(2, 0), rope3d.rope3d_options(0, 5),
-                 rope3d.rope3d_options(0, 0, (ctypes.c_int * 6)(0, 0, 1, 0, 0, 0))):
+                 rope3d.rope3d_options(0, 0, 7), rope3d.rope3d_options(0, 0, 0, 1),
+                 reserved_set):
         rc = lib.rope3d_qk_norm_rope_append_ex(
             dev[0].data_ptr(), dev[1].data_ptr(), dev[2].data_ptr(), qo.data_ptr(), 1, 2, D,
             rope3d.ROPE3D_F32, 0, 72, 0, 3, 4, 6, wq.data_ptr(), wq.data_ptr(), 1e-6,
