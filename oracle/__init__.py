@@ -86,6 +86,7 @@ def _declare(lib):
                                          _I64, _I64, _INT, _INT, _INT, _DBL, _INT, _INT], _INT),
         "rope3d_oracle_e4m3_value": ([_INT], _DBL),
         "rope3d_oracle_e4m3_encode": ([ctypes.c_float], _INT),
+        "rope3d_oracle_e4m3_scale_exponent": ([ctypes.c_float], _INT),
         "rope3d_oracle_quantize_head_e4m3": ([_F, _I64, _U8, _F], None),
         "rope3d_oracle_qk_norm_rope_append_fp8": ([_D, _D, _D, _D, _I64, _I64, _I64, _I64, _I64,
                                                    _I64, _I64, _I64, _I64, _D, _D, _DBL, _U8,
@@ -232,6 +233,9 @@ class Oracle:
 
     def e4m3_encode(self, x: float) -> int:
         return self.lib.rope3d_oracle_e4m3_encode(x)
+
+    def e4m3_scale_exponent(self, amax: float) -> int:
+        return self.lib.rope3d_oracle_e4m3_scale_exponent(amax)
 
     def quantize_head_e4m3(self, x):
         x = np.ascontiguousarray(x, dtype=np.float32).ravel()

@@ -475,9 +475,10 @@ int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t
 /* ------------------------------------------------------------------ FP8 KV cache
  *
  * Quantize-on-append: K and V rows go to the cache as FP8 E4M3 codes with one fp32
- * scale per (token, head), scale = amax(|x|) / 448 over the head's D values (1 when the
- * head is all zero).  Codes are E4M3(x * inv) with inv = 448 / amax (1 for a zero
- * head) -- one fp32 division per head, one multiply per element -- rounded to
+ * scale per (token, head).  The scale is a power of two, as in the OCP microscaling
+ * formats: the smallest 2^e (e >= -126) with amax(|x|) / 2^e <= 448 over the head's D
+ * values (1 when the head is all zero), so the head's largest value lands in
+ * (224, 448] and dividing by the scale is exact.  Codes are E4M3(x / scale) rounded to
  * nearest, ties to the even code, saturating at +-448.  A reader recovers
  * x ~ value(code) * scale.  The pages name
  * NVFP4 KV-cache quantization for Blackwell (the LongLive-2.0 abstract) but give no
@@ -523,6 +524,15 @@ int rope3d_oracle_e4m3_encode(float x)
     return sign | best;
 }
 
+/* Exponent of the power-of-two scale of a head whose largest magnitude is amax > 0:
+ * the smallest e >= -126 with amax <= 448 * 2^e, found by stepping e. */
+int rope3d_oracle_e4m3_scale_exponent(float amax)
+{
+    int e = -126;
+    while ((double)amax > ldexp(448.0, e)) ++e;
+    return e;
+}
+
 /* One head of n fp32 values -> codes and its scale. */
 void rope3d_oracle_quantize_head_e4m3(const float* x, int64_t n, unsigned char* codes,
                                       float* scale)
@@ -532,10 +542,10 @@ void rope3d_oracle_quantize_head_e4m3(const float* x, int64_t n, unsigned char* 
         float a = fabsf(x[e]);
         if (a > amax) amax = a;
     }
-    float s = amax > 0.0f ? amax / 448.0f : 1.0f;
-    float inv = amax > 0.0f ? 448.0f / amax : 1.0f;
-    for (int64_t e = 0; e < n; ++e) codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(x[e] * inv);
-    *scale = s;
+    int ex = amax > 0.0f ? rope3d_oracle_e4m3_scale_exponent(amax) : 0;
+    for (int64_t e = 0; e < n; ++e)
+        codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(ldexpf(x[e], -ex));  /* exact */
+    *scale = ldexpf(1.0f, ex);
 }
 
 /*

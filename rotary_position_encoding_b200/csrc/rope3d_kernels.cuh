@@ -440,10 +440,11 @@ __device__ __forceinline__ void norm_rotate_half_f(
 // ---------------------------------------------------------------- FP8 E4M3 cache rows
 //
 // Quantize-on-append: a head's K or V row goes to the cache as E4M3 codes with one fp32
-// scale, scale = amax / 448 (1 for an all-zero head); codes are E4M3(x * inv) with
-// inv = 448 / amax (1 for a zero head), rounded to nearest even with saturation -- one
-// division per head, one multiply per element.  The lanes holding a head (at one slot)
-// find its amax with a butterfly max; the head's first lane writes the scale.
+// scale.  The scale is a power of two (as in the OCP microscaling formats): the smallest
+// 2^e, e >= -126, with amax / 2^e <= 448 (1 for an all-zero head), read off amax's
+// exponent and mantissa bits; codes are E4M3(x * 2^-e) -- an exact scaling -- rounded to
+// nearest even with saturation.  The lanes holding a head (at one slot) find its amax
+// with a butterfly max; the head's first lane writes the scale.
 
 __device__ __forceinline__ float group_max(float x, int lanes) {
 #pragma unroll
@@ -463,9 +464,21 @@ struct Fp8Scale {
 };
 
 __device__ __forceinline__ Fp8Scale fp8_scale(float amax) {
+    int e = 0;
+    if (amax > 0.0f) {
+        const uint32_t b = __float_as_uint(amax);
+        const int field = (int)((b >> 23) & 0xFFu);
+        if (field == 0) {
+            e = -126;  // subnormal amax: already below 448 * 2^-126
+        } else {
+            // amax = 1.m * 2^(field-127); 448 = 1.75 * 2^8 = mantissa 0x600000 at 2^8
+            e = field - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+            if (e < -126) e = -126;
+        }
+    }
     Fp8Scale s;
-    s.scale = amax > 0.0f ? amax / 448.0f : 1.0f;
-    s.inv = amax > 0.0f ? 448.0f / amax : 1.0f;
+    s.scale = __uint_as_float((uint32_t)(e + 127) << 23);  // 2^e
+    s.inv = __uint_as_float((uint32_t)(127 - e) << 23);    // 2^-e
     return s;
 }
 

@@ -564,24 +564,33 @@ def check_e4m3_encode_matches_torch(orc):
     assert np.array_equal(got, ref)
 
 
+def check_e4m3_scale_exponent_closed_forms(orc):
+    """The power-of-two scale: smallest 2^e with amax / 2^e <= 448."""
+    cases = {448.0: 0, 449.0: 1, 1.0: -8, 3.5: -7, 3.5000002: -6, 224.0: -1, 224.00002: 0,
+             896.0: 1, 1e-3: -18, 3.0e38: 120}
+    for amax, e in cases.items():
+        assert orc.e4m3_scale_exponent(amax) == e, amax
+    assert orc.e4m3_scale_exponent(1e-40) == -126      # clamped at the smallest normal 2^e
+
+
 def check_e4m3_head_quantizer(orc):
-    """scale = amax / 448; codes are E4M3(x * (448 / amax)) in fp32; the largest magnitude
-    maps to +-448; every value is recovered within half an E4M3 step (plus the fp32
-    rounding of the multiply); an all-zero head has scale 1 and zero codes."""
+    """scale = 2^e with the head's largest magnitude in (224, 448] after scaling; codes are
+    E4M3(x / scale) of the exactly scaled values; every value is recovered within half an
+    E4M3 step; an all-zero head has scale 1 and zero codes."""
     rng = _rng(31)
     for _ in range(5):
         x = (rng.standard_normal(128) * rng.uniform(0.1, 5)).astype(np.float32)
         codes, scale = orc.quantize_head_e4m3(x)
-        amax = np.float32(np.max(np.abs(x)))
-        assert scale == amax / np.float32(448.0)
-        inv = np.float32(448.0) / amax
-        assert np.array_equal(codes, [orc.e4m3_encode(float(np.float32(v) * inv)) for v in x])
-        assert (codes[np.argmax(np.abs(x))] & 0x7F) == 0x7E
+        amax = float(np.max(np.abs(x)))
+        m, ex = math.frexp(scale)
+        assert m == 0.5 and 224.0 < amax / scale <= 448.0
+        assert np.array_equal(codes, [orc.e4m3_encode(float(np.float32(v) / np.float32(scale)))
+                                      for v in x])
         deq = np.array([orc.e4m3_value(int(c)) for c in codes]) * scale
         y = np.abs(x.astype(np.float64) / scale)
         step = np.where(y >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(y, 2.0 ** -6))) - 3),
                         2.0 ** -9)
-        assert np.all(np.abs(deq - x) <= (0.5 * step + 1e-6 * y) * scale * (1 + 1e-6))
+        assert np.all(np.abs(deq - x) <= 0.5 * step * scale * (1 + 1e-12))
     codes, scale = orc.quantize_head_e4m3(np.zeros(128, dtype=np.float32))
     assert scale == 1.0 and np.all((codes & 0x7F) == 0)
 

@@ -1,10 +1,12 @@
 """Quantize-on-append FP8 E4M3 KV cache on the GPU against the oracle.
 
-V is quantized from its exact input values, so its codes and scales must match the
-oracle bit for bit.  K is quantized from its fp32 value after RMSNorm and RoPE: the GPU's
-fp32 K and the oracle's fp64 K (rounded to fp32) can differ in the last bits, so a K code
-may differ where x / scale sits at a rounding midpoint; every other K code must match, and
-every dequantized K value must lie within half an E4M3 step of the oracle's K."""
+Scales are powers of two, so the scaling is exact.  V is quantized from its exact input
+values, so its codes and scales must match the oracle bit for bit.  K is quantized from its
+fp32 value after RMSNorm and RoPE: the GPU's fp32 K and the oracle's fp64 K (rounded to
+fp32) can differ in the last bits, so a K scale may differ where the head's amax sits at
+a power-of-two boundary and a K code may differ where x / scale sits at a rounding
+midpoint; every other code must match, and every dequantized K value must lie within half
+an E4M3 step of the oracle's K."""
 import numpy as np
 import pytest
 import torch
@@ -45,7 +47,15 @@ def _check_k(codes, scales, ref_codes, ref_scales, ref_k, rows_sel):
     """K codes equal except at rounding midpoints; dequantized K within half a step."""
     codes, ref_codes, ref_k = codes[rows_sel], ref_codes[rows_sel], ref_k[rows_sel]
     scales, ref_scales = scales[rows_sel], ref_scales[rows_sel]
-    assert np.allclose(scales, ref_scales, rtol=2e-6, atol=0), "K scales"
+    same_scale = scales == ref_scales
+    if not same_scale.all():  # only where amax sits at a power-of-two boundary of 448
+        r = ref_k.reshape(ref_k.shape[:-1] + (-1,))
+        amax = np.max(np.abs(r), axis=-1)[~same_scale]
+        edge = 448.0 * np.minimum(scales, ref_scales)[~same_scale]
+        assert np.all(np.abs(amax - edge) <= 1e-6 * edge), "K scales differ away from an edge"
+        keep = same_scale[..., None] & np.ones(codes.shape, dtype=bool)
+        codes, ref_codes, ref_k = codes * keep, ref_codes * keep, ref_k * keep
+        scales = np.where(same_scale, scales, ref_scales)
     ratio = ref_k / ref_scales[..., None].astype(np.float64)
     mism = codes != ref_codes
     if mism.any():

@@ -66,10 +66,12 @@ MUTANTS = {
     "e4m3_bias_8": ("else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
                     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "e4m3_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", "if (a >= 464.0) return sign | 0x7F;"),
-    "fp8_scale_240": ("float s = amax > 0.0f ? amax / 448.0f : 1.0f;",
-                      "float s = amax > 0.0f ? amax / 240.0f : 1.0f;"),
-    "fp8_codes_scaled_to_240": ("float inv = amax > 0.0f ? 448.0f / amax : 1.0f;",
-                                "float inv = amax > 0.0f ? 240.0f / amax : 1.0f;"),
+    "fp8_scale_exponent_240": ("while ((double)amax > ldexp(448.0, e)) ++e;",
+                               "while ((double)amax > ldexp(240.0, e)) ++e;"),
+    "fp8_scale_exponent_strict": ("while ((double)amax > ldexp(448.0, e)) ++e;",
+                                  "while ((double)amax >= ldexp(448.0, e)) ++e;"),
+    "fp8_codes_unscaled_by_half": ("codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(ldexpf(x[e], -ex));  /* exact */",
+                                   "codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(ldexpf(x[e], -ex - 1));"),
     "fp8_v_scale_from_k": ("rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, v_scale + scale_off);",
                            "rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, k_scale + scale_off);"),
 }
