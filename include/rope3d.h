@@ -100,8 +100,8 @@ extern "C" {
  *   FP8_E4M3 -- quantize-on-append: each head of an appended K or V row is stored as
  *               128 FP8 E4M3 codes (1 byte each; the OCP E4M3 format, max 448) with one
  *               fp32 power-of-two scale (as in the OCP microscaling formats): the
- *               smallest 2^e, e >= -126, with amax(|x|) / 2^e <= 448 over the head (1 if
- *               all zero); code = E4M3(x / 2^e) -- an exact scaling -- rounded to nearest
+ *               smallest 2^e, e >= -126, with amax(|x|) / 2^e <= 448 over the head
+ *               (2^-126 for an all-zero head); code = E4M3(x / 2^e) -- an exact scaling -- rounded to nearest
  *               even, saturating.  K is
  *               quantized from its fp32 value after RMSNorm and RoPE.  A reader recovers
  *               x ~ value(code) * scale.  Scales are laid out like the cache rows:

@@ -524,8 +524,9 @@ int rope3d_oracle_e4m3_encode(float x)
     return sign | best;
 }
 
-/* Exponent of the power-of-two scale of a head whose largest magnitude is amax > 0:
- * the smallest e >= -126 with amax <= 448 * 2^e, found by stepping e. */
+/* Exponent of the power-of-two scale of a head whose largest magnitude is amax >= 0:
+ * the smallest e >= -126 with amax <= 448 * 2^e, found by stepping e (-126 for an
+ * all-zero head, whose codes are zero under any scale). */
 int rope3d_oracle_e4m3_scale_exponent(float amax)
 {
     int e = -126;
@@ -542,7 +543,7 @@ void rope3d_oracle_quantize_head_e4m3(const float* x, int64_t n, unsigned char* 
         float a = fabsf(x[e]);
         if (a > amax) amax = a;
     }
-    int ex = amax > 0.0f ? rope3d_oracle_e4m3_scale_exponent(amax) : 0;
+    int ex = rope3d_oracle_e4m3_scale_exponent(amax);
     for (int64_t e = 0; e < n; ++e)
         codes[e] = (unsigned char)rope3d_oracle_e4m3_encode(ldexpf(x[e], -ex));  /* exact */
     *scale = ldexpf(1.0f, ex);

@@ -571,12 +571,16 @@ def check_e4m3_scale_exponent_closed_forms(orc):
     for amax, e in cases.items():
         assert orc.e4m3_scale_exponent(amax) == e, amax
     assert orc.e4m3_scale_exponent(1e-40) == -126      # clamped at the smallest normal 2^e
+    assert orc.e4m3_scale_exponent(0.0) == -126        # the same rule for an all-zero head
+    assert orc.e4m3_scale_exponent(448.0 * 2.0 ** -126) == -126
+    assert orc.e4m3_scale_exponent(float(np.nextafter(np.float32(448.0 * 2.0 ** -126),
+                                                      np.float32(1)))) == -125
 
 
 def check_e4m3_head_quantizer(orc):
     """scale = 2^e with the head's largest magnitude in (224, 448] after scaling; codes are
     E4M3(x / scale) of the exactly scaled values; every value is recovered within half an
-    E4M3 step; an all-zero head has scale 1 and zero codes."""
+    E4M3 step; an all-zero head has scale 2^-126 (the rule's smallest) and zero codes."""
     rng = _rng(31)
     for _ in range(5):
         x = (rng.standard_normal(128) * rng.uniform(0.1, 5)).astype(np.float32)
@@ -592,7 +596,7 @@ def check_e4m3_head_quantizer(orc):
                         2.0 ** -9)
         assert np.all(np.abs(deq - x) <= 0.5 * step * scale * (1 + 1e-12))
     codes, scale = orc.quantize_head_e4m3(np.zeros(128, dtype=np.float32))
-    assert scale == 1.0 and np.all((codes & 0x7F) == 0)
+    assert scale == 2.0 ** -126 and np.all((codes & 0x7F) == 0)
 
 
 def check_fp8_step_matches_layout_step(orc):
