@@ -394,8 +394,12 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pair
         if (stages >= 2) break;
     }
     if (teams < 1 || stages < 2) return ROPE3D_OK;  // does not fit: register kernel
+    // Measured on B200: the ring pays off for wide rows and long runs only, and not with an
+    // FP8 cache in adjacent pairing, where the register kernel's extra resident warps hide
+    // the quantizer's latency better (127 vs 139 us on the 720P chunk).
     if (!forced && (g.tpr < 96 || teams < 2 ||
-                    p.units < (int64_t)16 * info.sms * teams))
+                    p.units < (int64_t)16 * info.sms * teams ||
+                    (p.k_scale != nullptr && pairing == ROPE3D_PAIRING_ADJACENT)))
         return ROPE3D_OK;
     smem = tma_layout(p, teams, stages, warps_per_team);
     TmaKernelFn fn = pick_tma_kernel(dtype, trig, pairing, p.k_scale != nullptr, g.vpt);

@@ -441,21 +441,16 @@ __device__ __forceinline__ void norm_rotate_half_f(
 //
 // Quantize-on-append: a head's K or V row goes to the cache as E4M3 codes with one fp32
 // scale.  The scale is a power of two (as in the OCP microscaling formats): the smallest
-// 2^e, e >= -126, with amax / 2^e <= 448 (1 for an all-zero head), read off amax's
-// exponent and mantissa bits; codes are E4M3(x * 2^-e) -- an exact scaling -- rounded to
-// nearest even with saturation.  The lanes holding a head (at one slot) find its amax
-// with a butterfly max; the head's first lane writes the scale.
+// 2^e, e >= -126, with amax / 2^e <= 448; codes are E4M3(x * 2^-e) -- an exact scaling --
+// rounded to nearest even with saturation.  The lanes holding a head (at one slot) agree
+// on its scale through a butterfly maximum of integer keys, two heads per shuffle; the
+// head's first lane writes the scale.
 
-__device__ __forceinline__ float group_max(float x, int lanes) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        if (off < lanes) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-    return x;
-}
-
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-    // element a in the low byte (lower address)
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+// Key of a magnitude a >= 0: a's biased exponent, plus one when a's mantissa lies above
+// that of 1.75 (448 = 1.75 * 2^8), so that the smallest e with a <= 448 * 2^e is
+// key - 135.  The key is monotone in a, so a head's key is the maximum of its lanes'.
+__device__ __forceinline__ uint32_t fp8_key(float a) {
+    return (__float_as_uint(a) + 0x1FFFFFu) >> 23;
 }
 
 struct Fp8Scale {
@@ -463,45 +458,87 @@ struct Fp8Scale {
     float inv;    // codes are E4M3(x * inv)
 };
 
-__device__ __forceinline__ Fp8Scale fp8_scale(float amax) {
-    int e = 0;
-    if (amax > 0.0f) {
-        const uint32_t b = __float_as_uint(amax);
-        const int field = (int)((b >> 23) & 0xFFu);
-        if (field == 0) {
-            e = -126;  // subnormal amax: already below 448 * 2^-126
-        } else {
-            // amax = 1.m * 2^(field-127); 448 = 1.75 * 2^8 = mantissa 0x600000 at 2^8
-            e = field - 127 - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
-            if (e < -126) e = -126;
-        }
-    }
+__device__ __forceinline__ Fp8Scale fp8_scale_from_key(uint32_t key) {
+    key = max(key, 9u);  // e = key - 135 >= -126
     Fp8Scale s;
-    s.scale = __uint_as_float((uint32_t)(e + 127) << 23);  // 2^e
-    s.inv = __uint_as_float((uint32_t)(127 - e) << 23);    // 2^-e
+    s.scale = __uint_as_float((key - 8u) << 23);  // 2^e
+    s.inv = __uint_as_float((262u - key) << 23);  // 2^-e
     return s;
 }
 
-// Store E codes of one vector at vector index vi of an FP8 cache (E bytes per vector).
+// Three-input maximum (a single instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Scales of two heads from this lane's keys k0, k1: the keys travel packed in the halves
+// of one word, reduced over groups of `lanes` lanes (a power of two <= 32).
+__device__ __forceinline__ void fp8_scale_pair(uint32_t k0, uint32_t k1, int lanes,
+                                               Fp8Scale& s0, Fp8Scale& s1) {
+    uint32_t w = k0 | (k1 << 16);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        if (off < lanes) w = max_u16x2(w, __shfl_xor_sync(0xffffffffu, w, off));
+    s0 = fp8_scale_from_key(w & 0xFFFFu);
+    s1 = fp8_scale_from_key(w >> 16);
+}
+
+// Key of the largest magnitude in a vector of input elements.  For bf16 the magnitudes
+// are compared as 16-bit integers (ordered like the values), and the key of a bf16 value
+// with bits b is (b + 0x1F) >> 7, fp8_key of its fp32 widening b << 16.
+__device__ __forceinline__ uint32_t vec_key(const uint4& v) {
+    uint32_t m = max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.z & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.w & 0x7FFF7FFFu);
+    return (max(m & 0xFFFFu, m >> 16) + 0x1Fu) >> 7;
+}
+__device__ __forceinline__ uint32_t vec_key(const float4& v) {
+    return fp8_key(fmaxf(max3f(fabsf(v.x), fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
+}
+
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    // element a in the low byte (lower address)
+    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Store E codes of one vector at vector index vi of an FP8 cache (E bytes per vector);
+// the values are scaled two at a time (packed fp32x2 multiplies).
+__device__ __forceinline__ uint32_t e4m3x4_scaled(float a, float b, float c, float d,
+                                                  float2 inv2) {
+    const float2 x = __fmul2_rn(make_float2(a, b), inv2);
+    const float2 y = __fmul2_rn(make_float2(c, d), inv2);
+    return e4m3x2(x.x, x.y) | (e4m3x2(y.x, y.y) << 16);
+}
 __device__ __forceinline__ void store_fp8(void* cache, int64_t vi, const float (&v)[8],
                                           float inv) {
+    const float2 inv2 = make_float2(inv, inv);
     uint2 c;
-    c.x = e4m3x2(v[0] * inv, v[1] * inv) | (e4m3x2(v[2] * inv, v[3] * inv) << 16);
-    c.y = e4m3x2(v[4] * inv, v[5] * inv) | (e4m3x2(v[6] * inv, v[7] * inv) << 16);
+    c.x = e4m3x4_scaled(v[0], v[1], v[2], v[3], inv2);
+    c.y = e4m3x4_scaled(v[4], v[5], v[6], v[7], inv2);
     __stcs(reinterpret_cast<uint2*>(cache) + vi, c);
 }
 __device__ __forceinline__ void store_fp8(void* cache, int64_t vi, const float (&v)[4],
                                           float inv) {
-    const uint32_t c = e4m3x2(v[0] * inv, v[1] * inv) | (e4m3x2(v[2] * inv, v[3] * inv) << 16);
+    const uint32_t c = e4m3x4_scaled(v[0], v[1], v[2], v[3], make_float2(inv, inv));
     __stcs(reinterpret_cast<unsigned int*>(cache) + vi, c);
 }
 
 template <int E>
 __device__ __forceinline__ float abs_max(const float (&v)[E]) {
-    float m = 0.0f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) m = fmaxf(m, fabsf(v[e]));
-    return m;
+    static_assert(E == 4 || E == 8, "vectors hold 4 or 8 elements");
+    float m = max3f(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+    if constexpr (E == 4) return fmaxf(m, fabsf(v[3]));
+    m = max3f(m, fabsf(v[3]), fabsf(v[4]));
+    m = max3f(m, fabsf(v[5]), fabsf(v[6]));
+    return fmaxf(m, fabsf(v[7]));
 }
 
 __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, float* s_wk) {
@@ -518,22 +555,37 @@ __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, floa
 
 // ---------------------------------------------------------------- per-row output
 
+// Quantize one vector of V (its input elements) to the FP8 cache.
+template <typename T>
+__device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
+                                            const typename VecTraits<T>::Vec& x, float inv) {
+    using Tr = VecTraits<T>;
+    float v[Tr::kElems];
+#pragma unroll
+    for (int e = 0; e < Tr::kElems; ++e) v[e] = Tr::elem(x, e);
+    store_fp8(vc, vi, v, inv);
+}
+
 // Normalise, rotate and store this thread's vectors of one row: q_out, and in the fused
-// mode the K row into the cache (V is stored by store_v_row).  With rotate_half pairing
-// slots 2m and 2m+1 hold the two halves of the same pairs (see slot_vec).  With an FP8
-// cache (CFP8) the K values stay fp32 until they are quantized; every lane of the warp
-// takes part in the head-wise maximum, whether its slot holds a vector or not.
+// mode the K row into the cache.  With rotate_half pairing slots 2m and 2m+1 hold the two
+// halves of the same pairs (see slot_vec).  V goes to a same-dtype cache through
+// store_v_row; with an FP8 cache (CFP8) it is quantized here, beside K: the K values stay
+// fp32 until they are quantized, and the K and V keys of one head travel in one shuffle
+// word.  Every lane of the warp takes part in the head-wise maximum, whether its slots
+// hold vectors or not.
 template <typename T, int VPT, int PAIR, int MODE, bool CFP8>
 __device__ __forceinline__ void emit_row(
     const Params& p, int t, const RowPos& pos, int64_t row_vec,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
+    const typename VecTraits<T>::Vec (&xv)[VPT],
     float rq, float rk, const float* s_wq, const float* s_wk,
     const float (&cs)[PairCount<T, PAIR>::value], const float (&sn)[PairCount<T, PAIR>::value],
-    typename VecTraits<T>::Vec* qo, typename VecTraits<T>::Vec* kc) {
+    typename VecTraits<T>::Vec* qo, typename VecTraits<T>::Vec* kc,
+    typename VecTraits<T>::Vec* vc) {
     using Tr = VecTraits<T>;
-    using Vec = typename Tr::Vec;
     constexpr int EPV = Tr::kElems;
     constexpr bool NORM = MODE == kModeFused;
+    constexpr bool QUANT = MODE == kModeFused && CFP8;
     constexpr int VPH = Tr::kVecsPerHead;
     if constexpr (PAIR == kPairAdjacent) {
 #pragma unroll
@@ -543,20 +595,29 @@ __device__ __forceinline__ void emit_row(
             const int e0 = idx * EPV;
             if (valid)
                 store_out(qo + row_vec + idx, norm_rotate<T, NORM>(xq[s], rq, s_wq, e0, cs, sn));
-            if constexpr (MODE == kModeFused) {
-                if constexpr (CFP8) {
-                    float o[EPV];
-                    if (valid) norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
-                    const Fp8Scale sc = fp8_scale(group_max(valid ? abs_max<EPV>(o) : 0.0f, VPH));
-                    if (valid) {
-                        store_fp8(kc, cache_vec_index(p, pos, idx), o, sc.inv);
-                        if ((idx & (VPH - 1)) == 0)
-                            __stcs(p.k_scale + cache_scale_index(p, pos, idx / VPH), sc.scale);
-                    }
-                } else if (valid) {
-                    store_out(kc + cache_vec_index(p, pos, idx),
-                              norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
+            if constexpr (QUANT) {
+                float o[EPV];
+                uint32_t kk = 0, kv = 0;
+                if (valid) {
+                    norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
+                    kk = fp8_key(abs_max<EPV>(o));
+                    kv = vec_key(xv[s]);
                 }
+                Fp8Scale sk, sv;
+                fp8_scale_pair(kk, kv, VPH, sk, sv);
+                if (valid) {
+                    const int64_t vi = cache_vec_index(p, pos, idx);
+                    store_fp8(kc, vi, o, sk.inv);
+                    store_v_fp8<T>(vc, vi, xv[s], sv.inv);
+                    if ((idx & (VPH - 1)) == 0) {
+                        const int64_t si = cache_scale_index(p, pos, idx / VPH);
+                        __stcs(p.k_scale + si, sk.scale);
+                        __stcs(p.v_scale + si, sv.scale);
+                    }
+                }
+            } else if (MODE == kModeFused && valid) {
+                store_out(kc + cache_vec_index(p, pos, idx),
+                          norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
             }
         }
     } else {
@@ -578,13 +639,25 @@ __device__ __forceinline__ void emit_row(
                     norm_rotate_half_f<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV,
                                                 i_im * EPV, cs, sn, o_re, o_im);
                 if constexpr (CFP8) {
-                    const float local = valid ? fmaxf(abs_max<EPV>(o_re), abs_max<EPV>(o_im)) : 0.0f;
-                    const Fp8Scale sc = fp8_scale(group_max(local, VPH / 2));
+                    uint32_t kk = 0, kv = 0;
                     if (valid) {
-                        store_fp8(kc, cache_vec_index(p, pos, i_re), o_re, sc.inv);
-                        store_fp8(kc, cache_vec_index(p, pos, i_im), o_im, sc.inv);
-                        if ((i_re & (VPH - 1)) == 0)
-                            __stcs(p.k_scale + cache_scale_index(p, pos, i_re / VPH), sc.scale);
+                        kk = fp8_key(fmaxf(abs_max<EPV>(o_re), abs_max<EPV>(o_im)));
+                        kv = max(vec_key(xv[s]), vec_key(xv[s + 1]));
+                    }
+                    Fp8Scale sk, sv;
+                    fp8_scale_pair(kk, kv, VPH / 2, sk, sv);
+                    if (valid) {
+                        const int64_t vr = cache_vec_index(p, pos, i_re);
+                        const int64_t vm = cache_vec_index(p, pos, i_im);
+                        store_fp8(kc, vr, o_re, sk.inv);
+                        store_fp8(kc, vm, o_im, sk.inv);
+                        store_v_fp8<T>(vc, vr, xv[s], sv.inv);
+                        store_v_fp8<T>(vc, vm, xv[s + 1], sv.inv);
+                        if ((i_re & (VPH - 1)) == 0) {
+                            const int64_t si = cache_scale_index(p, pos, i_re / VPH);
+                            __stcs(p.k_scale + si, sk.scale);
+                            __stcs(p.v_scale + si, sv.scale);
+                        }
                     }
                 } else if (valid) {
                     store_out(kc + cache_vec_index(p, pos, i_re), Tr::pack_elems(o_re));
@@ -595,46 +668,15 @@ __device__ __forceinline__ void emit_row(
     }
 }
 
-// Store this thread's vectors of one row of V to the cache: a bit copy, or FP8 codes
-// with a per-head scale (every lane of the warp takes part in the head-wise maximum).
-template <typename T, int VPT, int PAIR, bool CFP8>
+// Store this thread's vectors of one row of V to a same-dtype cache: a bit copy.
+template <typename T, int VPT, int PAIR>
 __device__ __forceinline__ void store_v_row(const Params& p, int t, const RowPos& pos,
                                             const typename VecTraits<T>::Vec (&xv)[VPT],
                                             typename VecTraits<T>::Vec* vc) {
-    using Tr = VecTraits<T>;
-    constexpr int EPV = Tr::kElems;
-    constexpr int VPH = Tr::kVecsPerHead;
-    if constexpr (!CFP8) {
 #pragma unroll
-        for (int s = 0; s < VPT; ++s) {
-            const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
-            if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[s]);
-        }
-    } else {
-        constexpr int STEP = PAIR == kPairAdjacent ? 1 : 2;  // slots that share one head
-        constexpr int LANES = PAIR == kPairAdjacent ? VPH : VPH / 2;
-#pragma unroll
-        for (int s = 0; s < VPT; s += STEP) {
-            const int idx0 = slot_vec<T, PAIR>(t, s, p.tpr);
-            const bool valid = idx0 < p.dim_vecs;
-            float v[STEP][EPV];
-            float local = 0.0f;
-#pragma unroll
-            for (int j = 0; j < STEP; ++j) {
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) v[j][e] = valid ? Tr::elem(xv[s + j], e) : 0.0f;
-                local = fmaxf(local, abs_max<EPV>(v[j]));
-            }
-            const Fp8Scale sc = fp8_scale(group_max(local, LANES));
-            if (valid) {
-#pragma unroll
-                for (int j = 0; j < STEP; ++j)
-                    store_fp8(vc, cache_vec_index(p, pos, slot_vec<T, PAIR>(t, s + j, p.tpr)),
-                              v[j], sc.inv);
-                if ((idx0 & (VPH - 1)) == 0)
-                    __stcs(p.v_scale + cache_scale_index(p, pos, idx0 / VPH), sc.scale);
-            }
-        }
+    for (int s = 0; s < VPT; ++s) {
+        const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+        if (idx < p.dim_vecs) store_out(vc + cache_vec_index(p, pos, idx), xv[s]);
     }
 }
 
@@ -696,7 +738,7 @@ qk_norm_rope_kernel(const Params p) {
 
         float rq = 1.0f, rk = 1.0f;
         if (MODE == kModeFused) {
-            store_v_row<T, VPT, PAIR, CFP8>(p, t, pos, xv, vc);
+            if constexpr (!CFP8) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -704,8 +746,8 @@ qk_norm_rope_kernel(const Params p) {
             rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
-        emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, rq, rk, s_wq, s_wk, cs, sn,
-                                           qo, kc);
+        emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq, s_wk,
+                                           cs, sn, qo, kc, vc);
     }
 }
 
