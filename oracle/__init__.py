@@ -10,7 +10,9 @@ Paper: "Accelerating Video Generation Inference with Sequential-Parallel 3D
 Positional Encoding Using a Global Time Index" (Yuan & Li) -- Section 3.3.1 (complex
 rotation), Section 3.3.2 (global time index, localized formula), Algorithm 2 (per-axis
 tables, adjacent-pair complex view, fp64), Section 3.3.3 (local-to-global index decode)
-and Algorithms 1 and 3, step 5 (KV-cache update).
+and Algorithms 1 and 3, step 5 (KV-cache update).  ``Oracle.qk_norm_rope_append_sp`` adds
+the all-to-all of Algorithm 3 step 4 (Section 3.4.1 item 1: gather the sequence, scatter
+the heads) as plain per-head stores on top of the C step.
 """
 from __future__ import annotations
 
@@ -315,6 +317,43 @@ class Oracle:
             _f64(k_cache, "k_cache"), _f64(v_cache, "v_cache"), C, slot,
             n_t, n_h, n_w, theta, schedule, pairing, cache_layout, nthreads))
         return q_out
+
+    def qk_norm_rope_append_sp(self, q, k, v, token_begin, token_end, frame_offset, T, H, W,
+                               q_norm_w, k_norm_w, eps, q_dst, k_dst, v_dst, slot,
+                               q_row0=0, cache_layout=CACHE_TOKEN_MAJOR, n_t=N_T, n_h=N_H,
+                               n_w=N_W, theta=THETA, schedule=0):
+        """One rank's sequence-parallel step with the all-to-all (Algorithm 3, steps 3-5;
+        the FusedAllToAll of Section 3.4.1 item 1: gather over the sequence, scatter over
+        heads).  q, k, v: this rank's rows [B, n, N, D] for tokens [token_begin,
+        token_end), all heads.  The step is computed as usual; then every head n goes to
+        its owner rank r = n // (N/P) as local head n - r N/P: q to q_dst[r][b, i - q_row0],
+        K and V to k_dst[r], v_dst[r] at cache row (slot + i) mod C
+        ([B, C, N/P, D], or [B, N/P, C, D] head-major).  P = len(q_dst); the destination
+        arrays (float64) are written in place."""
+        B, n, N, D = q.shape
+        P = len(q_dst)
+        if N % P:
+            raise ValueError("heads do not split evenly over the ranks")
+        hl = N // P
+        if token_begin < q_row0 or token_end - q_row0 > q_dst[0].shape[1]:
+            raise ValueError("the token range is not inside the q buffers' rows")
+        C = k_dst[0].shape[1] if cache_layout == CACHE_TOKEN_MAJOR else k_dst[0].shape[2]
+        kc = np.zeros((B, C, N, D))
+        vc = np.zeros((B, C, N, D))
+        q_out = self.qk_norm_rope_append_layout(
+            q, k, v, token_begin, token_end, frame_offset, T, H, W, q_norm_w, k_norm_w, eps,
+            kc, vc, slot, PAIRING_ADJACENT, CACHE_TOKEN_MAJOR, n_t, n_h, n_w, theta, schedule)
+        i = np.arange(token_begin, token_end)
+        rows = (slot + i) % C
+        for head in range(N):
+            r, local = divmod(head, hl)
+            q_dst[r][:, i - q_row0, local] = q_out[:, :, head]
+            if cache_layout == CACHE_TOKEN_MAJOR:
+                k_dst[r][:, rows, local] = kc[:, rows, head]
+                v_dst[r][:, rows, local] = vc[:, rows, head]
+            else:
+                k_dst[r][:, local, rows] = kc[:, rows, head]
+                v_dst[r][:, local, rows] = vc[:, rows, head]
 
     def apply_pairing(self, x, token_begin, token_end, frame_offset, T, H, W, pairing,
                       n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):

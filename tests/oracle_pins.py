@@ -19,6 +19,12 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 D = 128
 P = 64
 NT, NH, NW = 22, 21, 21
+CACHE_TOKEN_MAJOR, CACHE_HEAD_MAJOR = 0, 1  # the oracle's cache layouts
+
+
+def _f32(x):
+    """float64 values that are exactly float32 (as the workloads' inputs are)."""
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
 
 
 def _rows(name):
@@ -626,6 +632,49 @@ def check_fp8_step_matches_layout_step(orc):
                     ev, esv = orc.quantize_head_e4m3(vf[idx])
                     assert np.array_equal(kc[idx], ek) and ks[idx] == esk
                     assert np.array_equal(vc[idx], ev) and vs[idx] == esv
+
+
+def check_sp_head_scatter_is_whole_step_split_by_heads(orc):
+    """Algorithm 3 steps 3-5 with the all-to-all folded in: ranks with uneven token
+    ranges, each storing every head at its owner, together leave in owner r exactly the
+    whole-sequence step's heads [r N/P, (r+1) N/P) -- q at rows i - q_row0 of its buffer,
+    K/V at the rolling cache rows -- and nothing else (sentinels elsewhere stay).  Both
+    cache layouts; P = 1, 2, 4; q buffers longer than the range, and buffers that start
+    mid-chunk (q_row0 > 0)."""
+    rng = _rng(41)
+    B, N, T, H, W, s, C, slot = 2, 4, 3, 4, 6, 6, 100, 90
+    L = T * H * W
+    q, k, v = (_f32(rng.standard_normal((B, L, N, D))) for _ in range(3))
+    wq, wk = (_f32(rng.uniform(0.5, 1.5, N * D)) for _ in range(2))
+    kw, vw = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    whole = orc.qk_norm_rope_append_layout(q, k, v, 0, L, s, T, H, W, wq, wk, 1e-6, kw, vw,
+                                           slot)
+    for P, cuts, q_row0, q_rows in ((1, [0, L], 0, L), (2, [0, 17, 40, L], 0, L + 9),
+                                    (4, [0, 17, 40, L], 0, L), (2, [24, 50, L], 24, L - 24 + 3)):
+        hl = N // P
+        span = np.arange(cuts[0], cuts[-1])
+        rows = (slot + span) % C
+        for layout in (CACHE_TOKEN_MAJOR, CACHE_HEAD_MAJOR):
+            cshape = (B, C, hl, D) if layout == CACHE_TOKEN_MAJOR else (B, hl, C, D)
+            q_dst = [np.full((B, q_rows, hl, D), 7.0) for _ in range(P)]
+            k_dst = [np.full(cshape, 7.0) for _ in range(P)]
+            v_dst = [np.full(cshape, 7.0) for _ in range(P)]
+            for a, e in zip(cuts[:-1], cuts[1:]):
+                orc.qk_norm_rope_append_sp(q[:, a:e].copy(), k[:, a:e].copy(),
+                                           v[:, a:e].copy(), a, e, s, T, H, W, wq, wk, 1e-6,
+                                           q_dst, k_dst, v_dst, slot, q_row0=q_row0,
+                                           cache_layout=layout)
+            for r in range(P):
+                heads = slice(r * hl, (r + 1) * hl)
+                got = q_dst[r][:, span - q_row0]
+                assert np.array_equal(got, whole[:, span][:, :, heads])
+                assert np.all(np.delete(q_dst[r], span - q_row0, axis=1) == 7.0)
+                kt, vt = k_dst[r], v_dst[r]
+                if layout == CACHE_HEAD_MAJOR:
+                    kt, vt = kt.transpose(0, 2, 1, 3), vt.transpose(0, 2, 1, 3)
+                assert np.array_equal(kt[:, rows], kw[:, rows][:, :, heads])
+                assert np.array_equal(vt[:, rows], v[:, span][:, :, heads])
+                assert np.all(np.delete(kt, rows, axis=1) == 7.0)
 
 
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -5,8 +5,12 @@ own token slice [r L/P, (r+1) L/P) with the global index offset Delta = r L_loca
 communication ("Accelerating Video Generation Inference with Sequential-Parallel 3D
 Positional Encoding Using a Global Time Index", Section 3.3.3; Algorithm 3 steps 2-3).
 These tests run ranks as processes: (1) each rank computes its slice with the oracle
-and rank 0 checks the gathered result against the whole sequence; (2) the benchmark's
-timing reduction takes the maximum over ranks and scales the token count by the ranks."""
+and rank 0 checks the gathered result against the whole sequence; (2) the oracle's
+sequence-parallel step with the all-to-all folded in (each head stored at the rank that
+owns it) equals the pages' separate FusedAllToAll -- an all-to-all that gathers the
+sequence and scatters the heads (Algorithm 3 step 4), here torch's gloo all_to_all_single
+-- applied to each rank's plain results; (3) the benchmark's timing reduction takes the
+maximum over ranks and scales the token count by the ranks."""
 import os
 import socket
 import sys
@@ -72,6 +76,62 @@ def _sp_rank(rank, world, port, q_path):
         dist.destroy_process_group()
 
 
+def _a2a_rank(rank, world, port, out_path):
+    _init(rank, world, port)
+    import datetime
+
+    import oracle
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        B, N, D, T, H, W, s, C, slot = 1, 4, 128, 3, 4, 6, 3, 96, 80
+        L = T * H * W
+        hl = N // world
+        rng = np.random.default_rng(77)  # the same inputs on every rank
+        q, k, v = (rng.standard_normal((B, L, N, D)).astype(np.float32).astype(np.float64)
+                   for _ in range(3))
+        wq, wk = (rng.uniform(0.5, 1.5, N * D).astype(np.float32).astype(np.float64)
+                  for _ in range(2))
+        n = L // world
+        a, e = rank * n, (rank + 1) * n  # Algorithm 3 step 2: Delta = r L_local
+        orc = oracle.default()
+        # the pages' order: local step, then an all-to-all over (sequence, heads)
+        kc = np.zeros((B, C, N, D))
+        vc = np.zeros_like(kc)
+        q_loc = orc.qk_norm_rope_append(q[:, a:e].copy(), k[:, a:e].copy(), v[:, a:e].copy(),
+                                        a, e, s, T, H, W, wq, wk, 1e-6, kc, vc, slot)
+        rows = (slot + np.arange(a, e)) % C
+
+        def exchange(x):  # x: [B, n, N, D] -> this rank's heads of every rank's rows
+            send = torch.from_numpy(np.ascontiguousarray(
+                x.reshape(B, n, world, hl, D).transpose(2, 0, 1, 3, 4)))
+            recv = torch.empty_like(send)
+            dist.all_to_all_single(recv, send)
+            return np.concatenate(list(recv.numpy()), axis=1)  # [B, L, hl, D]
+
+        q_a2a = exchange(q_loc)
+        k_a2a, v_a2a = exchange(kc[:, rows]), exchange(vc[:, rows])
+        # the fused form: every rank writes each head straight to its owner's buffers
+        q_dst = [np.zeros((B, L, hl, D)) for _ in range(world)]
+        k_dst = [np.zeros((B, C, hl, D)) for _ in range(world)]
+        v_dst = [np.zeros((B, C, hl, D)) for _ in range(world)]
+        orc.qk_norm_rope_append_sp(q[:, a:e].copy(), k[:, a:e].copy(), v[:, a:e].copy(), a, e,
+                                   s, T, H, W, wq, wk, 1e-6, q_dst, k_dst, v_dst, slot)
+        mine = []
+        for x in q_dst + k_dst + v_dst:  # land every rank's stores at the owner
+            t = torch.from_numpy(x)
+            dist.all_reduce(t)  # each element is written by exactly one rank
+            mine.append(t.numpy())
+        q_f, k_f, v_f = mine[rank], mine[world + rank], mine[2 * world + rank]
+        all_rows = (slot + np.arange(L)) % C
+        ok = (np.array_equal(q_f, q_a2a) and np.array_equal(k_f[:, all_rows], k_a2a) and
+              np.array_equal(v_f[:, all_rows], v_a2a) and
+              not np.delete(k_f, all_rows, axis=1).any())
+        with open(f"{out_path}.{rank}", "w") as f:
+            f.write("ok" if ok else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
 def _timing_rank(rank, world, port, out_path):
     _init(rank, world, port)
     import bench
@@ -93,6 +153,13 @@ def test_sequence_parallel_slices_on_two_ranks(tmp_path):
     mp.start_processes(_sp_rank, args=(2, _free_port(), out), nprocs=2, start_method="spawn",
                        join=True)
     assert open(out).read() == "ok"
+
+
+def test_fused_head_scatter_equals_all_to_all_on_two_ranks(tmp_path):
+    out = str(tmp_path / "a2a")
+    mp.start_processes(_a2a_rank, args=(2, _free_port(), out), nprocs=2, start_method="spawn",
+                       join=True)
+    assert [open(f"{out}.{r}").read() for r in range(2)] == ["ok", "ok"]
 
 
 def test_bench_timing_is_max_over_ranks(tmp_path):

@@ -111,3 +111,36 @@ def test_pins_catch_mutant(tmp_path, name):
         except Exception as e:  # a crash also counts as caught, but say which
             caught.append(f"{check.__name__} ({type(e).__name__})")
     assert caught, f"no pin catches the planted mistake {name}"
+
+
+# Planted mistakes in the oracle's Python-level head scatter (the sequence-parallel step's
+# all-to-all folded into stores): a copy of oracle/__init__.py with one line changed.
+PY_MUTANTS = {
+    "sp_round_robin_owner": ("r, local = divmod(head, hl)", "r, local = head % P, head // P"),
+    "sp_q_row_ignores_row0": ("q_dst[r][:, i - q_row0, local]", "q_dst[r][:, i, local]"),
+    "sp_cache_rows_drop_slot": ("rows = (slot + i) % C", "rows = i % C"),
+    "sp_head_major_as_token_major": (
+        "                k_dst[r][:, local, rows] = kc[:, rows, head]",
+        "                k_dst[r][:, rows, local] = kc[:, rows, head]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_python_mutant(name):
+    import types
+    old, new = PY_MUTANTS[name]
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, f"mutant site of {name} not found exactly once"
+    mod = types.ModuleType(f"oracle_{name}")
+    mod.__file__ = oracle.__file__
+    exec(compile(src.replace(old, new), oracle.__file__, "exec"), mod.__dict__)
+    orc = mod.Oracle()
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check(orc)
+        except AssertionError:
+            caught.append(check.__name__)
+        except Exception as e:
+            caught.append(f"{check.__name__} ({type(e).__name__})")
+    assert caught, f"no pin catches the planted mistake {name}"
