@@ -70,6 +70,10 @@ def parse_args(argv=None):
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
                          "fits in shared memory)")
+    ap.add_argument("--sp", type=int, default=0,
+                    help="sequence-parallel step with the all-to-all folded in: each chunk is "
+                         "cut into SP even token slices (the ranks of one node, emulated on "
+                         "this GPU as SP launches) whose heads go to SP destination buffers")
     ap.add_argument("--eager", action="store_true",
                     help="launch every chunk call from Python and time each launch with its "
                          "own CUDA event pair (default: capture one step -- all its chunk "
@@ -247,7 +251,7 @@ def recorded_traffic(workload_name: str, trig: str):
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    entry = rec.get(f"{workload_name}/{trig}")
+    entry = rec.get(workload_name if trig is None else f"{workload_name}/{trig}")
     if not entry or entry.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
     return entry.get("dram_bytes_per_launch")
@@ -309,17 +313,46 @@ def run_ours(args, dist: Dist):
                                       "registers": rope3d.ROPE3D_PATH_REGISTERS,
                                       "tma": rope3d.ROPE3D_PATH_TMA}[args.path])
 
+    P = args.sp
+    if P:
+        if w.N % P or n % P or fp8 or args.pairing != "adjacent":
+            raise SystemExit("--sp needs heads and tokens divisible by SP, adjacent pairing "
+                             "and a same-dtype cache")
+        hl = w.N // P
+        dshape = ((w.B, w.cache_tokens, hl, wl.HEAD_DIM) if args.cache_layout == "token"
+                  else (w.B, hl, w.cache_tokens, wl.HEAD_DIM))
+        sp_q = [torch.empty((w.B, n, hl, wl.HEAD_DIM), dtype=tdt, device=device)
+                for _ in range(P)]
+        sp_k = [torch.zeros(dshape, dtype=tdt, device=device) for _ in range(P)]
+        sp_v = [torch.zeros(dshape, dtype=tdt, device=device) for _ in range(P)]
+        k_cache = v_cache = None
+        # each emulated rank reads its own slice of the chunk's rows
+        sp_inputs = [[tuple(x[:, r * (n // P):(r + 1) * (n // P)].contiguous() for x in c)
+                      for r in range(P)] for c in inputs]
+        inputs = None
+
     def step(events=None):
+        j = 0
         for ci, chunk in enumerate(w.chunks):
-            q, k, v = inputs[ci]
-            if events is not None:
-                events[2 * ci].record(stream)
-            rope3d.rope3d_qk_norm_rope_append_ex(
-                q, k, v, q_out[ci], chunk.token_begin, chunk.token_end, chunk.frame_offset,
-                w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache, chunk.slot, tables, trig,
-                pairing, layout, k_scale, v_scale, stream)
-            if events is not None:
-                events[2 * ci + 1].record(stream)
+            for r in range(max(P, 1)):
+                if events is not None:
+                    events[2 * j].record(stream)
+                if P:
+                    q, k, v = sp_inputs[ci][r]
+                    a = chunk.token_begin + r * (n // P)
+                    rope3d.rope3d_qk_norm_rope_append_sp(
+                        q, k, v, a, a + n // P, chunk.frame_offset, w.T, w.H, w.W, wq_d, wk_d,
+                        w.eps, sp_q, sp_k, sp_v, chunk.slot, tables, trig, layout,
+                        q_row0=chunk.token_begin, stream=stream)
+                else:
+                    q, k, v = inputs[ci]
+                    rope3d.rope3d_qk_norm_rope_append_ex(
+                        q, k, v, q_out[ci], chunk.token_begin, chunk.token_end,
+                        chunk.frame_offset, w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache,
+                        chunk.slot, tables, trig, pairing, layout, k_scale, v_scale, stream)
+                if events is not None:
+                    events[2 * j + 1].record(stream)
+                j += 1
 
     clocks = ClockSampler(dist.local_rank) if dist.rank == 0 else None
     if clocks:
@@ -330,7 +363,9 @@ def run_ours(args, dist: Dist):
     torch.cuda.synchronize()
 
     # per-launch events of every timed launch (the kernel's own duration) and the region
-    n_launch = len(w.chunks)
+    n_launch = len(w.chunks) * max(P, 1)
+    if P:
+        bytes_per_launch //= P
     graph = None
     if (not args.eager):
         side = torch.cuda.Stream(device)
@@ -380,12 +415,14 @@ def run_ours(args, dist: Dist):
     kernel_used = {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
                    rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
         rope3d.rope3d_testing_last_path(), "unknown")
+    if P:
+        kernel_used += " (head-scatter stores)"
     device_status = rope3d.rope3d_check_device_status(tables)
     if device_status != rope3d.ROPE3D_OK:
         raise RuntimeError("a kernel wait timed out during the benchmark")
     e2e = None
-    if not args.no_e2e and (args.pairing, args.cache_layout, args.cache_dtype) != (
-            "adjacent", "token", "same"):
+    if not args.no_e2e and ((args.pairing, args.cache_layout, args.cache_dtype) != (
+            "adjacent", "token", "same") or P):
         args.no_e2e = True  # the e2e leg runs the default layout only
     if not args.no_e2e:
         e2e = run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch)
@@ -405,7 +442,8 @@ def run_ours(args, dist: Dist):
         "peak": peaks["hbm_gbs"],
         "unit": "GB/s",
         "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-        "traffic": recorded_traffic(w.name, args.trig),
+        "traffic": recorded_traffic(w.name + (f"/{args.trig}/sp{P}" if P else ""),
+                                    args.trig if not P else None),
         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
         else "fallback 6.65 TB/s",
         "kernel": kernel_used,
@@ -446,6 +484,9 @@ def run_ours(args, dist: Dist):
             "l2": "no flush: inputs larger than L2 (each launch streams "
                   f"{bytes_per_launch / 1e6:.1f} MB from its own buffers)",
             "parallelism": f"replicas x{dist.world} (independent streams, no collective)",
+            "sequence_parallel": (f"{P} ranks emulated on one GPU: {P} launches per chunk over "
+                                  f"even token slices, heads stored to {P} local destination "
+                                  f"buffers ({w.N // P} heads each)") if P else None,
         },
         "hbm_gbs": round(bytes_per_launch * n_launch * args.steps * dist.world
                          / (elapsed_ms / 1e3) / 1e9, 1),

@@ -203,6 +203,57 @@ ROPE3D_API int rope3d_qk_norm_rope_append_ex(
     const rope3d_options* options, void* cuda_stream);
 
 /*
+ * Sequence-parallel step with the all-to-all folded in: Algorithm 3 steps 3-5 ("Causal-RoPE
+ * SP", Section 3.3.3; the FusedAllToAll of Section 3.4.1 item 1 with scatter over heads and
+ * gather over the sequence).  This rank holds q, k, v for its own token range
+ * [token_begin, token_end) with all N heads (layout as for rope3d_qk_norm_rope_append).  The
+ * heads are split evenly over dest->ranks = P ranks: rank r owns heads
+ * [r N/P, (r+1) N/P).  For every token i of the range and head n the step computes the same
+ * values as rope3d_qk_norm_rope_append and stores them at the owner r of n, local head
+ * n' = n - r N/P:
+ *   q:  dest->q[r]        [B][dest->q_rows][N/P][D], row i - dest->q_row0 (the owner's
+ *                          buffer holds the gathered sequence; usually q_row0 = 0 and
+ *                          q_rows = T*H*W);
+ *   K:  dest->k_cache[r]  [B][cache_tokens][N/P][D] (or [B][N/P][cache_tokens][D] with
+ *                          options->cache_layout = ROPE3D_CACHE_HEAD_MAJOR), cache row
+ *                          (slot + i) mod cache_tokens;
+ *   V:  dest->v_cache[r]  likewise, a bit copy.
+ * Run on every rank with its own range and the same dest tables (each rank listing the
+ * ranks' buffers in rank order), the ranks together produce the whole-sequence result
+ * split by heads, bit-identical to rope3d_qk_norm_rope_append on the whole sequence.
+ *
+ * Destination pointers are device addresses valid on the calling device: this device's
+ * memory, or another GPU's memory mapped into this process (CUDA IPC, or a symmetric-memory
+ * mapping); stores to another GPU go over NVLink as plain peer stores.  The call does not
+ * synchronise with the other ranks: before a rank reads what others wrote, every rank's
+ * step must have completed (for example a stream synchronisation followed by a barrier of
+ * the process group).  Options: adjacent pairing and same-dtype caches only
+ * (ROPE3D_EINVAL otherwise); the cache layout option applies.  Errors: P outside
+ * [1, ROPE3D_SP_MAX_RANKS] or N not divisible by P (EINVAL); the token range outside
+ * [q_row0, q_row0 + q_rows) (ERANGE); a NULL or misaligned destination (EINVAL / EALIGN);
+ * destinations that overlap one another or an input, as far as their address ranges show
+ * it (EOVERLAP).  Other arguments and errors as for rope3d_qk_norm_rope_append.
+ */
+#define ROPE3D_SP_MAX_RANKS 8
+
+typedef struct rope3d_sp_dest {
+    int ranks;                               /* P                                      */
+    int reserved0;                           /* must be zero                           */
+    int64_t q_rows;                          /* rows per sample of each q buffer       */
+    int64_t q_row0;                          /* global token index of q row 0          */
+    void* q[ROPE3D_SP_MAX_RANKS];            /* rank r's q buffer (entries >= P unused) */
+    void* k_cache[ROPE3D_SP_MAX_RANKS];      /* rank r's K cache                       */
+    void* v_cache[ROPE3D_SP_MAX_RANKS];      /* rank r's V cache                       */
+} rope3d_sp_dest;
+
+ROPE3D_API int rope3d_qk_norm_rope_append_sp(
+    const void* q, const void* k, const void* v, int64_t B, int64_t N, int D, int dtype,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
+    const float* q_norm_w, const float* k_norm_w, float eps, const rope3d_sp_dest* dest,
+    int64_t cache_tokens, int64_t slot, const rope3d_tables* tables, int trig,
+    const rope3d_options* options, void* cuda_stream);
+
+/*
  * The rotation alone -- CausalRoPE of Algorithm 3 step 3 / Algorithm 2 -- on one
  * token range: out[b][r] = RoPE(x[b][r], pos(token_begin + r)).  x and out are
  * [B][n_tok][N][D] of dtype; out may be x (in place) or must not overlap it.  Other

@@ -218,7 +218,13 @@ KernelFn pick_pairing(int pairing, int trig, int vpt) {
 
 template <int MODE>
 KernelFn pick_kernel(int dtype, int trig, int pairing, bool fp8, int vpt) {
-    if constexpr (MODE == rope3d::kModeApply) {
+    if constexpr (MODE == rope3d::kModeFusedSP) {
+        // head-scatter stores: adjacent pairing and same-dtype caches only
+        if (pairing != ROPE3D_PAIRING_ADJACENT || fp8) return nullptr;
+        return dtype == ROPE3D_BF16
+                   ? pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent, false>(trig, vpt)
+                   : pick_trig<float, MODE, rope3d::kPairAdjacent, false>(trig, vpt);
+    } else if constexpr (MODE == rope3d::kModeApply) {
         return dtype == ROPE3D_BF16 ? pick_pairing<__nv_bfloat16, MODE, false>(pairing, trig, vpt)
                                     : pick_pairing<float, MODE, false>(pairing, trig, vpt);
     } else {
@@ -439,9 +445,10 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int d
     const int threads = teams * g.tpr;
     const int warps_per_team = g.tpr / 32;
     size_t smem = 0;
-    if (MODE == rope3d::kModeFused) {
+    if (MODE != rope3d::kModeApply) {
         smem = (size_t)2 * p.dim * sizeof(float);
         if (warps_per_team > 1) smem += (size_t)2 * teams * warps_per_team * sizeof(float2);
+        if (MODE == rope3d::kModeFusedSP) smem += 3 * rope3d::kMaxRanks * sizeof(void*);
     }
     if (smem > (size_t)info.max_smem_optin)
         return fail(ROPE3D_EINVAL, "N=%lld needs %zu bytes of shared memory (limit %d)",
@@ -821,6 +828,110 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
             return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);
     }
     rc = launch<rope3d::kModeFused>(p, N, dtype, trig, opt.pairing, dev, info, stream);
+    if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
+    return rc;
+}
+
+int rope3d_qk_norm_rope_append_sp(const void* q, const void* k, const void* v,
+                                  int64_t B, int64_t N, int D, int dtype,
+                                  int64_t token_begin, int64_t token_end, int64_t frame_offset,
+                                  int T, int H, int W,
+                                  const float* q_norm_w, const float* k_norm_w, float eps,
+                                  const rope3d_sp_dest* dest, int64_t cache_tokens,
+                                  int64_t slot, const rope3d_tables* tables, int trig,
+                                  const rope3d_options* options, void* cuda_stream) {
+    rope3d_options opt;
+    int rc = read_options(options, &opt, true);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_common(B, N, D, dtype, token_begin, token_end, frame_offset, T, H, W, tables,
+                      trig);
+    if (rc != ROPE3D_OK) return rc;
+    if (opt.pairing != ROPE3D_PAIRING_ADJACENT || opt.cache_dtype != ROPE3D_CACHE_SAME)
+        return fail(ROPE3D_EINVAL,
+                    "head-scatter stores support adjacent pairing and same-dtype caches");
+    if (!q || !k || !v || !q_norm_w || !k_norm_w || !dest)
+        return fail(ROPE3D_EINVAL, "a tensor pointer or dest is NULL");
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(ROPE3D_EINVAL, "eps must be >= 0");
+    const int P = dest->ranks;
+    if (P < 1 || P > ROPE3D_SP_MAX_RANKS)
+        return fail(ROPE3D_EINVAL, "dest->ranks %d is not in [1, %d]", P, ROPE3D_SP_MAX_RANKS);
+    if (N % P != 0)
+        return fail(ROPE3D_EINVAL, "N=%lld heads do not split evenly over %d ranks",
+                    (long long)N, P);
+    if (dest->reserved0 != 0) return fail(ROPE3D_EINVAL, "dest->reserved0 must be zero");
+    if (cache_tokens < 1) return fail(ROPE3D_EINVAL, "cache_tokens must be >= 1");
+    if (slot < 0) return fail(ROPE3D_EINVAL, "slot must be >= 0");
+    if (token_end - token_begin > cache_tokens)
+        return fail(ROPE3D_ERANGE, "%lld tokens do not fit a cache of %lld rows",
+                    (long long)(token_end - token_begin), (long long)cache_tokens);
+    if (dest->q_row0 < 0 || dest->q_rows < 1 || token_begin < dest->q_row0 ||
+        token_end > dest->q_row0 + dest->q_rows)
+        return fail(ROPE3D_ERANGE, "tokens [%lld, %lld) are not inside the q rows [%lld, %lld)",
+                    (long long)token_begin, (long long)token_end, (long long)dest->q_row0,
+                    (long long)(dest->q_row0 + dest->q_rows));
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_norm_w) ||
+        !aligned16(k_norm_w))
+        return fail(ROPE3D_EALIGN, "every tensor pointer must be 16-byte aligned");
+    for (int r = 0; r < P; ++r) {
+        if (!dest->q[r] || !dest->k_cache[r] || !dest->v_cache[r])
+            return fail(ROPE3D_EINVAL, "a destination pointer of rank %d is NULL", r);
+        if (!aligned16(dest->q[r]) || !aligned16(dest->k_cache[r]) ||
+            !aligned16(dest->v_cache[r]))
+            return fail(ROPE3D_EALIGN, "destination pointers must be 16-byte aligned");
+    }
+    // Overlap among the local inputs and the destinations is checked for destinations in
+    // this process's address space only as far as the ranges are known here: inputs must
+    // not overlap any destination range of a rank.
+    const size_t esz = dtype == ROPE3D_BF16 ? 2 : 4;
+    const size_t act = (size_t)B * (size_t)(token_end - token_begin) * (size_t)N * D * esz;
+    const size_t qd = (size_t)B * (size_t)dest->q_rows * (size_t)(N / P) * D * esz;
+    const size_t cd = (size_t)B * (size_t)cache_tokens * (size_t)(N / P) * D * esz;
+    for (int r = 0; r < P; ++r) {
+        const void* dsts[3] = {dest->q[r], dest->k_cache[r], dest->v_cache[r]};
+        const size_t dsz[3] = {qd, cd, cd};
+        for (int j = 0; j < 3; ++j)
+            if (overlap(dsts[j], dsz[j], q, act) || overlap(dsts[j], dsz[j], k, act) ||
+                overlap(dsts[j], dsz[j], v, act))
+                return fail(ROPE3D_EOVERLAP, "a destination of rank %d overlaps an input", r);
+        for (int r2 = 0; r2 < P; ++r2) {
+            const void* d2[3] = {dest->q[r2], dest->k_cache[r2], dest->v_cache[r2]};
+            for (int j = 0; j < 3; ++j)
+                for (int j2 = 0; j2 < 3; ++j2)
+                    if ((r2 != r || j2 != j) && overlap(dsts[j], dsz[j], d2[j2], dsz[j2]))
+                        return fail(ROPE3D_EOVERLAP, "destination buffers overlap");
+        }
+    }
+
+    DeviceInfo info;
+    int dev = 0;
+    rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_tables_device(tables, dev);
+    if (rc != ROPE3D_OK) return rc;
+
+    rope3d::Params p{};
+    fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.q_w = q_norm_w;
+    p.k_w = k_norm_w;
+    p.cache_tokens = cache_tokens;
+    p.slot = slot;
+    p.eps = eps;
+    fill_layout(p, N, dtype, opt);
+    p.sp_ranks = P;
+    p.sp_heads = (int)(N / P);
+    p.sp_q_rows = dest->q_rows;
+    p.sp_q_row0 = dest->q_row0;
+    for (int r = 0; r < P; ++r) {
+        p.sp_dst[3 * r] = dest->q[r];
+        p.sp_dst[3 * r + 1] = dest->k_cache[r];
+        p.sp_dst[3 * r + 2] = dest->v_cache[r];
+    }
+    set_small_idx(p);
+    rc = launch<rope3d::kModeFusedSP>(p, N, dtype, trig, opt.pairing, dev, info,
+                                      static_cast<cudaStream_t>(cuda_stream));
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
     return rc;
 }

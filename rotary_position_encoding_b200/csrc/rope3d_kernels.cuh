@@ -40,7 +40,10 @@ constexpr int kMaxTeamsPerBlock = 15;  // named barriers 1..15 (0 is __syncthrea
 constexpr int kMaxBlockThreads = 512;  // leaves up to 128 registers per thread
 constexpr int kTmaMaxBlockThreads = 320;  // ring kernel: one block per SM, up to 204 registers
 
-enum Mode : int { kModeFused = 0, kModeApply = 1 };
+// kModeFusedSP: the fused step with head-scatter stores (the sequence-parallel
+// all-to-all folded into the step): each head goes to the destination rank that owns it.
+enum Mode : int { kModeFused = 0, kModeApply = 1, kModeFusedSP = 2 };
+constexpr int kMaxRanks = 8;  // head-scatter destinations (one node)
 enum Trig : int { kTrigTable = 0, kTrigOnTheFly = 1 };
 // Pairing of a head's elements into complex pairs: adjacent (2j, 2j+1) -- the complex
 // view of Wan2.1 -- or rotate_half (j, j + 64), the cos/sin form of M-RoPE.
@@ -88,6 +91,12 @@ struct Params {
     int vph_log2;          // log2 of the 16-byte vectors per head
     float* k_scale;        // FP8 caches: per (token, head) scales, laid out like the cache rows
     float* v_scale;
+    // head-scatter destinations (kModeFusedSP): rank r owns heads [r*sp_heads, (r+1)*sp_heads)
+    int sp_ranks;
+    int sp_heads;          // heads per rank
+    int64_t sp_q_rows;     // rows per batch sample of a destination q buffer
+    int64_t sp_q_row0;     // global token index held by a destination q buffer's row 0
+    void* sp_dst[3 * kMaxRanks];  // rank r: q [B][sp_q_rows][sp_heads][D], k and v caches
     float inv_freq[kPairs];  // fp32 angle per unit position of every pair
 };
 
@@ -680,6 +689,71 @@ __device__ __forceinline__ void store_v_row(const Params& p, int t, const RowPos
     }
 }
 
+// ---------------------------------------------------------------- head-scatter stores
+//
+// The sequence-parallel all-to-all (sequence gather, head scatter) folded into the step:
+// a rank holds all heads of its token slice, and each head's q, K and V go straight to
+// the rank that owns the head -- q to row (i - sp_q_row0) of that rank's q buffer, K and
+// V to its caches at the token's cache row -- as plain stores (through peer mappings when
+// the destination is another GPU).  The destination of a slot depends on the thread
+// only: code = (rank << 16) | vector index within the destination's token row.
+
+__device__ __forceinline__ int sp_code(const Params& p, int idx) {
+    const int vph = 1 << p.vph_log2;
+    const int d = (idx >> p.vph_log2) / p.sp_heads;
+    return (d << 16) | (idx - d * p.sp_heads * vph);
+}
+
+// Vector index of local vector dv of a cache row in a destination cache of sp_heads heads.
+__device__ __forceinline__ int64_t sp_cache_index(const Params& p, const RowPos& pos, int dv) {
+    if (!p.cache_head_major)
+        return ((pos.b * p.cache_tokens + pos.crow) * p.sp_heads << p.vph_log2) + dv;
+    const int nl = dv >> p.vph_log2;
+    const int v = dv & ((1 << p.vph_log2) - 1);
+    return (((pos.b * p.sp_heads + nl) * p.cache_tokens + pos.crow) << p.vph_log2) + v;
+}
+
+template <typename T, int VPT>
+__device__ __forceinline__ void store_v_row_sp(const Params& p, int t, const RowPos& pos,
+                                               const typename VecTraits<T>::Vec (&xv)[VPT],
+                                               const int (&dst)[VPT], void* const* s_sp) {
+    using Vec = typename VecTraits<T>::Vec;
+#pragma unroll
+    for (int s = 0; s < VPT; ++s) {
+        if (slot_vec<T, kPairAdjacent>(t, s, p.tpr) < p.dim_vecs) {
+            Vec* vd = reinterpret_cast<Vec*>(s_sp[3 * (dst[s] >> 16) + 2]);
+            store_out(vd + sp_cache_index(p, pos, dst[s] & 0xFFFF), xv[s]);
+        }
+    }
+}
+
+template <typename T, int VPT>
+__device__ __forceinline__ void emit_row_sp(
+    const Params& p, int t, const RowPos& pos,
+    const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
+    float rq, float rk, const float* s_wq, const float* s_wk,
+    const float (&cs)[PairCount<T, kPairAdjacent>::value],
+    const float (&sn)[PairCount<T, kPairAdjacent>::value], const int (&dst)[VPT],
+    void* const* s_sp) {
+    using Tr = VecTraits<T>;
+    using Vec = typename Tr::Vec;
+    const int64_t q_row = (pos.b * p.sp_q_rows + (pos.i - p.sp_q_row0)) * p.sp_heads
+                          << p.vph_log2;
+#pragma unroll
+    for (int s = 0; s < VPT; ++s) {
+        const int idx = slot_vec<T, kPairAdjacent>(t, s, p.tpr);
+        if (idx < p.dim_vecs) {
+            const int d = dst[s] >> 16, dv = dst[s] & 0xFFFF;
+            const int e0 = idx * Tr::kElems;
+            Vec* qd = reinterpret_cast<Vec*>(s_sp[3 * d]);
+            Vec* kd = reinterpret_cast<Vec*>(s_sp[3 * d + 1]);
+            store_out(qd + q_row + dv, norm_rotate<T, true>(xq[s], rq, s_wq, e0, cs, sn));
+            store_out(kd + sp_cache_index(p, pos, dv),
+                      norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
+        }
+    }
+}
+
 // ---------------------------------------------------------------- register kernel
 
 template <typename T, int VPT, int TRIG, int MODE, int PAIR, bool CFP8>
@@ -688,11 +762,17 @@ qk_norm_rope_kernel(const Params p) {
     using Tr = VecTraits<T>;
     using Vec = typename Tr::Vec;
     constexpr int NP = PairCount<T, PAIR>::value;
+    constexpr bool FUSED = MODE != kModeApply;
+    constexpr bool SP = MODE == kModeFusedSP;
+    static_assert(!SP || (PAIR == kPairAdjacent && !CFP8),
+                  "head-scatter stores: adjacent pairing, same-dtype caches");
 
+    // dynamic shared memory: [SP: destination table] [q, k norm weights] [team partials]
     extern __shared__ float4 smem4[];
-    float* s_wq = reinterpret_cast<float*>(smem4);
-    float* s_wk = s_wq + (MODE == kModeFused ? p.dim : 0);
-    float2* s_part = reinterpret_cast<float2*>(s_wk + (MODE == kModeFused ? p.dim : 0));
+    void** s_sp = reinterpret_cast<void**>(smem4);
+    float* s_wq = reinterpret_cast<float*>(smem4 + (SP ? 3 * kMaxRanks / 2 : 0));
+    float* s_wk = s_wq + (FUSED ? p.dim : 0);
+    float2* s_part = reinterpret_cast<float2*>(s_wk + (FUSED ? p.dim : 0));
 
     const int tid = threadIdx.x;
     const int team = tid / p.tpr;
@@ -703,11 +783,21 @@ qk_norm_rope_kernel(const Params p) {
 
     pdl_launch_dependents();
     pdl_wait_previous_grid();
-    if (MODE == kModeFused) {
+    if (FUSED) {
+        if constexpr (SP) {
+#pragma unroll
+            for (int j = 0; j < 3 * kMaxRanks; ++j)
+                if (tid == j) s_sp[j] = p.sp_dst[j];  // constant indices into the parameters
+        }
         stage_weights(p, s_wq, s_wk);
         __syncthreads();
     }
     const PairInfo<NP> pi = pair_info<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
+    int dst[VPT];
+    if constexpr (SP) {
+#pragma unroll
+        for (int s = 0; s < VPT; ++s) dst[s] = sp_code(p, slot_vec<T, PAIR>(t, s, p.tpr));
+    }
 
     const Vec* qg = reinterpret_cast<const Vec*>(p.q);
     const Vec* kg = reinterpret_cast<const Vec*>(p.k);
@@ -727,7 +817,7 @@ qk_norm_rope_kernel(const Params p) {
             const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
             if (idx < p.dim_vecs) {
                 xq[s] = load_stream(qg + row_vec + idx);
-                if (MODE == kModeFused) {
+                if (FUSED) {
                     xk[s] = load_stream(kg + row_vec + idx);
                     xv[s] = load_stream(vg + row_vec + idx);
                 }
@@ -737,8 +827,9 @@ qk_norm_rope_kernel(const Params p) {
         pair_trig<TRIG>(pi, pos, cs, sn);
 
         float rq = 1.0f, rk = 1.0f;
-        if (MODE == kModeFused) {
-            if constexpr (!CFP8) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
+        if (FUSED) {
+            if constexpr (SP) store_v_row_sp<T, VPT>(p, t, pos, xv, dst, s_sp);
+            else if constexpr (!CFP8) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -746,8 +837,11 @@ qk_norm_rope_kernel(const Params p) {
             rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
-        emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq, s_wk,
-                                           cs, sn, qo, kc, vc);
+        if constexpr (SP)
+            emit_row_sp<T, VPT>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
+        else
+            emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq,
+                                               s_wk, cs, sn, qo, kc, vc);
     }
 }
 

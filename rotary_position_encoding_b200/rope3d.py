@@ -49,6 +49,17 @@ class rope3d_options(ctypes.Structure):
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
                 ("reserved", ctypes.c_int * 4)]
 
+ROPE3D_SP_MAX_RANKS = 8
+
+
+class rope3d_sp_dest(ctypes.Structure):
+    """struct rope3d_sp_dest of include/rope3d.h."""
+    _fields_ = [("ranks", ctypes.c_int), ("reserved0", ctypes.c_int),
+                ("q_rows", ctypes.c_int64), ("q_row0", ctypes.c_int64),
+                ("q", ctypes.c_void_p * ROPE3D_SP_MAX_RANKS),
+                ("k_cache", ctypes.c_void_p * ROPE3D_SP_MAX_RANKS),
+                ("v_cache", ctypes.c_void_p * ROPE3D_SP_MAX_RANKS)]
+
 # include/rope3d_testing.h
 ROPE3D_PATH_AUTO = 0
 ROPE3D_PATH_REGISTERS = 1
@@ -69,6 +80,10 @@ SIGNATURES = {
     "rope3d_qk_norm_rope_append_ex": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64,
                                        _I64, _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP,
                                        _VP, _I64, _I64, _VP, _INT,
+                                       ctypes.POINTER(rope3d_options), _VP], _INT),
+    "rope3d_qk_norm_rope_append_sp": ([_VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64,
+                                       _INT, _INT, _INT, _VP, _VP, ctypes.c_float,
+                                       ctypes.POINTER(rope3d_sp_dest), _I64, _I64, _VP, _INT,
                                        ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_apply": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT, _VP,
                       _INT, _VP], _INT),
@@ -276,6 +291,68 @@ def rope3d_qk_norm_rope_append_ex(q, k, v, q_out, token_begin: int, token_end: i
         B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,
         _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), C, slot,
+        tables.handle, trig, ctypes.byref(opts), _stream(stream)))
+
+
+def rope3d_qk_norm_rope_append_sp(q, k, v, token_begin: int, token_end: int,
+                                  frame_offset: int, T: int, H: int, W: int, q_norm_w, k_norm_w,
+                                  eps: float, q_dst, k_cache_dst, v_cache_dst, slot: int,
+                                  tables: Tables, trig: int = ROPE3D_TRIG_TABLE,
+                                  cache_layout: int = ROPE3D_CACHE_TOKEN_MAJOR, q_row0: int = 0,
+                                  q_rows: int | None = None, cache_tokens: int | None = None,
+                                  stream=None) -> None:
+    """The step with head-scatter stores: q, k, v are this rank's [B, n_tok, N, 128]; the
+    three destination lists hold, in rank order, each rank's q buffer [B, q_rows, N/P, 128]
+    and caches [B, C, N/P, 128] (head-major: [B, N/P, C, 128]) -- tensors on this device,
+    or integer device addresses of peer mappings (then q_rows and cache_tokens are given)."""
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k and v must all be [B, n_tok, N, D]")
+    B, n_tok, N, D = q.shape
+    if n_tok != token_end - token_begin:
+        raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
+    P = len(q_dst)
+    if not 1 <= P <= ROPE3D_SP_MAX_RANKS or len(k_cache_dst) != P or len(v_cache_dst) != P:
+        raise ValueError(f"one q, k and v destination per rank, 1 to {ROPE3D_SP_MAX_RANKS} ranks")
+    for name, t in (("k", k), ("v", v)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have q's dtype {q.dtype}")
+    if N % P:
+        raise ValueError(f"N={N} heads do not split evenly over {P} ranks")
+    hl = N // P
+    dest = rope3d_sp_dest()
+    dest.ranks = P
+    dest.q_row0 = q_row0
+
+    def addr(t, name, shape_ok):
+        if isinstance(t, int):
+            return t
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} must have q's dtype {q.dtype}")
+        if not shape_ok(tuple(t.shape)):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}")
+        return _dev_ptr(t, name)
+
+    for r in range(P):
+        if not isinstance(q_dst[r], int):
+            q_rows = q_dst[r].shape[1] if q_rows is None else q_rows
+        kc = k_cache_dst[r]
+        if not isinstance(kc, int):
+            c = kc.shape[2] if cache_layout == ROPE3D_CACHE_HEAD_MAJOR else kc.shape[1]
+            cache_tokens = c if cache_tokens is None else cache_tokens
+    if q_rows is None or cache_tokens is None:
+        raise ValueError("q_rows and cache_tokens are needed when every destination is an address")
+    cshape = ((B, hl, cache_tokens, D) if cache_layout == ROPE3D_CACHE_HEAD_MAJOR
+              else (B, cache_tokens, hl, D))
+    dest.q_rows = q_rows
+    for r in range(P):
+        dest.q[r] = addr(q_dst[r], f"q_dst[{r}]", lambda s: s == (B, q_rows, hl, D))
+        dest.k_cache[r] = addr(k_cache_dst[r], f"k_cache_dst[{r}]", lambda s: s == cshape)
+        dest.v_cache[r] = addr(v_cache_dst[r], f"v_cache_dst[{r}]", lambda s: s == cshape)
+    opts = rope3d_options(ROPE3D_PAIRING_ADJACENT, cache_layout)
+    _check(load_library().rope3d_qk_norm_rope_append_sp(
+        _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), B, N, D, _dtype_code(q),
+        token_begin, token_end, frame_offset, T, H, W, _dev_ptr(q_norm_w, "q_norm_w"),
+        _dev_ptr(k_norm_w, "k_norm_w"), eps, ctypes.byref(dest), cache_tokens, slot,
         tables.handle, trig, ctypes.byref(opts), _stream(stream)))
 
 

@@ -123,3 +123,37 @@ def test_options_struct_layout_matches_header(tmp_path):
     S = rope3d.rope3d_options
     assert got == [ctypes.sizeof(S), S.pairing.offset, S.cache_layout.offset,
                    S.cache_dtype.offset, S.k_scale.offset, S.v_scale.offset, S.reserved.offset]
+
+
+def test_sp_dest_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of rope3d_sp_dest has the C struct's size and field offsets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    fields = ("ranks", "reserved0", "q_rows", "q_row0", "q", "k_cache", "v_cache")
+    src = tmp_path / "layout_sp.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "rope3d.h"\n'
+                   'int main(void){printf("%zu", sizeof(rope3d_sp_dest));'
+                   + "".join(f'printf(" %zu", offsetof(rope3d_sp_dest, {f}));' for f in fields)
+                   + ' return 0;}\n')
+    exe = tmp_path / "layout_sp"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = list(map(int, subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()))
+    S = rope3d.rope3d_sp_dest
+    assert got == [ctypes.sizeof(S)] + [getattr(S, f).offset for f in fields]
+
+
+def test_sp_step_rejects_null_arguments_without_device(lib):
+    """NULL tables or a NULL destination table fail on the host (the destination checks that
+    need real tables run in the gpu-marked tests)."""
+    p = ctypes.c_void_p(0x10000)
+    dest = rope3d.rope3d_sp_dest()
+    dest.ranks, dest.q_rows, dest.q_row0 = 2, 72, 0
+    for r in range(2):
+        dest.q[r] = dest.k_cache[r] = dest.v_cache[r] = 0x100000 * (r + 1)
+    for d in (ctypes.byref(dest), None):
+        assert lib.rope3d_qk_norm_rope_append_sp(p, p, p, 1, 2, 128, 1, 0, 72, 0, 3, 4, 6, p, p,
+                                                 1e-6, d, 144, 0, None, 0, None,
+                                                 None) == rope3d.ROPE3D_EINVAL
