@@ -240,3 +240,41 @@ def test_argument_errors():
                                 scale.data_ptr())
     assert c_call(dest, ctypes.byref(fp8)) == rope3d.ROPE3D_EINVAL
     torch.cuda.synchronize()
+
+
+def test_symmetric_memory_wiring_one_rank():
+    """The multi-GPU wiring (one symmetric-memory allocation per rank, the table of every
+    rank's addresses, the step, the device barrier) on a one-rank NCCL group: the rank's
+    own buffers hold the plain step's results bit for bit.  Runs with more ranks need
+    more GPUs than this build has."""
+    import datetime
+    import socket
+
+    import torch.distributed as dist
+
+    from rotary_position_encoding_b200 import sp
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True)
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        st = Setup("bf16", B=2, N=4, T=2, H=3, W=5, s=4, C=64, slot=50, P=1, layout=TOKEN,
+                   seed=31)
+        wiring = sp.SequenceParallelStep(dist.group.WORLD, 0, 1, B=2, N=4, q_rows=st.L,
+                                         cache_tokens=64, dtype=torch.bfloat16, device="cuda")
+        wiring.q.fill_(3.0)
+        wiring.k_cache.fill_(2.0)
+        wiring.v_cache.fill_(-2.0)
+        q, k, v = st.dev
+        wiring.step(q, k, v, 0, st.L, 4, 2, 3, 5, st.wq, st.wk, 1e-6, 50, st.tables)
+        wiring.barrier()
+        torch.cuda.synchronize()
+        st.q_dst, st.k_dst, st.v_dst = [wiring.q], [wiring.k_cache], [wiring.v_cache]
+        st.check_against_plain(0, st.L)
+        del wiring, st
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()

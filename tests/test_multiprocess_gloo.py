@@ -132,6 +132,46 @@ def _a2a_rank(rank, world, port, out_path):
         dist.destroy_process_group()
 
 
+def _sp_table_rank(rank, world, port, out_path):
+    """The multi-GPU wiring's address bookkeeping with a CPU stand-in for the symmetric
+    allocation: every rank's destination table lists, in rank order, the regions that
+    each rank exposes as its own q and cache tensors."""
+    _init(rank, world, port)
+    import datetime
+
+    from rotary_position_encoding_b200 import rope3d, sp
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        def exchange(nbytes, device, group):
+            buf = torch.zeros(nbytes, dtype=torch.uint8)
+            bases = [None] * world
+            dist.all_gather_object(bases, buf.data_ptr(), group=group)
+            return buf, bases, lambda: dist.barrier(group=group)
+
+        ok = True
+        for layout in (rope3d.ROPE3D_CACHE_TOKEN_MAJOR, rope3d.ROPE3D_CACHE_HEAD_MAJOR):
+            st = sp.SequenceParallelStep(dist.group.WORLD, rank, world, B=2, N=6, q_rows=77,
+                                         cache_tokens=131, dtype=torch.bfloat16, device="cpu",
+                                         cache_layout=layout, exchange=exchange)
+            own = (st.q.data_ptr(), st.k_cache.data_ptr(), st.v_cache.data_ptr())
+            everyone = [None] * world
+            dist.all_gather_object(everyone, own)
+            ok &= [list(x) for x in zip(st.q_dst, st.k_dst, st.v_dst)] == [list(e) for e in everyone]
+            cshape = (2, 131, 3, 128) if layout == rope3d.ROPE3D_CACHE_TOKEN_MAJOR else (2, 3, 131, 128)
+            ok &= tuple(st.q.shape) == (2, 77, 3, 128) and tuple(st.k_cache.shape) == cshape
+            lay = st.layout  # regions start on 256-byte boundaries of the allocation
+            ok &= all(off % 256 == 0 for off in (lay.q_off, lay.k_off, lay.v_off, lay.nbytes))
+            ends = sorted((t.data_ptr(), t.data_ptr() + t.numel() * 2)
+                          for t in (st.q, st.k_cache, st.v_cache))
+            ok &= all(a[1] <= b[0] for a, b in zip(ends, ends[1:]))
+            ok &= ends[-1][1] <= st.buffer.data_ptr() + st.buffer.numel()
+            st.barrier()
+        with open(f"{out_path}.{rank}", "w") as f:
+            f.write("ok" if ok else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
 def _timing_rank(rank, world, port, out_path):
     _init(rank, world, port)
     import bench
@@ -159,6 +199,13 @@ def test_fused_head_scatter_equals_all_to_all_on_two_ranks(tmp_path):
     out = str(tmp_path / "a2a")
     mp.start_processes(_a2a_rank, args=(2, _free_port(), out), nprocs=2, start_method="spawn",
                        join=True)
+    assert [open(f"{out}.{r}").read() for r in range(2)] == ["ok", "ok"]
+
+
+def test_sp_destination_tables_on_two_ranks(tmp_path):
+    out = str(tmp_path / "sptab")
+    mp.start_processes(_sp_table_rank, args=(2, _free_port(), out), nprocs=2,
+                       start_method="spawn", join=True)
     assert [open(f"{out}.{r}").read() for r in range(2)] == ["ok", "ok"]
 
 
