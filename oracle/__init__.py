@@ -94,6 +94,14 @@ def _declare(lib):
                                                    _I64, _I64, _I64, _I64, _D, _D, _DBL, _U8,
                                                    _U8, _F, _F, _I64, _I64, _INT, _INT, _INT,
                                                    _DBL, _INT, _INT, _INT], _INT),
+        "rope3d_oracle_e2m1_value": ([_INT], _DBL),
+        "rope3d_oracle_e2m1_encode": ([ctypes.c_float], _INT),
+        "rope3d_oracle_quantize_block_nvfp4": ([_F, _I64, ctypes.c_float, _U8, _U8], None),
+        "rope3d_oracle_qk_norm_rope_append_nvfp4": ([_D, _D, _D, _D, _I64, _I64, _I64, _I64,
+                                                     _I64, _I64, _I64, _I64, _I64, _D, _D, _DBL,
+                                                     _U8, _U8, _U8, _U8, ctypes.c_float,
+                                                     ctypes.c_float, _I64, _I64, _INT, _INT,
+                                                     _INT, _DBL, _INT, _INT, _INT], _INT),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -264,6 +272,43 @@ class Oracle:
             _u8(k_codes, "k_codes"), _u8(v_codes, "v_codes"), _f32(k_scale, "k_scale"),
             _f32(v_scale, "v_scale"), C, slot, n_t, n_h, n_w, theta, schedule, pairing,
             cache_layout))
+        return q_out
+
+    # ---- NVFP4 KV cache
+
+    def e2m1_value(self, code: int) -> float:
+        return self.lib.rope3d_oracle_e2m1_value(code)
+
+    def e2m1_encode(self, x: float) -> int:
+        return self.lib.rope3d_oracle_e2m1_encode(x)
+
+    def quantize_block_nvfp4(self, x, g: float = 1.0):
+        """n (even) values -> (n/2 code bytes, E4M3 scale byte)."""
+        x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+        codes = np.zeros(x.size // 2, dtype=np.uint8)
+        scale = np.zeros(1, dtype=np.uint8)
+        self.lib.rope3d_oracle_quantize_block_nvfp4(_f32(x, "x"), x.size, g,
+                                                    _u8(codes, "codes"), _u8(scale, "scale"))
+        return codes, int(scale[0])
+
+    def qk_norm_rope_append_nvfp4(self, q, k, v, token_begin, token_end, frame_offset, T, H,
+                                  W, q_norm_w, k_norm_w, eps, k_codes, v_codes, k_scales,
+                                  v_scales, slot, k_global=1.0, v_global=1.0,
+                                  pairing=PAIRING_ADJACENT, cache_layout=CACHE_TOKEN_MAJOR,
+                                  n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
+        """Whole step with an NVFP4 cache: codes uint8 [B,C,N,D/2] / [B,N,C,D/2], block
+        scales uint8 [B,C,N,D/16] / [B,N,C,D/16], updated in place.  Returns q_out."""
+        B, n_tok, N, D = q.shape
+        C = k_codes.shape[1] if cache_layout == CACHE_TOKEN_MAJOR else k_codes.shape[2]
+        q_out = np.empty_like(q)
+        _check(self.lib.rope3d_oracle_qk_norm_rope_append_nvfp4(
+            _f64(q, "q"), _f64(k, "k"), _f64(v, "v"), _f64(q_out, "q_out"), B, N, D,
+            token_begin, token_end, frame_offset, T, H, W,
+            _f64(np.ascontiguousarray(q_norm_w, dtype=np.float64), "q_norm_w"),
+            _f64(np.ascontiguousarray(k_norm_w, dtype=np.float64), "k_norm_w"), eps,
+            _u8(k_codes, "k_codes"), _u8(v_codes, "v_codes"), _u8(k_scales, "k_scales"),
+            _u8(v_scales, "v_scales"), k_global, v_global, C, slot, n_t, n_h, n_w, theta,
+            schedule, pairing, cache_layout))
         return q_out
 
     def max_threads(self) -> int:

@@ -477,7 +477,7 @@ int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t
  * Quantize-on-append: K and V rows go to the cache as FP8 E4M3 codes with one fp32
  * scale per (token, head).  The scale is a power of two, as in the OCP microscaling
  * formats: the smallest 2^e (e >= -126) with amax(|x|) / 2^e <= 448 over the head's D
- * values (1 when the head is all zero), so the head's largest value lands in
+ * values (2^-126 when the head is all zero), so the head's largest value lands in
  * (224, 448] and dividing by the scale is exact.  Codes are E4M3(x / scale) rounded to
  * nearest, ties to the even code, saturating at +-448.  A reader recovers
  * x ~ value(code) * scale.  The pages name
@@ -603,6 +603,149 @@ int rope3d_oracle_qk_norm_rope_append_fp8(
                 rope3d_oracle_quantize_head_e4m3(head, D, k_codes + code_off, k_scale + scale_off);
                 for (int64_t e = 0; e < D; ++e) head[e] = (float)v_row[n * D + e];
                 rope3d_oracle_quantize_head_e4m3(head, D, v_codes + code_off, v_scale + scale_off);
+            }
+        }
+    }
+    free(k_row);
+    free(v_row);
+    free(head);
+    return rc;
+}
+
+/* ------------------------------------------------------------------ NVFP4 KV cache
+ *
+ * Quantize-on-append into NVFP4, the Blackwell 4-bit format the LongLive-2.0 abstract
+ * names for its KV cache (the pages give no further detail; this is the format as
+ * NVIDIA defines it): each block of 16 consecutive elements of a head holds 16 E2M1
+ * codes and one E4M3 block scale S; a per-tensor fp32 scale g (the caller's, one for K
+ * and one for V) sits above the block scales.  A reader recovers
+ * x ~ value(code) * value(S) * g.  This build's rounding recipe, in fp32:
+ *   S = E4M3(amax / (6 g))            amax = largest |x| in the block, 6 = E2M1's largest;
+ *   r = 1 / (value(S) g)  (0 if S is zero);
+ *   code = E2M1(x r)                   round to nearest, ties to the even code, saturating;
+ * every division, product and reciprocal a single fp32 operation rounded to nearest.
+ * Codes are packed two per byte, element 2j in the low nibble.
+ *
+ * E2M1: sign bit, 2 exponent bits with bias 1, 1 mantissa bit; exponent field 0 is
+ * subnormal (m/2); the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinity, no NaN.
+ */
+double rope3d_oracle_e2m1_value(int code)
+{
+    int sign = (code >> 3) & 1;
+    int e = (code >> 1) & 3;
+    int m = code & 1;
+    double v = e == 0 ? (double)m / 2.0 : ldexp(1.0 + (double)m / 2.0, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest E2M1 code of x (finite), ties to the even code, saturating at +-6; found by
+ * scanning the 8 non-negative codes in increasing order. */
+int rope3d_oracle_e2m1_encode(float x)
+{
+    int sign = signbit(x) ? 0x8 : 0;
+    double a = fabs((double)x);
+    if (a >= 6.0) return sign | 0x7;
+    int best = 0;
+    for (int c = 0; c < 7; ++c) {
+        double lo = rope3d_oracle_e2m1_value(c);
+        double hi = rope3d_oracle_e2m1_value(c + 1);
+        if (a >= lo && a <= hi) {
+            double dlo = a - lo, dhi = hi - a;
+            if (dlo < dhi) best = c;
+            else if (dhi < dlo) best = c + 1;
+            else best = (c % 2 == 0) ? c : c + 1;  /* tie: even mantissa */
+            break;
+        }
+    }
+    return sign | best;
+}
+
+/* One block of n (even) fp32 values -> n/2 code bytes and its E4M3 scale byte. */
+void rope3d_oracle_quantize_block_nvfp4(const float* x, int64_t n, float g,
+                                        unsigned char* codes, unsigned char* scale)
+{
+    float amax = 0.0f;
+    for (int64_t e = 0; e < n; ++e) {
+        float a = fabsf(x[e]);
+        if (a > amax) amax = a;
+    }
+    float c = 6.0f * g;
+    float sf = amax / c;
+    int S = rope3d_oracle_e4m3_encode(sf);
+    float sv = (float)rope3d_oracle_e4m3_value(S);
+    float r = sv > 0.0f ? 1.0f / (sv * g) : 0.0f;
+    for (int64_t e = 0; e < n; e += 2) {
+        float lo = x[e] * r;
+        float hi = x[e + 1] * r;
+        codes[e / 2] = (unsigned char)(rope3d_oracle_e2m1_encode(lo) |
+                                       (rope3d_oracle_e2m1_encode(hi) << 4));
+    }
+    *scale = (unsigned char)S;
+}
+
+/*
+ * The whole step with an NVFP4 cache.  q_out is returned in fp64 as above; the caches
+ * are code bytes [B][cache_tokens][N][D/2] (token-major) or [B][N][cache_tokens][D/2]
+ * (head-major) and the block scales E4M3 bytes [B][cache_tokens][N][D/16] or
+ * [B][N][cache_tokens][D/16].  K is quantized from its fp32 rounding, V exactly.
+ */
+int rope3d_oracle_qk_norm_rope_append_nvfp4(
+    const double* q, const double* k, const double* v, double* q_out,
+    int64_t B, int64_t N, int64_t D,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset,
+    int64_t T, int64_t H, int64_t W,
+    const double* q_norm_w, const double* k_norm_w, double eps,
+    unsigned char* k_codes, unsigned char* v_codes, unsigned char* k_scales,
+    unsigned char* v_scales, float k_global, float v_global,
+    int64_t cache_tokens, int64_t slot,
+    int n_t, int n_h, int n_w, double theta, int schedule, int pairing, int cache_layout)
+{
+    int rc = check_common(N, D, n_t, n_h, n_w, token_begin, token_end, frame_offset, T, H, W);
+    if (rc != ORACLE_OK) return rc;
+    if (B <= 0 || cache_tokens <= 0 || slot < 0 || D % 16 != 0) return ORACLE_EINVAL;
+    if (token_end - token_begin > cache_tokens) return ORACLE_EINVAL;
+    if (!(k_global > 0.0f) || !(v_global > 0.0f) || isinf(k_global) || isinf(v_global))
+        return ORACLE_EINVAL;
+    if (cache_layout != ORACLE_CACHE_TOKEN_MAJOR && cache_layout != ORACLE_CACHE_HEAD_MAJOR)
+        return ORACLE_EINVAL;
+    double inv[512];
+    rc = rope3d_oracle_inv_freq(n_t, n_h, n_w, theta, schedule, inv);
+    if (rc != ORACLE_OK) return rc;
+    int64_t n_tok = token_end - token_begin;
+    int64_t dim = N * D;
+    double* k_row = (double*)malloc((size_t)dim * sizeof(double));
+    double* v_row = (double*)malloc((size_t)dim * sizeof(double));
+    float* head = (float*)malloc((size_t)D * sizeof(float));
+    if (k_row == NULL || v_row == NULL || head == NULL) {
+        free(k_row); free(v_row); free(head);
+        return ORACLE_EINVAL;
+    }
+    for (int64_t b = 0; b < B && rc == ORACLE_OK; ++b) {
+        for (int64_t r = 0; r < n_tok; ++r) {
+            int64_t i = token_begin + r;
+            int64_t row = rope3d_oracle_cache_row(i, slot, cache_tokens);
+            int64_t in_off = (b * n_tok + r) * dim;
+            rc = rope3d_oracle_token_pairing(q + in_off, k + in_off, v + in_off, N, D, i,
+                                             frame_offset, T, H, W, q_norm_w, k_norm_w, eps,
+                                             slot, cache_tokens, n_t, n_h, n_w, inv, pairing,
+                                             q_out + in_off, k_row, v_row, NULL);
+            if (rc != ORACLE_OK) break;
+            for (int64_t n = 0; n < N; ++n) {
+                int64_t head_off = cache_layout == ORACLE_CACHE_TOKEN_MAJOR
+                                       ? (b * cache_tokens + row) * N + n
+                                       : (b * N + n) * cache_tokens + row;
+                for (int64_t blk = 0; blk < D / 16; ++blk) {
+                    int64_t code_off = head_off * (D / 2) + blk * 8;
+                    int64_t scale_off = head_off * (D / 16) + blk;
+                    for (int64_t e = 0; e < 16; ++e)
+                        head[e] = (float)k_row[n * D + blk * 16 + e];
+                    rope3d_oracle_quantize_block_nvfp4(head, 16, k_global, k_codes + code_off,
+                                                       k_scales + scale_off);
+                    for (int64_t e = 0; e < 16; ++e)
+                        head[e] = (float)v_row[n * D + blk * 16 + e];
+                    rope3d_oracle_quantize_block_nvfp4(head, 16, v_global, v_codes + code_off,
+                                                       v_scales + scale_off);
+                }
             }
         }
     }

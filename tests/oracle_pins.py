@@ -634,6 +634,107 @@ def check_fp8_step_matches_layout_step(orc):
                     assert np.array_equal(vc[idx], ev) and vs[idx] == esv
 
 
+# ---------------------------------------------------------------- NVFP4 cache
+
+E2M1_MAGNITUDES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]  # the format's 8 magnitudes
+
+
+def check_e2m1_closed_forms(orc):
+    """E2M1 (sign, 2 exponent bits with bias 1, 1 mantissa bit): codes 0..7 are the
+    magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 and codes 8..15 their negatives; every value
+    encodes to itself; midpoints go to the even code; magnitudes from 6 up saturate to
+    code 7; just off a midpoint goes to the nearer value; -0 keeps its sign."""
+    for c in range(16):
+        mag = E2M1_MAGNITUDES[c & 7]
+        assert orc.e2m1_value(c) == (-mag if c & 8 else mag), c
+        assert orc.e2m1_encode(float(orc.e2m1_value(c))) == (c if c != 8 else 8)
+    ties = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6}
+    for x, c in ties.items():
+        assert orc.e2m1_encode(x) == c, x
+        assert orc.e2m1_encode(-x) == c | 8, -x
+        lo, hi = np.nextafter(np.float32(x), np.float32(0)), np.nextafter(np.float32(x), np.float32(9))
+        assert orc.e2m1_encode(float(lo)) == E2M1_MAGNITUDES.index(max(m for m in E2M1_MAGNITUDES if m < x))
+        assert orc.e2m1_encode(float(hi)) == E2M1_MAGNITUDES.index(min(m for m in E2M1_MAGNITUDES if m > x))
+    for x in (6.0, 6.5, 7.0, 1e30):
+        assert orc.e2m1_encode(x) == 7 and orc.e2m1_encode(-x) == 15
+    assert orc.e2m1_encode(-0.0) == 8 and orc.e2m1_encode(0.0) == 0
+    assert orc.e2m1_encode(-0.2) == 8  # rounds to a negative zero
+
+
+def check_nvfp4_block_worked_example(orc):
+    """The block 0, 1, ..., 15 worked by hand: amax 15, S = E4M3(15 / 6 = 2.5) = 0x42
+    (1.25 * 2^1, exact), r = fp32(1 / 2.5), and x r = 0, 0.4, ..., 6.0 rounds to
+    0, 0.5, 1, 1, 1.5, 2, 2, 3, 3, 4, 4, 4, 4, 6, 6, 6, packed low nibble first."""
+    codes, scale = orc.quantize_block_nvfp4(np.arange(16, dtype=np.float32))
+    assert scale == 0x42
+    want = [0, 1, 2, 2, 3, 4, 4, 5, 5, 6, 6, 6, 6, 7, 7, 7]
+    assert list(codes) == [want[2 * j] | (want[2 * j + 1] << 4) for j in range(8)]
+
+
+def check_nvfp4_block_quantizer(orc):
+    """Block scale and codes follow the recipe (S = E4M3(amax / (6 g)), codes =
+    E2M1(x / (value(S) g)) through an fp32 reciprocal); every value is recovered within
+    half an E2M1 step of value(S) g, except where amax / (value(S) g) exceeds 6 and the
+    largest values saturate; a zero block has scale 0 and zero codes; a power-of-two
+    global scale g = 2^k gives the same codes and scale for x 2^k."""
+    rng = _rng(43)
+    for g in (1.0, 0.25, 3.0):
+        for _ in range(6):
+            x = (rng.standard_normal(16) * rng.uniform(0.05, 20)).astype(np.float32)
+            codes, S = orc.quantize_block_nvfp4(x, g)
+            amax = np.float32(np.max(np.abs(x)))
+            assert S == orc.e4m3_encode(float(amax / np.float32(6.0 * g)))
+            sv = np.float32(orc.e4m3_value(S))
+            r = np.float32(1.0) / np.float32(sv * np.float32(g))
+            got = [(c >> 4 * (e & 1)) & 15 for e, c in enumerate(np.repeat(codes, 2))]
+            assert got == [orc.e2m1_encode(float(np.float32(xe) * r)) for xe in x]
+            deq = np.array([orc.e2m1_value(c) for c in got]) * float(sv) * g
+            y = np.abs(x.astype(np.float64)) / (float(sv) * g)
+            step = np.where(y < 2, 0.5, np.where(y < 4, 1.0, 2.0))
+            bound = np.where(y <= 6, 0.5 * step, y - 6) * float(sv) * g
+            assert np.all(np.abs(deq - x) <= bound * (1 + 1e-6) + 1e-30)
+    codes, S = orc.quantize_block_nvfp4(np.zeros(16, dtype=np.float32))
+    assert S == 0 and not codes.any()
+    x = (rng.standard_normal(16) * 3).astype(np.float32)
+    c1, s1 = orc.quantize_block_nvfp4(x, 1.0)
+    c2, s2 = orc.quantize_block_nvfp4(x * np.float32(8.0), 8.0)
+    assert np.array_equal(c1, c2) and s1 == s2
+
+
+def check_nvfp4_step_matches_layout_step(orc):
+    """The NVFP4-cache step leaves q_out as the plain step does and stores, per block of
+    16 elements of each (token, head), the block quantization of the plain step's K and V
+    values (rounded to fp32) with the K and V global scales."""
+    B, N, T, H, W, s, slot, C = 1, 2, 3, 4, 6, 3, 100, 144
+    tb, te = 5, 60
+    kg, vg = 0.75, 2.0
+    q, k, v, wq, wk = _step_inputs(33, B, te - tb, N)
+    for pairing in (0, 1):
+        for layout in (0, 1):
+            shape = (B, C, N, D) if layout == 0 else (B, N, C, D)
+            kf, vf = np.zeros(shape), np.zeros(shape)
+            q0 = orc.qk_norm_rope_append_layout(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kf, vf,
+                                                slot, pairing, layout)
+            kc = np.zeros(shape[:3] + (D // 2,), dtype=np.uint8)
+            vc = np.zeros_like(kc)
+            ks = np.zeros(shape[:3] + (D // 16,), dtype=np.uint8)
+            vs = np.zeros_like(ks)
+            q1 = orc.qk_norm_rope_append_nvfp4(q, k, v, tb, te, s, T, H, W, wq, wk, 1e-6, kc, vc,
+                                               ks, vs, slot, kg, vg, pairing, layout)
+            assert np.array_equal(q0, q1)
+            for r in (0, 20, te - tb - 1):
+                row = (slot + tb + r) % C
+                for n in range(N):
+                    idx = (0, row, n) if layout == 0 else (0, n, row)
+                    for blk in range(D // 16):
+                        sl = slice(16 * blk, 16 * blk + 16)
+                        ek, esk = orc.quantize_block_nvfp4(kf[idx][sl], kg)
+                        ev, esv = orc.quantize_block_nvfp4(vf[idx][sl], vg)
+                        assert np.array_equal(kc[idx][8 * blk:8 * blk + 8], ek)
+                        assert np.array_equal(vc[idx][8 * blk:8 * blk + 8], ev)
+                        assert ks[idx][blk] == esk and vs[idx][blk] == esv
+
+
 def check_sp_head_scatter_is_whole_step_split_by_heads(orc):
     """Algorithm 3 steps 3-5 with the all-to-all folded in: ranks with uneven token
     ranges, each storing every head at its owner, together leave in owner r exactly the

@@ -10,6 +10,22 @@ import oracle
 from oracle_pins import ALL_CHECKS
 
 MUTANTS = {
+    "e2m1_ties_to_odd": ("            else best = (c % 2 == 0) ? c : c + 1;  /* tie: even mantissa */\n"
+                         "            break;\n        }\n    }\n    return sign | best;\n}\n\n/* One block",
+                         "            else best = (c % 2 == 0) ? c + 1 : c;\n"
+                         "            break;\n        }\n    }\n    return sign | best;\n}\n\n/* One block"),
+    "e2m1_no_saturation": ("if (a >= 6.0) return sign | 0x7;", "if (a >= 8.0) return sign | 0x7;"),
+    "nvfp4_scale_over_4": ("float c = 6.0f * g;", "float c = 4.0f * g;"),
+    "nvfp4_nibbles_swapped": ("codes[e / 2] = (unsigned char)(rope3d_oracle_e2m1_encode(lo) |\n"
+                              "                                       (rope3d_oracle_e2m1_encode(hi) << 4));",
+                              "codes[e / 2] = (unsigned char)(rope3d_oracle_e2m1_encode(hi) |\n"
+                              "                                       (rope3d_oracle_e2m1_encode(lo) << 4));"),
+    "nvfp4_one_scale_per_head": ("int64_t scale_off = head_off * (D / 16) + blk;",
+                                 "int64_t scale_off = head_off * (D / 16);"),
+    "nvfp4_v_uses_k_global": ("rope3d_oracle_quantize_block_nvfp4(head, 16, v_global, v_codes + code_off,",
+                              "rope3d_oracle_quantize_block_nvfp4(head, 16, k_global, v_codes + code_off,"),
+    "nvfp4_reciprocal_ignores_global": ("float r = sv > 0.0f ? 1.0f / (sv * g) : 0.0f;",
+                                        "float r = sv > 0.0f ? 1.0f / sv : 0.0f;"),
     "rotate_real_sign": ("y[n * head_dim + 2 * j] = a * c - b * s;",
                          "y[n * head_dim + 2 * j] = a * c + b * s;"),
     "rotate_imag_transposed": ("y[n * head_dim + 2 * j + 1] = a * s + b * c;",
