@@ -620,7 +620,8 @@ int rope3d_oracle_qk_norm_rope_append_fp8(
  * codes and one E4M3 block scale S; a per-tensor fp32 scale g (the caller's, one for K
  * and one for V) sits above the block scales.  A reader recovers
  * x ~ value(code) * value(S) * g.  This build's rounding recipe, in fp32:
- *   S = E4M3(amax / (6 g))            amax = largest |x| in the block, 6 = E2M1's largest;
+ *   k = 1 / (6 g)                      per tensor; 6 = E2M1's largest magnitude;
+ *   S = E4M3(amax k)                   amax = largest |x| in the block;
  *   r = 1 / (value(S) g)  (0 if S is zero);
  *   code = E2M1(x r)                   round to nearest, ties to the even code, saturating;
  * every division, product and reciprocal a single fp32 operation rounded to nearest.
@@ -669,8 +670,8 @@ void rope3d_oracle_quantize_block_nvfp4(const float* x, int64_t n, float g,
         float a = fabsf(x[e]);
         if (a > amax) amax = a;
     }
-    float c = 6.0f * g;
-    float sf = amax / c;
+    float k = 1.0f / (6.0f * g);
+    float sf = amax * k;
     int S = rope3d_oracle_e4m3_encode(sf);
     float sv = (float)rope3d_oracle_e4m3_value(S);
     float r = sv > 0.0f ? 1.0f / (sv * g) : 0.0f;

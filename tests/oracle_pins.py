@@ -662,8 +662,9 @@ def check_e2m1_closed_forms(orc):
 
 
 def check_nvfp4_block_worked_example(orc):
-    """The block 0, 1, ..., 15 worked by hand: amax 15, S = E4M3(15 / 6 = 2.5) = 0x42
-    (1.25 * 2^1, exact), r = fp32(1 / 2.5), and x r = 0, 0.4, ..., 6.0 rounds to
+    """The block 0, 1, ..., 15 worked by hand: amax 15, 15 fp32(1/6) rounds to 2.5 in
+    fp32, S = E4M3(2.5) = 0x42 (1.25 * 2^1, exact), r = fp32(1 / 2.5), and
+    x r = 0, 0.4, ..., 6.0 rounds to
     0, 0.5, 1, 1, 1.5, 2, 2, 3, 3, 4, 4, 4, 4, 6, 6, 6, packed low nibble first."""
     codes, scale = orc.quantize_block_nvfp4(np.arange(16, dtype=np.float32))
     assert scale == 0x42
@@ -672,7 +673,7 @@ def check_nvfp4_block_worked_example(orc):
 
 
 def check_nvfp4_block_quantizer(orc):
-    """Block scale and codes follow the recipe (S = E4M3(amax / (6 g)), codes =
+    """Block scale and codes follow the recipe (S = E4M3(amax fp32(1 / (6 g))), codes =
     E2M1(x / (value(S) g)) through an fp32 reciprocal); every value is recovered within
     half an E2M1 step of value(S) g, except where amax / (value(S) g) exceeds 6 and the
     largest values saturate; a zero block has scale 0 and zero codes; a power-of-two
@@ -683,7 +684,8 @@ def check_nvfp4_block_quantizer(orc):
             x = (rng.standard_normal(16) * rng.uniform(0.05, 20)).astype(np.float32)
             codes, S = orc.quantize_block_nvfp4(x, g)
             amax = np.float32(np.max(np.abs(x)))
-            assert S == orc.e4m3_encode(float(amax / np.float32(6.0 * g)))
+            k = np.float32(1.0) / np.float32(6.0 * g)
+            assert S == orc.e4m3_encode(float(amax * k))
             sv = np.float32(orc.e4m3_value(S))
             r = np.float32(1.0) / np.float32(sv * np.float32(g))
             got = [(c >> 4 * (e & 1)) & 15 for e, c in enumerate(np.repeat(codes, 2))]

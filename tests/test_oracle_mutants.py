@@ -15,7 +15,7 @@ MUTANTS = {
                          "            else best = (c % 2 == 0) ? c + 1 : c;\n"
                          "            break;\n        }\n    }\n    return sign | best;\n}\n\n/* One block"),
     "e2m1_no_saturation": ("if (a >= 6.0) return sign | 0x7;", "if (a >= 8.0) return sign | 0x7;"),
-    "nvfp4_scale_over_4": ("float c = 6.0f * g;", "float c = 4.0f * g;"),
+    "nvfp4_scale_over_4": ("float k = 1.0f / (6.0f * g);", "float k = 1.0f / (4.0f * g);"),
     "nvfp4_nibbles_swapped": ("codes[e / 2] = (unsigned char)(rope3d_oracle_e2m1_encode(lo) |\n"
                               "                                       (rope3d_oracle_e2m1_encode(hi) << 4));",
                               "codes[e / 2] = (unsigned char)(rope3d_oracle_e2m1_encode(hi) |\n"
