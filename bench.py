@@ -65,7 +65,7 @@ def parse_args(argv=None):
                     help="pairing of a head's elements (half: rotate_half, as in M-RoPE)")
     ap.add_argument("--cache-layout", choices=["token", "head"], default="token",
                     help="KV cache [B][C][N][D] (token) or [B][N][C][D] (head)")
-    ap.add_argument("--cache-dtype", choices=["same", "fp8"], default="same",
+    ap.add_argument("--cache-dtype", choices=["same", "fp8", "nvfp4"], default="same",
                     help="KV cache in the input dtype or FP8 E4M3 codes with per-head scales")
     ap.add_argument("--path", choices=["auto", "registers", "tma"], default="auto",
                     help="kernel path of the fused step (auto: the bulk-copy ring when it "
@@ -283,6 +283,10 @@ def run_ours(args, dist: Dist):
         # element plus one fp32 scale per head each
         e = w.elem_bytes
         bytes_per_launch = w.B * n * (w.dim * (4 * e + 2) + 2 * 4 * w.N)
+    elif args.cache_dtype == "nvfp4":
+        # K and V cache rows half a byte per element plus one E4M3 byte per 16 elements
+        e = w.elem_bytes
+        bytes_per_launch = w.B * n * (w.dim * 4 * e + 2 * (w.dim // 2 + w.dim // 16))
 
     host = make_inputs(w, seed_offset=dist.rank)
     wq, wk = wl.norm_weights(w.seed, w.dim)
@@ -302,10 +306,16 @@ def run_ours(args, dist: Dist):
     cache_shape = ((w.B, w.cache_tokens, w.N, wl.HEAD_DIM) if args.cache_layout == "token"
                    else (w.B, w.N, w.cache_tokens, wl.HEAD_DIM))
     fp8 = args.cache_dtype == "fp8"
-    k_cache = torch.zeros(cache_shape, dtype=torch.uint8 if fp8 else tdt, device=device)
-    v_cache = torch.zeros(cache_shape, dtype=torch.uint8 if fp8 else tdt, device=device)
-    k_scale = torch.zeros(cache_shape[:3], dtype=torch.float32, device=device) if fp8 else None
-    v_scale = torch.zeros(cache_shape[:3], dtype=torch.float32, device=device) if fp8 else None
+    fp4 = args.cache_dtype == "nvfp4"
+    if fp4:
+        cache_shape = cache_shape[:3] + (wl.HEAD_DIM // 2,)
+    quant = fp8 or fp4
+    k_cache = torch.zeros(cache_shape, dtype=torch.uint8 if quant else tdt, device=device)
+    v_cache = torch.zeros(cache_shape, dtype=torch.uint8 if quant else tdt, device=device)
+    sshape = cache_shape[:3] + ((wl.HEAD_DIM // 16,) if fp4 else ())
+    sdtype = torch.uint8 if fp4 else torch.float32
+    k_scale = torch.zeros(sshape, dtype=sdtype, device=device) if quant else None
+    v_scale = torch.zeros(sshape, dtype=sdtype, device=device) if quant else None
     max_t = max(c.frame_offset for c in w.chunks) + w.T
     tables = rope3d.rope3d_tables_init(max_t=max_t, max_h=w.H, max_w=w.W)
     stream = torch.cuda.current_stream(device)
@@ -315,7 +325,7 @@ def run_ours(args, dist: Dist):
 
     P = args.sp
     if P:
-        if w.N % P or n % P or fp8 or args.pairing != "adjacent":
+        if w.N % P or n % P or quant or args.pairing != "adjacent":
             raise SystemExit("--sp needs heads and tokens divisible by SP, adjacent pairing "
                              "and a same-dtype cache")
         hl = w.N // P
@@ -349,7 +359,7 @@ def run_ours(args, dist: Dist):
                     rope3d.rope3d_qk_norm_rope_append_ex(
                         q, k, v, q_out[ci], chunk.token_begin, chunk.token_end,
                         chunk.frame_offset, w.T, w.H, w.W, wq_d, wk_d, w.eps, k_cache, v_cache,
-                        chunk.slot, tables, trig, pairing, layout, k_scale, v_scale, stream)
+                        chunk.slot, tables, trig, pairing, layout, k_scale, v_scale, stream=stream)
                 if events is not None:
                     events[2 * j + 1].record(stream)
                 j += 1

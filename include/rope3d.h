@@ -110,6 +110,22 @@ extern "C" {
  *               format; E4M3 with per-head scales is this library's choice.) */
 #define ROPE3D_CACHE_SAME 0
 #define ROPE3D_CACHE_FP8_E4M3 1
+/*   NVFP4    -- quantize-on-append into NVFP4, the Blackwell 4-bit format (the
+ *               LongLive-2.0 abstract names NVFP4 for its KV cache): each block of 16
+ *               consecutive elements of a head holds 16 E2M1 codes (magnitudes 0, 0.5, 1,
+ *               1.5, 2, 3, 4, 6; two codes per byte, element 2j in the low nibble) and one
+ *               E4M3 block scale S, under a per-tensor fp32 scale g (options
+ *               nvfp4_k_global / nvfp4_v_global; 0 means 1).  In fp32, each operation
+ *               rounded to nearest:  k = 1 / (6 g) per tensor, S = E4M3(amax k) over the
+ *               block, r = 1 / (value(S) g) (0 if S is zero), code = E2M1(x r) rounded to
+ *               nearest even, saturating at 6.  A reader recovers x ~ value(code) value(S) g.  K is
+ *               quantized from its fp32 value after RMSNorm and RoPE, V from the input.
+ *               Caches hold D/2 = 64 bytes per (token, head): [B][cache_tokens][N][64]
+ *               (token-major) or [B][N][cache_tokens][64]; k_scale / v_scale then point to
+ *               BYTE arrays of D/16 = 8 E4M3 block scales per (token, head), laid out like
+ *               the cache rows ([B][cache_tokens][N][8] or [B][N][cache_tokens][8]),
+ *               8-byte aligned.  The register kernel runs it. */
+#define ROPE3D_CACHE_NVFP4 2
 
 /* Options of the _ex entry points; a NULL pointer or a zeroed struct gives the defaults
  * (adjacent pairing, token-major cache of the input dtype), i.e. the plain entry points'
@@ -119,9 +135,11 @@ typedef struct rope3d_options {
     int cache_layout;  /* ROPE3D_CACHE_TOKEN_MAJOR / _HEAD_MAJOR (fused step only)   */
     int cache_dtype;   /* ROPE3D_CACHE_SAME / _FP8_E4M3 (fused step only)            */
     int reserved0;     /* must be zero                                              */
-    float* k_scale;    /* FP8 cache: device fp32 scales of K (NULL otherwise)        */
-    float* v_scale;    /* FP8 cache: device fp32 scales of V (NULL otherwise)        */
-    int reserved[4];   /* must be zero                                              */
+    float* k_scale;    /* FP8: device fp32 scales of K; NVFP4: E4M3 block-scale bytes */
+    float* v_scale;    /* the same for V (NULL for a same-dtype cache)               */
+    float nvfp4_k_global; /* NVFP4: per-tensor scale g of K (0 = 1; else must be 0)   */
+    float nvfp4_v_global; /* NVFP4: per-tensor scale g of V (0 = 1; else must be 0)   */
+    int reserved[2];   /* must be zero                                              */
 } rope3d_options;
 
 /* Opaque frequency configuration: split, theta, schedule, the fp32 inverse

@@ -185,54 +185,62 @@ using KernelFn = void (*)(const rope3d::Params);
 // and vectors per thread.  Pairing rotate_half uses even VPT only (slots come in twos);
 // the rotation-only mode writes no cache.
 
-template <typename T, int TRIG, int MODE, int PAIR, bool CFP8>
+template <typename T, int TRIG, int MODE, int PAIR, int CF>
 KernelFn pick_vpt(int vpt) {
     if constexpr (PAIR == rope3d::kPairHalf) {
         switch (vpt) {
-            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CFP8>;
-            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CFP8>;
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CF>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CF>;
             default: return nullptr;
         }
     } else {
         switch (vpt) {
-            case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE, PAIR, CFP8>;
-            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CFP8>;
-            case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR, CFP8>;
-            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CFP8>;
+            case 1: return rope3d::qk_norm_rope_kernel<T, 1, TRIG, MODE, PAIR, CF>;
+            case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CF>;
+            case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR, CF>;
+            case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CF>;
             default: return nullptr;
         }
     }
 }
 
-template <typename T, int MODE, int PAIR, bool CFP8>
+template <typename T, int MODE, int PAIR, int CF>
 KernelFn pick_trig(int trig, int vpt) {
-    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<T, rope3d::kTrigTable, MODE, PAIR, CFP8>(vpt)
-                                     : pick_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR, CFP8>(vpt);
+    return trig == ROPE3D_TRIG_TABLE ? pick_vpt<T, rope3d::kTrigTable, MODE, PAIR, CF>(vpt)
+                                     : pick_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR, CF>(vpt);
 }
 
-template <typename T, int MODE, bool CFP8>
+template <typename T, int MODE, int CF>
 KernelFn pick_pairing(int pairing, int trig, int vpt) {
-    return pairing == ROPE3D_PAIRING_HALF ? pick_trig<T, MODE, rope3d::kPairHalf, CFP8>(trig, vpt)
-                                          : pick_trig<T, MODE, rope3d::kPairAdjacent, CFP8>(trig, vpt);
+    return pairing == ROPE3D_PAIRING_HALF ? pick_trig<T, MODE, rope3d::kPairHalf, CF>(trig, vpt)
+                                          : pick_trig<T, MODE, rope3d::kPairAdjacent, CF>(trig, vpt);
+}
+
+template <typename T, int MODE>
+KernelFn pick_format(int cache_fmt, int pairing, int trig, int vpt) {
+    switch (cache_fmt) {
+        case rope3d::kCacheFp8: return pick_pairing<T, MODE, rope3d::kCacheFp8>(pairing, trig, vpt);
+        case rope3d::kCacheNvfp4:
+            return pick_pairing<T, MODE, rope3d::kCacheNvfp4>(pairing, trig, vpt);
+        default: return pick_pairing<T, MODE, rope3d::kCacheSame>(pairing, trig, vpt);
+    }
 }
 
 template <int MODE>
-KernelFn pick_kernel(int dtype, int trig, int pairing, bool fp8, int vpt) {
+KernelFn pick_kernel(int dtype, int trig, int pairing, int cache_fmt, int vpt) {
     if constexpr (MODE == rope3d::kModeFusedSP) {
         // head-scatter stores: adjacent pairing and same-dtype caches only
-        if (pairing != ROPE3D_PAIRING_ADJACENT || fp8) return nullptr;
+        if (pairing != ROPE3D_PAIRING_ADJACENT || cache_fmt != rope3d::kCacheSame) return nullptr;
         return dtype == ROPE3D_BF16
-                   ? pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent, false>(trig, vpt)
-                   : pick_trig<float, MODE, rope3d::kPairAdjacent, false>(trig, vpt);
+                   ? pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent, rope3d::kCacheSame>(trig, vpt)
+                   : pick_trig<float, MODE, rope3d::kPairAdjacent, rope3d::kCacheSame>(trig, vpt);
     } else if constexpr (MODE == rope3d::kModeApply) {
-        return dtype == ROPE3D_BF16 ? pick_pairing<__nv_bfloat16, MODE, false>(pairing, trig, vpt)
-                                    : pick_pairing<float, MODE, false>(pairing, trig, vpt);
+        return dtype == ROPE3D_BF16
+                   ? pick_pairing<__nv_bfloat16, MODE, rope3d::kCacheSame>(pairing, trig, vpt)
+                   : pick_pairing<float, MODE, rope3d::kCacheSame>(pairing, trig, vpt);
     } else {
-        if (dtype == ROPE3D_BF16)
-            return fp8 ? pick_pairing<__nv_bfloat16, MODE, true>(pairing, trig, vpt)
-                       : pick_pairing<__nv_bfloat16, MODE, false>(pairing, trig, vpt);
-        return fp8 ? pick_pairing<float, MODE, true>(pairing, trig, vpt)
-                   : pick_pairing<float, MODE, false>(pairing, trig, vpt);
+        return dtype == ROPE3D_BF16 ? pick_format<__nv_bfloat16, MODE>(cache_fmt, pairing, trig, vpt)
+                                    : pick_format<float, MODE>(cache_fmt, pairing, trig, vpt);
     }
 }
 
@@ -381,6 +389,7 @@ size_t tma_layout(rope3d::Params& p, int teams, int stages, int warps_per_team) 
 int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int dev,
                      const DeviceInfo& info, cudaStream_t stream, bool forced, bool* launched) {
     *launched = false;
+    if (p.k_bscale != nullptr) return ROPE3D_OK;  // NVFP4 caches: register kernel only
     const Geometry g = geometry(N, dtype, pairing);
     if (g.tpr > rope3d::kTmaMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
     const int warps_per_team = g.tpr / 32;
@@ -449,11 +458,14 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int d
         smem = (size_t)2 * p.dim * sizeof(float);
         if (warps_per_team > 1) smem += (size_t)2 * teams * warps_per_team * sizeof(float2);
         if (MODE == rope3d::kModeFusedSP) smem += 3 * rope3d::kMaxRanks * sizeof(void*);
+        if (p.k_bscale != nullptr) smem += rope3d::kNvfp4TableFloats * sizeof(float);
     }
     if (smem > (size_t)info.max_smem_optin)
         return fail(ROPE3D_EINVAL, "N=%lld needs %zu bytes of shared memory (limit %d)",
                     (long long)N, smem, info.max_smem_optin);
-    KernelFn fn = pick_kernel<MODE>(dtype, trig, pairing, p.k_scale != nullptr, g.vpt);
+    const int cache_fmt = p.k_bscale != nullptr ? rope3d::kCacheNvfp4
+                          : p.k_scale != nullptr ? rope3d::kCacheFp8 : rope3d::kCacheSame;
+    KernelFn fn = pick_kernel<MODE>(dtype, trig, pairing, cache_fmt, g.vpt);
     if (fn == nullptr) return fail(ROPE3D_EINVAL, "no kernel for vpt=%d", g.vpt);
     int per_sm = 0;
     int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
@@ -511,18 +523,31 @@ int read_options(const rope3d_options* options, rope3d_options* out, bool with_c
                     o.cache_layout);
     if (!with_cache && o.cache_layout != ROPE3D_CACHE_TOKEN_MAJOR)
         return fail(ROPE3D_EINVAL, "options.cache_layout applies to the fused step only");
-    if (o.cache_dtype != ROPE3D_CACHE_SAME && o.cache_dtype != ROPE3D_CACHE_FP8_E4M3)
+    if (o.cache_dtype != ROPE3D_CACHE_SAME && o.cache_dtype != ROPE3D_CACHE_FP8_E4M3 &&
+        o.cache_dtype != ROPE3D_CACHE_NVFP4)
         return fail(ROPE3D_EINVAL, "options.cache_dtype %d is not a ROPE3D_CACHE_* value",
                     o.cache_dtype);
     if (!with_cache && (o.cache_dtype != ROPE3D_CACHE_SAME || o.k_scale || o.v_scale))
         return fail(ROPE3D_EINVAL, "options.cache_dtype and scales apply to the fused step only");
-    if (o.cache_dtype == ROPE3D_CACHE_FP8_E4M3) {
+    if (o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 || o.cache_dtype == ROPE3D_CACHE_NVFP4) {
         if (o.k_scale == nullptr || o.v_scale == nullptr)
-            return fail(ROPE3D_EINVAL, "an FP8 cache needs k_scale and v_scale");
-        if ((reinterpret_cast<uintptr_t>(o.k_scale) & 3u) || (reinterpret_cast<uintptr_t>(o.v_scale) & 3u))
-            return fail(ROPE3D_EALIGN, "k_scale and v_scale must be 4-byte aligned");
+            return fail(ROPE3D_EINVAL, "a quantized cache needs k_scale and v_scale");
+        const uintptr_t mask = o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 ? 3u : 7u;
+        if ((reinterpret_cast<uintptr_t>(o.k_scale) & mask) ||
+            (reinterpret_cast<uintptr_t>(o.v_scale) & mask))
+            return fail(ROPE3D_EALIGN, "k_scale and v_scale must be %d-byte aligned",
+                        (int)mask + 1);
     } else if (o.k_scale != nullptr || o.v_scale != nullptr) {
-        return fail(ROPE3D_EINVAL, "k_scale / v_scale are only for an FP8 cache");
+        return fail(ROPE3D_EINVAL, "k_scale / v_scale are only for a quantized cache");
+    }
+    if (o.cache_dtype == ROPE3D_CACHE_NVFP4) {
+        for (float g : {o.nvfp4_k_global, o.nvfp4_v_global})
+            if (!(g >= 0.0f) || !std::isfinite(g))
+                return fail(ROPE3D_EINVAL, "NVFP4 global scales must be finite and >= 0 (0 = 1)");
+        if (o.nvfp4_k_global == 0.0f) o.nvfp4_k_global = 1.0f;
+        if (o.nvfp4_v_global == 0.0f) o.nvfp4_v_global = 1.0f;
+    } else if (o.nvfp4_k_global != 0.0f || o.nvfp4_v_global != 0.0f) {
+        return fail(ROPE3D_EINVAL, "NVFP4 global scales are only for an NVFP4 cache");
     }
     if (o.reserved0 != 0) return fail(ROPE3D_EINVAL, "options.reserved0 must be zero");
     for (int r : o.reserved)
@@ -538,6 +563,15 @@ void fill_layout(rope3d::Params& p, int64_t N, int dtype, const rope3d_options& 
     p.vph_log2 = vph == 16 ? 4 : 5;
     p.k_scale = o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 ? o.k_scale : nullptr;
     p.v_scale = o.cache_dtype == ROPE3D_CACHE_FP8_E4M3 ? o.v_scale : nullptr;
+    const bool fp4 = o.cache_dtype == ROPE3D_CACHE_NVFP4;
+    p.k_bscale = fp4 ? reinterpret_cast<uint8_t*>(o.k_scale) : nullptr;
+    p.v_bscale = fp4 ? reinterpret_cast<uint8_t*>(o.v_scale) : nullptr;
+    p.k_global = fp4 ? o.nvfp4_k_global : 1.0f;
+    p.v_global = fp4 ? o.nvfp4_v_global : 1.0f;
+    // k = fp32(1 / fp32(6 g)), as the format's rounding recipe defines it
+    const float six_k = 6.0f * p.k_global, six_v = 6.0f * p.v_global;
+    p.k_inv6g = 1.0f / six_k;
+    p.v_inv6g = 1.0f / six_v;
 }
 
 int check_tables_device(const rope3d_tables* tables, int dev) {
@@ -771,9 +805,11 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
     const size_t row = (size_t)N * D * esz;
     const size_t act = (size_t)B * (size_t)(token_end - token_begin) * row;
     const bool fp8 = opt.cache_dtype == ROPE3D_CACHE_FP8_E4M3;
-    const size_t cache = (size_t)B * (size_t)cache_tokens * (size_t)N * D * (fp8 ? 1 : esz);
-    if (fp8) {
-        const size_t sc = (size_t)B * (size_t)cache_tokens * (size_t)N * sizeof(float);
+    const bool fp4 = opt.cache_dtype == ROPE3D_CACHE_NVFP4;
+    const size_t heads = (size_t)B * (size_t)cache_tokens * (size_t)N;
+    const size_t cache = fp4 ? heads * D / 2 : fp8 ? heads * D : heads * D * esz;
+    if (fp8 || fp4) {
+        const size_t sc = heads * (fp8 ? sizeof(float) : (size_t)D / 16);
         const void* bufs[6] = {q, k, v, q_out, k_cache, v_cache};
         const size_t sizes[6] = {act, act, act, act, cache, cache};
         for (int b2 = 0; b2 < 6; ++b2)
@@ -825,7 +861,8 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
         if (launched) g_last_path = ROPE3D_PATH_TMA;
         if (rc != ROPE3D_OK || launched) return rc;
         if (path == ROPE3D_PATH_TMA)
-            return fail(ROPE3D_EINVAL, "the TMA path does not fit N=%lld", (long long)N);
+            return fail(ROPE3D_EINVAL, "the TMA path does not take this call (N=%lld%s)",
+                        (long long)N, p.k_bscale ? ", NVFP4 cache" : "");
     }
     rc = launch<rope3d::kModeFused>(p, N, dtype, trig, opt.pairing, dev, info, stream);
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;

@@ -44,6 +44,8 @@ constexpr int kTmaMaxBlockThreads = 320;  // ring kernel: one block per SM, up t
 // all-to-all folded into the step): each head goes to the destination rank that owns it.
 enum Mode : int { kModeFused = 0, kModeApply = 1, kModeFusedSP = 2 };
 constexpr int kMaxRanks = 8;  // head-scatter destinations (one node)
+// KV-cache element formats of the fused step
+enum CacheFmt : int { kCacheSame = 0, kCacheFp8 = 1, kCacheNvfp4 = 2 };
 enum Trig : int { kTrigTable = 0, kTrigOnTheFly = 1 };
 // Pairing of a head's elements into complex pairs: adjacent (2j, 2j+1) -- the complex
 // view of Wan2.1 -- or rotate_half (j, j + 64), the cos/sin form of M-RoPE.
@@ -91,6 +93,10 @@ struct Params {
     int vph_log2;          // log2 of the 16-byte vectors per head
     float* k_scale;        // FP8 caches: per (token, head) scales, laid out like the cache rows
     float* v_scale;
+    uint8_t* k_bscale;     // NVFP4 caches: E4M3 scale per 16-element block, laid out like the rows
+    uint8_t* v_bscale;
+    float k_global, v_global;  // NVFP4 per-tensor scales g
+    float k_inv6g, v_inv6g;    // fp32(1 / fp32(6 g))
     // head-scatter destinations (kModeFusedSP): rank r owns heads [r*sp_heads, (r+1)*sp_heads)
     int sp_ranks;
     int sp_heads;          // heads per rank
@@ -512,10 +518,97 @@ __device__ __forceinline__ uint32_t vec_key(const uint4& v) {
 __device__ __forceinline__ uint32_t vec_key(const float4& v) {
     return fp8_key(fmaxf(max3f(fabsf(v.x), fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
 }
+// Largest magnitude of a vector of input elements (exact; bf16 magnitudes compare as
+// 16-bit integers).
+__device__ __forceinline__ float vec_abs_max(const uint4& v) {
+    uint32_t m = max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.z & 0x7FFF7FFFu);
+    m = max_u16x2(m, v.w & 0x7FFF7FFFu);
+    return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
+}
+__device__ __forceinline__ float vec_abs_max(const float4& v) {
+    return fmaxf(max3f(fabsf(v.x), fabsf(v.y), fabsf(v.z)), fabsf(v.w));
+}
 
 __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     // element a in the low byte (lower address)
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// ---------------------------------------------------------------- NVFP4 cache rows
+//
+// Each block of 16 consecutive elements of a head goes to the cache as 16 E2M1 codes
+// (two per byte, element 2j in the low nibble) with one E4M3 block scale S, under the
+// tensor's fp32 scale g: S = E4M3(amax * k) with k = 1 / (6 g), codes = E2M1(x * r) with
+// r = 1 / (value(S) g) (0 when S is zero), each operation one fp32 rounding to nearest.
+// r depends on S alone, so each block of threads tabulates it for the 256 codes once.
+// A block of 16 elements is 2 vectors (bf16) or 4 (fp32) held by as many neighbouring
+// lanes.
+
+constexpr int kNvfp4TableFloats = 512;  // r for the 256 codes, K then V
+
+// Value of a non-negative E4M3 code (exponent bias 7, 3 mantissa bits; field 0 is
+// subnormal m * 2^-9), built from its fields.
+__device__ __forceinline__ float e4m3_nonneg_value(uint32_t code) {
+    const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0x1p-9f;
+}
+
+__device__ __forceinline__ void fill_nvfp4_tables(const Params& p, float* s_r) {
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+        const float sv = e4m3_nonneg_value((uint32_t)c);
+        s_r[c] = sv > 0.0f ? __frcp_rn(__fmul_rn(sv, p.k_global)) : 0.0f;
+        s_r[256 + c] = sv > 0.0f ? __frcp_rn(__fmul_rn(sv, p.v_global)) : 0.0f;
+    }
+}
+
+struct Nvfp4Scale {
+    uint32_t code;  // E4M3 byte
+    float r;        // 1 / (value(S) g), or 0
+};
+
+__device__ __forceinline__ Nvfp4Scale nvfp4_scale(float amax, float inv6g, const float* s_r) {
+    Nvfp4Scale s;
+    s.code = e4m3x2(__fmul_rn(amax, inv6g), 0.0f) & 0xFFu;
+    s.r = s_r[s.code];
+    return s;
+}
+
+// E2M1 codes of 8 values in one 32-bit word, element 0 in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+    uint32_t r;
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        " mov.b32 %0, {b0, b1, b2, b3};\n}"
+        : "=r"(r)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+    return r;
+}
+
+// Store the codes of one vector at vector index vi of an NVFP4 cache (E/2 bytes per vector).
+__device__ __forceinline__ void store_fp4(void* cache, int64_t vi, const float (&v)[8], float r) {
+    const float2 r2 = make_float2(r, r);
+    const uint32_t c = e2m1x8(__fmul2_rn(make_float2(v[0], v[1]), r2),
+                              __fmul2_rn(make_float2(v[2], v[3]), r2),
+                              __fmul2_rn(make_float2(v[4], v[5]), r2),
+                              __fmul2_rn(make_float2(v[6], v[7]), r2));
+    __stcs(reinterpret_cast<unsigned int*>(cache) + vi, c);
+}
+__device__ __forceinline__ void store_fp4(void* cache, int64_t vi, const float (&v)[4], float r) {
+    const float2 r2 = make_float2(r, r);
+    const float2 z = make_float2(0.0f, 0.0f);
+    const uint32_t c = e2m1x8(__fmul2_rn(make_float2(v[0], v[1]), r2),
+                              __fmul2_rn(make_float2(v[2], v[3]), r2), z, z);
+    __stcs(reinterpret_cast<unsigned short*>(cache) + vi, (unsigned short)c);
+}
+
+// Maximum over the `lanes` neighbouring lanes that hold one block (1, 2 or 4).
+__device__ __forceinline__ float block_max(float x, int lanes) {
+    for (int off = 1; off < lanes; off <<= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+    return x;
 }
 
 // Store E codes of one vector at vector index vi of an FP8 cache (E bytes per vector);
@@ -578,11 +671,11 @@ __device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
 // Normalise, rotate and store this thread's vectors of one row: q_out, and in the fused
 // mode the K row into the cache.  With rotate_half pairing slots 2m and 2m+1 hold the two
 // halves of the same pairs (see slot_vec).  V goes to a same-dtype cache through
-// store_v_row; with an FP8 cache (CFP8) it is quantized here, beside K: the K values stay
+// store_v_row; with an FP8 or NVFP4 cache (CF) it is quantized here, beside K: the K values stay
 // fp32 until they are quantized, and the K and V keys of one head travel in one shuffle
 // word.  Every lane of the warp takes part in the head-wise maximum, whether its slots
 // hold vectors or not.
-template <typename T, int VPT, int PAIR, int MODE, bool CFP8>
+template <typename T, int VPT, int PAIR, int MODE, int CF>
 __device__ __forceinline__ void emit_row(
     const Params& p, int t, const RowPos& pos, int64_t row_vec,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -590,12 +683,14 @@ __device__ __forceinline__ void emit_row(
     float rq, float rk, const float* s_wq, const float* s_wk,
     const float (&cs)[PairCount<T, PAIR>::value], const float (&sn)[PairCount<T, PAIR>::value],
     typename VecTraits<T>::Vec* qo, typename VecTraits<T>::Vec* kc,
-    typename VecTraits<T>::Vec* vc) {
+    typename VecTraits<T>::Vec* vc, const float* s_r = nullptr) {
     using Tr = VecTraits<T>;
     constexpr int EPV = Tr::kElems;
     constexpr bool NORM = MODE == kModeFused;
-    constexpr bool QUANT = MODE == kModeFused && CFP8;
+    constexpr bool QUANT = MODE == kModeFused && CF == kCacheFp8;
+    constexpr bool QUANT4 = MODE == kModeFused && CF == kCacheNvfp4;
     constexpr int VPH = Tr::kVecsPerHead;
+    constexpr int VPB = 16 / EPV;  // vectors (lanes) per NVFP4 block
     if constexpr (PAIR == kPairAdjacent) {
 #pragma unroll
         for (int s = 0; s < VPT; ++s) {
@@ -624,6 +719,30 @@ __device__ __forceinline__ void emit_row(
                         __stcs(p.v_scale + si, sv.scale);
                     }
                 }
+            } else if constexpr (QUANT4) {
+                float o[EPV];
+                float ak = 0.0f, av = 0.0f;
+                if (valid) {
+                    norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
+                    ak = abs_max<EPV>(o);
+                    av = vec_abs_max(xv[s]);
+                }
+                ak = block_max(ak, VPB);
+                av = block_max(av, VPB);
+                if (valid) {
+                    const Nvfp4Scale sk = nvfp4_scale(ak, p.k_inv6g, s_r);
+                    const Nvfp4Scale sv = nvfp4_scale(av, p.v_inv6g, s_r + 256);
+                    const int64_t vi = cache_vec_index(p, pos, idx);
+                    float v[EPV];
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) v[e] = Tr::elem(xv[s], e);
+                    store_fp4(kc, vi, o, sk.r);
+                    store_fp4(vc, vi, v, sv.r);
+                    if ((idx & (VPB - 1)) == 0) {
+                        __stcs(reinterpret_cast<char*>(p.k_bscale + vi / VPB), (char)sk.code);
+                        __stcs(reinterpret_cast<char*>(p.v_bscale + vi / VPB), (char)sv.code);
+                    }
+                }
             } else if (MODE == kModeFused && valid) {
                 store_out(kc + cache_vec_index(p, pos, idx),
                           norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
@@ -647,7 +766,43 @@ __device__ __forceinline__ void emit_row(
                 if (valid)
                     norm_rotate_half_f<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV,
                                                 i_im * EPV, cs, sn, o_re, o_im);
-                if constexpr (CFP8) {
+                if constexpr (QUANT4) {
+                    // i_re and i_im lie in different blocks: each reduces over its own lanes
+                    float a_re = 0.0f, a_im = 0.0f, v_re = 0.0f, v_im = 0.0f;
+                    if (valid) {
+                        a_re = abs_max<EPV>(o_re);
+                        a_im = abs_max<EPV>(o_im);
+                        v_re = vec_abs_max(xv[s]);
+                        v_im = vec_abs_max(xv[s + 1]);
+                    }
+                    a_re = block_max(a_re, VPB);
+                    a_im = block_max(a_im, VPB);
+                    v_re = block_max(v_re, VPB);
+                    v_im = block_max(v_im, VPB);
+                    if (valid) {
+                        const int64_t vr = cache_vec_index(p, pos, i_re);
+                        const int64_t vm = cache_vec_index(p, pos, i_im);
+                        const Nvfp4Scale k_re = nvfp4_scale(a_re, p.k_inv6g, s_r);
+                        const Nvfp4Scale k_im = nvfp4_scale(a_im, p.k_inv6g, s_r);
+                        const Nvfp4Scale s_re = nvfp4_scale(v_re, p.v_inv6g, s_r + 256);
+                        const Nvfp4Scale s_im = nvfp4_scale(v_im, p.v_inv6g, s_r + 256);
+                        float v[EPV];
+                        store_fp4(kc, vr, o_re, k_re.r);
+                        store_fp4(kc, vm, o_im, k_im.r);
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) v[e] = Tr::elem(xv[s], e);
+                        store_fp4(vc, vr, v, s_re.r);
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) v[e] = Tr::elem(xv[s + 1], e);
+                        store_fp4(vc, vm, v, s_im.r);
+                        if ((i_re & (VPB - 1)) == 0) {
+                            __stcs(reinterpret_cast<char*>(p.k_bscale + vr / VPB), (char)k_re.code);
+                            __stcs(reinterpret_cast<char*>(p.k_bscale + vm / VPB), (char)k_im.code);
+                            __stcs(reinterpret_cast<char*>(p.v_bscale + vr / VPB), (char)s_re.code);
+                            __stcs(reinterpret_cast<char*>(p.v_bscale + vm / VPB), (char)s_im.code);
+                        }
+                    }
+                } else if constexpr (QUANT) {
                     uint32_t kk = 0, kv = 0;
                     if (valid) {
                         kk = fp8_key(fmaxf(abs_max<EPV>(o_re), abs_max<EPV>(o_im)));
@@ -756,7 +911,7 @@ __device__ __forceinline__ void emit_row_sp(
 
 // ---------------------------------------------------------------- register kernel
 
-template <typename T, int VPT, int TRIG, int MODE, int PAIR, bool CFP8>
+template <typename T, int VPT, int TRIG, int MODE, int PAIR, int CF>
 __global__ void __launch_bounds__(kMaxBlockThreads)
 qk_norm_rope_kernel(const Params p) {
     using Tr = VecTraits<T>;
@@ -764,13 +919,17 @@ qk_norm_rope_kernel(const Params p) {
     constexpr int NP = PairCount<T, PAIR>::value;
     constexpr bool FUSED = MODE != kModeApply;
     constexpr bool SP = MODE == kModeFusedSP;
-    static_assert(!SP || (PAIR == kPairAdjacent && !CFP8),
+    static_assert(!SP || (PAIR == kPairAdjacent && CF == kCacheSame),
                   "head-scatter stores: adjacent pairing, same-dtype caches");
 
-    // dynamic shared memory: [SP: destination table] [q, k norm weights] [team partials]
+    // dynamic shared memory: [SP: destination table | NVFP4: reciprocal tables]
+    // [q, k norm weights] [team partials]
+    constexpr bool FP4 = CF == kCacheNvfp4;
     extern __shared__ float4 smem4[];
     void** s_sp = reinterpret_cast<void**>(smem4);
-    float* s_wq = reinterpret_cast<float*>(smem4 + (SP ? 3 * kMaxRanks / 2 : 0));
+    float* s_r = reinterpret_cast<float*>(smem4);
+    float* s_wq = reinterpret_cast<float*>(
+        smem4 + (SP ? 3 * kMaxRanks / 2 : FP4 ? kNvfp4TableFloats / 4 : 0));
     float* s_wk = s_wq + (FUSED ? p.dim : 0);
     float2* s_part = reinterpret_cast<float2*>(s_wk + (FUSED ? p.dim : 0));
 
@@ -789,6 +948,7 @@ qk_norm_rope_kernel(const Params p) {
             for (int j = 0; j < 3 * kMaxRanks; ++j)
                 if (tid == j) s_sp[j] = p.sp_dst[j];  // constant indices into the parameters
         }
+        if constexpr (FP4) fill_nvfp4_tables(p, s_r);
         stage_weights(p, s_wq, s_wk);
         __syncthreads();
     }
@@ -829,7 +989,7 @@ qk_norm_rope_kernel(const Params p) {
         float rq = 1.0f, rk = 1.0f;
         if (FUSED) {
             if constexpr (SP) store_v_row_sp<T, VPT>(p, t, pos, xv, dst, s_sp);
-            else if constexpr (!CFP8) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
+            else if constexpr (CF == kCacheSame) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -840,8 +1000,8 @@ qk_norm_rope_kernel(const Params p) {
         if constexpr (SP)
             emit_row_sp<T, VPT>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
         else
-            emit_row<T, VPT, PAIR, MODE, CFP8>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq,
-                                               s_wk, cs, sn, qo, kc, vc);
+            emit_row<T, VPT, PAIR, MODE, CF>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq,
+                                             s_wk, cs, sn, qo, kc, vc, s_r);
     }
 }
 

@@ -189,8 +189,8 @@ qk_norm_rope_tma_kernel(const Params p) {
         const float rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         const int64_t row_vec = u * p.dim_vecs;
         if constexpr (!CFP8) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
-        emit_row<T, VPT, PAIR, kModeFused, CFP8>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq,
-                                                 s_wk, cs, sn, qo, kc, vc);
+        emit_row<T, VPT, PAIR, kModeFused, CFP8 ? kCacheFp8 : kCacheSame>(
+            p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq, s_wk, cs, sn, qo, kc, vc);
     }
 
     if (failed && t == 0) {

@@ -40,6 +40,7 @@ ROPE3D_CACHE_TOKEN_MAJOR = 0
 ROPE3D_CACHE_HEAD_MAJOR = 1
 ROPE3D_CACHE_SAME = 0
 ROPE3D_CACHE_FP8_E4M3 = 1
+ROPE3D_CACHE_NVFP4 = 2
 
 
 class rope3d_options(ctypes.Structure):
@@ -47,7 +48,8 @@ class rope3d_options(ctypes.Structure):
     _fields_ = [("pairing", ctypes.c_int), ("cache_layout", ctypes.c_int),
                 ("cache_dtype", ctypes.c_int), ("reserved0", ctypes.c_int),
                 ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
-                ("reserved", ctypes.c_int * 4)]
+                ("nvfp4_k_global", ctypes.c_float), ("nvfp4_v_global", ctypes.c_float),
+                ("reserved", ctypes.c_int * 2)]
 
 ROPE3D_SP_MAX_RANKS = 8
 
@@ -251,41 +253,52 @@ def rope3d_qk_norm_rope_append_ex(q, k, v, q_out, token_begin: int, token_end: i
                                   trig: int = ROPE3D_TRIG_TABLE,
                                   pairing: int = ROPE3D_PAIRING_ADJACENT,
                                   cache_layout: int = ROPE3D_CACHE_TOKEN_MAJOR,
-                                  k_scale=None, v_scale=None, stream=None) -> None:
-    """rope3d_qk_norm_rope_append with options; head-major caches are [B, N, C, 128].
-    Passing k_scale and v_scale (float32, [B, C, N] or [B, N, C]) selects the FP8 E4M3
-    cache: k_cache and v_cache are then uint8 code tensors."""
+                                  k_scale=None, v_scale=None, k_global: float = 0.0,
+                                  v_global: float = 0.0, stream=None) -> None:
+    """rope3d_qk_norm_rope_append with options; head-major caches are [B, N, C, ...].
+    Passing k_scale and v_scale selects a quantized cache (k_cache and v_cache are then
+    uint8 code tensors): float32 scales [B, C, N] / [B, N, C] for FP8 E4M3 (caches
+    [..., 128]); uint8 block scales [B, C, N, 8] / [B, N, C, 8] for NVFP4 (caches
+    [..., 64]) with per-tensor scales k_global, v_global (0 = 1)."""
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or q_out.shape != q.shape:
         raise ValueError("q, k, v and q_out must all be [B, n_tok, N, D]")
     B, n_tok, N, D = q.shape
+    quant = k_scale is not None or v_scale is not None
+    fp4 = quant and k_scale is not None and k_scale.dtype == torch.uint8
+    row = D // 2 if fp4 else D
     if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("k_cache and v_cache must have one 4-d shape")
     if cache_layout == ROPE3D_CACHE_HEAD_MAJOR:
         C = k_cache.shape[2]
-        ok = k_cache.shape[0] == B and k_cache.shape[1] == N and k_cache.shape[3] == D
+        ok = k_cache.shape[0] == B and k_cache.shape[1] == N and k_cache.shape[3] == row
     else:
         C = k_cache.shape[1]
-        ok = k_cache.shape[0] == B and k_cache.shape[2:] == q.shape[2:]
+        ok = k_cache.shape[0] == B and k_cache.shape[2] == N and k_cache.shape[3] == row
     if not ok:
         raise ValueError("cache shape does not match q and the cache layout")
     if n_tok != token_end - token_begin:
         raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
-    fp8 = k_scale is not None or v_scale is not None
     for name, t in (("k", k), ("v", v), ("q_out", q_out)) + (
-            () if fp8 else (("k_cache", k_cache), ("v_cache", v_cache))):
+            () if quant else (("k_cache", k_cache), ("v_cache", v_cache))):
         if t.dtype != q.dtype:
             raise TypeError(f"{name} must have q's dtype {q.dtype}")
     opts = rope3d_options(pairing, cache_layout)
-    if fp8:
+    if quant:
         if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8:
-            raise TypeError("an FP8 cache is uint8 codes")
+            raise TypeError("a quantized cache is uint8 codes")
         sshape = (B, C, N) if cache_layout == ROPE3D_CACHE_TOKEN_MAJOR else (B, N, C)
+        sdtype = torch.uint8 if fp4 else torch.float32
+        if fp4:
+            sshape = sshape + (D // 16,)
         for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
-            if t is None or t.dtype != torch.float32 or tuple(t.shape) != sshape:
-                raise ValueError(f"{name} must be float32 of shape {sshape}")
-        opts.cache_dtype = ROPE3D_CACHE_FP8_E4M3
+            if t is None or t.dtype != sdtype or tuple(t.shape) != sshape:
+                raise ValueError(f"{name} must be {sdtype} of shape {sshape}")
+        opts.cache_dtype = ROPE3D_CACHE_NVFP4 if fp4 else ROPE3D_CACHE_FP8_E4M3
         opts.k_scale = _dev_ptr(k_scale, "k_scale")
         opts.v_scale = _dev_ptr(v_scale, "v_scale")
+        if fp4:
+            opts.nvfp4_k_global = k_global
+            opts.nvfp4_v_global = v_global
     _check(load_library().rope3d_qk_norm_rope_append_ex(
         _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
         B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,

@@ -111,10 +111,12 @@ def test_options_struct_layout_matches_header(tmp_path):
         pytest.skip("needs gcc")
     src = tmp_path / "layout.c"
     src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "rope3d.h"\n'
-                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu", sizeof(rope3d_options),'
+                   'int main(void){printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu",'
+                   ' sizeof(rope3d_options),'
                    ' offsetof(rope3d_options, pairing), offsetof(rope3d_options, cache_layout),'
                    ' offsetof(rope3d_options, cache_dtype), offsetof(rope3d_options, k_scale),'
-                   ' offsetof(rope3d_options, v_scale), offsetof(rope3d_options, reserved));'
+                   ' offsetof(rope3d_options, v_scale), offsetof(rope3d_options, nvfp4_k_global),'
+                   ' offsetof(rope3d_options, nvfp4_v_global), offsetof(rope3d_options, reserved));'
                    ' return 0;}\n')
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
@@ -122,7 +124,8 @@ def test_options_struct_layout_matches_header(tmp_path):
     got = list(map(int, subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()))
     S = rope3d.rope3d_options
     assert got == [ctypes.sizeof(S), S.pairing.offset, S.cache_layout.offset,
-                   S.cache_dtype.offset, S.k_scale.offset, S.v_scale.offset, S.reserved.offset]
+                   S.cache_dtype.offset, S.k_scale.offset, S.v_scale.offset,
+                   S.nvfp4_k_global.offset, S.nvfp4_v_global.offset, S.reserved.offset]
 
 
 def test_sp_dest_struct_layout_matches_header(tmp_path):

@@ -191,7 +191,7 @@ def test_invalid_options_rejected():
     wq = torch.ones(256, device="cuda")
     tables = rope3d.rope3d_tables_init(max_t=6, max_h=4, max_w=6)
     reserved_set = rope3d.rope3d_options()
-    reserved_set.reserved[2] = 1
+    reserved_set.reserved[1] = 1
     for opts in (rope3d.rope3d_options(2, 0), rope3d.rope3d_options(0, 5),
                  rope3d.rope3d_options(0, 0, 7), rope3d.rope3d_options(0, 0, 0, 1),
                  reserved_set):
