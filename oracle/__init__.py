@@ -400,6 +400,41 @@ class Oracle:
                 k_dst[r][:, local, rows] = kc[:, rows, head]
                 v_dst[r][:, local, rows] = vc[:, rows, head]
 
+    # ---- QKV projection feeding the step (Algorithm 1/3 step 1, Section 3.4.1 item 3)
+
+    @staticmethod
+    def bf16_round(a):
+        return bf16_round(a)
+
+    @staticmethod
+    def qkv_project(x, w_qkv, b_qkv=None):
+        """q, k, v = QKV(x): x [B, n, dim_in] @ w_qkv.T + b_qkv, in fp64, with w_qkv
+        [3 dim, dim_in] holding the q rows, then the k rows, then the v rows (an
+        nn.Linear weight); each result is returned as [B, n, dim]."""
+        x = np.asarray(x, dtype=np.float64)
+        w = np.asarray(w_qkv, dtype=np.float64)
+        y = x @ w.T
+        if b_qkv is not None:
+            y = y + np.asarray(b_qkv, dtype=np.float64)
+        dim = w.shape[0] // 3
+        return y[..., :dim], y[..., dim:2 * dim], y[..., 2 * dim:]
+
+    def qkv_norm_rope_append(self, x, w_qkv, b_qkv, N, token_begin, token_end, frame_offset,
+                             T, H, W, q_norm_w, k_norm_w, eps, k_cache, v_cache, slot,
+                             round_bf16=True, **freq):
+        """Step 1 (the projection) then the step.  With round_bf16 the projected q, k, v
+        are rounded to bf16 first (round to nearest even), as a projection that stores
+        bf16 activations hands them on; the step then runs on those values."""
+        q, k, v = self.qkv_project(x, w_qkv, b_qkv)
+        if round_bf16:
+            q, k, v = (self.bf16_round(a) for a in (q, k, v))
+        B, n = q.shape[:2]
+        shape = (B, n, N, q.shape[-1] // N)
+        return self.qk_norm_rope_append_layout(
+            q.reshape(shape).copy(), k.reshape(shape).copy(), v.reshape(shape).copy(),
+            token_begin, token_end, frame_offset, T, H, W, q_norm_w, k_norm_w, eps, k_cache,
+            v_cache, slot, **freq)
+
     def apply_pairing(self, x, token_begin, token_end, frame_offset, T, H, W, pairing,
                       n_t=N_T, n_h=N_H, n_w=N_W, theta=THETA, schedule=0):
         B, n_tok, N, D = x.shape
@@ -408,6 +443,15 @@ class Oracle:
             _f64(x, "x"), _f64(out, "out"), B, N, D, token_begin, token_end, frame_offset,
             T, H, W, n_t, n_h, n_w, theta, schedule, pairing))
         return out
+
+
+def bf16_round(a):
+    """fp64 values rounded to the nearest bfloat16 (8 significant bits, ties to even,
+    the fp32 exponent range with its subnormal spacing 2^-133), returned as fp64."""
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)               # a = m 2^e with 0.5 <= |m| < 1
+    e = np.maximum(e, -125)          # below 2^-126 the spacing stays 2^-133
+    return np.ldexp(np.rint(np.ldexp(a, 8 - e)), e - 8)
 
 
 _default = None

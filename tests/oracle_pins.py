@@ -737,6 +737,65 @@ def check_nvfp4_step_matches_layout_step(orc):
                         assert ks[idx][blk] == esk and vs[idx][blk] == esv
 
 
+# ---------------------------------------------------------------- QKV projection
+
+def check_qkv_project_brute_force(orc):
+    """q, k, v = QKV(x) (Algorithm 1/3 step 1) as an nn.Linear: out[t][o] = sum_i x[t][i]
+    w[o][i] + b[o], with output rows [0, dim) -> q, [dim, 2 dim) -> k, [2 dim, 3 dim) -> v;
+    checked by explicit loops on a tiny case, with and without bias."""
+    rng = _rng(51)
+    B, n, din, dim = 2, 3, 5, 4
+    x = rng.standard_normal((B, n, din))
+    w = rng.standard_normal((3 * dim, din))
+    b = rng.standard_normal(3 * dim)
+    for bias in (b, None):
+        q, k, v = orc.qkv_project(x, w, bias)
+        for bb in range(B):
+            for t in range(n):
+                for o in range(3 * dim):
+                    acc = 0.0
+                    for i in range(din):
+                        acc += x[bb, t, i] * w[o, i]
+                    if bias is not None:
+                        acc += bias[o]
+                    got = (q, k, v)[o // dim][bb, t, o % dim]
+                    assert abs(got - acc) <= 1e-12 * (1 + abs(acc))
+
+
+def check_qkv_project_closed_forms(orc):
+    """A one-hot token e_j picks column j of each projection plus its bias; a zero token
+    gives the bias alone."""
+    rng = _rng(52)
+    din, dim = 6, 4
+    w = rng.standard_normal((3 * dim, din))
+    b = rng.standard_normal(3 * dim)
+    x = np.zeros((1, din + 1, din))
+    for j in range(din):
+        x[0, j, j] = 1.0
+    q, k, v = orc.qkv_project(x, w, b)
+    for j in range(din):
+        assert np.allclose(q[0, j], w[:dim, j] + b[:dim], rtol=0, atol=1e-15)
+        assert np.allclose(k[0, j], w[dim:2 * dim, j] + b[dim:2 * dim], rtol=0, atol=1e-15)
+        assert np.allclose(v[0, j], w[2 * dim:, j] + b[2 * dim:], rtol=0, atol=1e-15)
+    assert np.array_equal(np.concatenate([q[0, din], k[0, din], v[0, din]]), b)
+
+
+def check_bf16_round(orc):
+    """Rounding to bfloat16: equal to torch's float32 -> bfloat16 conversion (a library
+    routine) on float32 values across the exponent range; exact midpoints go to the even
+    significand; below 2^-126 the spacing is 2^-133."""
+    import torch
+    rng = _rng(53)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-80, 80, 20000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(orc.bf16_round(x.astype(np.float64)), ref)
+    ulp = 2.0 ** -7
+    mids = np.array([1 + ulp / 2, 1 + 3 * ulp / 2, -(1 + ulp / 2), 3 + ulp, 3 + 3 * ulp])
+    assert list(orc.bf16_round(mids)) == [1.0, 1 + 2 * ulp, -1.0, 3.0, 3 + 4 * ulp]
+    tiny = np.array([2.0 ** -133 * 2.5, 2.0 ** -133 * 3.5, 2.0 ** -126 * (1 + 2 ** -9)])
+    assert list(orc.bf16_round(tiny)) == [2.0 ** -132, 2.0 ** -131, 2.0 ** -126]
+
+
 def check_sp_head_scatter_is_whole_step_split_by_heads(orc):
     """Algorithm 3 steps 3-5 with the all-to-all folded in: ranks with uneven token
     ranges, each storing every head at its owner, together leave in owner r exactly the

@@ -132,6 +132,13 @@ def test_pins_catch_mutant(tmp_path, name):
 # Planted mistakes in the oracle's Python-level head scatter (the sequence-parallel step's
 # all-to-all folded into stores): a copy of oracle/__init__.py with one line changed.
 PY_MUTANTS = {
+    "qkv_weight_not_transposed": ("y = x @ w.T", "y = x @ w.reshape(w.shape[::-1])"),
+    "qkv_q_and_k_swapped": ("return y[..., :dim], y[..., dim:2 * dim], y[..., 2 * dim:]",
+                            "return y[..., dim:2 * dim], y[..., :dim], y[..., 2 * dim:]"),
+    "qkv_bias_dropped": ("            y = y + np.asarray(b_qkv, dtype=np.float64)",
+                         "            y = y + 0.0"),
+    "bf16_round_half_up": ("return np.ldexp(np.rint(np.ldexp(a, 8 - e)), e - 8)",
+                           "return np.ldexp(np.floor(np.ldexp(a, 8 - e) + 0.5), e - 8)"),
     "sp_round_robin_owner": ("r, local = divmod(head, hl)", "r, local = head % P, head // P"),
     "sp_q_row_ignores_row0": ("q_dst[r][:, i - q_row0, local]", "q_dst[r][:, i, local]"),
     "sp_cache_rows_drop_slot": ("rows = (slot + i) % C", "rows = i % C"),
