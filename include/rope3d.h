@@ -272,6 +272,37 @@ ROPE3D_API int rope3d_qk_norm_rope_append_sp(
     const rope3d_options* options, void* cuda_stream);
 
 /*
+ * The QKV projection that feeds the step (Algorithm 1/3 step 1, "q, k, v <- QKV(x)"; the
+ * paper fuses it with the rotary step, Section 3.4.1 item 3), on the tensor cores:
+ * y = x W^T + b with x [M][K] bf16 (token rows), w_qkv [3 N D][K] bf16 (an nn.Linear
+ * weight: the q rows, then the k rows, then the v rows) and b_qkv [3 N D] fp32 (NULL: no
+ * bias); fp32 accumulation, one round to nearest even to bf16.  The q, k and v column
+ * blocks of y go to q_out, k_out, v_out, each [M][N][D] bf16.  K must be a multiple of
+ * 64; x and w_qkv 16-byte aligned.  The kernel holds all of each SM's tensor memory while
+ * it runs: calls on concurrent streams serialise on it.
+ */
+ROPE3D_API int rope3d_qkv_project(const void* x, const void* w_qkv, const float* b_qkv, int64_t M,
+                                  int64_t K, int64_t N, int D, void* q_out, void* k_out,
+                                  void* v_out, void* cuda_stream);
+
+/*
+ * The projection and the step in one call: x [B][n_tok][K] bf16 holds the token rows of
+ * [token_begin, token_end); q, k, v = QKV(x) as in rope3d_qkv_project, each rounded to
+ * bf16, then the step of rope3d_qk_norm_rope_append on them.  The projection's epilogue
+ * stores v straight into the V cache at each token's cache row (the append, fused), q into
+ * q_out and k into the caller's work buffer k_work [B][n_tok][N][D]; the step then
+ * normalises and rotates q in place and k into the K cache.  bf16 only; options: the cache
+ * layout (adjacent pairing, bf16 caches).  Other arguments and errors as for
+ * rope3d_qk_norm_rope_append and rope3d_qkv_project.
+ */
+ROPE3D_API int rope3d_qkv_norm_rope_append(
+    const void* x, const void* w_qkv, const float* b_qkv, int64_t K, int64_t B, int64_t N, int D,
+    int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
+    const float* q_norm_w, const float* k_norm_w, float eps, void* q_out, void* k_work,
+    void* k_cache, void* v_cache, int64_t cache_tokens, int64_t slot, const rope3d_tables* tables,
+    int trig, const rope3d_options* options, void* cuda_stream);
+
+/*
  * The rotation alone -- CausalRoPE of Algorithm 3 step 3 / Algorithm 2 -- on one
  * token range: out[b][r] = RoPE(x[b][r], pos(token_begin + r)).  x and out are
  * [B][n_tok][N][D] of dtype; out may be x (in place) or must not overlap it.  Other

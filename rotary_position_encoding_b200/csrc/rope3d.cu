@@ -9,8 +9,10 @@
 #include "rope3d_testing.h"
 #include "rope3d_kernels.cuh"
 #include "rope3d_tma.cuh"
+#include "rope3d_gemm.cuh"
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
 #include <cstdarg>
@@ -228,7 +230,13 @@ KernelFn pick_format(int cache_fmt, int pairing, int trig, int vpt) {
 
 template <int MODE>
 KernelFn pick_kernel(int dtype, int trig, int pairing, int cache_fmt, int vpt) {
-    if constexpr (MODE == rope3d::kModeFusedSP) {
+    if constexpr (MODE == rope3d::kModeFusedNoV) {
+        // the step after the QKV projection: bf16, adjacent pairing, same-dtype K cache
+        if (pairing != ROPE3D_PAIRING_ADJACENT || cache_fmt != rope3d::kCacheSame ||
+            dtype != ROPE3D_BF16)
+            return nullptr;
+        return pick_trig<__nv_bfloat16, MODE, rope3d::kPairAdjacent, rope3d::kCacheSame>(trig, vpt);
+    } else if constexpr (MODE == rope3d::kModeFusedSP) {
         // head-scatter stores: adjacent pairing and same-dtype caches only
         if (pairing != ROPE3D_PAIRING_ADJACENT || cache_fmt != rope3d::kCacheSame) return nullptr;
         return dtype == ROPE3D_BF16
@@ -480,6 +488,69 @@ int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int d
         launch_pdl(reinterpret_cast<const void*>(fn), grid, threads, smem, stream, &p);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+// ---------------------------------------------------------------- QKV projection (tcgen05)
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D tensor map of a row-major bf16 matrix [rows][cols] read in boxes of box_rows x 64
+// with the 128-byte swizzle; rows past the end read as zero.
+int make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return fail(ROPE3D_ECUDA, "cuTensorMapEncodeTiled is not available");
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)rope3d::kGemmBK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ROPE3D_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return ROPE3D_OK;
+}
+
+int launch_qkv_gemm(const void* x, const void* w, rope3d::GemmParams& gp, int dev,
+                    const DeviceInfo& info, cudaStream_t stream) {
+    CUtensorMap map_x, map_w;
+    int rc = make_map_bf16(&map_x, x, gp.M, gp.K, rope3d::kGemmBM);
+    if (rc != ROPE3D_OK) return rc;
+    rc = make_map_bf16(&map_w, w, gp.n_out, gp.K, rope3d::kGemmBN);
+    if (rc != ROPE3D_OK) return rc;
+    gp.num_m = (gp.M + rope3d::kGemmBM - 1) / rope3d::kGemmBM;
+    gp.num_n = (gp.n_out + rope3d::kGemmBN - 1) / rope3d::kGemmBN;
+    gp.wait_limit_ns = g_wait_limit_ns.load();
+    const void* fn = reinterpret_cast<const void*>(rope3d::qkv_proj_kernel);
+    if ((int)rope3d::kGemmSmemBytes > info.max_smem_optin)
+        return fail(ROPE3D_EDEVICE, "the projection needs %zu bytes of shared memory",
+                    rope3d::kGemmSmemBytes);
+    static std::once_flag raised[64];
+    cudaError_t e = cudaSuccess;
+    std::call_once(raised[dev & 63], [&] {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)rope3d::kGemmSmemBytes);
+    });
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    const int tiles = gp.num_m * gp.num_n;
+    const int grid = tiles < info.sms ? tiles : info.sms;  // one CTA per SM (smem, TMEM)
+    void* args[] = {&map_x, &map_w, &gp};
+    e = cudaLaunchKernel(fn, dim3(grid), dim3(rope3d::kGemmThreads), args,
+                         rope3d::kGemmSmemBytes, stream);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "projection launch: %s", cudaGetErrorString(e));
+    return ROPE3D_OK;
 }
 
 void fill_common(rope3d::Params& p, int64_t B, int64_t N, int64_t token_begin, int64_t token_end,
@@ -969,6 +1040,158 @@ int rope3d_qk_norm_rope_append_sp(const void* q, const void* k, const void* v,
     set_small_idx(p);
     rc = launch<rope3d::kModeFusedSP>(p, N, dtype, trig, opt.pairing, dev, info,
                                       static_cast<cudaStream_t>(cuda_stream));
+    if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
+    return rc;
+}
+
+namespace {
+
+int check_projection(const void* x, const void* w_qkv, const float* b_qkv, int64_t M, int64_t K,
+                     int64_t N, int D) {
+    if (!x || !w_qkv) return fail(ROPE3D_EINVAL, "x or w_qkv is NULL");
+    if (D != rope3d::kHeadDim) return fail(ROPE3D_EINVAL, "head size D=%d must be 128", D);
+    if (N < 1 || M < 1) return fail(ROPE3D_EINVAL, "N=%lld and M=%lld must be >= 1",
+                                    (long long)N, (long long)M);
+    if (K < rope3d::kGemmBK || K % rope3d::kGemmBK != 0 || K > (1 << 20))
+        return fail(ROPE3D_EINVAL, "input features K=%lld must be a multiple of %d",
+                    (long long)K, rope3d::kGemmBK);
+    if (M > (1 << 30) || 3 * N * D > (1 << 24))
+        return fail(ROPE3D_ERANGE, "M=%lld or N=%lld is too large", (long long)M, (long long)N);
+    if (!aligned16(x) || !aligned16(w_qkv) ||
+        (b_qkv != nullptr && (reinterpret_cast<uintptr_t>(b_qkv) & 3u)))
+        return fail(ROPE3D_EALIGN, "x and w_qkv must be 16-byte aligned, b_qkv 4-byte");
+    return ROPE3D_OK;
+}
+
+}  // namespace
+
+int rope3d_qkv_project(const void* x, const void* w_qkv, const float* b_qkv, int64_t M,
+                       int64_t K, int64_t N, int D, void* q_out, void* k_out, void* v_out,
+                       void* cuda_stream) {
+    int rc = check_projection(x, w_qkv, b_qkv, M, K, N, D);
+    if (rc != ROPE3D_OK) return rc;
+    if (!q_out || !k_out || !v_out) return fail(ROPE3D_EINVAL, "an output pointer is NULL");
+    if (!aligned16(q_out) || !aligned16(k_out) || !aligned16(v_out))
+        return fail(ROPE3D_EALIGN, "outputs must be 16-byte aligned");
+    const size_t out = (size_t)M * N * D * 2;
+    const size_t xb = (size_t)M * K * 2, wb = (size_t)3 * N * D * K * 2;
+    const void* outs[3] = {q_out, k_out, v_out};
+    for (int a = 0; a < 3; ++a) {
+        if (overlap(outs[a], out, x, xb) || overlap(outs[a], out, w_qkv, wb))
+            return fail(ROPE3D_EOVERLAP, "an output overlaps x or w_qkv");
+        for (int b = a + 1; b < 3; ++b)
+            if (overlap(outs[a], out, outs[b], out)) return fail(ROPE3D_EOVERLAP, "outputs overlap");
+    }
+    DeviceInfo info;
+    int dev = 0;
+    rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    rope3d::GemmParams gp{};
+    gp.M = (int)M;
+    gp.K = (int)K;
+    gp.dim = (int)(N * D);
+    gp.n_out = 3 * gp.dim;
+    gp.bias = b_qkv;
+    gp.q_out = static_cast<__nv_bfloat16*>(q_out);
+    gp.k_out = static_cast<__nv_bfloat16*>(k_out);
+    gp.v_cache = static_cast<__nv_bfloat16*>(v_out);  // a cache of M rows, row = token
+    gp.n_tok = M;
+    gp.token_begin = 0;
+    gp.cache_tokens = M;
+    gp.slot = 0;
+    gp.n_heads = (int)N;
+    gp.cache_head_major = 0;
+    gp.status = nullptr;
+    return launch_qkv_gemm(x, w_qkv, gp, dev, info, static_cast<cudaStream_t>(cuda_stream));
+}
+
+int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b_qkv, int64_t K,
+                                int64_t B, int64_t N, int D, int64_t token_begin,
+                                int64_t token_end, int64_t frame_offset, int T, int H, int W,
+                                const float* q_norm_w, const float* k_norm_w, float eps,
+                                void* q_out, void* k_work, void* k_cache, void* v_cache,
+                                int64_t cache_tokens, int64_t slot, const rope3d_tables* tables,
+                                int trig, const rope3d_options* options, void* cuda_stream) {
+    rope3d_options opt;
+    int rc = read_options(options, &opt, true);
+    if (rc != ROPE3D_OK) return rc;
+    if (opt.pairing != ROPE3D_PAIRING_ADJACENT || opt.cache_dtype != ROPE3D_CACHE_SAME)
+        return fail(ROPE3D_EINVAL, "the projection-fed step supports adjacent pairing and "
+                                   "bf16 caches");
+    rc = check_common(B, N, D, ROPE3D_BF16, token_begin, token_end, frame_offset, T, H, W,
+                      tables, trig);
+    if (rc != ROPE3D_OK) return rc;
+    const int64_t n_tok = token_end - token_begin;
+    rc = check_projection(x, w_qkv, b_qkv, B * n_tok, K, N, D);
+    if (rc != ROPE3D_OK) return rc;
+    if (!q_out || !k_work || !k_cache || !v_cache || !q_norm_w || !k_norm_w)
+        return fail(ROPE3D_EINVAL, "a tensor pointer is NULL");
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(ROPE3D_EINVAL, "eps must be >= 0");
+    if (cache_tokens < 1) return fail(ROPE3D_EINVAL, "cache_tokens must be >= 1");
+    if (slot < 0) return fail(ROPE3D_EINVAL, "slot must be >= 0");
+    if (n_tok > cache_tokens)
+        return fail(ROPE3D_ERANGE, "%lld tokens do not fit a cache of %lld rows",
+                    (long long)n_tok, (long long)cache_tokens);
+    if (!aligned16(q_out) || !aligned16(k_work) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(q_norm_w) || !aligned16(k_norm_w))
+        return fail(ROPE3D_EALIGN, "every tensor pointer must be 16-byte aligned");
+    const size_t act = (size_t)B * n_tok * N * D * 2;
+    const size_t cache = (size_t)B * cache_tokens * N * D * 2;
+    const size_t xb = (size_t)B * n_tok * K * 2, wb = (size_t)3 * N * D * K * 2;
+    const void* bufs[4] = {q_out, k_work, k_cache, v_cache};
+    const size_t sizes[4] = {act, act, cache, cache};
+    for (int a = 0; a < 4; ++a) {
+        if (overlap(bufs[a], sizes[a], x, xb) || overlap(bufs[a], sizes[a], w_qkv, wb))
+            return fail(ROPE3D_EOVERLAP, "an output overlaps x or w_qkv");
+        for (int b = a + 1; b < 4; ++b)
+            if (overlap(bufs[a], sizes[a], bufs[b], sizes[b]))
+                return fail(ROPE3D_EOVERLAP, "q_out, k_work and the caches must not overlap");
+    }
+    DeviceInfo info;
+    int dev = 0;
+    rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+    rc = check_tables_device(tables, dev);
+    if (rc != ROPE3D_OK) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+
+    // 1. q, k, v = QKV(x): q into q_out, k into k_work, v into the V cache rows
+    rope3d::GemmParams gp{};
+    gp.M = (int)(B * n_tok);
+    gp.K = (int)K;
+    gp.dim = (int)(N * D);
+    gp.n_out = 3 * gp.dim;
+    gp.bias = b_qkv;
+    gp.q_out = static_cast<__nv_bfloat16*>(q_out);
+    gp.k_out = static_cast<__nv_bfloat16*>(k_work);
+    gp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+    gp.n_tok = n_tok;
+    gp.token_begin = token_begin;
+    gp.cache_tokens = cache_tokens;
+    gp.slot = slot;
+    gp.n_heads = (int)N;
+    gp.cache_head_major = opt.cache_layout == ROPE3D_CACHE_HEAD_MAJOR ? 1 : 0;
+    gp.status = tables->d_status;
+    rc = launch_qkv_gemm(x, w_qkv, gp, dev, info, stream);
+    if (rc != ROPE3D_OK) return rc;
+
+    // 2. the step on q (in place) and k; V is already in the cache
+    rope3d::Params p{};
+    fill_common(p, B, N, token_begin, token_end, frame_offset, H, W, tables);
+    p.q = q_out;
+    p.k = k_work;
+    p.v = nullptr;
+    p.q_out = q_out;
+    p.k_cache = k_cache;
+    p.v_cache = nullptr;
+    p.q_w = q_norm_w;
+    p.k_w = k_norm_w;
+    p.cache_tokens = cache_tokens;
+    p.slot = slot;
+    p.eps = eps;
+    fill_layout(p, N, ROPE3D_BF16, opt);
+    set_small_idx(p);
+    rc = launch<rope3d::kModeFusedNoV>(p, N, ROPE3D_BF16, trig, opt.pairing, dev, info, stream);
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
     return rc;
 }

@@ -42,7 +42,9 @@ constexpr int kTmaMaxBlockThreads = 320;  // ring kernel: one block per SM, up t
 
 // kModeFusedSP: the fused step with head-scatter stores (the sequence-parallel
 // all-to-all folded into the step): each head goes to the destination rank that owns it.
-enum Mode : int { kModeFused = 0, kModeApply = 1, kModeFusedSP = 2 };
+// kModeFusedNoV: the fused step for q and K only (V was appended by the producer of q,
+// k, v -- the QKV projection's epilogue).
+enum Mode : int { kModeFused = 0, kModeApply = 1, kModeFusedSP = 2, kModeFusedNoV = 3 };
 constexpr int kMaxRanks = 8;  // head-scatter destinations (one node)
 // KV-cache element formats of the fused step
 enum CacheFmt : int { kCacheSame = 0, kCacheFp8 = 1, kCacheNvfp4 = 2 };
@@ -919,6 +921,9 @@ qk_norm_rope_kernel(const Params p) {
     constexpr int NP = PairCount<T, PAIR>::value;
     constexpr bool FUSED = MODE != kModeApply;
     constexpr bool SP = MODE == kModeFusedSP;
+    constexpr bool HAS_V = FUSED && MODE != kModeFusedNoV;
+    constexpr int EMIT_MODE = MODE == kModeFusedNoV ? kModeFused : MODE;
+    static_assert(HAS_V || !FUSED || CF == kCacheSame, "no-V step: same-dtype K cache");
     static_assert(!SP || (PAIR == kPairAdjacent && CF == kCacheSame),
                   "head-scatter stores: adjacent pairing, same-dtype caches");
 
@@ -977,10 +982,8 @@ qk_norm_rope_kernel(const Params p) {
             const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
             if (idx < p.dim_vecs) {
                 xq[s] = load_stream(qg + row_vec + idx);
-                if (FUSED) {
-                    xk[s] = load_stream(kg + row_vec + idx);
-                    xv[s] = load_stream(vg + row_vec + idx);
-                }
+                if (FUSED) xk[s] = load_stream(kg + row_vec + idx);
+                if (HAS_V) xv[s] = load_stream(vg + row_vec + idx);
             }
         }
         float cs[NP], sn[NP];
@@ -989,7 +992,8 @@ qk_norm_rope_kernel(const Params p) {
         float rq = 1.0f, rk = 1.0f;
         if (FUSED) {
             if constexpr (SP) store_v_row_sp<T, VPT>(p, t, pos, xv, dst, s_sp);
-            else if constexpr (CF == kCacheSame) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
+            else if constexpr (CF == kCacheSame && HAS_V)
+                store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -1000,8 +1004,8 @@ qk_norm_rope_kernel(const Params p) {
         if constexpr (SP)
             emit_row_sp<T, VPT>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
         else
-            emit_row<T, VPT, PAIR, MODE, CF>(p, t, pos, row_vec, xq, xk, xv, rq, rk, s_wq,
-                                             s_wk, cs, sn, qo, kc, vc, s_r);
+            emit_row<T, VPT, PAIR, EMIT_MODE, CF>(p, t, pos, row_vec, xq, xk, xv, rq, rk,
+                                                  s_wq, s_wk, cs, sn, qo, kc, vc, s_r);
     }
 }
 

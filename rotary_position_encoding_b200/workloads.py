@@ -167,6 +167,22 @@ def chunk_inputs(w: Workload, chunk_index: int, n_tok: int | None = None):
     return tuple(normal_tensor(rng, shape, w.dtype) for _ in range(3))
 
 
+def hidden_states(w: Workload, chunk_index: int, K: int, n_tok: int | None = None):
+    """Token rows x [B, n_tok, K] entering the QKV projection: N(0,1), bf16 bits."""
+    n = w.tokens_per_chunk if n_tok is None else n_tok
+    rng = rng_for(w.seed, 2000 + chunk_index)
+    return f32_to_bf16_bits(rng.standard_normal(size=(w.B, n, K), dtype=np.float32))
+
+
+def projection_weights(seed: int, dim: int, K: int):
+    """A QKV projection: weight [3 dim, K] ~ N(0, 1/K) as bf16 bits (so that the projected
+    values are about N(0,1)) and bias [3 dim] ~ N(0, 0.1^2) float32."""
+    rng = rng_for(seed, 3000)
+    w = rng.standard_normal(size=(3 * dim, K), dtype=np.float32) * np.float32(1.0 / np.sqrt(K))
+    b = (rng.standard_normal(size=3 * dim, dtype=np.float32) * np.float32(0.1))
+    return f32_to_bf16_bits(w), b
+
+
 def to_f64(x: np.ndarray, dtype: str) -> np.ndarray:
     """Exact float64 view of a workload tensor (float32 or bf16 bits)."""
     if dtype == "f32":
