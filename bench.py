@@ -74,6 +74,9 @@ def parse_args(argv=None):
                     help="sequence-parallel step with the all-to-all folded in: each chunk is "
                          "cut into SP even token slices (the ranks of one node, emulated on "
                          "this GPU as SP launches) whose heads go to SP destination buffers")
+    ap.add_argument("--qkv", action="store_true",
+                    help="the QKV-projection-fed step: token rows x [n, N*128] through the "
+                         "tcgen05 projection (V appended by its epilogue), then the step")
     ap.add_argument("--eager", action="store_true",
                     help="launch every chunk call from Python and time each launch with its "
                          "own CUDA event pair (default: capture one step -- all its chunk "
@@ -510,6 +513,134 @@ def run_ours(args, dist: Dist):
     return line
 
 
+def run_qkv(args, dist: Dist):
+    """The step fed by the QKV projection: every chunk's token rows x [1, n, K] (K = N*128)
+    go through rope3d_qkv_norm_rope_append.  The roofline is the projection kernel's, on
+    the tensor cores: 2 n K (3 N 128) flops per launch over its own launch time, measured
+    by timing rope3d_qkv_project alone on the same shapes; cuBLAS (torch.matmul) on the
+    same GEMM is timed beside it for context."""
+    import torch
+
+    from rotary_position_encoding_b200 import rope3d
+
+    torch.cuda.set_device(dist.local_rank)
+    device = torch.device("cuda", dist.local_rank)
+    dist.init("nccl")
+    w = workload_for(args)
+    if w.dtype != "bf16":
+        raise SystemExit("--qkv runs bf16 workloads")
+    K = w.dim
+    n = w.tokens_per_chunk
+    trig = rope3d.ROPE3D_TRIG_TABLE if args.trig == "table" else rope3d.ROPE3D_TRIG_ONTHEFLY
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    xs = [dev_bf16(wl.hidden_states(w, ci, K)) for ci in range(len(w.chunks))]
+    w_bits, b = wl.projection_weights(w.seed, w.dim, K)
+    wt = dev_bf16(w_bits)
+    bt = torch.from_numpy(b).to(device)
+    wq, wk = (torch.from_numpy(a).to(device) for a in wl.norm_weights(w.seed, w.dim))
+    q_out = [torch.empty((w.B, n, w.N, wl.HEAD_DIM), dtype=torch.bfloat16, device=device)
+             for _ in w.chunks]
+    k_work = torch.empty_like(q_out[0])
+    shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    k_cache = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    v_cache = torch.zeros(shape, dtype=torch.bfloat16, device=device)
+    tables = rope3d.rope3d_tables_init(max_t=max(c.frame_offset for c in w.chunks) + w.T,
+                                       max_h=w.H, max_w=w.W)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for ci, c in enumerate(w.chunks):
+            rope3d.rope3d_qkv_norm_rope_append(
+                xs[ci], wt, bt, q_out[ci], k_work, c.token_begin, c.token_end, c.frame_offset,
+                w.T, w.H, w.W, wq, wk, w.eps, k_cache, v_cache, c.slot, tables, trig,
+                stream=stream)
+
+    clocks = ClockSampler(dist.local_rank) if dist.rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark("start")
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.mark("end")
+    dist.barrier()
+    elapsed_ms = dist.max(start.elapsed_time(end), device)
+    clock_info = clocks.stop() if clocks else None
+
+    # the projection kernel alone, and cuBLAS on the same GEMM
+    outs = [torch.empty_like(q_out[0]) for _ in range(3)]
+    reps = max(3, min(args.steps, 20)) * len(w.chunks)
+
+    def timed(fn):
+        for _ in range(3):
+            fn(0)
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for r in range(reps):
+            fn(r % len(w.chunks))
+        e.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(e) / reps
+
+    gemm_ms = timed(lambda ci: rope3d.rope3d_qkv_project(xs[ci], wt, bt, *outs, stream=stream))
+    y = torch.empty((n, 3 * w.dim), dtype=torch.bfloat16, device=device)
+    cublas_ms = timed(lambda ci: torch.matmul(xs[ci].view(n, K), wt.t(), out=y))
+    tables.close()
+    dist.close()
+    if dist.rank != 0:
+        return None
+    peaks, peak_kind = measured_peaks()
+    flops = 2.0 * w.B * n * K * 3 * w.dim
+    achieved = flops / (gemm_ms / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    tokens_per_step = w.B * n * len(w.chunks)
+    return {
+        "metric": "QKV projection + QK-RMSNorm + 3D RoPE + KV append tokens/s, 1 GPU",
+        "value": round(tokens_per_step * args.steps * dist.world / (elapsed_ms / 1e3), 1),
+        "unit": "tokens/s",
+        "n_gpus": dist.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) token rows, N(0,1/K) projection weights, N(0,0.01) "
+                "bias, U(0.5,1.5) norm weights)",
+        "config": {"workload": w.name + "+qkv", "K": K, "heads": w.N,
+                   "chunks_per_step": len(w.chunks), "tokens_per_step": tokens_per_step,
+                   "launch": "eager, one C-ABI call per chunk (projection + step)",
+                   "l2": "no flush: each chunk's x (110 MB) and the weight (157 MB) exceed L2 "
+                         "together"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained (back-to-back launches)",
+                     "kernel": "rope3d::qkv_proj_kernel",
+                     "algorithmic_flops_per_launch": flops,
+                     "avg_launch_ms": round(gemm_ms, 4),
+                     "cublas_same_gemm_ms": round(cublas_ms, 4),
+                     "cublas_tflops": round(flops / (cublas_ms / 1e3) / 1e12, 1)},
+        "gpu_launches": 2 * len(w.chunks) * args.steps,
+        "clocks": clock_info,
+    }
+
+
 def run_e2e(args, w, host, wq_d, wk_d, tables, trig, device, dist, rope3d, torch):
     """Same workload through the public call, with the step's inputs copied in from pinned
     host memory and its results (q_out and the appended K/V rows) copied back every step,
@@ -721,6 +852,8 @@ def main(argv=None):
     dist = Dist()
     if args.impl == "reference":
         line = run_reference(args, dist)
+    elif args.qkv:
+        line = run_qkv(args, dist)
     else:
         line = run_ours(args, dist)
     if line is not None and dist.rank == 0:
