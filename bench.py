@@ -48,8 +48,10 @@ WORKLOADS = {
     "longhorizon": wl.long_horizon,
 }
 METRIC = "fused norm+3D-RoPE+KV-append tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
+# the step kernels' sources and their launch planning (the per-launch traffic recorded in
+# profiles/traffic.json holds for these only)
 KERNEL_SOURCES = [os.path.join(ROOT, "rotary_position_encoding_b200", "csrc", f)
-                  for f in ("rope3d_kernels.cuh", "rope3d.cu")]
+                  for f in ("rope3d_kernels.cuh", "rope3d_tma.cuh", "rope3d.cu")]
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
