@@ -287,20 +287,31 @@ ROPE3D_API int rope3d_qkv_project(const void* x, const void* w_qkv, const float*
 
 /*
  * The projection and the step in one call: x [B][n_tok][K] bf16 holds the token rows of
- * [token_begin, token_end); q, k, v = QKV(x) as in rope3d_qkv_project, each rounded to
- * bf16, then the step of rope3d_qk_norm_rope_append on them.  The projection's epilogue
- * stores v straight into the V cache at each token's cache row (the append, fused), q into
- * q_out and k into the caller's work buffer k_work [B][n_tok][N][D]; the step then
- * normalises and rotates q in place and k into the K cache.  bf16 only; options: the cache
- * layout (adjacent pairing, bf16 caches).  Other arguments and errors as for
- * rope3d_qk_norm_rope_append and rope3d_qkv_project.
+ * [token_begin, token_end); q, k, v = QKV(x) as in rope3d_qkv_project (fp32 accumulation),
+ * then the step of rope3d_qk_norm_rope_append on them, with V stored straight into the V
+ * cache at each token's cache row by the projection's epilogue.
+ *   - When N D is a multiple of 256 (even head counts) the projection's epilogue applies
+ *     the RMSNorm weight and the rotation to the fp32 q and k tiles, stores them to q_out
+ *     and the K cache, and records each row's partial sum of squares per tile in the
+ *     workspace; a light second kernel then scales every q and K row by
+ *     1 / sqrt(mean(x^2) + eps) in place (a fixed-order sum, so results do not depend on
+ *     scheduling or on slicing).  The normalisation uses the fp32 projections, and q, K
+ *     are rounded to bf16 twice (before and after the scale).
+ *   - Otherwise the projection rounds q and k to bf16 (q into q_out, k into the workspace)
+ *     and the step then normalises and rotates them (V already in the cache).
+ * workspace: device scratch of rope3d_qkv_workspace_bytes(B, n_tok, N, D) bytes (no
+ * initialisation needed).  bf16 only; options: the cache layout (adjacent pairing, bf16
+ * caches).  Other arguments and errors as for rope3d_qk_norm_rope_append and
+ * rope3d_qkv_project.
  */
+ROPE3D_API size_t rope3d_qkv_workspace_bytes(int64_t B, int64_t n_tok, int64_t N, int D);
+
 ROPE3D_API int rope3d_qkv_norm_rope_append(
     const void* x, const void* w_qkv, const float* b_qkv, int64_t K, int64_t B, int64_t N, int D,
     int64_t token_begin, int64_t token_end, int64_t frame_offset, int T, int H, int W,
-    const float* q_norm_w, const float* k_norm_w, float eps, void* q_out, void* k_work,
-    void* k_cache, void* v_cache, int64_t cache_tokens, int64_t slot, const rope3d_tables* tables,
-    int trig, const rope3d_options* options, void* cuda_stream);
+    const float* q_norm_w, const float* k_norm_w, float eps, void* q_out, void* workspace,
+    size_t workspace_bytes, void* k_cache, void* v_cache, int64_t cache_tokens, int64_t slot,
+    const rope3d_tables* tables, int trig, const rope3d_options* options, void* cuda_stream);
 
 /*
  * The rotation alone -- CausalRoPE of Algorithm 3 step 3 / Algorithm 2 -- on one

@@ -19,7 +19,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "librope3d.so")
 SOURCES = [os.path.join(CSRC, "rope3d.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("rope3d_kernels.cuh", "rope3d_tma.cuh")] + \
+DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("rope3d_kernels.cuh", "rope3d_tma.cuh",
+                                                    "rope3d_gemm.cuh")] + \
     [os.path.join(INCLUDE, f) for f in ("rope3d.h", "rope3d_testing.h")]
 
 NVCC_FLAGS = [

@@ -1105,13 +1105,23 @@ int rope3d_qkv_project(const void* x, const void* w_qkv, const float* b_qkv, int
     return launch_qkv_gemm(x, w_qkv, gp, dev, info, static_cast<cudaStream_t>(cuda_stream));
 }
 
+size_t rope3d_qkv_workspace_bytes(int64_t B, int64_t n_tok, int64_t N, int D) {
+    if (B < 1 || n_tok < 1 || N < 1 || D != rope3d::kHeadDim) return 0;
+    const int64_t M = B * n_tok, dim = N * D;
+    if (dim % rope3d::kGemmBN == 0)  // fused epilogue: partial sums of squares per row and tile
+        return (size_t)(2 * M * (dim / rope3d::kGemmBN)) * sizeof(float);
+    return (size_t)(M * dim) * 2;  // odd head counts: k is staged for the step
+}
+
 int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b_qkv, int64_t K,
                                 int64_t B, int64_t N, int D, int64_t token_begin,
                                 int64_t token_end, int64_t frame_offset, int T, int H, int W,
                                 const float* q_norm_w, const float* k_norm_w, float eps,
-                                void* q_out, void* k_work, void* k_cache, void* v_cache,
-                                int64_t cache_tokens, int64_t slot, const rope3d_tables* tables,
-                                int trig, const rope3d_options* options, void* cuda_stream) {
+                                void* q_out, void* workspace, size_t workspace_bytes,
+                                void* k_cache, void* v_cache, int64_t cache_tokens, int64_t slot,
+                                const rope3d_tables* tables, int trig,
+                                const rope3d_options* options, void* cuda_stream) {
+    void* k_work = workspace;
     rope3d_options opt;
     int rc = read_options(options, &opt, true);
     if (rc != ROPE3D_OK) return rc;
@@ -1126,6 +1136,10 @@ int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b
     if (rc != ROPE3D_OK) return rc;
     if (!q_out || !k_work || !k_cache || !v_cache || !q_norm_w || !k_norm_w)
         return fail(ROPE3D_EINVAL, "a tensor pointer is NULL");
+    const size_t ws_need = rope3d_qkv_workspace_bytes(B, n_tok, N, D);
+    if (workspace_bytes < ws_need)
+        return fail(ROPE3D_EINVAL, "workspace of %zu bytes, %zu needed", workspace_bytes, ws_need);
+    const bool fused = (N * D) % rope3d::kGemmBN == 0;
     if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(ROPE3D_EINVAL, "eps must be >= 0");
     if (cache_tokens < 1) return fail(ROPE3D_EINVAL, "cache_tokens must be >= 1");
     if (slot < 0) return fail(ROPE3D_EINVAL, "slot must be >= 0");
@@ -1139,13 +1153,13 @@ int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b
     const size_t cache = (size_t)B * cache_tokens * N * D * 2;
     const size_t xb = (size_t)B * n_tok * K * 2, wb = (size_t)3 * N * D * K * 2;
     const void* bufs[4] = {q_out, k_work, k_cache, v_cache};
-    const size_t sizes[4] = {act, act, cache, cache};
+    const size_t sizes[4] = {act, ws_need, cache, cache};
     for (int a = 0; a < 4; ++a) {
         if (overlap(bufs[a], sizes[a], x, xb) || overlap(bufs[a], sizes[a], w_qkv, wb))
             return fail(ROPE3D_EOVERLAP, "an output overlaps x or w_qkv");
         for (int b = a + 1; b < 4; ++b)
             if (overlap(bufs[a], sizes[a], bufs[b], sizes[b]))
-                return fail(ROPE3D_EOVERLAP, "q_out, k_work and the caches must not overlap");
+                return fail(ROPE3D_EOVERLAP, "q_out, the workspace and the caches must not overlap");
     }
     DeviceInfo info;
     int dev = 0;
@@ -1172,6 +1186,47 @@ int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b
     gp.n_heads = (int)N;
     gp.cache_head_major = opt.cache_layout == ROPE3D_CACHE_HEAD_MAJOR ? 1 : 0;
     gp.status = tables->d_status;
+    if (fused) {
+        // 1+2. the projection with the normalisation and rotation in its epilogue
+        const int64_t M = B * n_tok;
+        gp.fused = 1;
+        gp.q_w = q_norm_w;
+        gp.k_w = k_norm_w;
+        gp.eps = eps;
+        gp.inv_dim = 1.0f / (float)(N * D);
+        gp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+        gp.psum = static_cast<float*>(workspace);
+        const bool table = trig == ROPE3D_TRIG_TABLE;
+        gp.tab_t = table ? tables->tab_t : nullptr;
+        gp.tab_h = table ? tables->tab_h : nullptr;
+        gp.tab_w = table ? tables->tab_w : nullptr;
+        gp.n_t = tables->n_t;
+        gp.n_h = tables->n_h;
+        gp.n_w = tables->n_w;
+        gp.H = H;
+        gp.W = W;
+        gp.hw = (int64_t)H * W;
+        gp.frame_offset = frame_offset;
+        for (int j = 0; j < rope3d::kPairs; ++j) gp.inv_freq[j] = tables->inv_freq[j];
+        rc = launch_qkv_gemm(x, w_qkv, gp, dev, info, stream);
+        if (rc != ROPE3D_OK) return rc;
+        // 3. the per-row scale 1 / sqrt(mean + eps) of q and K, in place
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)((2 * M + rope3d::kScaleWarps - 1) / rope3d::kScaleWarps));
+        cfg.blockDim = dim3(32 * rope3d::kScaleWarps);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        void* args[] = {&gp};
+        const cudaError_t e = cudaLaunchKernelExC(
+            &cfg, reinterpret_cast<const void*>(rope3d::qk_row_scale_kernel), args);
+        if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "row scale launch: %s", cudaGetErrorString(e));
+        g_last_path = ROPE3D_PATH_REGISTERS;
+        return ROPE3D_OK;
+    }
     rc = launch_qkv_gemm(x, w_qkv, gp, dev, info, stream);
     if (rc != ROPE3D_OK) return rc;
 

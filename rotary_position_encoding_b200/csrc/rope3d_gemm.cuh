@@ -40,8 +40,9 @@ constexpr int kGemmGroupM = 32;
 constexpr uint32_t kGemmStageA = kGemmBM * kGemmBK * 2;  // 16 KB
 constexpr uint32_t kGemmStageB = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr uint32_t kGemmTmemCols = 2 * kGemmBN;          // two accumulators
-// dynamic shared memory: 1 KB alignment slack, the stages, then the barriers
-constexpr size_t kGemmSmemBytes = 1024 + kGemmStages * (kGemmStageA + kGemmStageB) + 256;
+// dynamic shared memory: 1 KB alignment slack, the stages, then barriers and the
+// epilogue's row scales
+constexpr size_t kGemmSmemBytes = 1024 + kGemmStages * (kGemmStageA + kGemmStageB) + 1024;
 
 struct GemmParams {
     int M;                 // token rows (B * n_tok)
@@ -58,6 +59,23 @@ struct GemmParams {
     int cache_head_major;
     uint64_t wait_limit_ns;
     int* status;
+    // fused QK-RMSNorm + RoPE epilogue (dim a multiple of 256, so every tile is all q, all
+    // k or all v): q and K tiles are stored weighted and rotated but not yet normalised,
+    // with each row's partial sum of squares per tile; qk_row_scale_kernel then scales
+    // every row by 1 / sqrt(mean + eps) in place.
+    int fused;
+    const float* q_w;          // [dim] RMSNorm weights
+    const float* k_w;
+    float eps, inv_dim;
+    __nv_bfloat16* k_cache;    // [B][C][N][128] or [B][N][C][128]
+    float* psum;               // [2][M][dim / 256] partial sums of squares
+    const float2* tab_t;       // cos/sin tables, or null for on-the-fly fp32 sincos
+    const float2* tab_h;
+    const float2* tab_w;
+    int n_t, n_h, n_w;
+    int H, W;
+    int64_t hw, frame_offset;
+    float inv_freq[kPairs];
 };
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -122,6 +140,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Barrier 1 over the 4 epilogue warps, with the OR / AND of a predicate: every epilogue
+// thread gets the same answer, so the group always takes the same branch.
+__device__ __forceinline__ bool epi_vote_any(bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+                 " bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+                 : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool epi_vote_all(bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+                 " bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+                 : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
 }
 
 // Tile t -> (row block, column block), grouped kGemmGroupM row blocks at a time.
@@ -245,29 +280,43 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     } else {  // epilogue warps 2..5: lanes 32 (warp % 4) .. +32 of tensor memory
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
+        const int tiles_per_tensor = p.dim / kGemmBN;
         int it = 0;
-        for (int t = blockIdx.x; t < num_tiles && !*s_fail; t += gridDim.x, ++it) {
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+            if (epi_vote_any(*s_fail != 0)) break;  // the group leaves together
             int mb, nb;
             gemm_tile_coords(p, t, mb, nb);
             const int acc = it & 1;
             const int use = it >> 1;
-            if (!mbar_wait_bounded(tfull_bar + 8 * acc, use & 1, p.wait_limit_ns)) {
+            const bool got = mbar_wait_bounded(tfull_bar + 8 * acc, use & 1, p.wait_limit_ns);
+            if (!epi_vote_all(got)) {
                 *s_fail = 1;
                 break;
             }
             tmem_fence_after();
             const int row = mb * kGemmBM + row_in_tile;
             const bool live = row < p.M;
-            // destination of this row in the V cache
-            int64_t v_row = 0;
+            const int which_tile = (nb * kGemmBN) / p.dim;  // 0 q, 1 k, 2 v (fused layout)
+            const bool norm_tile = p.fused && which_tile < 2;
+            // this row's token: batch b, index i, position and cache row
+            int64_t b = 0, i = 0, crow = 0, t_g = 0;
+            int hh = 0, ww = 0;
             if (live) {
-                const int64_t b = row / p.n_tok;
-                const int64_t i = p.token_begin + (row - b * p.n_tok);
-                const int64_t crow = (p.slot + i) % p.cache_tokens;
-                v_row = p.cache_head_major ? (b * p.n_heads * p.cache_tokens + crow)
-                                           : (b * p.cache_tokens + crow);
+                b = row / p.n_tok;
+                i = p.token_begin + (row - b * p.n_tok);
+                crow = (p.slot + i) % p.cache_tokens;
+                if (norm_tile) {
+                    const int64_t tl = i / p.hw;
+                    const int64_t rem = i - tl * p.hw;
+                    t_g = p.frame_offset + tl;
+                    hh = (int)(rem / p.W);
+                    ww = (int)(rem - (int64_t)hh * p.W);
+                }
             }
+            const int64_t v_row = p.cache_head_major ? (b * p.n_heads * p.cache_tokens + crow)
+                                                     : (b * p.cache_tokens + crow);
             const uint32_t taddr = tmem + acc * kGemmBN + ((uint32_t)(quarter * 32) << 16);
+            float ss = 0.0f;  // this row's sum of squares over the tile (fixed order)
 #pragma unroll 1
             for (int c = 0; c < kGemmBN / 32; ++c) {
                 uint32_t r[32];
@@ -276,27 +325,91 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 if (!live || gc >= p.n_out) continue;
                 const int which = gc / p.dim;         // 0 q, 1 k, 2 v
                 const int col = gc - which * p.dim;
-                uint32_t packed[16];
+                float a[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float a = __uint_as_float(r[2 * j]), b = __uint_as_float(r[2 * j + 1]);
-                    if (p.bias != nullptr) {
-                        a += __ldg(p.bias + gc + 2 * j);
-                        b += __ldg(p.bias + gc + 2 * j + 1);
+                for (int j = 0; j < 32; ++j) a[j] = __uint_as_float(r[j]);
+                if (p.bias != nullptr) {  // 32 consecutive fp32: 8 aligned 16-byte loads
+                    const float4* b4 = reinterpret_cast<const float4*>(p.bias + gc);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 bb = __ldg(b4 + q);
+                        a[4 * q] += bb.x;
+                        a[4 * q + 1] += bb.y;
+                        a[4 * q + 2] += bb.z;
+                        a[4 * q + 3] += bb.w;
                     }
-                    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-                    packed[j] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                uint32_t packed[16];
+                if (norm_tile) {
+                    // every load of the chunk is issued before the arithmetic: the weights
+                    // (8 aligned 16-byte loads) and the 16 (cos, sin) pairs, whose table and
+                    // row are chosen without branches
+                    const float4* w4 =
+                        reinterpret_cast<const float4*>((which == 0 ? p.q_w : p.k_w) + col);
+                    float wv[32];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float4 t4 = __ldg(w4 + q);
+                        wv[4 * q] = t4.x;
+                        wv[4 * q + 1] = t4.y;
+                        wv[4 * q + 2] = t4.z;
+                        wv[4 * q + 3] = t4.w;
+                    }
+                    const int pair0 = (col & 127) >> 1;  // first pair of the chunk in its head
+                    float cs[16], sn[16];
+                    if (p.tab_t != nullptr) {
+                        float2 e[16];
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const int j = pair0 + m;
+                            const bool in_t = j < p.n_t, in_h = !in_t && j < p.n_t + p.n_h;
+                            const float2* tab = in_t ? p.tab_t : (in_h ? p.tab_h : p.tab_w);
+                            const int64_t at = in_t ? t_g * p.n_t + j
+                                               : in_h ? (int64_t)hh * p.n_h + (j - p.n_t)
+                                                      : (int64_t)ww * p.n_w + (j - p.n_t - p.n_h);
+                            e[m] = __ldg(tab + at);
+                        }
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            cs[m] = e[m].x;
+                            sn[m] = e[m].y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const int j = pair0 + m;
+                            const int64_t x = j < p.n_t ? t_g : (j < p.n_t + p.n_h ? hh : ww);
+                            sincosf((float)x * p.inv_freq[j], &sn[m], &cs[m]);
+                        }
+                    }
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        ss = fmaf(a[2 * m], a[2 * m], ss);
+                        ss = fmaf(a[2 * m + 1], a[2 * m + 1], ss);
+                        const float x0 = a[2 * m] * wv[2 * m];
+                        const float x1 = a[2 * m + 1] * wv[2 * m + 1];
+                        __nv_bfloat162 h = __floats2bfloat162_rn(x0 * cs[m] - x1 * sn[m],
+                                                                 x0 * sn[m] + x1 * cs[m]);
+                        packed[m] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * j], a[2 * j + 1]);
+                        packed[j] = *reinterpret_cast<uint32_t*>(&h);
+                    }
                 }
                 __nv_bfloat16* dst;
+                const int head = col >> 7;
                 if (which == 0) {
                     dst = p.q_out + (int64_t)row * p.dim + col;
-                } else if (which == 1) {
+                } else if (which == 1 && !p.fused) {
                     dst = p.k_out + (int64_t)row * p.dim + col;
-                } else if (!p.cache_head_major) {
-                    dst = p.v_cache + v_row * p.dim + col;
                 } else {
-                    const int head = col >> 7;
-                    dst = p.v_cache + (v_row + (int64_t)head * p.cache_tokens) * 128 + (col & 127);
+                    __nv_bfloat16* cache = which == 1 ? p.k_cache : p.v_cache;
+                    dst = !p.cache_head_major
+                              ? cache + v_row * p.dim + col
+                              : cache + (v_row + (int64_t)head * p.cache_tokens) * 128 + (col & 127);
                 }
                 uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -305,7 +418,12 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                                        packed[4 * j + 3]);
             }
             tmem_fence_before();
-            mbar_arrive(tempty_bar + 8 * acc);
+            mbar_arrive(tempty_bar + 8 * acc);  // the accumulator is free for the next tile
+            // record this row's partial sum of squares over the tile's columns
+            if (norm_tile && live) {
+                const int tile_in_tensor = nb - which_tile * tiles_per_tensor;
+                p.psum[((int64_t)which_tile * p.M + row) * tiles_per_tensor + tile_in_tensor] = ss;
+            }
         }
     }
 
@@ -317,6 +435,66 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         tmem_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                      ::"r"(tmem), "r"(kGemmTmemCols) : "memory");
+    }
+}
+
+// The normalisation that completes the fused epilogue: one warp per (tensor, row) sums
+// the row's partial sums of squares (lane-strided, then a butterfly: a fixed order, so
+// slices and wholes agree bit for bit) and scales the row's dim bf16 values -- q in q_out,
+// K in its cache row -- by 1 / sqrt(mean + eps) in place, 16 bytes per lane and access,
+// kScaleUnroll accesses in flight per lane.
+constexpr int kScaleWarps = 8;
+constexpr int kScaleUnroll = 4;
+
+__global__ void __launch_bounds__(32 * kScaleWarps)
+qk_row_scale_kernel(const GemmParams p) {
+    pdl_launch_dependents();
+    pdl_wait_previous_grid();
+    const int task = blockIdx.x * kScaleWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (task >= 2 * p.M) return;
+    const int which = task >= p.M ? 1 : 0;  // 0 q, 1 K
+    const int row = task - which * p.M;
+    const int tiles = p.dim / kGemmBN;
+    const float* ps = p.psum + ((int64_t)which * p.M + row) * tiles;
+    float part = 0.0f;
+    for (int k = lane; k < tiles; k += 32) part += __ldg(ps + k);
+    const float rs = rsqrtf(fmaf(warp_allreduce_sum(part), p.inv_dim, p.eps));
+    const int64_t b = row / p.n_tok;
+    const int64_t i = p.token_begin + (row - b * p.n_tok);
+    const int64_t crow = (p.slot + i) % p.cache_tokens;
+    const int vpr = p.dim / 8;
+    for (int v0 = lane; v0 < vpr; v0 += 32 * kScaleUnroll) {
+        uint4* ptr[kScaleUnroll];
+        uint4 x[kScaleUnroll];
+#pragma unroll
+        for (int u = 0; u < kScaleUnroll; ++u) {
+            const int v = v0 + 32 * u;
+            ptr[u] = nullptr;
+            if (v < vpr) {
+                const int col = v * 8;
+                ptr[u] = reinterpret_cast<uint4*>(
+                    which == 0 ? p.q_out + (int64_t)row * p.dim + col
+                    : !p.cache_head_major
+                        ? p.k_cache + (b * p.cache_tokens + crow) * p.dim + col
+                        : p.k_cache + ((b * p.n_heads + (col >> 7)) * p.cache_tokens + crow) * 128 +
+                              (col & 127));
+                x[u] = __ldcs(ptr[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kScaleUnroll; ++u) {
+            if (ptr[u] == nullptr) continue;
+            uint32_t* w4 = reinterpret_cast<uint32_t*>(&x[u]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w4[q]);
+                const float2 f = __bfloat1622float2(h);
+                h = __floats2bfloat162_rn(f.x * rs, f.y * rs);
+                w4[q] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            __stcs(ptr[u], x[u]);
+        }
     }
 }
 

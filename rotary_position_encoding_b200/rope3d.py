@@ -88,9 +88,10 @@ SIGNATURES = {
                                        ctypes.POINTER(rope3d_sp_dest), _I64, _I64, _VP, _INT,
                                        ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_qkv_project": ([_VP, _VP, _VP, _I64, _I64, _I64, _INT, _VP, _VP, _VP, _VP], _INT),
+    "rope3d_qkv_workspace_bytes": ([_I64, _I64, _I64, _INT], ctypes.c_size_t),
     "rope3d_qkv_norm_rope_append": ([_VP, _VP, _VP, _I64, _I64, _I64, _INT, _I64, _I64, _I64,
-                                     _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP, _VP, _VP,
-                                     _VP, _I64, _I64, _VP, _INT,
+                                     _INT, _INT, _INT, _VP, _VP, ctypes.c_float, _VP, _VP,
+                                     ctypes.c_size_t, _VP, _VP, _I64, _I64, _VP, _INT,
                                      ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_apply": ([_VP, _VP, _I64, _I64, _INT, _INT, _I64, _I64, _I64, _INT, _INT, _INT, _VP,
                       _INT, _VP], _INT),
@@ -399,38 +400,44 @@ def rope3d_qkv_project(x, w_qkv, b_qkv, q_out, k_out, v_out, stream=None) -> Non
         _stream(stream)))
 
 
-def rope3d_qkv_norm_rope_append(x, w_qkv, b_qkv, q_out, k_work, token_begin: int,
+def rope3d_qkv_workspace_bytes(B: int, n_tok: int, N: int, D: int = 128) -> int:
+    return int(load_library().rope3d_qkv_workspace_bytes(B, n_tok, N, D))
+
+
+def rope3d_qkv_norm_rope_append(x, w_qkv, b_qkv, q_out, workspace, token_begin: int,
                                 token_end: int, frame_offset: int, T: int, H: int, W: int,
                                 q_norm_w, k_norm_w, eps: float, k_cache, v_cache, slot: int,
                                 tables: Tables, trig: int = ROPE3D_TRIG_TABLE,
                                 cache_layout: int = ROPE3D_CACHE_TOKEN_MAJOR,
                                 stream=None) -> None:
     """x [B, n_tok, K] bf16 -> q_out [B, n_tok, N, 128] and the caches, through the QKV
-    projection (w_qkv [3 N 128, K], b_qkv [3 N 128] float32 or None); k_work is a
-    [B, n_tok, N, 128] bf16 work buffer."""
+    projection (w_qkv [3 N 128, K], b_qkv [3 N 128] float32 or None).  workspace: a uint8
+    device tensor of at least rope3d_qkv_workspace_bytes(B, n_tok, N) bytes (scratch)."""
     if x.dim() != 3 or q_out.dim() != 4:
         raise ValueError("x must be [B, n_tok, K] and q_out [B, n_tok, N, D]")
     B, n_tok, K = x.shape
     N, D = q_out.shape[2], q_out.shape[3]
-    if tuple(q_out.shape[:2]) != (B, n_tok) or k_work.shape != q_out.shape:
-        raise ValueError("q_out and k_work must be [B, n_tok, N, D]")
+    if tuple(q_out.shape[:2]) != (B, n_tok):
+        raise ValueError("q_out must be [B, n_tok, N, D]")
     if n_tok != token_end - token_begin:
         raise ValueError("x has n_tok rows but the range holds token_end - token_begin")
     if tuple(w_qkv.shape) != (3 * N * D, K):
         raise ValueError("w_qkv must be [3 N D, K]")
     C = k_cache.shape[2] if cache_layout == ROPE3D_CACHE_HEAD_MAJOR else k_cache.shape[1]
-    for name, t in (("x", x), ("w_qkv", w_qkv), ("q_out", q_out), ("k_work", k_work),
-                    ("k_cache", k_cache), ("v_cache", v_cache)):
+    for name, t in (("x", x), ("w_qkv", w_qkv), ("q_out", q_out), ("k_cache", k_cache),
+                    ("v_cache", v_cache)):
         if t.dtype != torch.bfloat16:
             raise TypeError(f"{name} must be bfloat16")
+    nbytes = workspace.numel() * workspace.element_size()
     opts = rope3d_options(ROPE3D_PAIRING_ADJACENT, cache_layout)
     _check(load_library().rope3d_qkv_norm_rope_append(
         _dev_ptr(x, "x"), _dev_ptr(w_qkv, "w_qkv"),
         None if b_qkv is None else _dev_ptr(b_qkv, "b_qkv"), K, B, N, D, token_begin,
         token_end, frame_offset, T, H, W, _dev_ptr(q_norm_w, "q_norm_w"),
         _dev_ptr(k_norm_w, "k_norm_w"), eps, _dev_ptr(q_out, "q_out"),
-        _dev_ptr(k_work, "k_work"), _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
-        C, slot, tables.handle, trig, ctypes.byref(opts), _stream(stream)))
+        _dev_ptr(workspace, "workspace"), nbytes, _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), C, slot, tables.handle, trig, ctypes.byref(opts),
+        _stream(stream)))
 
 
 def rope3d_apply_ex(x, out, token_begin: int, token_end: int, frame_offset: int, T: int, H: int,

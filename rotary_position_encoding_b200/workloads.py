@@ -175,10 +175,11 @@ def hidden_states(w: Workload, chunk_index: int, K: int, n_tok: int | None = Non
 
 
 def projection_weights(seed: int, dim: int, K: int):
-    """A QKV projection: weight [3 dim, K] ~ N(0, 1/K) as bf16 bits (so that the projected
-    values are about N(0,1)) and bias [3 dim] ~ N(0, 0.1^2) float32."""
+    """A QKV projection: weight [3 dim, K] ~ N(0, 4/K) as bf16 bits (so that the projected
+    values are about N(0, 4): the RMSNorm then halves them) and bias [3 dim] ~ N(0, 0.1^2)
+    float32."""
     rng = rng_for(seed, 3000)
-    w = rng.standard_normal(size=(3 * dim, K), dtype=np.float32) * np.float32(1.0 / np.sqrt(K))
+    w = rng.standard_normal(size=(3 * dim, K), dtype=np.float32) * np.float32(2.0 / np.sqrt(K))
     b = (rng.standard_normal(size=3 * dim, dtype=np.float32) * np.float32(0.1))
     return f32_to_bf16_bits(w), b
 
