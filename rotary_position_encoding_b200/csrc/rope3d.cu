@@ -533,6 +533,7 @@ int launch_qkv_gemm(const void* x, const void* w, rope3d::GemmParams& gp, int de
     gp.num_m = (gp.M + rope3d::kGemmBM - 1) / rope3d::kGemmBM;
     gp.num_n = (gp.n_out + rope3d::kGemmBN - 1) / rope3d::kGemmBN;
     gp.wait_limit_ns = g_wait_limit_ns.load();
+    gp.tx_extra = g_tx_extra.load();
     const void* fn = reinterpret_cast<const void*>(rope3d::qkv_proj_kernel);
     if ((int)rope3d::kGemmSmemBytes > info.max_smem_optin)
         return fail(ROPE3D_EDEVICE, "the projection needs %zu bytes of shared memory",

@@ -40,6 +40,9 @@ constexpr int kGemmGroupM = 32;
 constexpr uint32_t kGemmStageA = kGemmBM * kGemmBK * 2;  // 16 KB
 constexpr uint32_t kGemmStageB = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr uint32_t kGemmTmemCols = 2 * kGemmBN;          // two accumulators
+// Waits for work already issued (copies, tensor-core operations) before a CTA that gave up
+// leaves: independent of the test-adjustable limit, so nothing is left in flight.
+constexpr uint64_t kGemmDrainLimitNs = 250000000ull;  // 250 ms
 // dynamic shared memory: 1 KB alignment slack, the stages, then barriers and the
 // epilogue's row scales
 constexpr size_t kGemmSmemBytes = 1024 + kGemmStages * (kGemmStageA + kGemmStageB) + 1024;
@@ -58,6 +61,7 @@ struct GemmParams {
     int n_heads;
     int cache_head_major;
     uint64_t wait_limit_ns;
+    uint32_t tx_extra;         // extra bytes each stage waits for (0; tests use it to time out)
     int* status;
     // fused QK-RMSNorm + RoPE epilogue (dim a multiple of 256, so every tile is all q, all
     // k or all v): q and K tiles are stored weighted and rotated but not yet normalised,
@@ -229,7 +233,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                         *s_fail = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar + 8 * s, kGemmStageA + kGemmStageB);
+                    mbar_arrive_expect_tx(full_bar + 8 * s, kGemmStageA + kGemmStageB + p.tx_extra);
                     tma_load_2d(stage_a + s * kGemmStageA, &map_x, kk * kGemmBK, mb * kGemmBM,
                                 full_bar + 8 * s);
                     tma_load_2d(stage_b + s * kGemmStageB, &map_w, kk * kGemmBK, nb * kGemmBN,
@@ -241,7 +245,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             if (*s_fail) {  // let copies already issued land before the CTA can exit
                 for (int j = 0; j < armed; ++j) {
                     if (--s < 0) { s = kGemmStages - 1; phase ^= 1; }
-                    mbar_wait_bounded(full_bar + 8 * s, phase, p.wait_limit_ns);
+                    mbar_wait_bounded(full_bar + 8 * s, phase, kGemmDrainLimitNs);
                 }
             }
         }
@@ -275,7 +279,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 umma_commit(tfull_bar + 8 * acc);
             }
             umma_commit(drain_bar);  // every tensor-core operation of this CTA is done
-            mbar_wait_bounded(drain_bar, 0, p.wait_limit_ns);
+            mbar_wait_bounded(drain_bar, 0, kGemmDrainLimitNs);
         }
     } else {  // epilogue warps 2..5: lanes 32 (warp % 4) .. +32 of tensor memory
         const int quarter = warp & 3;

@@ -274,3 +274,30 @@ def test_argument_errors():
     assert fused(nbytes=ws.numel() - 1) == rope3d.ROPE3D_EINVAL
     assert rope3d.rope3d_qkv_workspace_bytes(0, 10, 4) == 0
     torch.cuda.synchronize()
+
+
+def test_projection_wait_timeout_reports_status():
+    """A projection whose stages can never fill (the test hook makes every stage wait for
+    16 bytes that no copy delivers) gives up after the wait limit: the tables' status word
+    reports ROPE3D_ETIMEOUT, the kernel's copies and tensor-core work are drained and its
+    tensor memory released, and the next call runs normally and correctly."""
+    c = _fused_case(TOKEN)
+    tables = rope3d.rope3d_tables_init(max_t=c["s"] + c["T"], max_h=c["H"], max_w=c["W"])
+    rope3d.rope3d_testing_set_waits(20_000_000, 16)  # 20 ms
+    try:
+        _run_fused(c, tables, 0, c["L"])
+        assert rope3d.rope3d_check_device_status(tables) == rope3d.ROPE3D_ETIMEOUT
+    finally:
+        rope3d.rope3d_testing_set_waits(0, 0)
+    assert rope3d.rope3d_check_device_status(tables) == rope3d.ROPE3D_OK
+    qo, _, kc, vc = _run_fused(c, tables, 0, c["L"])
+    assert rope3d.rope3d_check_device_status(tables) == rope3d.ROPE3D_OK
+    x64 = wl.bf16_bits_to_f64(c["x"])
+    w64 = wl.bf16_bits_to_f64(c["w"])
+    kr, vr = np.full(tuple(kc.shape), 2.0), np.full(tuple(vc.shape), -2.0)
+    q_ref = oracle.default().qkv_norm_rope_append(
+        x64, w64, c["b"], c["N"], 0, c["L"], c["s"], c["T"], c["H"], c["W"],
+        c["wq"].astype(np.float64), c["wk"].astype(np.float64), 1e-6, kr, vr, c["slot"],
+        round_bf16=False)
+    assert_close(to_f64(qo), q_ref, "bf16", "q_out after a timed-out call")
+    assert_close(to_f64(kc), kr, "bf16", "k_cache after a timed-out call")
