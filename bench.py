@@ -640,7 +640,7 @@ def run_qkv(args, dist: Dist):
                      "avg_launch_ms": round(gemm_ms, 4),
                      "cublas_same_gemm_ms": round(cublas_ms, 4),
                      "cublas_tflops": round(flops / (cublas_ms / 1e3) / 1e12, 1)},
-        "gpu_launches": (1 if (w.dim % 256 == 0) else 2) * len(w.chunks) * args.steps,
+        "gpu_launches": 2 * len(w.chunks) * args.steps,  # projection + row scale (or step)
         "clocks": clock_info,
     }
 
