@@ -79,6 +79,9 @@ def parse_args(argv=None):
     ap.add_argument("--qkv", action="store_true",
                     help="the QKV-projection-fed step: token rows x [n, N*128] through the "
                          "tcgen05 projection (V appended by its epilogue), then the step")
+    ap.add_argument("--gemm-form", type=int, choices=[0, 1, 2], default=0,
+                    help="--qkv: projection kernel form (1: one CTA per tile, 2: 2-CTA pairs, "
+                         "0: the library default, 2)")
     ap.add_argument("--eager", action="store_true",
                     help="launch every chunk call from Python and time each launch with its "
                          "own CUDA event pair (default: capture one step -- all its chunk "
@@ -553,6 +556,7 @@ def run_qkv(args, dist: Dist):
     tables = rope3d.rope3d_tables_init(max_t=max(c.frame_offset for c in w.chunks) + w.T,
                                        max_h=w.H, max_w=w.W)
     stream = torch.cuda.current_stream(device)
+    rope3d.rope3d_testing_gemm_cta_group(args.gemm_form)
 
     def step():
         for ci, c in enumerate(w.chunks):
@@ -635,7 +639,7 @@ def run_qkv(args, dist: Dist):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peak_kind} bf16_tflops_sustained (back-to-back launches)",
-                     "kernel": "rope3d::qkv_proj_kernel",
+                     "kernel": "rope3d::qkv_proj_kernel<%d>" % (args.gemm_form or 2),
                      "algorithmic_flops_per_launch": flops,
                      "avg_launch_ms": round(gemm_ms, 4),
                      "cublas_same_gemm_ms": round(cublas_ms, 4),

@@ -30,6 +30,11 @@ ROPE3D_API void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_ext
 /* Choose the kernel path for later launches (ROPE3D_PATH_*).  EINVAL for other values. */
 ROPE3D_API int rope3d_testing_force_path(int path);
 
+/* Form of the QKV projection kernel for later launches: 1 = one CTA per 128x256 tile
+ * (tcgen05 cta_group::1), 2 = a pair of CTAs in a cluster per 256x256 tile (cta_group::2,
+ * each CTA loading half of the weight rows), 0 = the default (2).  EINVAL otherwise. */
+ROPE3D_API int rope3d_testing_gemm_cta_group(int group);
+
 /* The path (ROPE3D_PATH_REGISTERS or ROPE3D_PATH_TMA) of the calling thread's most recent
  * successful rope3d_qk_norm_rope_append launch; ROPE3D_PATH_AUTO before the first. */
 ROPE3D_API int rope3d_testing_last_path(void);

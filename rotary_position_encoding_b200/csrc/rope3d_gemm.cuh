@@ -43,9 +43,10 @@ constexpr uint32_t kGemmTmemCols = 2 * kGemmBN;          // two accumulators
 // Waits for work already issued (copies, tensor-core operations) before a CTA that gave up
 // leaves: independent of the test-adjustable limit, so nothing is left in flight.
 constexpr uint64_t kGemmDrainLimitNs = 250000000ull;  // 250 ms
-// dynamic shared memory: 1 KB alignment slack, the stages, then barriers and the
-// epilogue's row scales
-constexpr size_t kGemmSmemBytes = 1024 + kGemmStages * (kGemmStageA + kGemmStageB) + 1024;
+// dynamic shared memory: 1 KB alignment slack, the stages, the barriers, and 16 KB that
+// keeps every tensor-core operand read of the pair form inside the allocation
+constexpr size_t kGemmSmemBytes =
+    1024 + kGemmStages * (kGemmStageA + kGemmStageB) + 1024 + 16384;
 
 struct GemmParams {
     int M;                 // token rows (B * n_tok)
@@ -163,6 +164,69 @@ __device__ __forceinline__ bool epi_vote_all(bool v) {
     return r != 0;
 }
 
+// ---- the pair form (cta_group::2): two CTAs of a cluster share each 256x256 tile; each
+// holds 128 rows of x and 128 rows of W per stage and 128 accumulator rows, and the even
+// CTA issues the tensor-core operations for both.
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The address of this CTA's shared-memory word `addr` in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.aligned;\nbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 ::"r"(cluster_addr) : "memory");
+}
+// 2-D TMA load into this CTA's shared memory completing on a barrier of either CTA of the
+// pair (no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x,
+                                                 int y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+// Instruction descriptor of the pair form: M = 256 across the two CTAs, N = 256.
+constexpr uint32_t kGemmIdescPair = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(kGemmBN >> 3) << 17) |
+                                    ((uint32_t)(2 * kGemmBM >> 4) << 24);
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kGemmIdescPair), "r"(accumulate)
+        : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the pair's
+// tensor-core operations issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+    asm volatile(
+        "{\n .reg .b16 m;\n mov.b16 m, 3;\n"
+        " tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], m;\n}" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+        ::"r"(bar) : "memory");
+}
+
+template <int G> struct GemmShape {
+    static constexpr int kStages = G == 1 ? kGemmStages : 6;
+    static constexpr uint32_t kStageB = (kGemmBN / G) * kGemmBK * 2;  // this CTA's W rows
+    static constexpr int kTileM = kGemmBM * G;                       // rows of a tile
+};
+
 // Tile t -> (row block, column block), grouped kGemmGroupM row blocks at a time.
 __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int t, int& mb, int& nb) {
     const int per_group = kGemmGroupM * p.num_n;
@@ -174,24 +238,31 @@ __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int t, int
     nb = r / rows;
 }
 
+template <int G>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                 const GemmParams p) {
+    constexpr int STAGES = GemmShape<G>::kStages;
+    constexpr uint32_t STAGE_B = GemmShape<G>::kStageB;
+    constexpr int TILE_M = GemmShape<G>::kTileM;
     extern __shared__ uint8_t gemm_smem_raw[];
     const uint32_t raw = smem_u32(gemm_smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // 1 KB aligned: the swizzle atoms
     const uint32_t stage_a = base;
-    const uint32_t stage_b = base + kGemmStages * kGemmStageA;
-    const uint32_t bars = stage_b + kGemmStages * kGemmStageB;
+    const uint32_t stage_b = base + STAGES * kGemmStageA;
+    const uint32_t bars = stage_b + STAGES * STAGE_B;
     // barriers: full[S], empty[S], tmem_full[2], tmem_empty[2], drain; then the TMEM
     // address and the failure flag
-    const uint32_t full_bar = bars, empty_bar = bars + 8 * kGemmStages;
-    const uint32_t tfull_bar = bars + 16 * kGemmStages, tempty_bar = tfull_bar + 16;
+    const uint32_t full_bar = bars, empty_bar = bars + 8 * STAGES;
+    const uint32_t tfull_bar = bars + 16 * STAGES, tempty_bar = tfull_bar + 16;
     const uint32_t drain_bar = tempty_bar + 16;
+    const uint32_t rank = G == 2 ? cluster_rank() : 0;
+    const int first_tile = G == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int tile_stride = G == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     uint8_t* gen_base = gemm_smem_raw + (base - raw);
     const uint32_t bars_off = bars - base;
-    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(gen_base + bars_off + 128);
-    volatile int* s_fail = reinterpret_cast<volatile int*>(gen_base + bars_off + 136);
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(gen_base + bars_off + 256);
+    volatile int* s_fail = reinterpret_cast<volatile int*>(gen_base + bars_off + 264);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -199,25 +270,32 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     const int k_steps = p.K / kGemmBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGemmStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar + 8 * s, 1);
             mbar_init(empty_bar + 8 * s, 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(tfull_bar + 8 * a, 1);
-            mbar_init(tempty_bar + 8 * a, 128);
+            mbar_init(tempty_bar + 8 * a, 128 * G);  // the epilogue threads of every CTA
         }
         mbar_init(drain_bar, 1);
         *s_fail = 0;
         fence_barrier_init();
     }
     if (warp == 1) {  // whole warp: allocate the accumulators' tensor memory
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     ::"r"(smem_u32((const void*)s_tmem)), "r"(kGemmTmemCols) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (G == 1) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32((const void*)s_tmem)), "r"(kGemmTmemCols) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32((const void*)s_tmem)), "r"(kGemmTmemCols) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        }
     }
     tmem_fence_before();
     __syncthreads();
+    if constexpr (G == 2) cluster_sync();  // both CTAs' barriers exist before any use
     tmem_fence_after();
     const uint32_t tmem = *s_tmem;
 
@@ -225,7 +303,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         if (lane == 0) {  // producer
             int s = 0, phase = 0;
             int armed = 0;  // stages armed and not yet known consumed (for the failure drain)
-            for (int t = blockIdx.x; t < num_tiles && !*s_fail; t += gridDim.x) {
+            for (int t = first_tile; t < num_tiles && !*s_fail; t += tile_stride) {
                 int mb, nb;
                 gemm_tile_coords(p, t, mb, nb);
                 for (int kk = 0; kk < k_steps; ++kk) {
@@ -233,26 +311,40 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                         *s_fail = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar + 8 * s, kGemmStageA + kGemmStageB + p.tx_extra);
-                    tma_load_2d(stage_a + s * kGemmStageA, &map_x, kk * kGemmBK, mb * kGemmBM,
-                                full_bar + 8 * s);
-                    tma_load_2d(stage_b + s * kGemmStageB, &map_w, kk * kGemmBK, nb * kGemmBN,
-                                full_bar + 8 * s);
-                    armed = min(armed + 1, kGemmStages);
-                    if (++s == kGemmStages) { s = 0; phase ^= 1; }
+                    if constexpr (G == 1) {
+                        mbar_arrive_expect_tx(full_bar + 8 * s,
+                                              kGemmStageA + STAGE_B + p.tx_extra);
+                        tma_load_2d(stage_a + s * kGemmStageA, &map_x, kk * kGemmBK,
+                                    mb * kGemmBM, full_bar + 8 * s);
+                        tma_load_2d(stage_b + s * STAGE_B, &map_w, kk * kGemmBK, nb * kGemmBN,
+                                    full_bar + 8 * s);
+                    } else {
+                        // both CTAs' copies complete on the even CTA's barrier, which
+                        // expects the pair's bytes
+                        const uint32_t bar = map_to_rank(full_bar + 8 * s, 0);
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(full_bar + 8 * s,
+                                                  2 * (kGemmStageA + STAGE_B) + p.tx_extra);
+                        tma_load_2d_pair(stage_a + s * kGemmStageA, &map_x, kk * kGemmBK,
+                                         mb * TILE_M + (int)rank * kGemmBM, bar);
+                        tma_load_2d_pair(stage_b + s * STAGE_B, &map_w, kk * kGemmBK,
+                                         nb * kGemmBN + (int)rank * (kGemmBN / 2), bar);
+                    }
+                    armed = min(armed + 1, STAGES);
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
             }
-            if (*s_fail) {  // let copies already issued land before the CTA can exit
+            if (*s_fail && (G == 1 || rank == 0)) {  // let copies already issued land
                 for (int j = 0; j < armed; ++j) {
-                    if (--s < 0) { s = kGemmStages - 1; phase ^= 1; }
+                    if (--s < 0) { s = STAGES - 1; phase ^= 1; }
                     mbar_wait_bounded(full_bar + 8 * s, phase, kGemmDrainLimitNs);
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {  // MMA issuer
+        if (lane == 0 && rank == 0) {  // MMA issuer (the even CTA of a pair)
             int s = 0, phase = 0, it = 0;
-            for (int t = blockIdx.x; t < num_tiles && !*s_fail; t += gridDim.x, ++it) {
+            for (int t = first_tile; t < num_tiles && !*s_fail; t += tile_stride, ++it) {
                 const int acc = it & 1;
                 const int use = it >> 1;  // how many times this accumulator was used before
                 if (!mbar_wait_bounded(tempty_bar + 8 * acc, (use & 1) ^ 1, p.wait_limit_ns)) {
@@ -268,17 +360,26 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     }
                     tmem_fence_after();
                     const uint64_t adesc = smem_desc_sw128(stage_a + s * kGemmStageA);
-                    const uint64_t bdesc = smem_desc_sw128(stage_b + s * kGemmStageB);
+                    const uint64_t bdesc = smem_desc_sw128(stage_b + s * STAGE_B);
 #pragma unroll
-                    for (int k = 0; k < kGemmBK / 16; ++k)  // 16 bf16 = 32 bytes along K
-                        umma_bf16(d, adesc + 2 * k, bdesc + 2 * k, (kk | k) != 0);
-                    umma_commit(empty_bar + 8 * s);  // the stage is free once these complete
-                    if (++s == kGemmStages) { s = 0; phase ^= 1; }
+                    for (int k = 0; k < kGemmBK / 16; ++k) {  // 16 bf16 = 32 bytes along K
+                        if constexpr (G == 1)
+                            umma_bf16(d, adesc + 2 * k, bdesc + 2 * k, (kk | k) != 0);
+                        else
+                            umma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, (kk | k) != 0);
+                    }
+                    // the stage is free (in every CTA) once these complete
+                    if constexpr (G == 1) umma_commit(empty_bar + 8 * s);
+                    else umma_commit_pair_both(empty_bar + 8 * s);
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
                 if (*s_fail) break;
-                umma_commit(tfull_bar + 8 * acc);
+                if constexpr (G == 1) umma_commit(tfull_bar + 8 * acc);
+                else umma_commit_pair_both(tfull_bar + 8 * acc);
             }
-            umma_commit(drain_bar);  // every tensor-core operation of this CTA is done
+            // every tensor-core operation of this CTA (pair) is done
+            if constexpr (G == 1) umma_commit(drain_bar);
+            else umma_commit_pair(drain_bar);
             mbar_wait_bounded(drain_bar, 0, kGemmDrainLimitNs);
         }
     } else {  // epilogue warps 2..5: lanes 32 (warp % 4) .. +32 of tensor memory
@@ -286,7 +387,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const int row_in_tile = quarter * 32 + lane;
         const int tiles_per_tensor = p.dim / kGemmBN;
         int it = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+        for (int t = first_tile; t < num_tiles; t += tile_stride, ++it) {
             if (epi_vote_any(*s_fail != 0)) break;  // the group leaves together
             int mb, nb;
             gemm_tile_coords(p, t, mb, nb);
@@ -298,7 +399,7 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 break;
             }
             tmem_fence_after();
-            const int row = mb * kGemmBM + row_in_tile;
+            const int row = mb * TILE_M + (int)rank * kGemmBM + row_in_tile;
             const bool live = row < p.M;
             const int which_tile = (nb * kGemmBN) / p.dim;  // 0 q, 1 k, 2 v (fused layout)
             const bool norm_tile = p.fused && which_tile < 2;
@@ -422,7 +523,9 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                                        packed[4 * j + 3]);
             }
             tmem_fence_before();
-            mbar_arrive(tempty_bar + 8 * acc);  // the accumulator is free for the next tile
+            // the accumulator is free for the next tile (the even CTA's barrier counts both)
+            if constexpr (G == 1) mbar_arrive(tempty_bar + 8 * acc);
+            else mbar_arrive_cluster(map_to_rank(tempty_bar + 8 * acc, 0));
             // record this row's partial sum of squares over the tile's columns
             if (norm_tile && live) {
                 const int tile_in_tensor = nb - which_tile * tiles_per_tensor;
@@ -434,11 +537,18 @@ qkv_proj_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __syncwarp();  // the role lanes rejoin their warps
     tmem_fence_before();
     __syncthreads();
+    // the pair stays resident until the even CTA's last operations on the odd CTA's
+    // shared memory and barriers are done
+    if constexpr (G == 2) cluster_sync();
     if (*s_fail && threadIdx.x == 0 && p.status != nullptr) atomicExch(p.status, kStatusWaitTimeout);
     if (warp == 1) {
         tmem_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     ::"r"(tmem), "r"(kGemmTmemCols) : "memory");
+        if constexpr (G == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                         ::"r"(tmem), "r"(kGemmTmemCols) : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                         ::"r"(tmem), "r"(kGemmTmemCols) : "memory");
     }
 }
 

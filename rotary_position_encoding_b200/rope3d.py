@@ -108,6 +108,7 @@ SIGNATURES = {
     "rope3d_version": ([], _INT),
     "rope3d_testing_set_waits": ([ctypes.c_uint64, ctypes.c_uint32], None),
     "rope3d_testing_force_path": ([_INT], _INT),
+    "rope3d_testing_gemm_cta_group": ([_INT], _INT),
     "rope3d_testing_last_path": ([], _INT),
 }
 
@@ -492,6 +493,10 @@ def rope3d_testing_set_waits(wait_limit_ns: int = 0, tx_extra_bytes: int = 0) ->
 
 def rope3d_testing_force_path(path: int = ROPE3D_PATH_AUTO) -> None:
     _check(load_library().rope3d_testing_force_path(path))
+
+
+def rope3d_testing_gemm_cta_group(group: int = 0) -> None:
+    _check(load_library().rope3d_testing_gemm_cta_group(group))
 
 
 def rope3d_testing_last_path() -> int:

@@ -53,9 +53,18 @@ def _check_projection(x_bits, w_bits, b, outs, rows=None):
     assert np.all(err <= bound), f"{int((err > bound).sum())} projected values out of bound"
 
 
+@pytest.fixture(params=[1, 2], ids=["cta1", "pair"])
+def gemm_form(request):
+    """Both forms of the projection kernel: one CTA per tile, or a 2-CTA pair."""
+    rope3d.rope3d_testing_gemm_cta_group(request.param)
+    yield request.param
+    rope3d.rope3d_testing_gemm_cta_group(0)
+
+
 @pytest.mark.parametrize("M,K,N,bias", [(200, 128, 2, True), (130, 256, 5, False),
-                                        (1, 64, 1, True), (384, 1536, 12, True)])
-def test_projection_small(M, K, N, bias):
+                                        (1, 64, 1, True), (384, 1536, 12, True),
+                                        (700, 512, 4, True)])
+def test_projection_small(M, K, N, bias, gemm_form):
     rng = np.random.default_rng(M + K + N)
     x_bits = wl.f32_to_bf16_bits(rng.standard_normal((M, K), dtype=np.float32))
     w_bits = wl.f32_to_bf16_bits(rng.standard_normal((3 * N * D, K), dtype=np.float32)
@@ -105,7 +114,7 @@ def _run_fused(c, tables, tb, te, ws=None):
 @pytest.mark.parametrize("layout", [TOKEN, HEAD])
 @pytest.mark.parametrize("N", [4, 5])
 @pytest.mark.parametrize("trig", [rope3d.ROPE3D_TRIG_TABLE, rope3d.ROPE3D_TRIG_ONTHEFLY])
-def test_fused_small_against_oracle(layout, N, trig):
+def test_fused_small_against_oracle(layout, N, trig, gemm_form):
     c = _fused_case(layout, N=N)
     tables = rope3d.rope3d_tables_init(max_t=c["s"] + c["T"], max_h=c["H"], max_w=c["W"])
     cshape = ((c["B"], c["C"], N, D) if layout == TOKEN else (c["B"], N, c["C"], D))
@@ -149,7 +158,7 @@ def test_fused_small_against_oracle(layout, N, trig):
 
 @pytest.mark.parametrize("layout", [TOKEN, HEAD])
 @pytest.mark.parametrize("N", [12, 5])
-def test_fused_against_projection_then_step(layout, N):
+def test_fused_against_projection_then_step(layout, N, gemm_form):
     """Against rope3d_qkv_project followed by the plain step on its outputs: V cache rows
     bit-identical always; q and K bit-identical for odd head counts (the same two passes)
     and within the bf16 tolerance of each other for even ones (the epilogue normalises the
@@ -195,7 +204,7 @@ def test_fused_against_projection_then_step(layout, N):
 
 
 @pytest.mark.slow
-def test_720p_chunk_sampled_rows():
+def test_720p_chunk_sampled_rows(gemm_form):
     """The Wan-14B-shaped 720P chunk: 10800 tokens of 5120 features, 40 heads; sampled
     rows of the projection and of the step against the oracle."""
     w = wl.chunk_720p()
@@ -276,7 +285,7 @@ def test_argument_errors():
     torch.cuda.synchronize()
 
 
-def test_projection_wait_timeout_reports_status():
+def test_projection_wait_timeout_reports_status(gemm_form):
     """A projection whose stages can never fill (the test hook makes every stage wait for
     16 bytes that no copy delivers) gives up after the wait limit: the tables' status word
     reports ROPE3D_ETIMEOUT, the kernel's copies and tensor-core work are drained and its
