@@ -36,7 +36,7 @@ constexpr int kGemmBN = 256;
 constexpr int kGemmBK = 64;   // 64 bf16 = 128 bytes: one swizzle row
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;
-constexpr int kGemmGroupM = 32;
+constexpr int kGemmGroupM = 16;
 constexpr uint32_t kGemmStageA = kGemmBM * kGemmBK * 2;  // 16 KB
 constexpr uint32_t kGemmStageB = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr uint32_t kGemmTmemCols = 2 * kGemmBN;          // two accumulators
