@@ -217,3 +217,22 @@ def test_bench_timing_is_max_over_ranks(tmp_path):
     assert int(world) == 2
     assert float(worst) == 20.0
     assert float(value) == pytest.approx(75600 * 3 * 2 / 0.020)
+
+
+def test_sp_plan_layout():
+    """The per-rank allocation plan: regions 256-byte aligned, in order q, K, V, sized for
+    the rank's heads; uneven head splits are refused."""
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    from rotary_position_encoding_b200 import rope3d, sp
+    lay = sp.plan(B=2, N=40, P=8, q_rows=10800, cache_tokens=75600, dtype=torch.bfloat16)
+    assert lay.q_shape == (2, 10800, 5, 128) and lay.cache_shape == (2, 75600, 5, 128)
+    q_bytes = 2 * 10800 * 5 * 128 * 2
+    c_bytes = 2 * 75600 * 5 * 128 * 2
+    assert lay.q_off == 0 and lay.k_off >= q_bytes and lay.v_off >= lay.k_off + c_bytes
+    assert lay.nbytes >= lay.v_off + c_bytes
+    assert all(x % 256 == 0 for x in (lay.k_off, lay.v_off, lay.nbytes))
+    head = sp.plan(1, 12, 4, 100, 64, torch.bfloat16, rope3d.ROPE3D_CACHE_HEAD_MAJOR)
+    assert head.cache_shape == (1, 3, 64, 128)
+    with pytest.raises(ValueError):
+        sp.plan(1, 12, 5, 100, 64, torch.bfloat16)
