@@ -482,7 +482,7 @@ int rope3d_oracle_apply_pairing(const double* x, double* out, int64_t B, int64_t
  * nearest, ties to the even code, saturating at +-448.  A reader recovers
  * x ~ value(code) * scale.  The pages name
  * NVFP4 KV-cache quantization for Blackwell (the LongLive-2.0 abstract) but give no
- * format details; E4M3 with per-head scales is this build's reading.  The decision
+ * format details; E4M3 with per-head scales is the reading taken here.  The decision
  * runs in fp32 (the precision the kernel computes the rows in): the oracle rounds its
  * fp64 K row to fp32 first; V is exact.
  *
@@ -619,7 +619,7 @@ int rope3d_oracle_qk_norm_rope_append_fp8(
  * NVIDIA defines it): each block of 16 consecutive elements of a head holds 16 E2M1
  * codes and one E4M3 block scale S; a per-tensor fp32 scale g (the caller's, one for K
  * and one for V) sits above the block scales.  A reader recovers
- * x ~ value(code) * value(S) * g.  This build's rounding recipe, in fp32:
+ * x ~ value(code) * value(S) * g.  The rounding recipe used here, in fp32:
  *   k = 1 / (6 g)                      per tensor; 6 = E2M1's largest magnitude;
  *   S = E4M3(amax k)                   amax = largest |x| in the block;
  *   r = 1 / (value(S) g)  (0 if S is zero);

@@ -246,7 +246,7 @@ def test_symmetric_memory_wiring_one_rank():
     """The multi-GPU wiring (one symmetric-memory allocation per rank, the table of every
     rank's addresses, the step, the device barrier) on a one-rank NCCL group: the rank's
     own buffers hold the plain step's results bit for bit.  Runs with more ranks need
-    more GPUs than this build has."""
+    more than one GPU."""
     import datetime
     import socket
 
