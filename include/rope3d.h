@@ -279,7 +279,12 @@ ROPE3D_API int rope3d_qk_norm_rope_append_sp(
  * bias); fp32 accumulation, one round to nearest even to bf16.  The q, k and v column
  * blocks of y go to q_out, k_out, v_out, each [M][N][D] bf16.  K must be a multiple of
  * 64; x and w_qkv 16-byte aligned.  The kernel holds all of each SM's tensor memory while
- * it runs: calls on concurrent streams serialise on it.
+ * it runs: calls on concurrent streams serialise on it.  The caller owns every buffer; the
+ * call allocates nothing.  Its pipeline waits are bounded (2 s each); a launch that gives
+ * up leaves its outputs incomplete and, having no tables, reports nothing.  Errors: NULL
+ * pointers, D != 128, N < 1, M < 1, or K not a multiple of 64 or above 2^20 (EINVAL);
+ * M > 2^30 or 3 N D > 2^24 (ERANGE); misaligned pointers, a bias not 4-byte aligned
+ * (EALIGN); outputs that overlap x, w_qkv or one another (EOVERLAP); EDEVICE, ECUDA.
  */
 ROPE3D_API int rope3d_qkv_project(const void* x, const void* w_qkv, const float* b_qkv, int64_t M,
                                   int64_t K, int64_t N, int D, void* q_out, void* k_out,
@@ -300,9 +305,12 @@ ROPE3D_API int rope3d_qkv_project(const void* x, const void* w_qkv, const float*
  *   - Otherwise the projection rounds q and k to bf16 (q into q_out, k into the workspace)
  *     and the step then normalises and rotates them (V already in the cache).
  * workspace: device scratch of rope3d_qkv_workspace_bytes(B, n_tok, N, D) bytes (no
- * initialisation needed).  bf16 only; options: the cache layout (adjacent pairing, bf16
- * caches).  Other arguments and errors as for rope3d_qk_norm_rope_append and
- * rope3d_qkv_project.
+ * initialisation needed; 0 is returned for invalid sizes).  bf16 only; options: the cache
+ * layout (adjacent pairing, bf16 caches; EINVAL otherwise).  A workspace smaller than
+ * needed is EINVAL; q_out, the workspace and the caches must not overlap one another, x
+ * or w_qkv (EOVERLAP).  A wait that gives up is recorded in the tables' status word
+ * (rope3d_check_device_status).  Other arguments and errors as for
+ * rope3d_qk_norm_rope_append and rope3d_qkv_project.
  */
 ROPE3D_API size_t rope3d_qkv_workspace_bytes(int64_t B, int64_t n_tok, int64_t N, int D);
 
