@@ -775,8 +775,8 @@ class OracleSample:
                 have += w.B * (e - a)
         self.prepared = have
 
-    def run(self, budget_s: float, max_tokens=None):
-        """Returns (tokens, oracle seconds, threads)."""
+    def run(self, budget_s: float, max_tokens=None, nthreads=0):
+        """Returns (tokens, oracle seconds, threads); nthreads 0 means every core."""
         w = self.w
         done, spent, i = 0, 0.0, 0
         while True:
@@ -790,21 +790,27 @@ class OracleSample:
             t0 = time.perf_counter()
             self.orc.qk_norm_rope_append(f[0], f[1], f[2], a, e, chunk.frame_offset, w.T, w.H,
                                          w.W, self.wq64, self.wk64, w.eps, kc, vc, (-a) % m,
-                                         nthreads=0)
+                                         nthreads=nthreads)
             spent += time.perf_counter() - t0
             done += w.B * m
             if spent >= budget_s or (max_tokens is not None and done >= max_tokens):
-                return done, spent, self.orc.max_threads()
+                return done, spent, nthreads or self.orc.max_threads()
 
 
 def cpu_baseline(w, host, budget_s):
+    """The oracle on every host core for budget_s seconds, then on one core for a third of
+    that."""
     sampler = OracleSample(w, host)
     tokens, secs, threads = sampler.run(budget_s)
+    tok1, secs1, _ = sampler.run(budget_s / 3.0, nthreads=1)
     return {"value": round(tokens / secs, 1), "unit": "tokens/s", "cores": threads,
             "kind": "oracle",
             "sample": f"{tokens} tokens: the first {sampler.prepared} tokens of the step "
                       f"({w.name}) in 512-token sub-batches, cycled for {secs:.1f} s of fp64 "
-                      f"oracle time on {threads} OpenMP threads"}
+                      f"oracle time on {threads} OpenMP threads",
+            "single_thread": {"value": round(tok1 / secs1, 1), "unit": "tokens/s",
+                              "sample": f"{tok1} tokens of the same sample in {secs1:.1f} s "
+                                        f"on one thread"}}
 
 
 def run_reference(args, dist: Dist):

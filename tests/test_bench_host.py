@@ -66,3 +66,14 @@ def test_recorded_traffic_file_is_well_formed():
     for key, entry in rec.items():
         assert len(entry["kernel_source_sha256_16"]) == 16, key
         assert entry["dram_bytes_per_launch"] > 0, key
+
+
+def test_cpu_baseline_reports_all_cores_and_one():
+    w = bench.WORKLOADS["chunk480p"]()
+    w.chunks = w.chunks[:1]
+    host = bench.make_inputs(w, seed_offset=0)
+    cb = bench.cpu_baseline(w, host, 0.6)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s"
+    assert cb["value"] > 0 and cb["cores"] >= 1
+    one = cb["single_thread"]
+    assert one["value"] > 0 and one["unit"] == "tokens/s" and "one thread" in one["sample"]
