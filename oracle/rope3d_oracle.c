@@ -23,7 +23,8 @@
  *     instead takes one head-wide schedule theta^(-2j/D) for pair j = 0..D/2-1 and
  *     hands the first n_t pairs to t, the next n_h to h and the last n_w to w.
  *     The paper names the three per-axis frequency sets but prints no formula, so
- *     which schedule is meant is not pinned by it.
+ *     which schedule is meant is parity unpinned: both are computed here, and each
+ *     is pinned by its own closed forms.
  *   - h and w decode: the paper gives only the time index; h and w follow from
  *     the row-major (F, H, W) expansion of the frequency tables in its
  *     Algorithm 2, so h = floor(i / W) mod H and w = i mod W.
