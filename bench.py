@@ -90,6 +90,10 @@ def parse_args(argv=None):
     ap.add_argument("--chunks", type=int, default=0,
                     help="use only the first CHUNKS chunk calls per step (profiling captures "
                          "of a smaller case; 0 = the whole step)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads measured after the default 720P headline "
+                         "(480P chunk, whole 480P vs 8 slices, long horizon, FP8 and NVFP4 "
+                         "caches, 8-rank sequence-parallel step, QKV projection)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -181,6 +185,7 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.rows = None
         self.t_start = self.t_end = None
 
     def start(self):
@@ -198,7 +203,9 @@ class ClockSampler:
         setattr(self, "t_" + which, time.time())
 
     def stop(self):
+        """Stop sampling; the clock record of the timed region (marks "start" and "end")."""
         if self.proc is None:
+            self.rows = None
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.1)
         self.proc.terminate()
@@ -206,30 +213,38 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
+        self.rows = []
         with open(self.path) as f:
             for rec in csv.reader(f):
                 if len(rec) >= 10:
-                    rows.append([x.strip() for x in rec])
+                    self.rows.append([x.strip() for x in rec])
         os.unlink(self.path)
+        return self.window(self.t_start, self.t_end, "timed region")
+
+    @staticmethod
+    def _stamp(r):
+        try:
+            return time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S")) + \
+                float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
+        except ValueError:
+            return None
+
+    def window(self, t0, t1, name="window"):
+        """Median SM clock, maximum clock and throttle reasons of the samples taken between
+        host times t0 and t1 (all samples if none fall inside)."""
+        if self.rows is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = self.rows
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        # keep the samples taken inside the timed region when there are any
-        def stamp(r):
-            try:
-                return time.mktime(time.strptime(r[0].split(".")[0], "%Y/%m/%d %H:%M:%S")) + \
-                    float("0." + r[0].split(".")[1]) if "." in r[0] else 0.0
-            except ValueError:
-                return None
-        if self.t_start is not None and self.t_end is not None:
-            inside = [r for r in rows if (stamp(r) is not None
-                                          and self.t_start - 0.06 <= stamp(r) <= self.t_end + 0.06)]
-            window = "timed region"
+        window = "whole run"
+        if t0 is not None and t1 is not None:
+            inside = [r for r in rows if (self._stamp(r) is not None
+                                          and t0 - 0.06 <= self._stamp(r) <= t1 + 0.06)]
+            window = name
             if not inside:
-                inside, window = rows, "whole run (timed region shorter than the sampling period)"
+                inside, window = rows, f"whole run ({name} shorter than the sampling period)"
             rows = inside
-        else:
-            window = "whole run"
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
@@ -423,6 +438,15 @@ def run_ours(args, dist: Dist):
     else:
         launch_ms = [ev[2 * j].elapsed_time(ev[2 * j + 1]) for ev in per_step_events
                      for j in range(n_launch)]
+    headline_path = rope3d.rope3d_testing_last_path()
+    configs = None
+    if (not args.no_configs and dist.world == 1 and graph is not None and not P
+            and args.workload == "chunk720p" and not args.chunks
+            and (args.trig, args.pairing, args.cache_layout, args.cache_dtype, args.path)
+            == ("table", "adjacent", "token", "same", "auto")):
+        graph = None
+        configs = run_configs(torch, rope3d, device, stream, clocks, measured_peaks()[0],
+                              (w, inputs, q_out, wq_d, wk_d, tables))
     clock_info = clocks.stop() if clocks else None
 
     elapsed_ms = dist.max(elapsed_ms, device)
@@ -432,7 +456,7 @@ def run_ours(args, dist: Dist):
 
     kernel_used = {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
                    rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
-        rope3d.rope3d_testing_last_path(), "unknown")
+        headline_path, "unknown")
     if P:
         kernel_used += " (head-scatter stores)"
     device_status = rope3d.rope3d_check_device_status(tables)
@@ -513,9 +537,262 @@ def run_ours(args, dist: Dist):
         "clocks": clock_info,
         "e2e": e2e,
     }
+    if configs is not None:
+        line["configs"] = configs
     if not args.no_cpu_baseline and dist.world == 1:
         line["cpu_baseline"] = cpu_baseline(w, host, args.cpu_seconds)
     return line
+
+
+def graph_launch_us(torch, step, n_launch, stream, budget_ms=250.0):
+    """Capture step() (n_launch kernel launches) in a CUDA graph, replay it for about
+    budget_ms after warm-up, and return (mean device time per launch in us, host start and
+    end time of the timed replays)."""
+    step()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(stream.device)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step()
+    torch.cuda.synchronize()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        graph.replay()
+    a.record(stream)
+    graph.replay()
+    e.record(stream)
+    torch.cuda.synchronize()
+    reps = max(5, int(budget_ms / max(a.elapsed_time(e), 1e-3)))
+    t0 = time.time()
+    a.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    e.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    us = a.elapsed_time(e) * 1e3 / (reps * n_launch)
+    del graph
+    return us, (t0, t1)
+
+
+def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
+    """The other workloads of the step, each measured like the headline (graph replay of
+    one step, device time per launch, clocks of its own window): the 480P chunk loop, the
+    whole 480P sequence against its 8 slices (with a bit-identity check), the batch-2
+    long-horizon rollout with table and on-the-fly cos/sin, the 720P step with FP8 and
+    NVFP4 caches (on the headline's inputs), and the QKV projection on the tensor cores
+    with cuBLAS on the same GEMM beside it.  Inputs of the extra workloads are drawn on
+    the device (torch.randn with a fixed seed, rounded to bf16; norm weights U(0.5, 1.5))."""
+    hbm = peaks["hbm_gbs"]
+    out = {}
+    gen = torch.Generator(device=device)
+
+    def randn_bf16(shape, seed):
+        gen.manual_seed(seed)
+        return torch.randn(shape, generator=gen, device=device).to(torch.bfloat16)
+
+    def weights(dim, seed):
+        gen.manual_seed(seed)
+        return (torch.rand(dim, generator=gen, device=device) + 0.5,
+                torch.rand(dim, generator=gen, device=device) + 0.5)
+
+    def entry(name, us, nbytes, window, **extra):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        d = {"avg_launch_us": round(us, 2), "algorithmic_bytes_per_launch": nbytes,
+             "achieved_gbs": round(gbs, 1), "frac": round(gbs / hbm, 4),
+             "kernel": {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
+                        rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
+                 rope3d.rope3d_testing_last_path(), "unknown"),
+             "clocks": clocks.window(*window, name=name) if clocks else None}
+        d.update(extra)
+        out[name] = d
+
+    def plain_step(w, ins, q_out, kc, vc, tables, trig=rope3d.ROPE3D_TRIG_TABLE, chunks=None):
+        chunks = w.chunks if chunks is None else chunks
+
+        def step():
+            for j, c in enumerate(chunks):
+                q, k, v = ins[j % len(ins)]
+                rope3d.rope3d_qk_norm_rope_append(
+                    q, k, v, q_out[j % len(q_out)], c.token_begin, c.token_end, c.frame_offset,
+                    w.T, w.H, w.W, ins_w[0], ins_w[1], w.eps, kc, vc, c.slot, tables, trig,
+                    stream=stream)
+        return step
+
+    # 480P chunk loop: 7 calls of 4680 tokens x 12 heads
+    w = wl.chunk_480p()
+    n = w.tokens_per_chunk
+    shape = (w.B, n, w.N, wl.HEAD_DIM)
+    ins = [tuple(randn_bf16(shape, 100 + 3 * j + t) for t in range(3)) for j in range(len(w.chunks))]
+    ins_w = weights(w.dim, 99)
+    q_out = [torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in w.chunks]
+    cshape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    kc = torch.zeros(cshape, dtype=torch.bfloat16, device=device)
+    vc = torch.zeros_like(kc)
+    tables = rope3d.rope3d_tables_init(max_t=21, max_h=w.H, max_w=w.W)
+    us, win = graph_launch_us(torch, plain_step(w, ins, q_out, kc, vc, tables), len(w.chunks), stream)
+    entry("chunk480p_3x30x52_h12_bf16", us, w.algorithmic_bytes(n), win,
+          launches_per_step=len(w.chunks),
+          note="7 chunk calls (start frames 0..18) into a 32760-token cache, graph replay; "
+               "inputs 604 MB per step, above L2")
+    del ins, q_out
+
+    # whole 480P sequence (one call of 32760 tokens) against 8 slices of 4095 tokens
+    w = wl.full_480p()
+    n = w.tokens_per_chunk
+    shape = (w.B, n, w.N, wl.HEAD_DIM)
+    q, k, v = (randn_bf16(shape, 200 + t) for t in range(3))
+    qo_whole, qo_sl = torch.empty_like(q), torch.empty_like(q)
+    kw_, vw_ = torch.zeros_like(q), torch.zeros_like(q)
+    ks_, vs_ = torch.zeros_like(q), torch.zeros_like(q)
+
+    def whole():
+        rope3d.rope3d_qk_norm_rope_append(q, k, v, qo_whole, 0, n, 0, w.T, w.H, w.W, ins_w[0],
+                                          ins_w[1], w.eps, kw_, vw_, 0, tables, stream=stream)
+    parts = wl.slices(n, 8)
+
+    def sliced():
+        for a, b in parts:
+            rope3d.rope3d_qk_norm_rope_append(
+                q[:, a:b], k[:, a:b], v[:, a:b], qo_sl[:, a:b], a, b, 0, w.T, w.H, w.W,
+                ins_w[0], ins_w[1], w.eps, ks_, vs_, 0, tables, stream=stream)
+    us_w, win_w = graph_launch_us(torch, whole, 1, stream)
+    kern_w = rope3d.rope3d_testing_last_path()
+    us_s, win_s = graph_launch_us(torch, sliced, len(parts), stream)
+    torch.cuda.synchronize()
+    same = all(torch.equal(a.view(torch.int16), b.view(torch.int16))
+               for a, b in ((qo_whole, qo_sl), (kw_, ks_), (vw_, vs_)))
+    nbytes = w.algorithmic_bytes(n)
+    entry("full480p_21x30x52_h12_bf16/8slices", us_s, nbytes // len(parts), win_s,
+          slice_tokens=[b - a for a, b in parts], slices_bit_identical_to_whole=same,
+          whole={"avg_launch_us": round(us_w, 2), "algorithmic_bytes_per_launch": nbytes,
+                 "frac": round(nbytes / (us_w * 1e-6) / 1e9 / hbm, 4),
+                 "kernel": {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
+                            rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
+                     kern_w, "unknown"),
+                 "clocks": clocks.window(*win_w, name="whole") if clocks else None},
+          note="slices: 8 calls of 4095 tokens cutting through frames and rows; each call is "
+               "a separate launch (one graph of 8 launches)")
+    del q, k, v, qo_whole, qo_sl, kw_, vw_, ks_, vs_
+    tables.close()
+
+    # long-horizon rollout: batch 2, 80 chunks (global frames 0..239), rolling 21-frame cache
+    w = wl.long_horizon()
+    n = w.tokens_per_chunk
+    shape = (w.B, n, w.N, wl.HEAD_DIM)
+    nsets = 8  # input sets cycled over the 80 calls: 1.4 GB, so every launch reads HBM
+    ins = [tuple(randn_bf16(shape, 300 + 3 * j + t) for t in range(3)) for j in range(nsets)]
+    q_out = [torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(nsets)]
+    cshape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    kc = torch.zeros(cshape, dtype=torch.bfloat16, device=device)
+    vc = torch.zeros_like(kc)
+    tables = rope3d.rope3d_tables_init(max_t=240, max_h=w.H, max_w=w.W)
+    for trig, tname in ((rope3d.ROPE3D_TRIG_TABLE, "table"),
+                        (rope3d.ROPE3D_TRIG_ONTHEFLY, "onthefly")):
+        us, win = graph_launch_us(torch, plain_step(w, ins, q_out, kc, vc, tables, trig),
+                                  len(w.chunks), stream)
+        entry(f"longhorizon_b2_3x30x52_h12_bf16/{tname}", us, w.algorithmic_bytes(n), win,
+              launches_per_step=len(w.chunks),
+              note="80 chunk calls of 2 x 4680 tokens, start frames 0..237, cache slots "
+                   "wrapping every 21 frames; 8 input sets cycled")
+    del ins, q_out, kc, vc
+    tables.close()
+
+    # the 720P step with quantized caches, on the headline's inputs
+    w, ins, q_out, wq_d, wk_d, tables = headline
+    n = w.tokens_per_chunk
+    ins_w = (wq_d, wk_d)
+    for fmt in ("fp8", "nvfp4"):
+        fp4 = fmt == "nvfp4"
+        cshape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM // 2 if fp4 else wl.HEAD_DIM)
+        kc = torch.zeros(cshape, dtype=torch.uint8, device=device)
+        vc = torch.zeros_like(kc)
+        sshape = cshape[:3] + ((wl.HEAD_DIM // 16,) if fp4 else ())
+        sdt = torch.uint8 if fp4 else torch.float32
+        ks_, vs_ = (torch.zeros(sshape, dtype=sdt, device=device) for _ in range(2))
+        e = w.elem_bytes
+        nbytes = (w.B * n * (w.dim * 4 * e + 2 * (w.dim // 2 + w.dim // 16)) if fp4
+                  else w.B * n * (w.dim * (4 * e + 2) + 2 * 4 * w.N))
+
+        def qstep():
+            for j, c in enumerate(w.chunks):
+                q, k, v = ins[j]
+                rope3d.rope3d_qk_norm_rope_append_ex(
+                    q, k, v, q_out[j], c.token_begin, c.token_end, c.frame_offset, w.T, w.H,
+                    w.W, wq_d, wk_d, w.eps, kc, vc, c.slot, tables, k_scale=ks_, v_scale=vs_,
+                    k_global=0.5 if fp4 else 0.0, v_global=0.25 if fp4 else 0.0, stream=stream)
+        us, win = graph_launch_us(torch, qstep, len(w.chunks), stream)
+        entry(f"{w.name}/{fmt}_cache", us, nbytes, win, launches_per_step=len(w.chunks),
+              note="q, k, v read and q_out written in bf16; K and V cache rows as "
+                   + ("E2M1 codes with E4M3 scales per 16 elements" if fp4
+                      else "E4M3 codes with an fp32 scale per head"))
+        del kc, vc, ks_, vs_
+
+    # the 8-rank sequence-parallel step emulated on this GPU: each chunk's 8 token slices
+    # (1350 tokens, all 40 heads) store each head's q, K and V at the rank that owns it
+    P = 8
+    hl = w.N // P
+    sp_q = [torch.empty((w.B, n, hl, wl.HEAD_DIM), dtype=torch.bfloat16, device=device)
+            for _ in range(P)]
+    sp_k = [torch.zeros((w.B, w.cache_tokens, hl, wl.HEAD_DIM), dtype=torch.bfloat16,
+                        device=device) for _ in range(P)]
+    sp_v = [torch.zeros_like(sp_k[0]) for _ in range(P)]
+    sl = n // P
+    sp_in = [[tuple(x[:, r * sl:(r + 1) * sl].contiguous() for x in c) for r in range(P)]
+             for c in ins]
+
+    def sp_step():
+        for j, c in enumerate(w.chunks):
+            for r in range(P):
+                q, k, v = sp_in[j][r]
+                a = c.token_begin + r * sl
+                rope3d.rope3d_qk_norm_rope_append_sp(
+                    q, k, v, a, a + sl, c.frame_offset, w.T, w.H, w.W, wq_d, wk_d, w.eps, sp_q,
+                    sp_k, sp_v, c.slot, tables, q_row0=c.token_begin, stream=stream)
+    us, win = graph_launch_us(torch, sp_step, P * len(w.chunks), stream)
+    entry(f"{w.name}/sp8", us, w.algorithmic_bytes(sl), win, launches_per_step=P * len(w.chunks),
+          note="8 ranks emulated as 8 launches per chunk over 1350-token slices; every head "
+               "stored to its owner's buffers (5 heads each, all on this GPU)")
+    del sp_q, sp_k, sp_v, sp_in
+
+    # the QKV projection on the tensor cores (timed alone: the burst peak applies)
+    K = w.dim
+    xs = [randn_bf16((w.B * n, K), 400 + j) for j in range(3)]
+    gen.manual_seed(499)
+    wt = (torch.randn((3 * w.dim, K), generator=gen, device=device) * (2.0 / K ** 0.5)).to(
+        torch.bfloat16)
+    bt = torch.zeros(3 * w.dim, device=device)
+    outs = [torch.empty((w.B, n, w.N, wl.HEAD_DIM), dtype=torch.bfloat16, device=device)
+            for _ in range(3)]
+
+    def proj():
+        for j in range(3):
+            rope3d.rope3d_qkv_project(xs[j], wt, bt, *outs, stream=stream)
+    us, win = graph_launch_us(torch, proj, 3, stream)
+    y = torch.empty((w.B * n, 3 * w.dim), dtype=torch.bfloat16, device=device)
+
+    def cublas():
+        for j in range(3):
+            torch.matmul(xs[j], wt.t(), out=y)
+    us_cb, _ = graph_launch_us(torch, cublas, 3, stream)
+    flops = 2.0 * w.B * n * K * 3 * w.dim
+    burst = peaks.get("bf16_tflops", 1590.0)
+    tf = flops / (us * 1e-6) / 1e12
+    out[f"{w.name}/qkv_projection"] = {
+        "bound": "tensor", "avg_launch_us": round(us, 2), "algorithmic_flops_per_launch": flops,
+        "achieved_tflops": round(tf, 1), "peak_tflops": burst,
+        "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst: the kernel is timed alone)",
+        "frac": round(tf / burst, 4), "kernel": "rope3d::qkv_proj_kernel<2>",
+        "cublas_same_gemm_us": round(us_cb, 2),
+        "cublas_tflops": round(flops / (us_cb * 1e-6) / 1e12, 1),
+        "clocks": clocks.window(*win, name="projection") if clocks else None,
+        "note": "x [10800, 5120] bf16 times W^T, W [15360, 5120] bf16, fp32 accumulate, bf16 "
+                "out; 3 input sets, graph replay"}
+    del xs, wt, outs, y
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_qkv(args, dist: Dist):

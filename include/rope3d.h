@@ -60,6 +60,7 @@ extern "C" {
 #define ROPE3D_EALIGN (-5)   /* a tensor pointer is not 16-byte aligned                */
 #define ROPE3D_EOVERLAP (-6) /* output buffers overlap each other or an input          */
 #define ROPE3D_ETIMEOUT (-7) /* a kernel gave up a bounded wait (see check_device_status) */
+#define ROPE3D_EINDEX (-8)   /* checked build: a kernel skipped an out-of-extent row */
 
 /* Element types of q, k, v, q_out and the caches (all the same type). */
 #define ROPE3D_F32 0
@@ -356,6 +357,16 @@ ROPE3D_API int rope3d_decode_positions(int64_t token_begin, int64_t token_end, i
  * cuda_stream, reads and clears that word, and returns ROPE3D_ETIMEOUT if any launch
  * since the last check gave up, else ROPE3D_OK (ECUDA / EDEVICE / EINVAL on failure to
  * read it).  Not needed on the normal path; intended for health checks.
+ *
+ * A library built with -DROPE3D_DEVICE_CHECKS (rotary_position_encoding_b200.build
+ * --checked, librope3d_checked.so) also tests, in the step kernels, every cache row,
+ * table row and sequence-parallel destination q row it derives against the extents of
+ * the call.  A token row whose cache row (or destination q row) lies outside is not
+ * stored at all; a table row outside its table is not read (cos and sin are taken as 1
+ * and 0).  Either is recorded in the same word, which this call then reports as
+ * ROPE3D_EINDEX.  The host checks of
+ * every entry point make that unreachable for valid arguments; the checked build guards
+ * the kernels' own index arithmetic.  No kernel traps in either build.
  */
 ROPE3D_API int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream);
 
@@ -373,10 +384,14 @@ ROPE3D_API int rope3d_check_device_status(const rope3d_tables* tables, void* cud
  * holds until the process exits: a status word and room for 8192 (cos, sin) entries.
  * With trig = ROPE3D_TRIG_TABLE each call computes, in fp64 on the host, the cos/sin rows
  * of its own positions -- (frames touched) * n_t + H * n_h + W * n_w entries -- and
- * copies them into that array on cuda_stream (a copy from pageable host memory, so the
- * call waits for the stream to drain before it returns); a call needing more than 8192
- * entries returns ROPE3D_ERANGE and launches nothing.  With ROPE3D_TRIG_ONTHEFLY nothing
- * is copied.  Each call first clears the status word.  Outputs are bit-identical to
+ * copies them into that array with cudaMemcpyAsync on cuda_stream, ahead of the call's
+ * kernel in stream order.  The rows come from a library-owned pageable host buffer: the
+ * runtime has taken them (staged or copied) when the copy call returns, and the library
+ * holds a lock from the rows' computation until then, so a later call cannot overwrite
+ * them.  Nothing here waits for cuda_stream to drain; the runtime may do so for a
+ * pageable copy.  A call needing more than 8192 entries returns ROPE3D_ERANGE and
+ * launches nothing.  With ROPE3D_TRIG_ONTHEFLY nothing is copied.  Each call first
+ * clears the status word.  Outputs are bit-identical to
  * rope3d_qk_norm_rope_append with tables built from the same configuration.
  *
  * Every call shares the array and it keeps the last call's contents; calls that overlap

@@ -35,6 +35,17 @@ ROPE3D_API int rope3d_testing_force_path(int path);
  * each CTA loading half of the weight rows), 0 = the default (2).  EINVAL otherwise. */
 ROPE3D_API int rope3d_testing_gemm_cta_group(int group);
 
+/*
+ * Checked build only (librope3d_checked.so; a no-op in librope3d.so): for later launches
+ * of the step kernels, the device-side check of a cache row accepts rows below
+ * cache_tokens - shrink_rows instead of below cache_tokens.  Rows at or above that bound
+ * are then treated as out of extent: the kernel skips all of that token row's stores
+ * (q_out, K and V) and records ROPE3D_EINDEX in the status word.  The skipped rows lie
+ * inside the caller's buffers, so the check's firing path is exercised without any access
+ * outside them.  0 (the default) restores the plain check; negative values are EINVAL.
+ */
+ROPE3D_API int rope3d_testing_shrink_checked_cache(int64_t shrink_rows);
+
 /* The path (ROPE3D_PATH_REGISTERS or ROPE3D_PATH_TMA) of the calling thread's most recent
  * successful rope3d_qk_norm_rope_append launch; ROPE3D_PATH_AUTO before the first. */
 ROPE3D_API int rope3d_testing_last_path(void);

@@ -61,6 +61,7 @@ std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<uint32_t> g_tx_extra{0};
 std::atomic<int> g_force_path{ROPE3D_PATH_AUTO};
 std::atomic<int> g_gemm_cta_group{2};  // the projection's form: 1 CTA or a 2-CTA pair per tile
+std::atomic<int64_t> g_check_shrink{0};  // checked build: cache rows the row check withholds
 thread_local int g_last_path = ROPE3D_PATH_AUTO;  // path of this thread's last fused launch
 
 int fail(int status, const char* fmt, ...) {
@@ -588,6 +589,10 @@ void fill_common(rope3d::Params& p, int64_t B, int64_t N, int64_t token_begin, i
     p.tab_t = tables->tab_t;
     p.tab_h = tables->tab_h;
     p.tab_w = tables->tab_w;
+    p.tab_rows_t = tables->max_t;
+    p.tab_rows_h = tables->max_h;
+    p.tab_rows_w = tables->max_w;
+    p.check_shrink = g_check_shrink.load();
     std::memcpy(p.inv_freq, tables->inv_freq, sizeof(p.inv_freq));
     p.status = tables->d_status;
     p.cache_tokens = 1;  // the fused entry point overwrites these two
@@ -686,6 +691,7 @@ const char* rope3d_strerror(int status) {
         case ROPE3D_EALIGN: return "tensor pointer not 16-byte aligned";
         case ROPE3D_EOVERLAP: return "output buffers overlap";
         case ROPE3D_ETIMEOUT: return "a kernel wait timed out";
+        case ROPE3D_EINDEX: return "a device-side index check failed (checked build)";
         default: return "unknown status";
     }
 }
@@ -833,6 +839,9 @@ int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream) {
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "status read: %s", cudaGetErrorString(e));
     if (word & rope3d::kStatusWaitTimeout)
         return fail(ROPE3D_ETIMEOUT, "a kernel gave up waiting for a shared-memory stage to fill");
+    if (word & rope3d::kStatusIndexRange)
+        return fail(ROPE3D_EINDEX, "a kernel of the checked build derived a cache, table or "
+                                   "destination row outside its extent and skipped it");
     return ok();
 }
 
@@ -842,6 +851,12 @@ void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes) {
 }
 
 int rope3d_testing_last_path(void) { return g_last_path; }
+
+int rope3d_testing_shrink_checked_cache(int64_t shrink_rows) {
+    if (shrink_rows < 0) return fail(ROPE3D_EINVAL, "shrink_rows %lld < 0", (long long)shrink_rows);
+    g_check_shrink.store(shrink_rows);
+    return ok();
+}
 
 int rope3d_testing_gemm_cta_group(int group) {
     if (group != 0 && group != 1 && group != 2)
@@ -1486,7 +1501,9 @@ extern "C" int rope3d_qk_norm_rope_append_noalloc(
                 h[off++] = make_float2((float)std::cos(phi), (float)std::sin(phi));
             }
         float2* d_tab = reinterpret_cast<float2*>(scratch + kNoAllocStatusBytes);
-        // From pageable memory the copy has consumed the host rows when it returns.
+        // A copy from pageable memory has taken the host rows (staged or copied) when it
+        // returns, so the next call may refill g_noalloc_host once it holds the lock; the
+        // device array is written in stream order, ahead of this call's kernel.
         e = cudaMemcpyAsync(d_tab, h, off * sizeof(float2), cudaMemcpyHostToDevice, stream);
         if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "table upload: %s", cudaGetErrorString(e));
         tb.d_tab = d_tab;

@@ -131,10 +131,12 @@ qk_norm_rope_tma_kernel(const Params p) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     pdl_wait_previous_grid();
-    stage_weights(p, s_wq, s_wk);
-    __syncthreads();
+    // The first S rows are requested before the block stages its weights, so the two
+    // latencies overlap at the start of the launch.
     if (t == 0)
         for (int kk = 0; kk < S; ++kk) issue(kk);
+    stage_weights(p, s_wq, s_wk);
+    __syncthreads();
 
     const PairInfo<NP> pi = pair_info<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
     Vec* qo = reinterpret_cast<Vec*>(p.q_out);
@@ -188,7 +190,7 @@ qk_norm_rope_tma_kernel(const Params p) {
 
         const RowPos pos = decode_row(p, u);
         float cs[NP], sn[NP];
-        pair_trig<TRIG>(pi, pos, cs, sn);
+        pair_trig<TRIG>(p, pi, pos, cs, sn);
         const float rq = rsqrtf(fmaf(tot.x, p.inv_dim, p.eps));
         const float rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         const int64_t row_vec = u * p.dim_vecs;

@@ -24,6 +24,7 @@ ROPE3D_EDEVICE = -4
 ROPE3D_EALIGN = -5
 ROPE3D_EOVERLAP = -6
 ROPE3D_ETIMEOUT = -7
+ROPE3D_EINDEX = -8
 
 ROPE3D_F32 = 0
 ROPE3D_BF16 = 1
@@ -110,6 +111,7 @@ SIGNATURES = {
     "rope3d_testing_force_path": ([_INT], _INT),
     "rope3d_testing_gemm_cta_group": ([_INT], _INT),
     "rope3d_testing_last_path": ([], _INT),
+    "rope3d_testing_shrink_checked_cache": ([_I64], _INT),
 }
 
 _lib = None
@@ -205,12 +207,11 @@ def rope3d_tables_destroy(tables: Tables) -> None:
     tables.close()
 
 
-def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
-                               frame_offset: int, T: int, H: int, W: int, q_norm_w, k_norm_w,
-                               eps: float, k_cache, v_cache, slot: int, tables: Tables,
-                               trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
-    """q, k, v, q_out: [B, n_tok, N, 128]; k_cache, v_cache: [B, cache_tokens, N, 128];
-    q_norm_w, k_norm_w: [N*128] float32.  Enqueued on ``stream`` (default: current)."""
+def _check_step_tensors(q, k, v, q_out, token_begin: int, token_end: int, q_norm_w, k_norm_w,
+                        k_cache, v_cache):
+    """Shape and dtype checks of the fused step's tensors, shared by every wrapper that
+    passes same-dtype caches: the C ABI sees only pointers and sizes, so a mismatch here
+    would make the kernel read or write past the end of a tensor.  Returns (B, N, D)."""
     if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or q_out.shape != q.shape:
         raise ValueError("q, k, v and q_out must all be [B, n_tok, N, D]")
     if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
@@ -220,7 +221,7 @@ def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
         raise ValueError("cache shape does not match q")
     if n_tok != token_end - token_begin:
         raise ValueError("q has n_tok rows but the range holds token_end - token_begin")
-    code = _dtype_code(q)
+    _dtype_code(q)
     for name, t in (("k", k), ("v", v), ("q_out", q_out), ("k_cache", k_cache),
                     ("v_cache", v_cache)):
         if t.dtype != q.dtype:
@@ -228,9 +229,20 @@ def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
     for name, t in (("q_norm_w", q_norm_w), ("k_norm_w", k_norm_w)):
         if t.dtype != torch.float32 or t.numel() != N * D:
             raise ValueError(f"{name} must be float32 with N*D elements")
+    return B, N, D
+
+
+def rope3d_qk_norm_rope_append(q, k, v, q_out, token_begin: int, token_end: int,
+                               frame_offset: int, T: int, H: int, W: int, q_norm_w, k_norm_w,
+                               eps: float, k_cache, v_cache, slot: int, tables: Tables,
+                               trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
+    """q, k, v, q_out: [B, n_tok, N, 128]; k_cache, v_cache: [B, cache_tokens, N, 128];
+    q_norm_w, k_norm_w: [N*128] float32.  Enqueued on ``stream`` (default: current)."""
+    B, N, D = _check_step_tensors(q, k, v, q_out, token_begin, token_end, q_norm_w, k_norm_w,
+                                  k_cache, v_cache)
     _check(load_library().rope3d_qk_norm_rope_append(
         _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
-        B, N, D, code, token_begin, token_end, frame_offset, T, H, W,
+        B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,
         _dev_ptr(q_norm_w, "q_norm_w"), _dev_ptr(k_norm_w, "k_norm_w"), eps,
         _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"), k_cache.shape[1], slot,
         tables.handle, trig, _stream(stream)))
@@ -244,8 +256,10 @@ def rope3d_qk_norm_rope_append_noalloc(q, k, v, q_out, token_begin: int, token_e
                                        schedule: int = ROPE3D_SCHEDULE_PER_AXIS,
                                        trig: int = ROPE3D_TRIG_TABLE, stream=None) -> None:
     """The fused step with no device allocation (frequency configuration passed directly;
-    its cos/sin rows and status word live in the library's fixed scratch array)."""
-    B, n_tok, N, D = q.shape
+    its cos/sin rows and status word live in the library's fixed scratch array).  The
+    tensors are checked as in rope3d_qk_norm_rope_append."""
+    B, N, D = _check_step_tensors(q, k, v, q_out, token_begin, token_end, q_norm_w, k_norm_w,
+                                  k_cache, v_cache)
     _check(load_library().rope3d_qk_norm_rope_append_noalloc(
         _dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"), _dev_ptr(q_out, "q_out"),
         B, N, D, _dtype_code(q), token_begin, token_end, frame_offset, T, H, W,
@@ -480,9 +494,10 @@ def rope3d_decode_positions(token_begin: int, token_end: int, frame_offset: int,
 
 def rope3d_check_device_status(tables: Tables, stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status of kernels launched
-    with these tables: ROPE3D_OK or ROPE3D_ETIMEOUT.  Raises on a failure to read it."""
+    with these tables: ROPE3D_OK, ROPE3D_ETIMEOUT, or (checked build) ROPE3D_EINDEX.
+    Raises on a failure to read it."""
     status = load_library().rope3d_check_device_status(tables.handle, _stream(stream))
-    if status not in (ROPE3D_OK, ROPE3D_ETIMEOUT):
+    if status not in (ROPE3D_OK, ROPE3D_ETIMEOUT, ROPE3D_EINDEX):
         _check(status)
     return status
 
@@ -497,6 +512,10 @@ def rope3d_testing_force_path(path: int = ROPE3D_PATH_AUTO) -> None:
 
 def rope3d_testing_gemm_cta_group(group: int = 0) -> None:
     _check(load_library().rope3d_testing_gemm_cta_group(group))
+
+
+def rope3d_testing_shrink_checked_cache(shrink_rows: int = 0) -> None:
+    _check(load_library().rope3d_testing_shrink_checked_cache(shrink_rows))
 
 
 def rope3d_testing_last_path() -> int:

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from rotary_position_encoding_b200 import build as native_build
 from rotary_position_encoding_b200 import rope3d
@@ -96,6 +97,19 @@ def test_testing_hooks_validate_without_device(lib):
     assert lib.rope3d_testing_force_path(rope3d.ROPE3D_PATH_AUTO) == rope3d.ROPE3D_OK
     lib.rope3d_testing_set_waits(0, 0)
     assert lib.rope3d_check_device_status(None, None) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_testing_shrink_checked_cache(-1) == rope3d.ROPE3D_EINVAL
+    assert lib.rope3d_testing_shrink_checked_cache(0) == rope3d.ROPE3D_OK
+
+
+def test_checked_build_compiles_and_exports_every_declared_symbol():
+    """librope3d_checked.so is the same source built with -DROPE3D_DEVICE_CHECKS."""
+    native_build.build_all()
+    checked = rope3d.load_library(native_build.CHECKED_LIBRARY)
+    assert checked is not rope3d.load_library()
+    for name in header_functions():
+        assert hasattr(checked, name), name
+    assert checked.rope3d_strerror(rope3d.ROPE3D_EINDEX).decode().startswith("a device-side")
+    assert checked.rope3d_version() == rope3d.load_library().rope3d_version()
 
 
 def test_missing_library_fails_loudly(tmp_path):
@@ -160,3 +174,31 @@ def test_sp_step_rejects_null_arguments_without_device(lib):
         assert lib.rope3d_qk_norm_rope_append_sp(p, p, p, 1, 2, 128, 1, 0, 72, 0, 3, 4, 6, p, p,
                                                  1e-6, d, 144, 0, None, 0, None,
                                                  None) == rope3d.ROPE3D_EINVAL
+
+
+@pytest.mark.parametrize("entry", ["rope3d_qk_norm_rope_append",
+                                   "rope3d_qk_norm_rope_append_noalloc"])
+def test_step_wrappers_check_tensors_before_any_call(entry):
+    """Both step wrappers check shapes and dtypes before the C call (host logic only: the
+    tensors here never reach the library)."""
+    fn = getattr(rope3d, entry)
+    extra = {"tables": None} if entry == "rope3d_qk_norm_rope_append" else {}
+    q = torch.zeros((1, 4, 2, 128), dtype=torch.bfloat16)
+    kc = torch.zeros((1, 8, 2, 128), dtype=torch.bfloat16)
+    wq = torch.ones(256)
+    args = dict(frame_offset=0, T=1, H=2, W=4, q_norm_w=wq, k_norm_w=wq, eps=1e-6, slot=0,
+                **extra)
+    with pytest.raises(ValueError, match="n_tok"):
+        fn(q, q, q, q.clone(), token_begin=0, token_end=5, k_cache=kc, v_cache=kc.clone(), **args)
+    with pytest.raises(TypeError, match="k_cache"):
+        fn(q, q, q, q.clone(), token_begin=0, token_end=4, k_cache=kc.float(),
+           v_cache=kc.float(), **args)
+    with pytest.raises(ValueError, match="cache shape"):
+        fn(q, q, q, q.clone(), token_begin=0, token_end=4, k_cache=kc[:, :, :1].contiguous(),
+           v_cache=kc[:, :, :1].contiguous(), **args)
+    with pytest.raises(ValueError, match="float32"):
+        fn(q, q, q, q.clone(), token_begin=0, token_end=4, k_cache=kc, v_cache=kc.clone(),
+           **dict(args, q_norm_w=wq[:8]))
+    with pytest.raises(ValueError, match="all be"):
+        fn(q, q[:, :3], q, q.clone(), token_begin=0, token_end=4, k_cache=kc, v_cache=kc.clone(),
+           **args)

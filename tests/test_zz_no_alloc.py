@@ -63,8 +63,9 @@ def test_noalloc_matches_existing_entry_point_on_two_calls(trig):
 
 def test_noalloc_rejects_tables_beyond_its_scratch():
     lib = rope3d.load_library()
-    # 21 frames of a 45 x 80 grid need 21*22 + 45*21 + 80*21 = 3087 entries: fits; a
-    # 400 x 400 grid needs 3*22 + 2*400*21 = 16866 entries: more than the 8192 it holds
+    # 21 frames of a 45 x 80 grid need 21*22 + 45*21 + 80*21 = 3087 entries: fits.  The
+    # range [0, 4) of a 400 x 400 grid touches frame 0 only, and needs 1*22 + 2*400*21 =
+    # 16822 entries (frames touched * n_t + H * n_h + W * n_w): more than the 8192 it holds
     w = wl.chunk_480p()
     T, H, W = 3, 400, 400
     q = torch.zeros((1, 4, 2, wl.HEAD_DIM), dtype=torch.bfloat16, device="cuda")
@@ -84,3 +85,25 @@ def test_noalloc_rejects_tables_beyond_its_scratch():
     assert rc == rope3d.ROPE3D_OK, rope3d.rope3d_last_error()
     torch.cuda.synchronize()
     assert bool((qo.float() == 0.0).all())
+
+
+def test_noalloc_wrapper_checks_tensors_before_the_call():
+    """The Python wrapper checks shapes and dtypes as the ordinary wrapper does: the C ABI
+    sees only pointers and sizes, so a short q or a cache of another dtype would otherwise
+    make the kernel read or write past the end of a tensor."""
+    q = torch.zeros((1, 4, 2, wl.HEAD_DIM), dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros((1, 8, 2, wl.HEAD_DIM), dtype=torch.bfloat16, device="cuda")
+    wq = torch.ones(2 * wl.HEAD_DIM, device="cuda")
+    args = dict(frame_offset=0, T=1, H=2, W=4, q_norm_w=wq, k_norm_w=wq, eps=1e-6, slot=0)
+    with pytest.raises(ValueError):  # the range holds 5 rows, q holds 4
+        rope3d.rope3d_qk_norm_rope_append_noalloc(q, q, q, q.clone(), token_begin=0,
+                                                  token_end=5, k_cache=kc, v_cache=kc.clone(),
+                                                  **args)
+    with pytest.raises(TypeError):  # fp32 caches with bf16 q
+        rope3d.rope3d_qk_norm_rope_append_noalloc(q, q, q, q.clone(), token_begin=0,
+                                                  token_end=4, k_cache=kc.float(),
+                                                  v_cache=kc.float(), **args)
+    with pytest.raises(ValueError):  # weights of the wrong length
+        rope3d.rope3d_qk_norm_rope_append_noalloc(q, q, q, q.clone(), token_begin=0,
+                                                  token_end=4, k_cache=kc, v_cache=kc.clone(),
+                                                  **dict(args, q_norm_w=wq[:8]))
