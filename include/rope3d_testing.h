@@ -17,6 +17,8 @@ extern "C" {
 #define ROPE3D_PATH_AUTO 0       /* the path measured faster for the shape (see rope3d.cu)     */
 #define ROPE3D_PATH_REGISTERS 1  /* rows loaded straight into registers                        */
 #define ROPE3D_PATH_TMA 2        /* rows streamed through shared memory (EINVAL if it does not fit) */
+#define ROPE3D_PATH_STREAM 3     /* rows staged in shared memory by a producer warp and consumed
+                                    from there in two passes (EINVAL if it does not fit) */
 
 /*
  * Bounded-wait settings of the bulk-copy ring kernel for later launches:
@@ -45,6 +47,14 @@ ROPE3D_API int rope3d_testing_gemm_cta_group(int group);
  * outside them.  0 (the default) restores the plain check; negative values are EINVAL.
  */
 ROPE3D_API int rope3d_testing_shrink_checked_cache(int64_t shrink_rows);
+
+/*
+ * The kernels' 32-bit position decode divides by the token count, H * W, W and the cache
+ * length with a multiply-and-shift instead of a divide instruction.  This runs the same
+ * arithmetic on the host: floor(n / d) for n < 2^31 and 1 <= d < 2^31, or 0xFFFFFFFF for
+ * arguments outside that range.
+ */
+ROPE3D_API uint32_t rope3d_testing_fast_divide(uint32_t n, uint32_t d);
 
 /* The path (ROPE3D_PATH_REGISTERS or ROPE3D_PATH_TMA) of the calling thread's most recent
  * successful rope3d_qk_norm_rope_append launch; ROPE3D_PATH_AUTO before the first. */

@@ -9,6 +9,7 @@
 #include "rope3d_testing.h"
 #include "rope3d_kernels.cuh"
 #include "rope3d_tma.cuh"
+#include "rope3d_stream.cuh"
 #include "rope3d_gemm.cuh"
 
 #include <cuda_runtime.h>
@@ -449,6 +450,132 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pair
     return ok();
 }
 
+// ---------------------------------------------------------------- staged-row kernel
+
+template <typename T, int TRIG, int MODE, int PAIR, int CF>
+KernelFn pick_stream_vpt(int vpt) {
+    if constexpr (PAIR == rope3d::kPairHalf) {
+        switch (vpt) {
+            case 2: return rope3d::qk_norm_rope_stream_kernel<T, 2, TRIG, MODE, PAIR, CF>;
+            case 4: return rope3d::qk_norm_rope_stream_kernel<T, 4, TRIG, MODE, PAIR, CF>;
+            default: return nullptr;
+        }
+    } else {
+        switch (vpt) {
+            case 1: return rope3d::qk_norm_rope_stream_kernel<T, 1, TRIG, MODE, PAIR, CF>;
+            case 2: return rope3d::qk_norm_rope_stream_kernel<T, 2, TRIG, MODE, PAIR, CF>;
+            case 3: return rope3d::qk_norm_rope_stream_kernel<T, 3, TRIG, MODE, PAIR, CF>;
+            case 4: return rope3d::qk_norm_rope_stream_kernel<T, 4, TRIG, MODE, PAIR, CF>;
+            default: return nullptr;
+        }
+    }
+}
+
+template <typename T, int MODE, int PAIR, int CF>
+KernelFn pick_stream_trig(int trig, int vpt) {
+    return trig == ROPE3D_TRIG_TABLE ? pick_stream_vpt<T, rope3d::kTrigTable, MODE, PAIR, CF>(vpt)
+                                     : pick_stream_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR, CF>(vpt);
+}
+
+template <typename T, int CF>
+KernelFn pick_stream_pairing(int pairing, int trig, int vpt) {
+    return pairing == ROPE3D_PAIRING_HALF
+               ? pick_stream_trig<T, rope3d::kModeFused, rope3d::kPairHalf, CF>(trig, vpt)
+               : pick_stream_trig<T, rope3d::kModeFused, rope3d::kPairAdjacent, CF>(trig, vpt);
+}
+
+template <typename T>
+KernelFn pick_stream_type(int mode, int cache_fmt, int pairing, int trig, int vpt) {
+    if (mode == rope3d::kModeFusedSP)
+        return pairing == ROPE3D_PAIRING_ADJACENT && cache_fmt == rope3d::kCacheSame
+                   ? pick_stream_trig<T, rope3d::kModeFusedSP, rope3d::kPairAdjacent,
+                                      rope3d::kCacheSame>(trig, vpt)
+                   : nullptr;
+    switch (cache_fmt) {
+        case rope3d::kCacheFp8: return pick_stream_pairing<T, rope3d::kCacheFp8>(pairing, trig, vpt);
+        case rope3d::kCacheNvfp4:
+            return pick_stream_pairing<T, rope3d::kCacheNvfp4>(pairing, trig, vpt);
+        default: return pick_stream_pairing<T, rope3d::kCacheSame>(pairing, trig, vpt);
+    }
+}
+
+KernelFn pick_stream_kernel(int mode, int dtype, int trig, int pairing, int cache_fmt, int vpt) {
+    return dtype == ROPE3D_BF16
+               ? pick_stream_type<__nv_bfloat16>(mode, cache_fmt, pairing, trig, vpt)
+               : pick_stream_type<float>(mode, cache_fmt, pairing, trig, vpt);
+}
+
+// Shared-memory plan of the staged-row kernel: [aux_bytes: SP destination table or NVFP4
+// reciprocals] [full and empty barriers] [failure flags] [partials] [weights] [stages].
+size_t stream_layout(rope3d::Params& p, int teams, int stages, int warps_per_team,
+                     size_t aux_bytes) {
+    size_t off = align_up(aux_bytes, 16);
+    p.off_bars = (uint32_t)off;
+    off += (size_t)2 * stages * sizeof(uint64_t);
+    p.off_fail = (uint32_t)off;
+    off += (size_t)teams * sizeof(int);
+    off = align_up(off, 16);
+    p.off_part = (uint32_t)off;
+    off += (size_t)2 * teams * warps_per_team * sizeof(float2);
+    off = align_up(off, 16);
+    p.off_w = (uint32_t)off;
+    off += (size_t)2 * p.dim * sizeof(float);
+    off = align_up(off, 128);
+    p.off_stage = (uint32_t)off;
+    off += (size_t)stages * 3 * p.row_bytes;
+    return off;
+}
+
+#ifndef ROPE3D_STREAM_MAX_STAGES
+#define ROPE3D_STREAM_MAX_STAGES 32
+#endif
+
+// The fused step through the staged-row kernel: one block per SM, a producer warp and as
+// many teams as kStreamMaxThreads allows (at most kMaxTeamsPerBlock), and as many stages
+// as fit in shared memory (at least 2, at most ROPE3D_STREAM_MAX_STAGES).  *launched
+// stays false if the shape does not fit.
+int launch_fused_stream(rope3d::Params& p, int mode, int64_t N, int dtype, int trig, int pairing,
+                        int dev, const DeviceInfo& info, cudaStream_t stream, bool* launched) {
+    *launched = false;
+    const Geometry g = geometry(N, dtype, pairing);
+    if (g.tpr + 32 > rope3d::kStreamMaxThreads || g.vpt > 4) return ROPE3D_OK;
+    const int warps_per_team = g.tpr / 32;
+    p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
+    int teams = (rope3d::kStreamMaxThreads - 32) / g.tpr;
+    if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
+    const size_t aux = mode == rope3d::kModeFusedSP ? 3 * rope3d::kMaxRanks * sizeof(void*)
+                       : p.k_bscale != nullptr ? rope3d::kNvfp4TableFloats * sizeof(float) : 0;
+    int stages = (int)((info.max_smem_optin - stream_layout(p, teams, 0, warps_per_team, aux)) /
+                       (3 * (size_t)p.row_bytes + 2 * sizeof(uint64_t)));
+    if (stages > ROPE3D_STREAM_MAX_STAGES) stages = ROPE3D_STREAM_MAX_STAGES;
+    while (stages >= 2 &&
+           stream_layout(p, teams, stages, warps_per_team, aux) > (size_t)info.max_smem_optin)
+        --stages;
+    if (stages < 2) return ROPE3D_OK;
+    const size_t smem = stream_layout(p, teams, stages, warps_per_team, aux);
+    const int cache_fmt = p.k_bscale != nullptr ? rope3d::kCacheNvfp4
+                          : p.k_scale != nullptr ? rope3d::kCacheFp8 : rope3d::kCacheSame;
+    KernelFn fn = pick_stream_kernel(mode, dtype, trig, pairing, cache_fmt, g.vpt);
+    if (fn == nullptr) return ROPE3D_OK;
+    const int threads = 32 + teams * g.tpr;
+    int per_sm = 0;
+    int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
+    if (rc != ROPE3D_OK) return rc;
+    int64_t grid = info.sms;
+    if (grid > p.units) grid = p.units;
+    p.dim_vecs = g.dim_vecs;
+    p.tpr = g.tpr;
+    p.teams = teams;
+    p.stages = stages;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.tx_extra = g_tx_extra.load();
+    const cudaError_t e =
+        launch_pdl(reinterpret_cast<const void*>(fn), grid, threads, smem, stream, &p);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
+    *launched = true;
+    return ok();
+}
+
 template <int MODE>
 int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int dev,
            const DeviceInfo& info, cudaStream_t stream) {
@@ -603,6 +730,12 @@ void set_small_idx(rope3d::Params& p) {
     const int64_t lim = (int64_t)1 << 31;
     p.small_idx = (p.units < lim && p.token_begin + p.n_tok + p.slot < lim &&
                    p.cache_tokens < lim && p.hw < lim) ? 1 : 0;
+    if (p.small_idx) {
+        p.div_ntok = rope3d::make_fastdiv((uint32_t)p.n_tok);
+        p.div_hw = rope3d::make_fastdiv((uint32_t)p.hw);
+        p.div_w = rope3d::make_fastdiv((uint32_t)p.W);
+        p.div_cache = rope3d::make_fastdiv((uint32_t)p.cache_tokens);
+    }
 }
 
 // The options of a call (NULL = all defaults), checked.
@@ -852,6 +985,11 @@ void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes) {
 
 int rope3d_testing_last_path(void) { return g_last_path; }
 
+uint32_t rope3d_testing_fast_divide(uint32_t n, uint32_t d) {
+    if (d == 0 || d >= (1u << 31) || n >= (1u << 31)) return 0xFFFFFFFFu;
+    return rope3d::fast_div(n, rope3d::make_fastdiv(d));
+}
+
 int rope3d_testing_shrink_checked_cache(int64_t shrink_rows) {
     if (shrink_rows < 0) return fail(ROPE3D_EINVAL, "shrink_rows %lld < 0", (long long)shrink_rows);
     g_check_shrink.store(shrink_rows);
@@ -866,7 +1004,8 @@ int rope3d_testing_gemm_cta_group(int group) {
 }
 
 int rope3d_testing_force_path(int path) {
-    if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA)
+    if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA &&
+        path != ROPE3D_PATH_STREAM)
         return fail(ROPE3D_EINVAL, "path %d is not a ROPE3D_PATH_* value", path);
     g_force_path.store(path);
     return ok();
@@ -965,6 +1104,15 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
     set_small_idx(p);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     const int path = g_force_path.load();
+    if (path == ROPE3D_PATH_STREAM) {
+        bool launched = false;
+        rc = launch_fused_stream(p, rope3d::kModeFused, N, dtype, trig, opt.pairing, dev, info,
+                                 stream, &launched);
+        if (launched) g_last_path = ROPE3D_PATH_STREAM;
+        if (rc != ROPE3D_OK || launched) return rc;
+        return fail(ROPE3D_EINVAL, "the staged-row path does not take this call (N=%lld)",
+                    (long long)N);
+    }
     if (path != ROPE3D_PATH_REGISTERS) {
         bool launched = false;
         rc = launch_fused_tma(p, N, dtype, trig, opt.pairing, dev, info, stream,
@@ -1078,6 +1226,15 @@ int rope3d_qk_norm_rope_append_sp(const void* q, const void* k, const void* v,
         p.sp_dst[3 * r + 2] = dest->v_cache[r];
     }
     set_small_idx(p);
+    if (g_force_path.load() == ROPE3D_PATH_STREAM) {
+        bool launched = false;
+        rc = launch_fused_stream(p, rope3d::kModeFusedSP, N, dtype, trig, opt.pairing, dev,
+                                 info, static_cast<cudaStream_t>(cuda_stream), &launched);
+        if (launched) g_last_path = ROPE3D_PATH_STREAM;
+        if (rc != ROPE3D_OK || launched) return rc;
+        return fail(ROPE3D_EINVAL, "the staged-row path does not take this call (N=%lld)",
+                    (long long)N);
+    }
     rc = launch<rope3d::kModeFusedSP>(p, N, dtype, trig, opt.pairing, dev, info,
                                       static_cast<cudaStream_t>(cuda_stream));
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;

@@ -64,6 +64,28 @@ enum Trig : int { kTrigTable = 0, kTrigOnTheFly = 1 };
 // view of Wan2.1 -- or rotate_half (j, j + 64), the cos/sin form of M-RoPE.
 enum Pairing : int { kPairAdjacent = 0, kPairHalf = 1 };
 
+// Division of n < 2^31 by a fixed divisor d in [1, 2^31) without a divide instruction:
+// q = floor(n m / 2^s) with l = ceil(log2 d), s = 31 + l and m = floor(2^s / d) + 1 < 2^32
+// (the round-up method for dividends of 31 bits; m d = 2^s + e with 0 < e <= d, so the
+// error term n e / (d 2^s) stays below 2^-l <= 1/d and the floor is exact).
+struct FastDiv {
+    uint32_t m;
+    uint32_t s;
+};
+
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 31 && (1u << l) < d) ++l;
+    FastDiv f;
+    f.s = 31 + l;
+    f.m = (uint32_t)((1ull << f.s) / d + 1);
+    return f;
+}
+
+__host__ __device__ __forceinline__ uint32_t fast_div(uint32_t n, FastDiv f) {
+    return (uint32_t)(((uint64_t)n * f.m) >> f.s);
+}
+
 struct Params {
     const void* q;        // fused: q;  apply: x
     const void* k;
@@ -92,6 +114,7 @@ struct Params {
     int tpr;              // threads per team (multiple of 32)
     int teams;            // teams per block
     int small_idx;        // all index arithmetic fits in 32 bits
+    FastDiv div_ntok, div_hw, div_w, div_cache;  // for the 32-bit decode
     float eps;
     float inv_dim;        // 1 / dim
     int n_t, n_h, n_w;
@@ -257,20 +280,21 @@ __device__ __forceinline__ RowPos decode_row(const Params& p, int64_t u) {
     RowPos q;
     if (p.small_idx) {
         const uint32_t uu = (uint32_t)u, ntok = (uint32_t)p.n_tok;
-        const uint32_t b = uu / ntok;
+        const uint32_t b = fast_div(uu, p.div_ntok);
         const uint32_t r = uu - b * ntok;
         const uint32_t i = (uint32_t)p.token_begin + r;
         const uint32_t hw = (uint32_t)p.hw, W = (uint32_t)p.W;
-        const uint32_t tl = i / hw;
+        const uint32_t tl = fast_div(i, p.div_hw);
         const uint32_t rem = i - tl * hw;
-        const uint32_t h = rem / W;
+        const uint32_t h = fast_div(rem, p.div_w);
         q.b = b;
         q.r = r;
         q.i = i;
         q.t_g = p.frame_offset + tl;
         q.h = (int)h;
         q.w = (int)(rem - h * W);
-        q.crow = ((uint32_t)p.slot + i) % (uint32_t)p.cache_tokens;
+        const uint32_t si = (uint32_t)p.slot + i;
+        q.crow = si - fast_div(si, p.div_cache) * (uint32_t)p.cache_tokens;
     } else {
         q.b = u / p.n_tok;
         q.r = u - q.b * p.n_tok;
@@ -366,30 +390,59 @@ __device__ __forceinline__ void pair_trig(const Params& p, const PairInfo<PPV>& 
     }
 }
 
+// acc + lo^2 + hi^2 for the two bf16 halves of a 32-bit word (lo, the element at the lower
+// address, first), without widening them: fma.rn.f32.bf16 multiplies two bf16 operands
+// (the product of two 8-bit significands is exact in fp32) and adds an fp32 operand with
+// one rounding -- the same result as fmaf on the widened values.
+__device__ __forceinline__ float fma_squares_bf16x2(uint32_t u, float acc) {
+    asm("{\n"
+        "  .reg .b16 lo, hi;\n"
+        "  mov.b32 {lo, hi}, %1;\n"
+        "  fma.rn.f32.bf16 %0, lo, lo, %0;\n"
+        "  fma.rn.f32.bf16 %0, hi, hi, %0;\n"
+        "}"
+        : "+f"(acc)
+        : "r"(u));
+    return acc;
+}
+
+// Adds the squares of one vector of q and one of k to (sq, sk), in element order.  Every
+// kernel sums a thread's vectors with this in slot order, so the sums are bit-identical
+// across kernels.
+__device__ __forceinline__ void accumulate_squares(const uint4& xq, const uint4& xk, float& sq,
+                                                   float& sk) {
+    sq = fma_squares_bf16x2(xq.x, sq);
+    sq = fma_squares_bf16x2(xq.y, sq);
+    sq = fma_squares_bf16x2(xq.z, sq);
+    sq = fma_squares_bf16x2(xq.w, sq);
+    sk = fma_squares_bf16x2(xk.x, sk);
+    sk = fma_squares_bf16x2(xk.y, sk);
+    sk = fma_squares_bf16x2(xk.z, sk);
+    sk = fma_squares_bf16x2(xk.w, sk);
+}
+__device__ __forceinline__ void accumulate_squares(const float4& xq, const float4& xk, float& sq,
+                                                   float& sk) {
+    sq = fmaf(xq.x, xq.x, sq);
+    sq = fmaf(xq.y, xq.y, sq);
+    sq = fmaf(xq.z, xq.z, sq);
+    sq = fmaf(xq.w, xq.w, sq);
+    sk = fmaf(xk.x, xk.x, sk);
+    sk = fmaf(xk.y, xk.y, sk);
+    sk = fmaf(xk.z, xk.z, sk);
+    sk = fmaf(xk.w, xk.w, sk);
+}
+
 // Sum of squares of this thread's share of one row of q and of k (fixed order).
 template <typename T, int VPT, int PAIR>
 __device__ __forceinline__ void partial_sum_squares(const typename VecTraits<T>::Vec (&xq)[VPT],
                                                     const typename VecTraits<T>::Vec (&xk)[VPT],
                                                     int t, int tpr, int dim_vecs, float& sq,
                                                     float& sk) {
-    using Tr = VecTraits<T>;
     sq = 0.f;
     sk = 0.f;
 #pragma unroll
-    for (int s = 0; s < VPT; ++s) {
-        if (slot_vec<T, PAIR>(t, s, tpr) < dim_vecs) {
-#pragma unroll
-            for (int m = 0; m < Tr::kPairsPerVec; ++m) {
-                float a, c;
-                Tr::pair(xq[s], m, a, c);
-                sq = fmaf(a, a, sq);
-                sq = fmaf(c, c, sq);
-                Tr::pair(xk[s], m, a, c);
-                sk = fmaf(a, a, sk);
-                sk = fmaf(c, c, sk);
-            }
-        }
-    }
+    for (int s = 0; s < VPT; ++s)
+        if (slot_vec<T, PAIR>(t, s, tpr) < dim_vecs) accumulate_squares(xq[s], xk[s], sq, sk);
 }
 
 // Team-wide totals of (sq, sk): warp butterfly, then the warps' partials in warp order.
@@ -416,44 +469,89 @@ __device__ __forceinline__ float2 team_sum(float sq, float sk, float2* s_part, i
     return make_float2(sq, sk);
 }
 
-// y = x * rs * w (RMSNorm), then (y_re + i y_im) * (cos + i sin) (RoPE), for the
-// pairs of one vector, as fp32 in element order; weights come from shared memory.
-template <typename T, bool NORM>
-__device__ __forceinline__ void norm_rotate_f(
-    const typename VecTraits<T>::Vec& x, float rs, const float* s_w, int e0,
-    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec],
-    float (&out)[VecTraits<T>::kElems]) {
-    using Tr = VecTraits<T>;
-    constexpr int PPV = Tr::kPairsPerVec;
-    float w[2 * PPV];
-    if (NORM) {
+// The norm weights sit in shared memory permuted inside every group of four elements --
+// (w0, w2, w1, w3) -- so that one 16-byte read gives the weights of the real parts of two
+// neighbouring pairs and, as the other half, those of their imaginary parts: the operand
+// layout of the packed fp32x2 arithmetic below.  Weights of elements e .. e + 3 (e a
+// multiple of 4) in element order:
+__device__ __forceinline__ float4 weights4(const float* s_w, int e) {
+    const float4 a = *reinterpret_cast<const float4*>(s_w + e);
+    return make_float4(a.x, a.z, a.y, a.w);
+}
+
+// A row's rotation for the thread's pairs, scaled by the row's RMSNorm factor rs, as
+// fp32x2 lanes (pairs 2h and 2h + 1): c = rs cos, s = rs sin, ns = -(rs sin).
+template <int PPV>
+struct RowRot {
+    float2 c[PPV / 2], s[PPV / 2], ns[PPV / 2];
+};
+
+template <int PPV>
+__device__ __forceinline__ RowRot<PPV> row_rot(float rs, const float (&cs)[PPV],
+                                               const float (&sn)[PPV]) {
+    RowRot<PPV> r;
+    const float2 p = make_float2(rs, rs), n = make_float2(-rs, -rs);
 #pragma unroll
-        for (int c = 0; c < 2 * PPV / 4; ++c) {
-            const float4 a = *reinterpret_cast<const float4*>(s_w + e0 + 4 * c);
-            w[4 * c] = a.x; w[4 * c + 1] = a.y; w[4 * c + 2] = a.z; w[4 * c + 3] = a.w;
-        }
+    for (int h = 0; h < PPV / 2; ++h) {
+        const float2 c = make_float2(cs[2 * h], cs[2 * h + 1]);
+        const float2 sv = make_float2(sn[2 * h], sn[2 * h + 1]);
+        r.c[h] = __fmul2_rn(c, p);
+        r.s[h] = __fmul2_rn(sv, p);
+        r.ns[h] = __fmul2_rn(sv, n);
     }
+    return r;
+}
+
+// RMSNorm and RoPE of one vector: y = x w (the weight), then (y_re + i y_im) times
+// rs (cos + i sin) -- the row's 1/rms folded into the rotation -- two pairs per packed
+// fp32x2 operation; the result as fp32 in element order.
+template <typename T>
+__device__ __forceinline__ void norm_rotate_f(
+    const typename VecTraits<T>::Vec& x, const float* s_w, int e0,
+    const RowRot<VecTraits<T>::kPairsPerVec>& r, float (&out)[VecTraits<T>::kElems]) {
+    using Tr = VecTraits<T>;
 #pragma unroll
-    for (int m = 0; m < PPV; ++m) {
-        float a, c;
-        Tr::pair(x, m, a, c);
-        if (NORM) {
-            a = a * rs * w[2 * m];
-            c = c * rs * w[2 * m + 1];
-        }
-        out[2 * m] = a * cs[m] - c * sn[m];
-        out[2 * m + 1] = a * sn[m] + c * cs[m];
+    for (int h = 0; h < Tr::kPairsPerVec / 2; ++h) {
+        const float4 w = *reinterpret_cast<const float4*>(s_w + e0 + 4 * h);  // permuted
+        float a0, c0, a1, c1;
+        Tr::pair(x, 2 * h, a0, c0);
+        Tr::pair(x, 2 * h + 1, a1, c1);
+        const float2 y_re = __fmul2_rn(make_float2(a0, a1), make_float2(w.x, w.y));
+        const float2 y_im = __fmul2_rn(make_float2(c0, c1), make_float2(w.z, w.w));
+        const float2 o_re = __ffma2_rn(y_im, r.ns[h], __fmul2_rn(y_re, r.c[h]));
+        const float2 o_im = __ffma2_rn(y_im, r.c[h], __fmul2_rn(y_re, r.s[h]));
+        out[4 * h] = o_re.x;
+        out[4 * h + 1] = o_im.x;
+        out[4 * h + 2] = o_re.y;
+        out[4 * h + 3] = o_im.y;
     }
 }
 
 // The same, rounded once to the element type.
-template <typename T, bool NORM>
+template <typename T>
 __device__ __forceinline__ typename VecTraits<T>::Vec norm_rotate(
-    const typename VecTraits<T>::Vec& x, float rs, const float* s_w, int e0,
-    const float (&cs)[VecTraits<T>::kPairsPerVec], const float (&sn)[VecTraits<T>::kPairsPerVec]) {
+    const typename VecTraits<T>::Vec& x, const float* s_w, int e0,
+    const RowRot<VecTraits<T>::kPairsPerVec>& r) {
     float out[VecTraits<T>::kElems];
-    norm_rotate_f<T, NORM>(x, rs, s_w, e0, cs, sn, out);
+    norm_rotate_f<T>(x, s_w, e0, r, out);
     return VecTraits<T>::pack_elems(out);
+}
+
+// RoPE alone (the rotation-only entry point), rounded once to the element type.
+template <typename T>
+__device__ __forceinline__ typename VecTraits<T>::Vec rotate_only(
+    const typename VecTraits<T>::Vec& x, const float (&cs)[VecTraits<T>::kPairsPerVec],
+    const float (&sn)[VecTraits<T>::kPairsPerVec]) {
+    using Tr = VecTraits<T>;
+    float out[Tr::kElems];
+#pragma unroll
+    for (int m = 0; m < Tr::kPairsPerVec; ++m) {
+        float a, c;
+        Tr::pair(x, m, a, c);
+        out[2 * m] = a * cs[m] - c * sn[m];
+        out[2 * m + 1] = a * sn[m] + c * cs[m];
+    }
+    return Tr::pack_elems(out);
 }
 
 // rotate_half pairing: `re_v` is a head's first-half vector at some position and
@@ -472,8 +570,8 @@ __device__ __forceinline__ void norm_rotate_half_f(
     if (NORM) {
 #pragma unroll
         for (int c = 0; c < E / 4; ++c) {
-            const float4 a = *reinterpret_cast<const float4*>(s_w + e_re + 4 * c);
-            const float4 b = *reinterpret_cast<const float4*>(s_w + e_im + 4 * c);
+            const float4 a = weights4(s_w, e_re + 4 * c);
+            const float4 b = weights4(s_w, e_im + 4 * c);
             wr[4 * c] = a.x; wr[4 * c + 1] = a.y; wr[4 * c + 2] = a.z; wr[4 * c + 3] = a.w;
             wi[4 * c] = b.x; wi[4 * c + 1] = b.y; wi[4 * c + 2] = b.z; wi[4 * c + 3] = b.w;
         }
@@ -689,8 +787,9 @@ __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, floa
     float4* sq4 = reinterpret_cast<float4*>(s_wq);
     float4* sk4 = reinterpret_cast<float4*>(s_wk);
     for (int e = threadIdx.x; e < p.dim / 4; e += blockDim.x) {
-        sq4[e] = __ldg(gq + e);
-        sk4[e] = __ldg(gk + e);
+        const float4 a = __ldg(gq + e), b = __ldg(gk + e);
+        sq4[e] = make_float4(a.x, a.z, a.y, a.w);  // (w0, w2, w1, w3): see weights4
+        sk4[e] = make_float4(b.x, b.z, b.y, b.w);
     }
 }
 
@@ -714,7 +813,12 @@ __device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
 // fp32 until they are quantized, and the K and V keys of one head travel in one shuffle
 // word.  Every lane of the warp takes part in the head-wise maximum, whether its slots
 // hold vectors or not.
-template <typename T, int VPT, int PAIR, int MODE, int CF>
+// Parts of a row's output: q (q_out), K (the K cache row, with V where V is quantized), or
+// both.  The register kernel emits q and K separately so that it can request the next
+// row's q while this row's K is still being written.
+enum EmitPart : int { kEmitQ = 1, kEmitK = 2, kEmitAll = 3 };
+
+template <typename T, int VPT, int PAIR, int MODE, int CF, int PART = kEmitAll>
 __device__ __forceinline__ void emit_row(
     const Params& p, int t, const RowPos& pos, int64_t row_vec,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -731,60 +835,80 @@ __device__ __forceinline__ void emit_row(
     constexpr int VPH = Tr::kVecsPerHead;
     constexpr int VPB = 16 / EPV;  // vectors (lanes) per NVFP4 block
     if constexpr (PAIR == kPairAdjacent) {
+        // q first, for every slot, then K (and V where it is quantized): one row rotation
+        // (RowRot) is live at a time
+        if constexpr (!(PART & kEmitQ)) {
+        } else if constexpr (NORM) {
+            const RowRot<Tr::kPairsPerVec> rot_q = row_rot(rq, cs, sn);
 #pragma unroll
-        for (int s = 0; s < VPT; ++s) {
-            const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
-            const bool valid = idx < p.dim_vecs && (!kDeviceChecks || pos.ok);
-            const int e0 = idx * EPV;
-            if (valid)
-                store_out(qo + row_vec + idx, norm_rotate<T, NORM>(xq[s], rq, s_wq, e0, cs, sn));
-            if constexpr (QUANT) {
-                float o[EPV];
-                uint32_t kk = 0, kv = 0;
-                if (valid) {
-                    norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
-                    kk = fp8_key(abs_max<EPV>(o));
-                    kv = vec_key(xv[s]);
-                }
-                Fp8Scale sk, sv;
-                fp8_scale_pair(kk, kv, VPH, sk, sv);
-                if (valid) {
-                    const int64_t vi = cache_vec_index(p, pos, idx);
-                    store_fp8(kc, vi, o, sk.inv);
-                    store_v_fp8<T>(vc, vi, xv[s], sv.inv);
-                    if ((idx & (VPH - 1)) == 0) {
-                        const int64_t si = cache_scale_index(p, pos, idx / VPH);
-                        __stcs(p.k_scale + si, sk.scale);
-                        __stcs(p.v_scale + si, sv.scale);
-                    }
-                }
-            } else if constexpr (QUANT4) {
-                float o[EPV];
-                float ak = 0.0f, av = 0.0f;
-                if (valid) {
-                    norm_rotate_f<T, true>(xk[s], rk, s_wk, e0, cs, sn, o);
-                    ak = abs_max<EPV>(o);
-                    av = vec_abs_max(xv[s]);
-                }
-                ak = block_max(ak, VPB);
-                av = block_max(av, VPB);
-                if (valid) {
-                    const Nvfp4Scale sk = nvfp4_scale(ak, p.k_inv6g, s_r);
-                    const Nvfp4Scale sv = nvfp4_scale(av, p.v_inv6g, s_r + 256);
-                    const int64_t vi = cache_vec_index(p, pos, idx);
-                    float v[EPV];
+            for (int s = 0; s < VPT; ++s) {
+                const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+                if (idx < p.dim_vecs && (!kDeviceChecks || pos.ok))
+                    store_out(qo + row_vec + idx, norm_rotate<T>(xq[s], s_wq, idx * EPV, rot_q));
+            }
+        } else {
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) v[e] = Tr::elem(xv[s], e);
-                    store_fp4(kc, vi, o, sk.r);
-                    store_fp4(vc, vi, v, sv.r);
-                    if ((idx & (VPB - 1)) == 0) {
-                        __stcs(reinterpret_cast<char*>(p.k_bscale + vi / VPB), (char)sk.code);
-                        __stcs(reinterpret_cast<char*>(p.v_bscale + vi / VPB), (char)sv.code);
+            for (int s = 0; s < VPT; ++s) {
+                const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+                if (idx < p.dim_vecs && (!kDeviceChecks || pos.ok))
+                    store_out(qo + row_vec + idx, rotate_only<T>(xq[s], cs, sn));
+            }
+        }
+        if constexpr (MODE == kModeFused && (PART & kEmitK)) {
+            const RowRot<Tr::kPairsPerVec> rot_k = row_rot(rk, cs, sn);
+#pragma unroll
+            for (int s = 0; s < VPT; ++s) {
+                const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
+                const bool valid = idx < p.dim_vecs && (!kDeviceChecks || pos.ok);
+                const int e0 = idx * EPV;
+                if constexpr (QUANT) {
+                    float o[EPV];
+                    uint32_t kk = 0, kv = 0;
+                    if (valid) {
+                        norm_rotate_f<T>(xk[s], s_wk, e0, rot_k, o);
+                        kk = fp8_key(abs_max<EPV>(o));
+                        kv = vec_key(xv[s]);
                     }
+                    Fp8Scale sk, sv;
+                    fp8_scale_pair(kk, kv, VPH, sk, sv);
+                    if (valid) {
+                        const int64_t vi = cache_vec_index(p, pos, idx);
+                        store_fp8(kc, vi, o, sk.inv);
+                        store_v_fp8<T>(vc, vi, xv[s], sv.inv);
+                        if ((idx & (VPH - 1)) == 0) {
+                            const int64_t si = cache_scale_index(p, pos, idx / VPH);
+                            __stcs(p.k_scale + si, sk.scale);
+                            __stcs(p.v_scale + si, sv.scale);
+                        }
+                    }
+                } else if constexpr (QUANT4) {
+                    float o[EPV];
+                    float ak = 0.0f, av = 0.0f;
+                    if (valid) {
+                        norm_rotate_f<T>(xk[s], s_wk, e0, rot_k, o);
+                        ak = abs_max<EPV>(o);
+                        av = vec_abs_max(xv[s]);
+                    }
+                    ak = block_max(ak, VPB);
+                    av = block_max(av, VPB);
+                    if (valid) {
+                        const Nvfp4Scale sk = nvfp4_scale(ak, p.k_inv6g, s_r);
+                        const Nvfp4Scale sv = nvfp4_scale(av, p.v_inv6g, s_r + 256);
+                        const int64_t vi = cache_vec_index(p, pos, idx);
+                        float v[EPV];
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) v[e] = Tr::elem(xv[s], e);
+                        store_fp4(kc, vi, o, sk.r);
+                        store_fp4(vc, vi, v, sv.r);
+                        if ((idx & (VPB - 1)) == 0) {
+                            __stcs(reinterpret_cast<char*>(p.k_bscale + vi / VPB), (char)sk.code);
+                            __stcs(reinterpret_cast<char*>(p.v_bscale + vi / VPB), (char)sv.code);
+                        }
+                    }
+                } else if (valid) {
+                    store_out(kc + cache_vec_index(p, pos, idx),
+                              norm_rotate<T>(xk[s], s_wk, e0, rot_k));
                 }
-            } else if (MODE == kModeFused && valid) {
-                store_out(kc + cache_vec_index(p, pos, idx),
-                          norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
             }
         }
     } else {
@@ -795,13 +919,13 @@ __device__ __forceinline__ void emit_row(
             const int i_im = slot_vec<T, PAIR>(t, s + 1, p.tpr);
             const bool valid = i_re < p.dim_vecs && (!kDeviceChecks || pos.ok);
             float o_re[EPV], o_im[EPV];
-            if (valid) {
+            if ((PART & kEmitQ) && valid) {
                 norm_rotate_half_f<T, NORM>(xq[s], xq[s + 1], rq, s_wq, i_re * EPV, i_im * EPV,
                                             cs, sn, o_re, o_im);
                 store_out(qo + row_vec + i_re, Tr::pack_elems(o_re));
                 store_out(qo + row_vec + i_im, Tr::pack_elems(o_im));
             }
-            if constexpr (MODE == kModeFused) {
+            if constexpr (MODE == kModeFused && (PART & kEmitK)) {
                 if (valid)
                     norm_rotate_half_f<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV,
                                                 i_im * EPV, cs, sn, o_re, o_im);
@@ -922,7 +1046,7 @@ __device__ __forceinline__ void store_v_row_sp(const Params& p, int t, const Row
     }
 }
 
-template <typename T, int VPT>
+template <typename T, int VPT, int PART = kEmitAll>
 __device__ __forceinline__ void emit_row_sp(
     const Params& p, int t, const RowPos& pos,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -939,41 +1063,44 @@ __device__ __forceinline__ void emit_row_sp(
         ok = pos.ok && pos.i >= p.sp_q_row0 && pos.i - p.sp_q_row0 < p.sp_q_rows;
         if (pos.ok && !ok) record_index_error(p);
     }
+    if constexpr (PART & kEmitQ) {
+    const RowRot<Tr::kPairsPerVec> rot_q = row_rot(rq, cs, sn);
 #pragma unroll
     for (int s = 0; s < VPT; ++s) {
         const int idx = slot_vec<T, kPairAdjacent>(t, s, p.tpr);
         if (idx < p.dim_vecs && ok) {
-            const int d = dst[s] >> 16, dv = dst[s] & 0xFFFF;
-            const int e0 = idx * Tr::kElems;
-            Vec* qd = reinterpret_cast<Vec*>(s_sp[3 * d]);
-            Vec* kd = reinterpret_cast<Vec*>(s_sp[3 * d + 1]);
-            store_out(qd + q_row + dv, norm_rotate<T, true>(xq[s], rq, s_wq, e0, cs, sn));
-            store_out(kd + sp_cache_index(p, pos, dv),
-                      norm_rotate<T, true>(xk[s], rk, s_wk, e0, cs, sn));
+            Vec* qd = reinterpret_cast<Vec*>(s_sp[3 * (dst[s] >> 16)]);
+            store_out(qd + q_row + (dst[s] & 0xFFFF),
+                      norm_rotate<T>(xq[s], s_wq, idx * Tr::kElems, rot_q));
         }
+    }
+    }
+    if constexpr (PART & kEmitK) {
+    const RowRot<Tr::kPairsPerVec> rot_k = row_rot(rk, cs, sn);
+#pragma unroll
+    for (int s = 0; s < VPT; ++s) {
+        const int idx = slot_vec<T, kPairAdjacent>(t, s, p.tpr);
+        if (idx < p.dim_vecs && ok) {
+            Vec* kd = reinterpret_cast<Vec*>(s_sp[3 * (dst[s] >> 16) + 1]);
+            store_out(kd + sp_cache_index(p, pos, dst[s] & 0xFFFF),
+                      norm_rotate<T>(xk[s], s_wk, idx * Tr::kElems, rot_k));
+        }
+    }
     }
 }
 
 // ---------------------------------------------------------------- register kernel
 
-// This thread's vectors of token row u of q, k and v (v and k only where the mode has them).
-template <typename T, int VPT, int PAIR, bool HAS_K, bool HAS_V>
-__device__ __forceinline__ void load_row(const Params& p, int t, int64_t u,
-                                         const typename VecTraits<T>::Vec* qg,
-                                         const typename VecTraits<T>::Vec* kg,
-                                         const typename VecTraits<T>::Vec* vg,
-                                         typename VecTraits<T>::Vec (&xq)[VPT],
-                                         typename VecTraits<T>::Vec (&xk)[VPT],
-                                         typename VecTraits<T>::Vec (&xv)[VPT]) {
+// This thread's vectors of one tensor's token row u.
+template <typename T, int VPT, int PAIR>
+__device__ __forceinline__ void load_vecs(const Params& p, int t, int64_t u,
+                                          const typename VecTraits<T>::Vec* g,
+                                          typename VecTraits<T>::Vec (&x)[VPT]) {
     const int64_t row_vec = u * p.dim_vecs;
 #pragma unroll
     for (int s = 0; s < VPT; ++s) {
         const int idx = slot_vec<T, PAIR>(t, s, p.tpr);
-        if (idx < p.dim_vecs) {
-            xq[s] = load_stream(qg + row_vec + idx);
-            if (HAS_K) xk[s] = load_stream(kg + row_vec + idx);
-            if (HAS_V) xv[s] = load_stream(vg + row_vec + idx);
-        }
+        if (idx < p.dim_vecs) x[s] = load_stream(g + row_vec + idx);
     }
 }
 
@@ -987,6 +1114,9 @@ qk_norm_rope_kernel(const Params p) {
     constexpr bool SP = MODE == kModeFusedSP;
     constexpr bool HAS_V = FUSED && MODE != kModeFusedNoV;
     constexpr int EMIT_MODE = MODE == kModeFusedNoV ? kModeFused : MODE;
+    // V leaves the registers right after its row arrives (a bit copy) unless it is
+    // quantized beside K
+    constexpr bool V_EARLY = HAS_V && (SP || CF == kCacheSame);
     static_assert(HAS_V || !FUSED || CF == kCacheSame, "no-V step: same-dtype K cache");
     static_assert(!SP || (PAIR == kPairAdjacent && CF == kCacheSame),
                   "head-scatter stores: adjacent pairing, same-dtype caches");
@@ -1023,7 +1153,11 @@ qk_norm_rope_kernel(const Params p) {
     // The team's first row is requested before the block stages its weights, so the two
     // latencies overlap instead of adding up at the start of every launch.
     Vec xq[VPT], xk[VPT], xv[VPT];
-    if (u0 < p.units) load_row<T, VPT, PAIR, FUSED, HAS_V>(p, t, u0, qg, kg, vg, xq, xk, xv);
+    if (u0 < p.units) {
+        load_vecs<T, VPT, PAIR>(p, t, u0, qg, xq);
+        if (FUSED) load_vecs<T, VPT, PAIR>(p, t, u0, kg, xk);
+        if (HAS_V) load_vecs<T, VPT, PAIR>(p, t, u0, vg, xv);
+    }
     if (FUSED) {
         if constexpr (SP) {
 #pragma unroll
@@ -1041,8 +1175,14 @@ qk_norm_rope_kernel(const Params p) {
         for (int s = 0; s < VPT; ++s) dst[s] = sp_code(p, slot_vec<T, PAIR>(t, s, p.tpr));
     }
 
+    // Rolling prefetch: each tensor's registers are refilled with the team's next row as
+    // soon as this row is done with them -- V right after its bit copy, q after q_out, K
+    // (and a quantized V) after the cache row -- so the next row's loads overlap this row's
+    // reduction and arithmetic without a second set of row registers.
     int parity = 0;
     for (int64_t u = u0; u < p.units; u += stride) {
+        const int64_t next = u + stride;
+        const bool more = next < p.units;
         const RowPos pos = decode_row(p, u);
         const int64_t row_vec = u * p.dim_vecs;
         float cs[NP], sn[NP];
@@ -1051,8 +1191,8 @@ qk_norm_rope_kernel(const Params p) {
         float rq = 1.0f, rk = 1.0f;
         if (FUSED) {
             if constexpr (SP) store_v_row_sp<T, VPT>(p, t, pos, xv, dst, s_sp);
-            else if constexpr (CF == kCacheSame && HAS_V)
-                store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
+            else if constexpr (V_EARLY) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
+            if (V_EARLY && more) load_vecs<T, VPT, PAIR>(p, t, next, vg, xv);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -1061,15 +1201,25 @@ qk_norm_rope_kernel(const Params p) {
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
         if constexpr (SP)
-            emit_row_sp<T, VPT>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
+            emit_row_sp<T, VPT, kEmitQ>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
         else
-            emit_row<T, VPT, PAIR, EMIT_MODE, CF>(p, t, pos, row_vec, xq, xk, xv, rq, rk,
-                                                  s_wq, s_wk, cs, sn, qo, kc, vc, s_r);
-        // The team's next row, requested after this row's stores: one row in registers at a
-        // time keeps the blocks per SM up (a second row prefetched into registers measured
-        // 20-40% slower on B200, from the lost occupancy).
-        if (u + stride < p.units)
-            load_row<T, VPT, PAIR, FUSED, HAS_V>(p, t, u + stride, qg, kg, vg, xq, xk, xv);
+            emit_row<T, VPT, PAIR, EMIT_MODE, CF, kEmitQ>(p, t, pos, row_vec, xq, xk, xv, rq,
+                                                          rk, s_wq, s_wk, cs, sn, qo, kc, vc,
+                                                          s_r);
+        if (more) load_vecs<T, VPT, PAIR>(p, t, next, qg, xq);
+        if constexpr (FUSED) {
+            if constexpr (SP)
+                emit_row_sp<T, VPT, kEmitK>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst,
+                                            s_sp);
+            else
+                emit_row<T, VPT, PAIR, EMIT_MODE, CF, kEmitK>(p, t, pos, row_vec, xq, xk, xv,
+                                                              rq, rk, s_wq, s_wk, cs, sn, qo,
+                                                              kc, vc, s_r);
+            if (more) {
+                load_vecs<T, VPT, PAIR>(p, t, next, kg, xk);
+                if (HAS_V && !V_EARLY) load_vecs<T, VPT, PAIR>(p, t, next, vg, xv);
+            }
+        }
     }
 }
 

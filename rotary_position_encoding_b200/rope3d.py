@@ -67,6 +67,7 @@ class rope3d_sp_dest(ctypes.Structure):
 ROPE3D_PATH_AUTO = 0
 ROPE3D_PATH_REGISTERS = 1
 ROPE3D_PATH_TMA = 2
+ROPE3D_PATH_STREAM = 3
 
 _VP = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -112,6 +113,7 @@ SIGNATURES = {
     "rope3d_testing_gemm_cta_group": ([_INT], _INT),
     "rope3d_testing_last_path": ([], _INT),
     "rope3d_testing_shrink_checked_cache": ([_I64], _INT),
+    "rope3d_testing_fast_divide": ([ctypes.c_uint32, ctypes.c_uint32], ctypes.c_uint32),
 }
 
 _lib = None

@@ -202,3 +202,25 @@ def test_step_wrappers_check_tensors_before_any_call(entry):
     with pytest.raises(ValueError, match="all be"):
         fn(q, q[:, :3], q, q.clone(), token_begin=0, token_end=4, k_cache=kc, v_cache=kc.clone(),
            **args)
+
+
+def test_fast_divide_matches_integer_division(lib):
+    """The multiply-and-shift division the kernels' 32-bit decode uses, on the host: exact
+    floor(n / d) for every dividend below 2^31, at random and at the edges (powers of two
+    and their neighbours, the grid sizes of the workloads, n = q d - 1, q d, q d + 1)."""
+    import numpy as np
+    rng = np.random.default_rng(11)
+    top = (1 << 31) - 1
+    divisors = {1, 2, 3, 5, 7, 52, 80, 1560, 3600, 4680, 10800, 32760, 75600, top, top - 1}
+    divisors |= {(1 << k) + e for k in range(1, 31) for e in (-1, 0, 1)}
+    divisors |= set(int(x) for x in rng.integers(1, top, 300))
+    for d in sorted(x for x in divisors if 1 <= x <= top):
+        ns = {0, 1, d - 1, d, d + 1, top, top - 1, top - d}
+        for q in (1, 2, 3, top // d, top // d - 1):
+            ns |= {q * d - 1, q * d, q * d + 1}
+        ns |= set(int(x) for x in rng.integers(0, top + 1, 40))
+        for n in ns:
+            if 0 <= n <= top:
+                assert lib.rope3d_testing_fast_divide(n, d) == n // d, (n, d)
+    assert lib.rope3d_testing_fast_divide(5, 0) == 0xFFFFFFFF
+    assert lib.rope3d_testing_fast_divide(1 << 31, 3) == 0xFFFFFFFF
