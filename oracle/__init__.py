@@ -400,6 +400,26 @@ class Oracle:
                 k_dst[r][:, local, rows] = kc[:, rows, head]
                 v_dst[r][:, local, rows] = vc[:, rows, head]
 
+    @staticmethod
+    def sp_output_all_to_all(o_ranks, cuts):
+        """The all-to-all after attention (Algorithm 3, last step: o <- AllToAll(o,
+        scatter_dim=1, gather_dim=2)).  Rank r holds o_ranks[r] = [B, L, N/P, D]: the whole
+        sequence for its own heads [r N/P, (r+1) N/P).  Afterwards rank r' holds its token
+        slice [cuts[r'], cuts[r'+1]) with every head: out[r'][b, i - cuts[r'], r N/P + h]
+        = o_ranks[r][b, i, h].  Returns the P outputs [B, cuts[r'+1] - cuts[r'], N, D]."""
+        P = len(o_ranks)
+        B, L, hl, D = o_ranks[0].shape
+        if len(cuts) != P + 1 or cuts[0] != 0 or cuts[-1] != L or any(
+                cuts[j] > cuts[j + 1] for j in range(P)):
+            raise ValueError("cuts must rise from 0 to L with one slice per rank")
+        outs = [np.zeros((B, cuts[r + 1] - cuts[r], P * hl, D), dtype=o_ranks[0].dtype)
+                for r in range(P)]
+        for r in range(P):              # source rank: its heads
+            for dst in range(P):        # destination rank: its tokens
+                a, e = cuts[dst], cuts[dst + 1]
+                outs[dst][:, :, r * hl:(r + 1) * hl] = o_ranks[r][:, a:e]
+        return outs
+
     # ---- QKV projection feeding the step (Algorithm 1/3 step 1, Section 3.4.1 item 3)
 
     @staticmethod

@@ -839,4 +839,48 @@ def check_sp_head_scatter_is_whole_step_split_by_heads(orc):
                 assert np.all(np.delete(kt, rows, axis=1) == 7.0)
 
 
+def check_sp_output_all_to_all_inverts_the_head_split(orc):
+    """Algorithm 3's last step, o <- AllToAll(o, scatter_dim=1, gather_dim=2): if every
+    rank holds the whole sequence for its own heads -- a tensor X split by heads -- then
+    afterwards rank r holds its token slice of X with every head, i.e. X split by tokens
+    (numpy.split on the other axis).  P = 1, 2, 4, uneven slices and an empty one."""
+    rng = _rng(43)
+    B, L, N = 2, 23, 8
+    X = rng.standard_normal((B, L, N, D))
+    for P, cuts in ((1, [0, L]), (2, [0, 9, L]), (4, [0, 5, 5, 17, L]), (4, [0, 6, 12, 18, L])):
+        hl = N // P
+        o_ranks = np.split(X, P, axis=2)  # rank r: heads [r hl, (r+1) hl), all tokens
+        outs = orc.sp_output_all_to_all([x.copy() for x in o_ranks], cuts)
+        want = np.split(X, cuts[1:-1], axis=1)  # rank r: tokens [cuts[r], cuts[r+1])
+        assert len(outs) == P
+        for got, ref in zip(outs, want):
+            assert got.shape == ref.shape and np.array_equal(got, ref)
+
+
+def check_sp_round_trip_returns_each_slice_with_every_head(orc):
+    """The two exchanges of Algorithm 3 compose: rank slices through the step with the
+    head scatter (step 4 folded into the stores) give each owner the whole sequence for
+    its heads; the output all-to-all then gives each rank back its own token slice with
+    every head, equal to the whole-sequence step's rows of that slice."""
+    rng = _rng(44)
+    B, N, T, H, W, s, C, slot = 1, 4, 2, 3, 5, 3, 40, 7
+    L = T * H * W
+    q, k, v = (_f32(rng.standard_normal((B, L, N, D))) for _ in range(3))
+    wq, wk = (_f32(rng.uniform(0.5, 1.5, N * D)) for _ in range(2))
+    kw, vw = np.zeros((B, C, N, D)), np.zeros((B, C, N, D))
+    whole = orc.qk_norm_rope_append_layout(q, k, v, 0, L, s, T, H, W, wq, wk, 1e-6, kw, vw,
+                                           slot)
+    P, cuts = 2, [0, 11, L]
+    hl = N // P
+    q_dst = [np.zeros((B, L, hl, D)) for _ in range(P)]
+    k_dst = [np.zeros((B, C, hl, D)) for _ in range(P)]
+    v_dst = [np.zeros((B, C, hl, D)) for _ in range(P)]
+    for a, e in zip(cuts[:-1], cuts[1:]):
+        orc.qk_norm_rope_append_sp(q[:, a:e].copy(), k[:, a:e].copy(), v[:, a:e].copy(), a, e,
+                                   s, T, H, W, wq, wk, 1e-6, q_dst, k_dst, v_dst, slot)
+    back = orc.sp_output_all_to_all(q_dst, cuts)
+    for r in range(P):
+        assert np.array_equal(back[r], whole[:, cuts[r]:cuts[r + 1]])
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

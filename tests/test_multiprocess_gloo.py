@@ -132,6 +132,37 @@ def _a2a_rank(rank, world, port, out_path):
         dist.destroy_process_group()
 
 
+def _out_a2a_rank(rank, world, port, out_path):
+    """Algorithm 3's last step on two gloo ranks: torch's all_to_all_single with the
+    sequence scattered and the heads gathered (uneven token slices) against the oracle's
+    definition."""
+    _init(rank, world, port)
+    import datetime
+
+    import oracle
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        B, L, hl, D = 2, 13, 3, 128
+        cuts = [0, 5, L]
+        o_mine = np.random.default_rng(300 + rank).standard_normal((B, L, hl, D))
+        # all_to_all_single splits dim 0: tokens first, then [B, hl, D]
+        send = torch.from_numpy(np.ascontiguousarray(o_mine.transpose(1, 0, 2, 3)))
+        mine = cuts[rank + 1] - cuts[rank]
+        recv = torch.empty((world * mine, B, hl, D), dtype=torch.float64)
+        dist.all_to_all_single(recv, send,
+                               output_split_sizes=[mine] * world,
+                               input_split_sizes=[cuts[j + 1] - cuts[j] for j in range(world)])
+        got = np.concatenate([c.transpose(1, 0, 2, 3) for c in np.split(recv.numpy(), world)],
+                             axis=2)  # source rank j's heads at [j hl, (j+1) hl)
+        everyone = [None] * world
+        dist.all_gather_object(everyone, o_mine)
+        ref = oracle.Oracle.sp_output_all_to_all(everyone, cuts)[rank]
+        with open(f"{out_path}.{rank}", "w") as f:
+            f.write("ok" if got.shape == ref.shape and np.array_equal(got, ref) else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
 def _sp_table_rank(rank, world, port, out_path):
     """The multi-GPU wiring's address bookkeeping with a CPU stand-in for the symmetric
     allocation: every rank's destination table lists, in rank order, the regions that
@@ -200,6 +231,13 @@ def test_fused_head_scatter_equals_all_to_all_on_two_ranks(tmp_path):
     mp.start_processes(_a2a_rank, args=(2, _free_port(), out), nprocs=2, start_method="spawn",
                        join=True)
     assert [open(f"{out}.{r}").read() for r in range(2)] == ["ok", "ok"]
+
+
+def test_output_all_to_all_equals_torch_all_to_all_on_two_ranks(tmp_path):
+    out = str(tmp_path / "oa2a")
+    mp.start_processes(_out_a2a_rank, args=(2, _free_port(), out), nprocs=2,
+                       start_method="spawn", join=True)
+    assert open(out + ".0").read() == "ok" and open(out + ".1").read() == "ok"
 
 
 def test_sp_destination_tables_on_two_ranks(tmp_path):

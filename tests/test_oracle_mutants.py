@@ -142,6 +142,11 @@ PY_MUTANTS = {
     "sp_round_robin_owner": ("r, local = divmod(head, hl)", "r, local = head % P, head // P"),
     "sp_q_row_ignores_row0": ("q_dst[r][:, i - q_row0, local]", "q_dst[r][:, i, local]"),
     "sp_cache_rows_drop_slot": ("rows = (slot + i) % C", "rows = i % C"),
+    "sp_out_heads_at_destination_offset": (
+        "outs[dst][:, :, r * hl:(r + 1) * hl] = o_ranks[r][:, a:e]",
+        "outs[dst][:, :, dst * hl:(dst + 1) * hl] = o_ranks[r][:, a:e]"),
+    "sp_out_tokens_of_source_slice": ("a, e = cuts[dst], cuts[dst + 1]",
+                                      "a, e = cuts[r], cuts[r + 1]"),
     "sp_head_major_as_token_major": (
         "                k_dst[r][:, local, rows] = kc[:, rows, head]",
         "                k_dst[r][:, rows, local] = kc[:, rows, head]"),
