@@ -273,6 +273,37 @@ ROPE3D_API int rope3d_qk_norm_rope_append_sp(
     const rope3d_options* options, void* cuda_stream);
 
 /*
+ * The all-to-all after attention, Algorithm 3's last step (o <- AllToAll(o,
+ * scatter_dim=1, gather_dim=2)): the inverse exchange of the head scatter above.  Rank
+ * dest->rank = r holds o [B][L][heads_per_rank][D] -- the whole sequence of L tokens for
+ * its own heads [r hl, (r+1) hl), hl = heads_per_rank -- and stores every token i to the
+ * rank r' whose slice [dest->cuts[r'], dest->cuts[r'+1]) contains i, as that rank's rows
+ * with all N = P hl heads:
+ *   dest->out[r'] [B][cuts[r'+1] - cuts[r']][N][D], row i - cuts[r'], heads
+ *   [r hl, (r+1) hl) of that row.
+ * Run on every rank with the same cuts and out tables (each listing the ranks' buffers in
+ * rank order), the ranks together leave in rank r' its token slice with every head.  A
+ * bit copy of 16-byte vectors: o and every out[r'] must be 16-byte aligned.  Destinations
+ * are device addresses valid on the calling device (this device's memory, or another
+ * GPU's memory mapped into this process); stores to another GPU are plain peer stores over
+ * NVLink.  The call does not synchronise with the other ranks (as for the head scatter).
+ * Errors: dest->ranks outside [1, ROPE3D_SP_MAX_RANKS] or rank outside [0, P) (EINVAL);
+ * cuts not rising from 0 to L (ERANGE); D != 128, an unknown dtype, a NULL o or a NULL
+ * out[r'] whose slice is not empty (EINVAL); a misaligned pointer (EALIGN); outputs that
+ * overlap one another or o (EOVERLAP).
+ */
+typedef struct rope3d_sp_out_dest {
+    int ranks;                               /* P                                      */
+    int rank;                                /* this rank r, 0 <= r < P                */
+    int64_t cuts[ROPE3D_SP_MAX_RANKS + 1];   /* rank r' holds tokens [cuts[r'], cuts[r'+1]) */
+    void* out[ROPE3D_SP_MAX_RANKS];          /* rank r's output buffer (entries >= P unused) */
+} rope3d_sp_out_dest;
+
+ROPE3D_API int rope3d_sp_output_all_to_all(const void* o, int64_t B, int64_t L,
+                                           int64_t heads_per_rank, int D, int dtype,
+                                           const rope3d_sp_out_dest* dest, void* cuda_stream);
+
+/*
  * The QKV projection that feeds the step (Algorithm 1/3 step 1, "q, k, v <- QKV(x)"; the
  * paper fuses it with the rotary step, Section 3.4.1 item 3), on the tensor cores:
  * y = x W^T + b with x [M][K] bf16 (token rows), w_qkv [3 N D][K] bf16 (an nn.Linear

@@ -17,8 +17,6 @@ extern "C" {
 #define ROPE3D_PATH_AUTO 0       /* the path measured faster for the shape (see rope3d.cu)     */
 #define ROPE3D_PATH_REGISTERS 1  /* rows loaded straight into registers                        */
 #define ROPE3D_PATH_TMA 2        /* rows streamed through shared memory (EINVAL if it does not fit) */
-#define ROPE3D_PATH_STREAM 3     /* rows staged in shared memory by a producer warp and consumed
-                                    from there in two passes (EINVAL if it does not fit) */
 
 /*
  * Bounded-wait settings of the bulk-copy ring kernel for later launches:

@@ -26,7 +26,7 @@ CHECKED_LIBRARY = os.path.join(PKG, "librope3d_checked.so")
 CHECKED_FLAGS = ("-DROPE3D_DEVICE_CHECKS",)
 SOURCES = [os.path.join(CSRC, "rope3d.cu")]
 DEPENDS = SOURCES + [os.path.join(CSRC, f) for f in ("rope3d_kernels.cuh", "rope3d_tma.cuh",
-                                                    "rope3d_stream.cuh", "rope3d_gemm.cuh")] + \
+                                                    "rope3d_gemm.cuh")] + \
     [os.path.join(INCLUDE, f) for f in ("rope3d.h", "rope3d_testing.h")]
 
 NVCC_FLAGS = [

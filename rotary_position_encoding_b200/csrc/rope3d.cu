@@ -9,7 +9,6 @@
 #include "rope3d_testing.h"
 #include "rope3d_kernels.cuh"
 #include "rope3d_tma.cuh"
-#include "rope3d_stream.cuh"
 #include "rope3d_gemm.cuh"
 
 #include <cuda_runtime.h>
@@ -26,6 +25,9 @@
 
 #ifndef ROPE3D_VPT_TARGET
 #define ROPE3D_VPT_TARGET 4  // vectors per thread per tensor the team size aims for
+#endif
+#ifndef ROPE3D_MAX_VPT
+#define ROPE3D_MAX_VPT 4     // kernels are instantiated for 1 .. ROPE3D_MAX_VPT vectors
 #endif
 // Threads per block the team count aims for, per kernel path.  Measured on B200 at the
 // 720P shape (40 heads, TPR 160): the register kernel is fastest with one team per
@@ -196,6 +198,9 @@ KernelFn pick_vpt(int vpt) {
         switch (vpt) {
             case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CF>;
             case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CF>;
+#if ROPE3D_MAX_VPT >= 6
+            case 6: return rope3d::qk_norm_rope_kernel<T, 6, TRIG, MODE, PAIR, CF>;
+#endif
             default: return nullptr;
         }
     } else {
@@ -204,6 +209,10 @@ KernelFn pick_vpt(int vpt) {
             case 2: return rope3d::qk_norm_rope_kernel<T, 2, TRIG, MODE, PAIR, CF>;
             case 3: return rope3d::qk_norm_rope_kernel<T, 3, TRIG, MODE, PAIR, CF>;
             case 4: return rope3d::qk_norm_rope_kernel<T, 4, TRIG, MODE, PAIR, CF>;
+#if ROPE3D_MAX_VPT >= 6
+            case 5: return rope3d::qk_norm_rope_kernel<T, 5, TRIG, MODE, PAIR, CF>;
+            case 6: return rope3d::qk_norm_rope_kernel<T, 6, TRIG, MODE, PAIR, CF>;
+#endif
             default: return nullptr;
         }
     }
@@ -263,6 +272,9 @@ TmaKernelFn pick_tma_vpt(int vpt) {
         switch (vpt) {
             case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR, CFP8>;
             case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR, CFP8>;
+#if ROPE3D_MAX_VPT >= 6
+            case 6: return rope3d::qk_norm_rope_tma_kernel<T, 6, TRIG, PAIR, CFP8>;
+#endif
             default: return nullptr;
         }
     } else {
@@ -271,6 +283,10 @@ TmaKernelFn pick_tma_vpt(int vpt) {
             case 2: return rope3d::qk_norm_rope_tma_kernel<T, 2, TRIG, PAIR, CFP8>;
             case 3: return rope3d::qk_norm_rope_tma_kernel<T, 3, TRIG, PAIR, CFP8>;
             case 4: return rope3d::qk_norm_rope_tma_kernel<T, 4, TRIG, PAIR, CFP8>;
+#if ROPE3D_MAX_VPT >= 6
+            case 5: return rope3d::qk_norm_rope_tma_kernel<T, 5, TRIG, PAIR, CFP8>;
+            case 6: return rope3d::qk_norm_rope_tma_kernel<T, 6, TRIG, PAIR, CFP8>;
+#endif
             default: return nullptr;
         }
     }
@@ -402,7 +418,7 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pair
     *launched = false;
     if (p.k_bscale != nullptr) return ROPE3D_OK;  // NVFP4 caches: register kernel only
     const Geometry g = geometry(N, dtype, pairing);
-    if (g.tpr > rope3d::kTmaMaxBlockThreads || g.vpt > 4) return ROPE3D_OK;
+    if (g.tpr > rope3d::kTmaMaxBlockThreads || g.vpt > ROPE3D_MAX_VPT) return ROPE3D_OK;
     const int warps_per_team = g.tpr / 32;
     p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
     int teams = (ROPE3D_TMA_BLOCK_TARGET < rope3d::kTmaMaxBlockThreads
@@ -450,141 +466,16 @@ int launch_fused_tma(rope3d::Params& p, int64_t N, int dtype, int trig, int pair
     return ok();
 }
 
-// ---------------------------------------------------------------- staged-row kernel
-
-template <typename T, int TRIG, int MODE, int PAIR, int CF>
-KernelFn pick_stream_vpt(int vpt) {
-    if constexpr (PAIR == rope3d::kPairHalf) {
-        switch (vpt) {
-            case 2: return rope3d::qk_norm_rope_stream_kernel<T, 2, TRIG, MODE, PAIR, CF>;
-            case 4: return rope3d::qk_norm_rope_stream_kernel<T, 4, TRIG, MODE, PAIR, CF>;
-            default: return nullptr;
-        }
-    } else {
-        switch (vpt) {
-            case 1: return rope3d::qk_norm_rope_stream_kernel<T, 1, TRIG, MODE, PAIR, CF>;
-            case 2: return rope3d::qk_norm_rope_stream_kernel<T, 2, TRIG, MODE, PAIR, CF>;
-            case 3: return rope3d::qk_norm_rope_stream_kernel<T, 3, TRIG, MODE, PAIR, CF>;
-            case 4: return rope3d::qk_norm_rope_stream_kernel<T, 4, TRIG, MODE, PAIR, CF>;
-            default: return nullptr;
-        }
-    }
-}
-
-template <typename T, int MODE, int PAIR, int CF>
-KernelFn pick_stream_trig(int trig, int vpt) {
-    return trig == ROPE3D_TRIG_TABLE ? pick_stream_vpt<T, rope3d::kTrigTable, MODE, PAIR, CF>(vpt)
-                                     : pick_stream_vpt<T, rope3d::kTrigOnTheFly, MODE, PAIR, CF>(vpt);
-}
-
-template <typename T, int CF>
-KernelFn pick_stream_pairing(int pairing, int trig, int vpt) {
-    return pairing == ROPE3D_PAIRING_HALF
-               ? pick_stream_trig<T, rope3d::kModeFused, rope3d::kPairHalf, CF>(trig, vpt)
-               : pick_stream_trig<T, rope3d::kModeFused, rope3d::kPairAdjacent, CF>(trig, vpt);
-}
-
-template <typename T>
-KernelFn pick_stream_type(int mode, int cache_fmt, int pairing, int trig, int vpt) {
-    if (mode == rope3d::kModeFusedSP)
-        return pairing == ROPE3D_PAIRING_ADJACENT && cache_fmt == rope3d::kCacheSame
-                   ? pick_stream_trig<T, rope3d::kModeFusedSP, rope3d::kPairAdjacent,
-                                      rope3d::kCacheSame>(trig, vpt)
-                   : nullptr;
-    switch (cache_fmt) {
-        case rope3d::kCacheFp8: return pick_stream_pairing<T, rope3d::kCacheFp8>(pairing, trig, vpt);
-        case rope3d::kCacheNvfp4:
-            return pick_stream_pairing<T, rope3d::kCacheNvfp4>(pairing, trig, vpt);
-        default: return pick_stream_pairing<T, rope3d::kCacheSame>(pairing, trig, vpt);
-    }
-}
-
-KernelFn pick_stream_kernel(int mode, int dtype, int trig, int pairing, int cache_fmt, int vpt) {
-    return dtype == ROPE3D_BF16
-               ? pick_stream_type<__nv_bfloat16>(mode, cache_fmt, pairing, trig, vpt)
-               : pick_stream_type<float>(mode, cache_fmt, pairing, trig, vpt);
-}
-
-// Shared-memory plan of the staged-row kernel: [aux_bytes: SP destination table or NVFP4
-// reciprocals] [full and empty barriers] [failure flags] [partials] [weights] [stages].
-size_t stream_layout(rope3d::Params& p, int teams, int stages, int warps_per_team,
-                     size_t aux_bytes) {
-    size_t off = align_up(aux_bytes, 16);
-    p.off_bars = (uint32_t)off;
-    off += (size_t)2 * stages * sizeof(uint64_t);
-    p.off_fail = (uint32_t)off;
-    off += (size_t)teams * sizeof(int);
-    off = align_up(off, 16);
-    p.off_part = (uint32_t)off;
-    off += (size_t)2 * teams * warps_per_team * sizeof(float2);
-    off = align_up(off, 16);
-    p.off_w = (uint32_t)off;
-    off += (size_t)2 * p.dim * sizeof(float);
-    off = align_up(off, 128);
-    p.off_stage = (uint32_t)off;
-    off += (size_t)stages * 3 * p.row_bytes;
-    return off;
-}
-
-#ifndef ROPE3D_STREAM_MAX_STAGES
-#define ROPE3D_STREAM_MAX_STAGES 32
-#endif
-
-// The fused step through the staged-row kernel: one block per SM, a producer warp and as
-// many teams as kStreamMaxThreads allows (at most kMaxTeamsPerBlock), and as many stages
-// as fit in shared memory (at least 2, at most ROPE3D_STREAM_MAX_STAGES).  *launched
-// stays false if the shape does not fit.
-int launch_fused_stream(rope3d::Params& p, int mode, int64_t N, int dtype, int trig, int pairing,
-                        int dev, const DeviceInfo& info, cudaStream_t stream, bool* launched) {
-    *launched = false;
-    const Geometry g = geometry(N, dtype, pairing);
-    if (g.tpr + 32 > rope3d::kStreamMaxThreads || g.vpt > 4) return ROPE3D_OK;
-    const int warps_per_team = g.tpr / 32;
-    p.row_bytes = (uint32_t)(N * rope3d::kHeadDim * (dtype == ROPE3D_BF16 ? 2 : 4));
-    int teams = (rope3d::kStreamMaxThreads - 32) / g.tpr;
-    if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
-    const size_t aux = mode == rope3d::kModeFusedSP ? 3 * rope3d::kMaxRanks * sizeof(void*)
-                       : p.k_bscale != nullptr ? rope3d::kNvfp4TableFloats * sizeof(float) : 0;
-    int stages = (int)((info.max_smem_optin - stream_layout(p, teams, 0, warps_per_team, aux)) /
-                       (3 * (size_t)p.row_bytes + 2 * sizeof(uint64_t)));
-    if (stages > ROPE3D_STREAM_MAX_STAGES) stages = ROPE3D_STREAM_MAX_STAGES;
-    while (stages >= 2 &&
-           stream_layout(p, teams, stages, warps_per_team, aux) > (size_t)info.max_smem_optin)
-        --stages;
-    if (stages < 2) return ROPE3D_OK;
-    const size_t smem = stream_layout(p, teams, stages, warps_per_team, aux);
-    const int cache_fmt = p.k_bscale != nullptr ? rope3d::kCacheNvfp4
-                          : p.k_scale != nullptr ? rope3d::kCacheFp8 : rope3d::kCacheSame;
-    KernelFn fn = pick_stream_kernel(mode, dtype, trig, pairing, cache_fmt, g.vpt);
-    if (fn == nullptr) return ROPE3D_OK;
-    const int threads = 32 + teams * g.tpr;
-    int per_sm = 0;
-    int rc = occupancy(dev, fn, threads, smem, info.max_smem_optin, &per_sm);
-    if (rc != ROPE3D_OK) return rc;
-    int64_t grid = info.sms;
-    if (grid > p.units) grid = p.units;
-    p.dim_vecs = g.dim_vecs;
-    p.tpr = g.tpr;
-    p.teams = teams;
-    p.stages = stages;
-    p.wait_limit_ns = g_wait_limit_ns.load();
-    p.tx_extra = g_tx_extra.load();
-    const cudaError_t e =
-        launch_pdl(reinterpret_cast<const void*>(fn), grid, threads, smem, stream, &p);
-    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
-    *launched = true;
-    return ok();
-}
-
 template <int MODE>
 int launch(rope3d::Params& p, int64_t N, int dtype, int trig, int pairing, int dev,
            const DeviceInfo& info, cudaStream_t stream) {
     const Geometry g = geometry(N, dtype, pairing);
-    if (g.tpr > rope3d::kMaxBlockThreads || g.vpt > 4)
+    const int max_threads = g.vpt > 4 ? rope3d::kMaxBlockThreads / 2 : rope3d::kMaxBlockThreads;
+    if (g.tpr > max_threads || g.vpt > ROPE3D_MAX_VPT)
         return fail(ROPE3D_EINVAL, "N=%lld heads is more than one row team can hold",
                     (long long)N);
-    int teams = (ROPE3D_REG_BLOCK_TARGET < rope3d::kMaxBlockThreads ? ROPE3D_REG_BLOCK_TARGET
-                                                                    : rope3d::kMaxBlockThreads) / g.tpr;
+    int teams = (ROPE3D_REG_BLOCK_TARGET < max_threads ? ROPE3D_REG_BLOCK_TARGET
+                                                       : max_threads) / g.tpr;
     if (teams < 1) teams = 1;
     if (teams > rope3d::kMaxTeamsPerBlock) teams = rope3d::kMaxTeamsPerBlock;
     if ((int64_t)teams > p.units) teams = (int)p.units;
@@ -1004,8 +895,7 @@ int rope3d_testing_gemm_cta_group(int group) {
 }
 
 int rope3d_testing_force_path(int path) {
-    if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA &&
-        path != ROPE3D_PATH_STREAM)
+    if (path != ROPE3D_PATH_AUTO && path != ROPE3D_PATH_REGISTERS && path != ROPE3D_PATH_TMA)
         return fail(ROPE3D_EINVAL, "path %d is not a ROPE3D_PATH_* value", path);
     g_force_path.store(path);
     return ok();
@@ -1104,15 +994,6 @@ int rope3d_qk_norm_rope_append_ex(const void* q, const void* k, const void* v, v
     set_small_idx(p);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     const int path = g_force_path.load();
-    if (path == ROPE3D_PATH_STREAM) {
-        bool launched = false;
-        rc = launch_fused_stream(p, rope3d::kModeFused, N, dtype, trig, opt.pairing, dev, info,
-                                 stream, &launched);
-        if (launched) g_last_path = ROPE3D_PATH_STREAM;
-        if (rc != ROPE3D_OK || launched) return rc;
-        return fail(ROPE3D_EINVAL, "the staged-row path does not take this call (N=%lld)",
-                    (long long)N);
-    }
     if (path != ROPE3D_PATH_REGISTERS) {
         bool launched = false;
         rc = launch_fused_tma(p, N, dtype, trig, opt.pairing, dev, info, stream,
@@ -1226,15 +1107,6 @@ int rope3d_qk_norm_rope_append_sp(const void* q, const void* k, const void* v,
         p.sp_dst[3 * r + 2] = dest->v_cache[r];
     }
     set_small_idx(p);
-    if (g_force_path.load() == ROPE3D_PATH_STREAM) {
-        bool launched = false;
-        rc = launch_fused_stream(p, rope3d::kModeFusedSP, N, dtype, trig, opt.pairing, dev,
-                                 info, static_cast<cudaStream_t>(cuda_stream), &launched);
-        if (launched) g_last_path = ROPE3D_PATH_STREAM;
-        if (rc != ROPE3D_OK || launched) return rc;
-        return fail(ROPE3D_EINVAL, "the staged-row path does not take this call (N=%lld)",
-                    (long long)N);
-    }
     rc = launch<rope3d::kModeFusedSP>(p, N, dtype, trig, opt.pairing, dev, info,
                                       static_cast<cudaStream_t>(cuda_stream));
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
@@ -1446,6 +1318,86 @@ int rope3d_qkv_norm_rope_append(const void* x, const void* w_qkv, const float* b
     rc = launch<rope3d::kModeFusedNoV>(p, N, ROPE3D_BF16, trig, opt.pairing, dev, info, stream);
     if (rc == ROPE3D_OK) g_last_path = ROPE3D_PATH_REGISTERS;
     return rc;
+}
+
+int rope3d_sp_output_all_to_all(const void* o, int64_t B, int64_t L, int64_t heads_per_rank,
+                                int D, int dtype, const rope3d_sp_out_dest* dest,
+                                void* cuda_stream) {
+    if (o == nullptr || dest == nullptr) return fail(ROPE3D_EINVAL, "o or dest is NULL");
+    if (D != rope3d::kHeadDim) return fail(ROPE3D_EINVAL, "head size D=%d, not %d", D,
+                                           rope3d::kHeadDim);
+    if (dtype != ROPE3D_F32 && dtype != ROPE3D_BF16)
+        return fail(ROPE3D_EINVAL, "dtype %d is neither ROPE3D_F32 nor ROPE3D_BF16", dtype);
+    if (B < 1 || L < 1 || heads_per_rank < 1)
+        return fail(ROPE3D_EINVAL, "B=%lld, L=%lld and heads_per_rank=%lld must be >= 1",
+                    (long long)B, (long long)L, (long long)heads_per_rank);
+    const int P = dest->ranks;
+    if (P < 1 || P > ROPE3D_SP_MAX_RANKS)
+        return fail(ROPE3D_EINVAL, "dest->ranks %d is not in [1, %d]", P, ROPE3D_SP_MAX_RANKS);
+    if (dest->rank < 0 || dest->rank >= P)
+        return fail(ROPE3D_EINVAL, "dest->rank %d is not in [0, %d)", dest->rank, P);
+    if (dest->cuts[0] != 0 || dest->cuts[P] != L)
+        return fail(ROPE3D_ERANGE, "cuts must run from 0 to L = %lld", (long long)L);
+    for (int r = 0; r < P; ++r)
+        if (dest->cuts[r + 1] < dest->cuts[r])
+            return fail(ROPE3D_ERANGE, "cuts must not fall (cuts[%d] > cuts[%d])", r, r + 1);
+    if (!aligned16(o)) return fail(ROPE3D_EALIGN, "o must be 16-byte aligned");
+    const size_t esz = dtype == ROPE3D_BF16 ? 2 : 4;
+    const size_t row = (size_t)heads_per_rank * D * esz;
+    const size_t o_bytes = (size_t)B * (size_t)L * row;
+    size_t out_bytes[ROPE3D_SP_MAX_RANKS];
+    for (int r = 0; r < P; ++r) {
+        out_bytes[r] = (size_t)B * (size_t)(dest->cuts[r + 1] - dest->cuts[r]) * row * P;
+        if (out_bytes[r] == 0) continue;
+        if (dest->out[r] == nullptr)
+            return fail(ROPE3D_EINVAL, "dest->out[%d] is NULL but its slice is not empty", r);
+        if (!aligned16(dest->out[r]))
+            return fail(ROPE3D_EALIGN, "dest->out[%d] must be 16-byte aligned", r);
+        if (overlap(dest->out[r], out_bytes[r], o, o_bytes))
+            return fail(ROPE3D_EOVERLAP, "dest->out[%d] overlaps o", r);
+        for (int r2 = 0; r2 < r; ++r2)
+            if (out_bytes[r2] && overlap(dest->out[r], out_bytes[r], dest->out[r2], out_bytes[r2]))
+                return fail(ROPE3D_EOVERLAP, "dest->out[%d] overlaps dest->out[%d]", r, r2);
+    }
+    DeviceInfo info;
+    int dev = 0;
+    int rc = device_info(&info, &dev);
+    if (rc != ROPE3D_OK) return rc;
+
+    rope3d::SpOutParams sp{};
+    sp.o = static_cast<const uint4*>(o);
+    for (int r = 0; r < P; ++r) sp.out[r] = static_cast<uint4*>(dest->out[r]);
+    for (int r = 0; r <= P; ++r) sp.cuts[r] = dest->cuts[r];
+    for (int r = P + 1; r <= rope3d::kMaxRanks; ++r) sp.cuts[r] = L;
+    sp.L = L;
+    sp.ranks = P;
+    sp.rank = dest->rank;
+    sp.row_vecs = (int)(row / 16);
+    sp.out_row_vecs = sp.row_vecs * P;
+    sp.total = B * L * sp.row_vecs;
+    sp.small = sp.total < ((int64_t)1 << 31) ? 1 : 0;
+    if (sp.small) {
+        sp.div_row = rope3d::make_fastdiv((uint32_t)sp.row_vecs);
+        sp.div_L = rope3d::make_fastdiv((uint32_t)L);
+    }
+    const int threads = 256;
+    int64_t grid = (sp.total + threads - 1) / threads;
+    const int64_t cap = (int64_t)info.sms * 8;
+    if (grid > cap) grid = cap;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(threads);
+    cfg.stream = static_cast<cudaStream_t>(cuda_stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&sp};
+    const cudaError_t e = cudaLaunchKernelExC(
+        &cfg, reinterpret_cast<const void*>(rope3d::sp_output_all_to_all_kernel), args);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
+    return ok();
 }
 
 int rope3d_apply(const void* x, void* out, int64_t B, int64_t N, int D, int dtype,

@@ -813,12 +813,7 @@ __device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
 // fp32 until they are quantized, and the K and V keys of one head travel in one shuffle
 // word.  Every lane of the warp takes part in the head-wise maximum, whether its slots
 // hold vectors or not.
-// Parts of a row's output: q (q_out), K (the K cache row, with V where V is quantized), or
-// both.  The register kernel emits q and K separately so that it can request the next
-// row's q while this row's K is still being written.
-enum EmitPart : int { kEmitQ = 1, kEmitK = 2, kEmitAll = 3 };
-
-template <typename T, int VPT, int PAIR, int MODE, int CF, int PART = kEmitAll>
+template <typename T, int VPT, int PAIR, int MODE, int CF>
 __device__ __forceinline__ void emit_row(
     const Params& p, int t, const RowPos& pos, int64_t row_vec,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -837,8 +832,7 @@ __device__ __forceinline__ void emit_row(
     if constexpr (PAIR == kPairAdjacent) {
         // q first, for every slot, then K (and V where it is quantized): one row rotation
         // (RowRot) is live at a time
-        if constexpr (!(PART & kEmitQ)) {
-        } else if constexpr (NORM) {
+        if constexpr (NORM) {
             const RowRot<Tr::kPairsPerVec> rot_q = row_rot(rq, cs, sn);
 #pragma unroll
             for (int s = 0; s < VPT; ++s) {
@@ -854,7 +848,7 @@ __device__ __forceinline__ void emit_row(
                     store_out(qo + row_vec + idx, rotate_only<T>(xq[s], cs, sn));
             }
         }
-        if constexpr (MODE == kModeFused && (PART & kEmitK)) {
+        if constexpr (MODE == kModeFused) {
             const RowRot<Tr::kPairsPerVec> rot_k = row_rot(rk, cs, sn);
 #pragma unroll
             for (int s = 0; s < VPT; ++s) {
@@ -919,13 +913,13 @@ __device__ __forceinline__ void emit_row(
             const int i_im = slot_vec<T, PAIR>(t, s + 1, p.tpr);
             const bool valid = i_re < p.dim_vecs && (!kDeviceChecks || pos.ok);
             float o_re[EPV], o_im[EPV];
-            if ((PART & kEmitQ) && valid) {
+            if (valid) {
                 norm_rotate_half_f<T, NORM>(xq[s], xq[s + 1], rq, s_wq, i_re * EPV, i_im * EPV,
                                             cs, sn, o_re, o_im);
                 store_out(qo + row_vec + i_re, Tr::pack_elems(o_re));
                 store_out(qo + row_vec + i_im, Tr::pack_elems(o_im));
             }
-            if constexpr (MODE == kModeFused && (PART & kEmitK)) {
+            if constexpr (MODE == kModeFused) {
                 if (valid)
                     norm_rotate_half_f<T, true>(xk[s], xk[s + 1], rk, s_wk, i_re * EPV,
                                                 i_im * EPV, cs, sn, o_re, o_im);
@@ -1046,7 +1040,7 @@ __device__ __forceinline__ void store_v_row_sp(const Params& p, int t, const Row
     }
 }
 
-template <typename T, int VPT, int PART = kEmitAll>
+template <typename T, int VPT>
 __device__ __forceinline__ void emit_row_sp(
     const Params& p, int t, const RowPos& pos,
     const typename VecTraits<T>::Vec (&xq)[VPT], const typename VecTraits<T>::Vec (&xk)[VPT],
@@ -1063,7 +1057,6 @@ __device__ __forceinline__ void emit_row_sp(
         ok = pos.ok && pos.i >= p.sp_q_row0 && pos.i - p.sp_q_row0 < p.sp_q_rows;
         if (pos.ok && !ok) record_index_error(p);
     }
-    if constexpr (PART & kEmitQ) {
     const RowRot<Tr::kPairsPerVec> rot_q = row_rot(rq, cs, sn);
 #pragma unroll
     for (int s = 0; s < VPT; ++s) {
@@ -1074,8 +1067,6 @@ __device__ __forceinline__ void emit_row_sp(
                       norm_rotate<T>(xq[s], s_wq, idx * Tr::kElems, rot_q));
         }
     }
-    }
-    if constexpr (PART & kEmitK) {
     const RowRot<Tr::kPairsPerVec> rot_k = row_rot(rk, cs, sn);
 #pragma unroll
     for (int s = 0; s < VPT; ++s) {
@@ -1085,7 +1076,6 @@ __device__ __forceinline__ void emit_row_sp(
             store_out(kd + sp_cache_index(p, pos, dst[s] & 0xFFFF),
                       norm_rotate<T>(xk[s], s_wk, idx * Tr::kElems, rot_k));
         }
-    }
     }
 }
 
@@ -1105,7 +1095,7 @@ __device__ __forceinline__ void load_vecs(const Params& p, int t, int64_t u,
 }
 
 template <typename T, int VPT, int TRIG, int MODE, int PAIR, int CF>
-__global__ void __launch_bounds__(kMaxBlockThreads)
+__global__ void __launch_bounds__(VPT > 4 ? kMaxBlockThreads / 2 : kMaxBlockThreads)
 qk_norm_rope_kernel(const Params p) {
     using Tr = VecTraits<T>;
     using Vec = typename Tr::Vec;
@@ -1114,9 +1104,6 @@ qk_norm_rope_kernel(const Params p) {
     constexpr bool SP = MODE == kModeFusedSP;
     constexpr bool HAS_V = FUSED && MODE != kModeFusedNoV;
     constexpr int EMIT_MODE = MODE == kModeFusedNoV ? kModeFused : MODE;
-    // V leaves the registers right after its row arrives (a bit copy) unless it is
-    // quantized beside K
-    constexpr bool V_EARLY = HAS_V && (SP || CF == kCacheSame);
     static_assert(HAS_V || !FUSED || CF == kCacheSame, "no-V step: same-dtype K cache");
     static_assert(!SP || (PAIR == kPairAdjacent && CF == kCacheSame),
                   "head-scatter stores: adjacent pairing, same-dtype caches");
@@ -1175,14 +1162,8 @@ qk_norm_rope_kernel(const Params p) {
         for (int s = 0; s < VPT; ++s) dst[s] = sp_code(p, slot_vec<T, PAIR>(t, s, p.tpr));
     }
 
-    // Rolling prefetch: each tensor's registers are refilled with the team's next row as
-    // soon as this row is done with them -- V right after its bit copy, q after q_out, K
-    // (and a quantized V) after the cache row -- so the next row's loads overlap this row's
-    // reduction and arithmetic without a second set of row registers.
     int parity = 0;
     for (int64_t u = u0; u < p.units; u += stride) {
-        const int64_t next = u + stride;
-        const bool more = next < p.units;
         const RowPos pos = decode_row(p, u);
         const int64_t row_vec = u * p.dim_vecs;
         float cs[NP], sn[NP];
@@ -1191,8 +1172,8 @@ qk_norm_rope_kernel(const Params p) {
         float rq = 1.0f, rk = 1.0f;
         if (FUSED) {
             if constexpr (SP) store_v_row_sp<T, VPT>(p, t, pos, xv, dst, s_sp);
-            else if constexpr (V_EARLY) store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
-            if (V_EARLY && more) load_vecs<T, VPT, PAIR>(p, t, next, vg, xv);
+            else if constexpr (CF == kCacheSame && HAS_V)
+                store_v_row<T, VPT, PAIR>(p, t, pos, xv, vc);
             float sq, sk;
             partial_sum_squares<T, VPT, PAIR>(xq, xk, t, p.tpr, p.dim_vecs, sq, sk);
             const float2 tot = team_sum(sq, sk, s_part, team, p.teams, warp_in_team,
@@ -1201,25 +1182,70 @@ qk_norm_rope_kernel(const Params p) {
             rk = rsqrtf(fmaf(tot.y, p.inv_dim, p.eps));
         }
         if constexpr (SP)
-            emit_row_sp<T, VPT, kEmitQ>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
+            emit_row_sp<T, VPT>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst, s_sp);
         else
-            emit_row<T, VPT, PAIR, EMIT_MODE, CF, kEmitQ>(p, t, pos, row_vec, xq, xk, xv, rq,
-                                                          rk, s_wq, s_wk, cs, sn, qo, kc, vc,
-                                                          s_r);
-        if (more) load_vecs<T, VPT, PAIR>(p, t, next, qg, xq);
-        if constexpr (FUSED) {
-            if constexpr (SP)
-                emit_row_sp<T, VPT, kEmitK>(p, t, pos, xq, xk, rq, rk, s_wq, s_wk, cs, sn, dst,
-                                            s_sp);
-            else
-                emit_row<T, VPT, PAIR, EMIT_MODE, CF, kEmitK>(p, t, pos, row_vec, xq, xk, xv,
-                                                              rq, rk, s_wq, s_wk, cs, sn, qo,
-                                                              kc, vc, s_r);
-            if (more) {
-                load_vecs<T, VPT, PAIR>(p, t, next, kg, xk);
-                if (HAS_V && !V_EARLY) load_vecs<T, VPT, PAIR>(p, t, next, vg, xv);
-            }
+            emit_row<T, VPT, PAIR, EMIT_MODE, CF>(p, t, pos, row_vec, xq, xk, xv, rq, rk,
+                                                  s_wq, s_wk, cs, sn, qo, kc, vc, s_r);
+        // The team's next row, requested after this row's stores: one row in registers at a
+        // time keeps the blocks per SM up.  Measured on B200: a second row prefetched into
+        // registers cost 20-40% (lost occupancy), and refilling each tensor's registers as
+        // soon as the row was done with them cost 8-15% (480P and 720P chunks).
+        if (u + stride < p.units) {
+            load_vecs<T, VPT, PAIR>(p, t, u + stride, qg, xq);
+            if (FUSED) load_vecs<T, VPT, PAIR>(p, t, u + stride, kg, xk);
+            if (HAS_V) load_vecs<T, VPT, PAIR>(p, t, u + stride, vg, xv);
         }
+    }
+}
+
+// ---------------------------------------------------------------- output all-to-all
+//
+// The exchange after attention (Algorithm 3, last step): this rank's o [B][L][hl][D] --
+// every token for its own heads -- goes out token by token to the rank whose slice holds
+// the token, at head offset rank * hl of that rank's [B][slice][N][D] buffer.  A bit copy
+// in 16-byte vectors, one vector per thread and step; the source and each destination
+// row segment are contiguous, so loads and stores are coalesced on both sides.
+
+struct SpOutParams {
+    const uint4* o;
+    uint4* out[kMaxRanks];
+    int64_t cuts[kMaxRanks + 1];
+    int64_t L;
+    int64_t total;        // B * L * row_vecs
+    int ranks;
+    int rank;
+    int row_vecs;         // vectors of one token of o (hl heads)
+    int out_row_vecs;     // vectors of one token of an output (all heads)
+    int small;            // total < 2^31: 32-bit index arithmetic
+    FastDiv div_row, div_L;
+};
+
+__global__ void sp_output_all_to_all_kernel(const SpOutParams p) {
+    pdl_launch_dependents();
+    pdl_wait_previous_grid();
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < p.total; v += step) {
+        int64_t row, b, i;
+        if (p.small) {
+            const uint32_t r32 = fast_div((uint32_t)v, p.div_row);
+            const uint32_t b32 = fast_div(r32, p.div_L);
+            row = r32;
+            b = b32;
+            i = r32 - b32 * (uint32_t)p.L;
+        } else {
+            row = v / p.row_vecs;
+            b = row / p.L;
+            i = row - b * p.L;
+        }
+        const int j = (int)(v - row * p.row_vecs);
+        int d = 0;
+#pragma unroll
+        for (int r = 0; r < kMaxRanks; ++r)
+            if (r < p.ranks && i >= p.cuts[r] && i < p.cuts[r + 1]) d = r;
+        const int64_t rows_d = p.cuts[d + 1] - p.cuts[d];
+        const int64_t dst = ((b * rows_d + (i - p.cuts[d])) * p.out_row_vecs) +
+                            (int64_t)p.rank * p.row_vecs + j;
+        __stcs(p.out[d] + dst, __ldcs(p.o + v));
     }
 }
 

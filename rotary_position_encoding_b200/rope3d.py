@@ -55,6 +55,13 @@ class rope3d_options(ctypes.Structure):
 ROPE3D_SP_MAX_RANKS = 8
 
 
+class rope3d_sp_out_dest(ctypes.Structure):
+    """struct rope3d_sp_out_dest of include/rope3d.h."""
+    _fields_ = [("ranks", ctypes.c_int), ("rank", ctypes.c_int),
+                ("cuts", ctypes.c_int64 * (ROPE3D_SP_MAX_RANKS + 1)),
+                ("out", ctypes.c_void_p * ROPE3D_SP_MAX_RANKS)]
+
+
 class rope3d_sp_dest(ctypes.Structure):
     """struct rope3d_sp_dest of include/rope3d.h."""
     _fields_ = [("ranks", ctypes.c_int), ("reserved0", ctypes.c_int),
@@ -67,7 +74,6 @@ class rope3d_sp_dest(ctypes.Structure):
 ROPE3D_PATH_AUTO = 0
 ROPE3D_PATH_REGISTERS = 1
 ROPE3D_PATH_TMA = 2
-ROPE3D_PATH_STREAM = 3
 
 _VP = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -89,6 +95,8 @@ SIGNATURES = {
                                        _INT, _INT, _INT, _VP, _VP, ctypes.c_float,
                                        ctypes.POINTER(rope3d_sp_dest), _I64, _I64, _VP, _INT,
                                        ctypes.POINTER(rope3d_options), _VP], _INT),
+    "rope3d_sp_output_all_to_all": ([_VP, _I64, _I64, _I64, _INT, _INT,
+                                     ctypes.POINTER(rope3d_sp_out_dest), _VP], _INT),
     "rope3d_qkv_project": ([_VP, _VP, _VP, _I64, _I64, _I64, _INT, _VP, _VP, _VP, _VP], _INT),
     "rope3d_qkv_workspace_bytes": ([_I64, _I64, _I64, _INT], ctypes.c_size_t),
     "rope3d_qkv_norm_rope_append": ([_VP, _VP, _VP, _I64, _I64, _I64, _INT, _I64, _I64, _I64,
@@ -390,6 +398,40 @@ def rope3d_qk_norm_rope_append_sp(q, k, v, token_begin: int, token_end: int,
         token_begin, token_end, frame_offset, T, H, W, _dev_ptr(q_norm_w, "q_norm_w"),
         _dev_ptr(k_norm_w, "k_norm_w"), eps, ctypes.byref(dest), cache_tokens, slot,
         tables.handle, trig, ctypes.byref(opts), _stream(stream)))
+
+
+def rope3d_sp_output_all_to_all(o, out, rank: int, cuts=None, stream=None) -> None:
+    """Algorithm 3's last step on this rank: o is [B, L, N/P, D] (every token, this rank's
+    heads); out lists, in rank order, each rank's output [B, cuts[r'+1] - cuts[r'], N, D]
+    -- tensors on this device, or integer device addresses of peer mappings.  cuts
+    defaults to the even split r L // P."""
+    if o.dim() != 4:
+        raise ValueError("o must be [B, L, N/P, D]")
+    B, L, hl, D = o.shape
+    P = len(out)
+    if not 1 <= P <= ROPE3D_SP_MAX_RANKS:
+        raise ValueError(f"1 to {ROPE3D_SP_MAX_RANKS} ranks")
+    if cuts is None:
+        cuts = [(r * L) // P for r in range(P + 1)]
+    if len(cuts) != P + 1:
+        raise ValueError("one slice per rank: len(cuts) == P + 1")
+    dest = rope3d_sp_out_dest()
+    dest.ranks = P
+    dest.rank = rank
+    for r in range(P + 1):
+        dest.cuts[r] = cuts[r]
+    for r in range(P):
+        t = out[r]
+        if isinstance(t, int):
+            dest.out[r] = t
+            continue
+        if t.dtype != o.dtype:
+            raise TypeError(f"out[{r}] must have o's dtype {o.dtype}")
+        if tuple(t.shape) != (B, cuts[r + 1] - cuts[r], P * hl, D):
+            raise ValueError(f"out[{r}] has shape {tuple(t.shape)}")
+        dest.out[r] = _dev_ptr(t, f"out[{r}]")
+    _check(load_library().rope3d_sp_output_all_to_all(
+        _dev_ptr(o, "o"), B, L, hl, D, _dtype_code(o), ctypes.byref(dest), _stream(stream)))
 
 
 def rope3d_qkv_project(x, w_qkv, b_qkv, q_out, k_out, v_out, stream=None) -> None:

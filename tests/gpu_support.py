@@ -118,5 +118,4 @@ def kernel_path(path: int):
         rope3d.rope3d_testing_force_path(rope3d.ROPE3D_PATH_AUTO)
 
 
-PATHS = {"tma": rope3d.ROPE3D_PATH_TMA, "registers": rope3d.ROPE3D_PATH_REGISTERS,
-         "staged": rope3d.ROPE3D_PATH_STREAM}
+PATHS = {"tma": rope3d.ROPE3D_PATH_TMA, "registers": rope3d.ROPE3D_PATH_REGISTERS}

@@ -162,6 +162,64 @@ def test_sp_dest_struct_layout_matches_header(tmp_path):
     assert got == [ctypes.sizeof(S)] + [getattr(S, f).offset for f in fields]
 
 
+def test_sp_out_dest_struct_layout_matches_header(tmp_path):
+    """The ctypes mirror of rope3d_sp_out_dest has the C struct's size and field offsets."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    fields = ("ranks", "rank", "cuts", "out")
+    src = tmp_path / "layout_spo.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "rope3d.h"\n'
+                   'int main(void){printf("%zu", sizeof(rope3d_sp_out_dest));'
+                   + "".join(f'printf(" %zu", offsetof(rope3d_sp_out_dest, {f}));'
+                             for f in fields)
+                   + ' return 0;}\n')
+    exe = tmp_path / "layout_spo"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    got = list(map(int, subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()))
+    S = rope3d.rope3d_sp_out_dest
+    assert got == [ctypes.sizeof(S)] + [getattr(S, f).offset for f in fields]
+
+
+def test_sp_output_all_to_all_rejects_bad_arguments_without_device(lib):
+    """Every host-side check of the output all-to-all fails before any CUDA call."""
+    o = 0x100000
+    dest = rope3d.rope3d_sp_out_dest()
+    dest.ranks, dest.rank = 2, 0
+    dest.cuts[0], dest.cuts[1], dest.cuts[2] = 0, 5, 10
+    dest.out[0], dest.out[1] = 0x200000, 0x300000
+
+    def call(o=o, B=1, L=10, hl=2, D=128, dtype=rope3d.ROPE3D_BF16, d=dest):
+        return lib.rope3d_sp_output_all_to_all(o, B, L, hl, D, dtype,
+                                               None if d is None else ctypes.byref(d), None)
+    assert call(o=0) == rope3d.ROPE3D_EINVAL
+    assert call(d=None) == rope3d.ROPE3D_EINVAL
+    assert call(D=64) == rope3d.ROPE3D_EINVAL
+    assert call(dtype=7) == rope3d.ROPE3D_EINVAL
+    assert call(L=11) == rope3d.ROPE3D_ERANGE  # cuts end at 10
+    assert call(o=o + 8) == rope3d.ROPE3D_EALIGN
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.rank = 2
+    assert call(d=bad) == rope3d.ROPE3D_EINVAL
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.ranks = 9
+    assert call(d=bad) == rope3d.ROPE3D_EINVAL
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.cuts[1] = 11
+    assert call(d=bad) == rope3d.ROPE3D_ERANGE  # cuts fall
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.out[1] = 0
+    assert call(d=bad) == rope3d.ROPE3D_EINVAL
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.out[1] = 0x200000 + 16
+    assert call(d=bad) == rope3d.ROPE3D_EOVERLAP  # outputs overlap each other
+    bad = rope3d.rope3d_sp_out_dest.from_buffer_copy(dest)
+    bad.out[0] = o + 16
+    assert call(d=bad) == rope3d.ROPE3D_EOVERLAP  # an output overlaps o
+
+
 def test_sp_step_rejects_null_arguments_without_device(lib):
     """NULL tables or a NULL destination table fail on the host (the destination checks that
     need real tables run in the gpu-marked tests)."""

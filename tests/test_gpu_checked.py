@@ -91,8 +91,7 @@ def _bits(t):
     return t.contiguous().view(torch.uint8).cpu().numpy()
 
 
-@pytest.mark.parametrize("path", [rope3d.ROPE3D_PATH_REGISTERS, rope3d.ROPE3D_PATH_TMA,
-                                  rope3d.ROPE3D_PATH_STREAM])
+@pytest.mark.parametrize("path", [rope3d.ROPE3D_PATH_REGISTERS, rope3d.ROPE3D_PATH_TMA])
 @pytest.mark.parametrize("trig", [rope3d.ROPE3D_TRIG_TABLE, rope3d.ROPE3D_TRIG_ONTHEFLY])
 def test_checked_build_reports_ok_and_matches_plain_build(path, trig):
     w = wl.chunk_480p()
@@ -123,8 +122,7 @@ def test_checked_build_fp8_cache_and_sp_scatter():
             assert np.array_equal(_bits(a), _bits(b)), kw
 
 
-@pytest.mark.parametrize("path", [rope3d.ROPE3D_PATH_REGISTERS, rope3d.ROPE3D_PATH_TMA,
-                                  rope3d.ROPE3D_PATH_STREAM])
+@pytest.mark.parametrize("path", [rope3d.ROPE3D_PATH_REGISTERS, rope3d.ROPE3D_PATH_TMA])
 def test_checked_build_withholds_rows_beyond_the_check_bound(path):
     """With the row check told to accept cache rows below C - 100 only, the launch writing
     the cache's last rows skips exactly those token rows (q_out, K and V untouched) and

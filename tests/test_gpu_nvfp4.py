@@ -105,8 +105,7 @@ def _written(layout, rows):
 @pytest.mark.parametrize("layout", [TOKEN, HEAD])
 @pytest.mark.parametrize("pairing", [ADJ, HALF])
 @pytest.mark.parametrize("kg,vg", [(0.0, 0.0), (0.4, 3.0)])
-@pytest.mark.parametrize("path", ["registers", "staged"])
-def test_nvfp4_cache_480p_chunk(layout, pairing, kg, vg, path):
+def test_nvfp4_cache_480p_chunk(layout, pairing, kg, vg):
     w = wl.chunk_480p()
     chunk = w.chunks[3]
     raw = wl.chunk_inputs(w, 3)
@@ -114,11 +113,10 @@ def test_nvfp4_cache_480p_chunk(layout, pairing, kg, vg, path):
     wq_np, wk_np = wl.norm_weights(w.seed, w.dim)
     tables = rope3d.rope3d_tables_init(max_t=21, max_h=w.H, max_w=w.W)
     caches, scales = _alloc(w, layout)
-    with kernel_path(PATHS[path]):
-        qo = _run_gpu(w, dev_in, chunk, tables, torch.from_numpy(wq_np).cuda(),
-                      torch.from_numpy(wk_np).cuda(), caches, scales, pairing, layout, kg, vg)
+    qo = _run_gpu(w, dev_in, chunk, tables, torch.from_numpy(wq_np).cuda(),
+                  torch.from_numpy(wk_np).cuda(), caches, scales, pairing, layout, kg, vg)
     torch.cuda.synchronize()
-    assert rope3d.rope3d_testing_last_path() == PATHS[path]
+    assert rope3d.rope3d_testing_last_path() == rope3d.ROPE3D_PATH_REGISTERS
     heads = tuple(caches[0].shape[:3])
     q_ref, ref_codes, ref_sc, ref_k = _oracle(w, raw, chunk, wq_np, wk_np, pairing, layout,
                                               heads, kg, vg)

@@ -18,7 +18,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_support import PATHS, assert_close, kernel_path, to_bits, to_device, to_f64, torch_dtype
+from gpu_support import assert_close, to_bits, to_device, to_f64, torch_dtype
 from rotary_position_encoding_b200 import rope3d, workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -116,14 +116,12 @@ def _cuts(L, P, uneven):
                                        ("bf16", 12, 3), ("bf16", 40, 8), ("bf16", 8, 8)])
 @pytest.mark.parametrize("layout", [TOKEN, HEAD])
 @pytest.mark.parametrize("uneven", [False, True])
-@pytest.mark.parametrize("path", ["registers", "staged"])
-def test_small_every_element(dtype, N, P, layout, uneven, path):
+def test_small_every_element(dtype, N, P, layout, uneven):
     st = Setup(dtype, B=2, N=N, T=2, H=3, W=5, s=4, C=64, slot=50, P=P, layout=layout,
                seed=500 + N + P, extra_rows=3)
     cuts = _cuts(st.L, P, uneven)
-    with kernel_path(PATHS[path]):
-        for a, e in zip(cuts[:-1], cuts[1:]):
-            st.run_rank(a, e)
+    for a, e in zip(cuts[:-1], cuts[1:]):
+        st.run_rank(a, e)
     torch.cuda.synchronize()
     q_ref, k_ref, v_ref = st.oracle_dst(cuts)
     for r in range(P):
@@ -135,17 +133,14 @@ def test_small_every_element(dtype, N, P, layout, uneven, path):
 
 @pytest.mark.parametrize("P", [2, 3, 4, 6])
 @pytest.mark.parametrize("trig", [rope3d.ROPE3D_TRIG_TABLE, rope3d.ROPE3D_TRIG_ONTHEFLY])
-@pytest.mark.parametrize("path", ["registers", "staged"])
-def test_480p_chunk_matches_plain_step_and_oracle(P, trig, path):
+def test_480p_chunk_matches_plain_step_and_oracle(P, trig):
     w = wl.chunk_480p()
     st = Setup("bf16", B=1, N=w.N, T=w.T, H=w.H, W=w.W, s=12, C=w.cache_tokens,
                slot=12 * 1560, P=P, layout=TOKEN, seed=600 + P, trig=trig)
     cuts = _cuts(st.L, P, uneven=False)  # the pages' even split L / P
-    with kernel_path(PATHS[path]):
-        for a, e in zip(cuts[:-1], cuts[1:]):
-            st.run_rank(a, e)
+    for a, e in zip(cuts[:-1], cuts[1:]):
+        st.run_rank(a, e)
     torch.cuda.synchronize()
-    assert rope3d.rope3d_testing_last_path() == PATHS[path]
     st.check_against_plain(0, st.L)
     if P == 4:
         q_ref, k_ref, v_ref = st.oracle_dst(cuts)
@@ -158,16 +153,14 @@ def test_480p_chunk_matches_plain_step_and_oracle(P, trig, path):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("layout", [TOKEN, HEAD])
-@pytest.mark.parametrize("path", ["registers", "staged"])
-def test_720p_chunk_eight_ranks(layout, path):
+def test_720p_chunk_eight_ranks(layout):
     """40 heads over 8 ranks (5 heads each), the pages' even split of 10800 tokens."""
     w = wl.chunk_720p()
     st = Setup("bf16", B=1, N=w.N, T=w.T, H=w.H, W=w.W, s=18, C=w.cache_tokens,
                slot=18 * 3600, P=8, layout=layout, seed=700)
     cuts = _cuts(st.L, 8, uneven=False)
-    with kernel_path(PATHS[path]):
-        for a, e in zip(cuts[:-1], cuts[1:]):
-            st.run_rank(a, e)
+    for a, e in zip(cuts[:-1], cuts[1:]):
+        st.run_rank(a, e)
     torch.cuda.synchronize()
     st.check_against_plain(0, st.L)
     orc = oracle.default()

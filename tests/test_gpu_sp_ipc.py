@@ -12,7 +12,10 @@ sequence with a destination table that mixes its own buffers and the other proce
 mapped ones.  The kernels never wait on each other; the processes meet only on the host
 (a barrier) after both have synchronised.  Then each process checks its own buffers
 against the plain step on the whole sequence split by heads: bit-identical, so every
-store through the mapped addresses landed where it belongs and nothing else moved."""
+store through the mapped addresses landed where it belongs and nothing else moved.  Then
+the output all-to-all (Algorithm 3, last step) runs the other way across the processes:
+each sends its gathered q rows back as the other's token slice with every head, and each
+checks that it got exactly the plain step's rows of its own slice."""
 import os
 import sys
 
@@ -79,7 +82,28 @@ def _worker(rank, shared, barrier, results):
         ok = all(torch.equal(x.view(torch.int16), y.contiguous().view(torch.int16))
                  for x, y in ((mine[0], qo[:, :, heads]), (mine[1], kc[:, :, heads]),
                               (mine[2], vc[:, :, heads])))
-        results.put((rank, ok, "" if ok else "destination buffers differ from the plain step"))
+        # Algorithm 3's last step across the processes: each one sends its gathered q rows
+        # (every token, its heads) back as the other's token slice with all heads
+        cuts = wl.slices(L, P)
+        cuts = [c[0] for c in cuts] + [L]
+        back = torch.full((1, cuts[rank + 1] - cuts[rank], N, D), 9.0, dtype=torch.bfloat16,
+                          device="cuda")
+        torch.cuda.synchronize()            # the fill lands before the other process writes
+        shared[rank].put(back)
+        their_back = shared[1 - rank].get(timeout=60)
+        outs = [None, None]
+        outs[rank], outs[1 - rank] = back, their_back
+        barrier.wait(timeout=60)            # both outputs are mapped before either writes
+        rope3d.rope3d_sp_output_all_to_all(mine[0], outs, rank, cuts)
+        torch.cuda.synchronize()
+        barrier.wait(timeout=60)            # both processes' stores are done
+        ok2 = torch.equal(back.view(torch.int16),
+                          qo[:, cuts[rank]:cuts[rank + 1]].contiguous().view(torch.int16))
+        msg = ("" if ok and ok2 else
+               "destination buffers differ from the plain step" if not ok else
+               "the output all-to-all did not return this rank's slice")
+        results.put((rank, ok and ok2, msg))
+        del their_back, outs
         del theirs, dst
         torch.cuda.synchronize()
         barrier.wait(timeout=60)            # the mapping is released before either exits

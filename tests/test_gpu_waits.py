@@ -1,9 +1,8 @@
-"""Bounded waits of the two kernels that stage rows in shared memory (the bulk-copy ring
-and the staged-row kernel).  A test setting makes every stage wait for 16 bytes more than
-its copies deliver, so no stage ever fills: the kernel must give up after the (shortened)
-limit, report ROPE3D_ETIMEOUT through the tables' status word, leave the GPU usable, and
-the next normal launch must be correct.  No fault is caused: every copy lands; only the
-wait runs out."""
+"""Bounded waits of the bulk-copy ring kernel.  A test setting makes every stage wait for
+16 bytes more than its copies deliver, so no stage ever fills: the kernel must give up
+after the (shortened) limit, report ROPE3D_ETIMEOUT through the tables' status word,
+leave the GPU usable, and the next normal launch must be correct.  No fault is caused:
+every copy lands; only the wait runs out."""
 import numpy as np
 import pytest
 import torch
@@ -15,7 +14,7 @@ from rotary_position_encoding_b200 import rope3d, workloads as wl
 pytestmark = pytest.mark.gpu
 
 
-PATHS = [rope3d.ROPE3D_PATH_TMA, rope3d.ROPE3D_PATH_STREAM]
+PATHS = [rope3d.ROPE3D_PATH_TMA]
 
 
 @pytest.mark.parametrize("path", PATHS)
