@@ -448,6 +448,14 @@ def run_ours(args, dist: Dist):
         configs = run_configs(torch, rope3d, device, stream, clocks, measured_peaks()[0],
                               (w, inputs, q_out, wq_d, wk_d, tables))
     clock_info = clocks.stop() if clocks else None
+    if configs is not None:
+        # each workload's clock record, from the samples inside its own timed replays
+        for entry in [e for e in configs.values()] + [e["whole"] for e in configs.values()
+                                                       if "whole" in e]:
+            w_ = entry.get("clocks")
+            if isinstance(w_, dict) and "window" in w_:
+                entry["clocks"] = (clocks.window(*w_["window"], name=w_["name"]) if clocks
+                                   else None)
 
     elapsed_ms = dist.max(elapsed_ms, device)
     avg_launch_ms = dist.max(statistics.fmean(launch_ms), device)
@@ -605,7 +613,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
              "kernel": {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
                         rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
                  rope3d.rope3d_testing_last_path(), "unknown"),
-             "clocks": clocks.window(*window, name=name) if clocks else None}
+             "clocks": {"window": window, "name": name}}
         d.update(extra)
         out[name] = d
 
@@ -617,8 +625,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                 q, k, v = ins[j % len(ins)]
                 rope3d.rope3d_qk_norm_rope_append(
                     q, k, v, q_out[j % len(q_out)], c.token_begin, c.token_end, c.frame_offset,
-                    w.T, w.H, w.W, ins_w[0], ins_w[1], w.eps, kc, vc, c.slot, tables, trig,
-                    stream=stream)
+                    w.T, w.H, w.W, ins_w[0], ins_w[1], w.eps, kc, vc, c.slot, tables, trig)
         return step
 
     # 480P chunk loop: 7 calls of 4680 tokens x 12 heads
@@ -650,14 +657,14 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
 
     def whole():
         rope3d.rope3d_qk_norm_rope_append(q, k, v, qo_whole, 0, n, 0, w.T, w.H, w.W, ins_w[0],
-                                          ins_w[1], w.eps, kw_, vw_, 0, tables, stream=stream)
+                                          ins_w[1], w.eps, kw_, vw_, 0, tables)
     parts = wl.slices(n, 8)
 
     def sliced():
         for a, b in parts:
             rope3d.rope3d_qk_norm_rope_append(
                 q[:, a:b], k[:, a:b], v[:, a:b], qo_sl[:, a:b], a, b, 0, w.T, w.H, w.W,
-                ins_w[0], ins_w[1], w.eps, ks_, vs_, 0, tables, stream=stream)
+                ins_w[0], ins_w[1], w.eps, ks_, vs_, 0, tables)
     us_w, win_w = graph_launch_us(torch, whole, 1, stream)
     kern_w = rope3d.rope3d_testing_last_path()
     us_s, win_s = graph_launch_us(torch, sliced, len(parts), stream)
@@ -672,7 +679,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                  "kernel": {rope3d.ROPE3D_PATH_TMA: "rope3d::qk_norm_rope_tma_kernel",
                             rope3d.ROPE3D_PATH_REGISTERS: "rope3d::qk_norm_rope_kernel"}.get(
                      kern_w, "unknown"),
-                 "clocks": clocks.window(*win_w, name="whole") if clocks else None},
+                 "clocks": {"window": win_w, "name": "whole"}},
           note="slices: 8 calls of 4095 tokens cutting through frames and rows; each call is "
                "a separate launch (one graph of 8 launches)")
     del q, k, v, qo_whole, qo_sl, kw_, vw_, ks_, vs_
@@ -722,7 +729,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                 rope3d.rope3d_qk_norm_rope_append_ex(
                     q, k, v, q_out[j], c.token_begin, c.token_end, c.frame_offset, w.T, w.H,
                     w.W, wq_d, wk_d, w.eps, kc, vc, c.slot, tables, k_scale=ks_, v_scale=vs_,
-                    k_global=0.5 if fp4 else 0.0, v_global=0.25 if fp4 else 0.0, stream=stream)
+                    k_global=0.5 if fp4 else 0.0, v_global=0.25 if fp4 else 0.0)
         us, win = graph_launch_us(torch, qstep, len(w.chunks), stream)
         entry(f"{w.name}/{fmt}_cache", us, nbytes, win, launches_per_step=len(w.chunks),
               note="q, k, v read and q_out written in bf16; K and V cache rows as "
@@ -750,7 +757,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                 a = c.token_begin + r * sl
                 rope3d.rope3d_qk_norm_rope_append_sp(
                     q, k, v, a, a + sl, c.frame_offset, w.T, w.H, w.W, wq_d, wk_d, w.eps, sp_q,
-                    sp_k, sp_v, c.slot, tables, q_row0=c.token_begin, stream=stream)
+                    sp_k, sp_v, c.slot, tables, q_row0=c.token_begin)
     us, win = graph_launch_us(torch, sp_step, P * len(w.chunks), stream)
     entry(f"{w.name}/sp8", us, w.algorithmic_bytes(sl), win, launches_per_step=P * len(w.chunks),
           note="8 ranks emulated as 8 launches per chunk over 1350-token slices; every head "
@@ -769,7 +776,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
 
     def proj():
         for j in range(3):
-            rope3d.rope3d_qkv_project(xs[j], wt, bt, *outs, stream=stream)
+            rope3d.rope3d_qkv_project(xs[j], wt, bt, *outs)
     us, win = graph_launch_us(torch, proj, 3, stream)
     y = torch.empty((w.B * n, 3 * w.dim), dtype=torch.bfloat16, device=device)
 
@@ -787,7 +794,7 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
         "frac": round(tf / burst, 4), "kernel": "rope3d::qkv_proj_kernel<2>",
         "cublas_same_gemm_us": round(us_cb, 2),
         "cublas_tflops": round(flops / (us_cb * 1e-6) / 1e12, 1),
-        "clocks": clocks.window(*win, name="projection") if clocks else None,
+        "clocks": {"window": win, "name": "projection"},
         "note": "x [10800, 5120] bf16 times W^T, W [15360, 5120] bf16, fp32 accumulate, bf16 "
                 "out; 3 input sets, graph replay"}
     del xs, wt, outs, y
