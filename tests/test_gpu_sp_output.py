@@ -31,9 +31,12 @@ def _run(dtype, B, L, N, P, cuts, seed):
     for r in range(P):  # rank r's launch: its heads of every token
         rope3d.rope3d_sp_output_all_to_all(o[r], out, r, cuts)
     torch.cuda.synchronize()
-    ref = oracle.Oracle.sp_output_all_to_all(raw, cuts)
+    ref = oracle.Oracle.sp_output_all_to_all(raw, cuts)  # float32 values or bf16 bits
     for r in range(P):
-        assert np.array_equal(to_bits(out[r]), ref[r]), f"rank {r}"
+        want = np.ascontiguousarray(ref[r])
+        if dtype == "f32":
+            want = want.view(np.uint32)
+        assert np.array_equal(to_bits(out[r]), want), f"rank {r}"
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
