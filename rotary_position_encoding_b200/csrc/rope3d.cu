@@ -1126,6 +1126,12 @@ int check_projection(const void* x, const void* w_qkv, const float* b_qkv, int64
                     (long long)K, rope3d::kGemmBK);
     if (M > (1 << 30) || 3 * N * D > (1 << 24))
         return fail(ROPE3D_ERANGE, "M=%lld or N=%lld is too large", (long long)M, (long long)N);
+    // the kernels count output tiles (128 x 256 at the smallest) in an int
+    const int64_t tiles = ((M + rope3d::kGemmBM - 1) / rope3d::kGemmBM) *
+                          ((3 * N * D + rope3d::kGemmBN - 1) / rope3d::kGemmBN);
+    if (tiles >= ((int64_t)1 << 31))
+        return fail(ROPE3D_ERANGE, "M=%lld x 3 N D=%lld is %lld output tiles, over 2^31 - 1",
+                    (long long)M, (long long)(3 * N * D), (long long)tiles);
     if (!aligned16(x) || !aligned16(w_qkv) ||
         (b_qkv != nullptr && (reinterpret_cast<uintptr_t>(b_qkv) & 3u)))
         return fail(ROPE3D_EALIGN, "x and w_qkv must be 16-byte aligned, b_qkv 4-byte");

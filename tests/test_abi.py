@@ -282,3 +282,12 @@ def test_fast_divide_matches_integer_division(lib):
                 assert lib.rope3d_testing_fast_divide(n, d) == n // d, (n, d)
     assert lib.rope3d_testing_fast_divide(5, 0) == 0xFFFFFFFF
     assert lib.rope3d_testing_fast_divide(1 << 31, 3) == 0xFFFFFFFF
+
+
+def test_projection_rejects_a_tile_count_over_int_range(lib):
+    """M = 2^30 token rows against 3 N D = 3 * 43690 * 128 output columns passes the per-size
+    limits but is 2^23 x 65535 output tiles: ERANGE before any device work."""
+    p = 0x100000
+    rc = lib.rope3d_qkv_project(p, p, None, 1 << 30, 64, 43690, 128, p, p, p, None)
+    assert rc == rope3d.ROPE3D_ERANGE
+    assert "tiles" in lib.rope3d_last_error().decode()
