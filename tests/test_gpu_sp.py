@@ -274,7 +274,13 @@ def test_symmetric_memory_wiring_one_rank():
         torch.cuda.synchronize()
         st.q_dst, st.k_dst, st.v_dst = [wiring.q], [wiring.k_cache], [wiring.v_cache]
         st.check_against_plain(0, st.L)
-        del wiring, st
+        # the exchange back after attention (identity on one rank): the gathered q rows
+        # land in the output region as [B, L, N, 128]
+        back = wiring.output_all_to_all(wiring.q)
+        wiring.barrier()
+        torch.cuda.synchronize()
+        assert torch.equal(back.view(torch.int16), wiring.q.view(torch.int16))
+        del wiring, st, back
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()

@@ -184,16 +184,19 @@ def _sp_table_rank(rank, world, port, out_path):
             st = sp.SequenceParallelStep(dist.group.WORLD, rank, world, B=2, N=6, q_rows=77,
                                          cache_tokens=131, dtype=torch.bfloat16, device="cpu",
                                          cache_layout=layout, exchange=exchange)
-            own = (st.q.data_ptr(), st.k_cache.data_ptr(), st.v_cache.data_ptr())
+            own = (st.q.data_ptr(), st.k_cache.data_ptr(), st.v_cache.data_ptr(),
+                   st.out(st.layout.out_rows).data_ptr())
             everyone = [None] * world
             dist.all_gather_object(everyone, own)
-            ok &= [list(x) for x in zip(st.q_dst, st.k_dst, st.v_dst)] == [list(e) for e in everyone]
+            ok &= ([list(x) for x in zip(st.q_dst, st.k_dst, st.v_dst, st.out_dst)]
+                   == [list(e) for e in everyone])
             cshape = (2, 131, 3, 128) if layout == rope3d.ROPE3D_CACHE_TOKEN_MAJOR else (2, 3, 131, 128)
             ok &= tuple(st.q.shape) == (2, 77, 3, 128) and tuple(st.k_cache.shape) == cshape
             lay = st.layout  # regions start on 256-byte boundaries of the allocation
-            ok &= all(off % 256 == 0 for off in (lay.q_off, lay.k_off, lay.v_off, lay.nbytes))
+            ok &= all(off % 256 == 0 for off in (lay.q_off, lay.k_off, lay.v_off, lay.out_off,
+                                                 lay.nbytes))
             ends = sorted((t.data_ptr(), t.data_ptr() + t.numel() * 2)
-                          for t in (st.q, st.k_cache, st.v_cache))
+                          for t in (st.q, st.k_cache, st.v_cache, st.out(st.layout.out_rows)))
             ok &= all(a[1] <= b[0] for a, b in zip(ends, ends[1:]))
             ok &= ends[-1][1] <= st.buffer.data_ptr() + st.buffer.numel()
             st.barrier()
@@ -268,8 +271,12 @@ def test_sp_plan_layout():
     q_bytes = 2 * 10800 * 5 * 128 * 2
     c_bytes = 2 * 75600 * 5 * 128 * 2
     assert lay.q_off == 0 and lay.k_off >= q_bytes and lay.v_off >= lay.k_off + c_bytes
-    assert lay.nbytes >= lay.v_off + c_bytes
-    assert all(x % 256 == 0 for x in (lay.k_off, lay.v_off, lay.nbytes))
+    o_bytes = 2 * 1350 * 40 * 128 * 2  # the largest of 8 even slices of 10800 tokens
+    assert lay.out_rows == 1350 and lay.out_off >= lay.v_off + c_bytes
+    assert lay.nbytes >= lay.out_off + o_bytes
+    assert all(x % 256 == 0 for x in (lay.k_off, lay.v_off, lay.out_off, lay.nbytes))
+    assert sp.even_cuts(10, 4) == [0, 2, 5, 7, 10]
+    assert sp.plan(1, 12, 4, 10, 64, torch.bfloat16).out_rows == 3
     head = sp.plan(1, 12, 4, 100, 64, torch.bfloat16, rope3d.ROPE3D_CACHE_HEAD_MAJOR)
     assert head.cache_shape == (1, 3, 64, 128)
     with pytest.raises(ValueError):
