@@ -764,6 +764,26 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                "stored to its owner's buffers (5 heads each, all on this GPU)")
     del sp_q, sp_k, sp_v, sp_in
 
+    # the exchange back after attention for the same 8 ranks: each rank's o [1, 10800, 5,
+    # 128] (every token, its heads) goes to the 8 ranks' [1, 1350, 40, 128] slices; three
+    # chunks' worth of buffers (331 MB of o) so that every launch reads HBM
+    o_sets = [[randn_bf16((w.B, n, hl, wl.HEAD_DIM), 500 + 8 * c + r) for r in range(P)]
+              for c in range(3)]
+    o_out = [[torch.empty((w.B, sl, w.N, wl.HEAD_DIM), dtype=torch.bfloat16, device=device)
+              for _ in range(P)] for _ in range(3)]
+
+    def out_step():
+        for c in range(3):
+            for r in range(P):
+                rope3d.rope3d_sp_output_all_to_all(o_sets[c][r], o_out[c], r)
+    us, win = graph_launch_us(torch, out_step, 3 * P, stream)
+    out_bytes = 2 * w.B * n * hl * wl.HEAD_DIM * 2  # read o, write it out
+    entry(f"{w.name}/sp8_output_all_to_all", us, out_bytes, win, launches_per_step=3 * P,
+          kernel="rope3d::sp_output_all_to_all_kernel",
+          note="Algorithm 3's last step for 8 emulated ranks: each launch moves one rank's "
+               "13.8 MB of o (every token, 5 heads) to the 8 ranks' token slices")
+    del o_sets, o_out
+
     # the QKV projection on the tensor cores (timed alone: the burst peak applies)
     K = w.dim
     xs = [randn_bf16((w.B * n, K), 400 + j) for j in range(3)]
