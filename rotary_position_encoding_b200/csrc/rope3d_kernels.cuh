@@ -795,15 +795,43 @@ __device__ __forceinline__ void stage_weights(const Params& p, float* s_wq, floa
 
 // ---------------------------------------------------------------- per-row output
 
+// The two bf16 halves of u (low half first) times a power of two s (given as its bf16
+// bits), as fp32: one mixed-precision FMA per element widens and scales at once.  The
+// product of a bf16 value and a power of two is exact in fp32 (the -0 addend keeps the
+// sign of a zero product), so this equals widening and then multiplying in fp32.
+__device__ __forceinline__ float2 bf16x2_times_pow2(uint32_t u, unsigned short s) {
+    float2 r;
+    asm("{\n"
+        "  .reg .b16 lo, hi;\n"
+        "  mov.b32 {lo, hi}, %2;\n"
+        "  fma.rn.f32.bf16 %0, lo, %3, 0f80000000;\n"
+        "  fma.rn.f32.bf16 %1, hi, %3, 0f80000000;\n"
+        "}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(u), "h"(s));
+    return r;
+}
+
 // Quantize one vector of V (its input elements) to the FP8 cache.
 template <typename T>
 __device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
                                             const typename VecTraits<T>::Vec& x, float inv) {
     using Tr = VecTraits<T>;
-    float v[Tr::kElems];
+    if constexpr (Tr::kElems == 8) {
+        // bf16: inv is a power of two, so its bf16 bits are the top half of its fp32 bits
+        const unsigned short s = (unsigned short)(__float_as_uint(inv) >> 16);
+        const float2 a = bf16x2_times_pow2(x.x, s), b = bf16x2_times_pow2(x.y, s);
+        const float2 c = bf16x2_times_pow2(x.z, s), d = bf16x2_times_pow2(x.w, s);
+        uint2 w;
+        w.x = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
+        w.y = e4m3x2(c.x, c.y) | (e4m3x2(d.x, d.y) << 16);
+        __stcs(reinterpret_cast<uint2*>(vc) + vi, w);
+    } else {
+        float v[Tr::kElems];
 #pragma unroll
-    for (int e = 0; e < Tr::kElems; ++e) v[e] = Tr::elem(x, e);
-    store_fp8(vc, vi, v, inv);
+        for (int e = 0; e < Tr::kElems; ++e) v[e] = Tr::elem(x, e);
+        store_fp8(vc, vi, v, inv);
+    }
 }
 
 // Normalise, rotate and store this thread's vectors of one row: q_out, and in the fused
