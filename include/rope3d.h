@@ -283,7 +283,8 @@ ROPE3D_API int rope3d_qk_norm_rope_append_sp(
  *   [r hl, (r+1) hl) of that row.
  * Run on every rank with the same cuts and out tables (each listing the ranks' buffers in
  * rank order), the ranks together leave in rank r' its token slice with every head.  A
- * bit copy of 16-byte vectors: o and every out[r'] must be 16-byte aligned.  Destinations
+ * bit copy: o and every out[r'] must be 16-byte aligned; when all of them are 32-byte
+ * aligned the copy moves 32-byte units, otherwise 16-byte ones.  Destinations
  * are device addresses valid on the calling device (this device's memory, or another
  * GPU's memory mapped into this process); stores to another GPU are plain peer stores over
  * NVLink.  The call does not synchronise with the other ranks (as for the head scatter).

@@ -38,6 +38,14 @@
 #ifndef ROPE3D_TMA_BLOCK_TARGET
 #define ROPE3D_TMA_BLOCK_TARGET 320
 #endif
+// Output all-to-all: units per thread per step, and whether 32-byte units are used when
+// the pointers allow them.
+#ifndef ROPE3D_A2A_UNROLL
+#define ROPE3D_A2A_UNROLL 2
+#endif
+#ifndef ROPE3D_A2A_WIDE
+#define ROPE3D_A2A_WIDE 1
+#endif
 
 struct rope3d_tables {
     int device;
@@ -116,6 +124,7 @@ int device_info(DeviceInfo* out, int* device) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -1370,24 +1379,30 @@ int rope3d_sp_output_all_to_all(const void* o, int64_t B, int64_t L, int64_t hea
     int rc = device_info(&info, &dev);
     if (rc != ROPE3D_OK) return rc;
 
+    // 32-byte units when o, every destination and the row length allow them
+    bool wide = ROPE3D_A2A_WIDE && row % 32 == 0 && aligned32(o);
+    for (int r = 0; r < P; ++r)
+        if (out_bytes[r] && !aligned32(dest->out[r])) wide = false;
+    const int unit = wide ? 32 : 16;
     rope3d::SpOutParams sp{};
-    sp.o = static_cast<const uint4*>(o);
-    for (int r = 0; r < P; ++r) sp.out[r] = static_cast<uint4*>(dest->out[r]);
+    sp.o = static_cast<const unsigned char*>(o);
+    for (int r = 0; r < P; ++r) sp.out[r] = static_cast<unsigned char*>(dest->out[r]);
     for (int r = 0; r <= P; ++r) sp.cuts[r] = dest->cuts[r];
     for (int r = P + 1; r <= rope3d::kMaxRanks; ++r) sp.cuts[r] = L;
     sp.L = L;
     sp.ranks = P;
     sp.rank = dest->rank;
-    sp.row_vecs = (int)(row / 16);
-    sp.out_row_vecs = sp.row_vecs * P;
-    sp.total = B * L * sp.row_vecs;
+    sp.row_units = (int)(row / unit);
+    sp.out_row_units = sp.row_units * P;
+    sp.total = B * L * sp.row_units;
     sp.small = sp.total < ((int64_t)1 << 31) ? 1 : 0;
     if (sp.small) {
-        sp.div_row = rope3d::make_fastdiv((uint32_t)sp.row_vecs);
+        sp.div_row = rope3d::make_fastdiv((uint32_t)sp.row_units);
         sp.div_L = rope3d::make_fastdiv((uint32_t)L);
     }
+    constexpr int U = ROPE3D_A2A_UNROLL;
     const int threads = 256;
-    int64_t grid = (sp.total + threads - 1) / threads;
+    int64_t grid = (sp.total + (int64_t)threads * U - 1) / ((int64_t)threads * U);
     const int64_t cap = (int64_t)info.sms * 8;
     if (grid > cap) grid = cap;
     cudaLaunchConfig_t cfg{};
@@ -1400,8 +1415,9 @@ int rope3d_sp_output_all_to_all(const void* o, int64_t B, int64_t L, int64_t hea
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&sp};
-    const cudaError_t e = cudaLaunchKernelExC(
-        &cfg, reinterpret_cast<const void*>(rope3d::sp_output_all_to_all_kernel), args);
+    const void* fn = wide ? reinterpret_cast<const void*>(rope3d::sp_output_all_to_all_kernel<32, U>)
+                          : reinterpret_cast<const void*>(rope3d::sp_output_all_to_all_kernel<16, U>);
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }

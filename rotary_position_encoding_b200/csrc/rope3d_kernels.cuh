@@ -1231,49 +1231,91 @@ qk_norm_rope_kernel(const Params p) {
 // The exchange after attention (Algorithm 3, last step): this rank's o [B][L][hl][D] --
 // every token for its own heads -- goes out token by token to the rank whose slice holds
 // the token, at head offset rank * hl of that rank's [B][slice][N][D] buffer.  A bit copy
-// in 16-byte vectors, one vector per thread and step; the source and each destination
-// row segment are contiguous, so loads and stores are coalesced on both sides.
+// in W-byte units (16, or 32 when every pointer allows it); the source and each
+// destination row segment are contiguous, so loads and stores are coalesced on both
+// sides.  Each thread takes U units a step, all U loads issued before the first store,
+// so that U units per thread are in flight.
 
 struct SpOutParams {
-    const uint4* o;
-    uint4* out[kMaxRanks];
+    const unsigned char* o;
+    unsigned char* out[kMaxRanks];
     int64_t cuts[kMaxRanks + 1];
     int64_t L;
-    int64_t total;        // B * L * row_vecs
+    int64_t total;        // B * L * row_units
     int ranks;
     int rank;
-    int row_vecs;         // vectors of one token of o (hl heads)
-    int out_row_vecs;     // vectors of one token of an output (all heads)
+    int row_units;        // units of one token of o (hl heads)
+    int out_row_units;    // units of one token of an output (all heads)
     int small;            // total < 2^31: 32-bit index arithmetic
     FastDiv div_row, div_L;
 };
 
+template <int W>
+struct CopyUnit;
+template <>
+struct CopyUnit<16> {
+    uint4 v;
+    __device__ __forceinline__ void load(const unsigned char* p) {
+        v = __ldcs(reinterpret_cast<const uint4*>(p));
+    }
+    __device__ __forceinline__ void store(unsigned char* p) const {
+        __stcs(reinterpret_cast<uint4*>(p), v);
+    }
+};
+template <>
+struct CopyUnit<32> {  // one 256-bit access (sm_100)
+    uint32_t w[8];
+    __device__ __forceinline__ void load(const unsigned char* p) {
+        asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]),
+                       "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                     : "l"(p));
+    }
+    __device__ __forceinline__ void store(unsigned char* p) const {
+        asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]),
+                       "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    }
+};
+
+template <int W, int U>
 __global__ void sp_output_all_to_all_kernel(const SpOutParams p) {
     pdl_launch_dependents();
     pdl_wait_previous_grid();
     const int64_t step = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < p.total; v += step) {
-        int64_t row, b, i;
-        if (p.small) {
-            const uint32_t r32 = fast_div((uint32_t)v, p.div_row);
-            const uint32_t b32 = fast_div(r32, p.div_L);
-            row = r32;
-            b = b32;
-            i = r32 - b32 * (uint32_t)p.L;
-        } else {
-            row = v / p.row_vecs;
-            b = row / p.L;
-            i = row - b * p.L;
-        }
-        const int j = (int)(v - row * p.row_vecs);
-        int d = 0;
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 < p.total;
+         v0 += U * step) {
+        CopyUnit<W> x[U];
 #pragma unroll
-        for (int r = 0; r < kMaxRanks; ++r)
-            if (r < p.ranks && i >= p.cuts[r] && i < p.cuts[r + 1]) d = r;
-        const int64_t rows_d = p.cuts[d + 1] - p.cuts[d];
-        const int64_t dst = ((b * rows_d + (i - p.cuts[d])) * p.out_row_vecs) +
-                            (int64_t)p.rank * p.row_vecs + j;
-        __stcs(p.out[d] + dst, __ldcs(p.o + v));
+        for (int j = 0; j < U; ++j)
+            if (v0 + j * step < p.total) x[j].load(p.o + (v0 + j * step) * W);
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int64_t v = v0 + j * step;
+            if (v >= p.total) break;
+            int64_t row, b, i;
+            if (p.small) {
+                const uint32_t r32 = fast_div((uint32_t)v, p.div_row);
+                const uint32_t b32 = fast_div(r32, p.div_L);
+                row = r32;
+                b = b32;
+                i = r32 - b32 * (uint32_t)p.L;
+            } else {
+                row = v / p.row_units;
+                b = row / p.L;
+                i = row - b * p.L;
+            }
+            const int c = (int)(v - row * p.row_units);
+            int d = 0;
+#pragma unroll
+            for (int r = 0; r < kMaxRanks; ++r)
+                if (r < p.ranks && i >= p.cuts[r] && i < p.cuts[r + 1]) d = r;
+            const int64_t rows_d = p.cuts[d + 1] - p.cuts[d];
+            const int64_t dst = ((b * rows_d + (i - p.cuts[d])) * p.out_row_units) +
+                                (int64_t)p.rank * p.row_units + c;
+            x[j].store(p.out[d] + dst * W);
+        }
     }
 }
 

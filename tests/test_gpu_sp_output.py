@@ -46,6 +46,42 @@ def test_small_every_element(dtype, P, cuts):
     _run(dtype, B=2, L=23, N=8 if P != 3 else 6, P=P, cuts=cuts, seed=800 + P)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_buffers_aligned_to_16_bytes_only(dtype):
+    """o and every output start 16 bytes past a 32-byte boundary: the copy falls back from
+    32-byte to 16-byte units, with the same result."""
+    B, L, N, P = 2, 23, 8, 4
+    cuts = [0, 5, 5, 17, 23]
+    hl = N // P
+    td = torch_dtype(dtype)
+    pad = 16 // torch.empty((), dtype=td).element_size()
+    rng = np.random.default_rng(840)
+    raw = [wl.normal_tensor(rng, (B, L, hl, D), dtype) for _ in range(P)]
+
+    def shifted(shape, fill):
+        n = int(np.prod(shape))
+        buf = torch.full((n + pad,), fill, dtype=td, device="cuda")
+        t = buf[pad:].view(shape)
+        assert t.data_ptr() % 32 == 16
+        return t
+
+    o = []
+    for x in raw:
+        t = shifted((B, L, hl, D), 0.0)
+        t.copy_(to_device(x, dtype))
+        o.append(t)
+    out = [shifted((B, cuts[r + 1] - cuts[r], N, D), 5.0) for r in range(P)]
+    for r in range(P):
+        rope3d.rope3d_sp_output_all_to_all(o[r], out, r, cuts)
+    torch.cuda.synchronize()
+    ref = oracle.Oracle.sp_output_all_to_all(raw, cuts)
+    for r in range(P):
+        want = np.ascontiguousarray(ref[r])
+        if dtype == "f32":
+            want = want.view(np.uint32)
+        assert np.array_equal(to_bits(out[r]), want), f"rank {r}"
+
+
 def test_720p_eight_ranks_even_split():
     """The 720P chunk of a 40-head backbone over 8 ranks: 1350 tokens and 5 heads each."""
     _run("bf16", B=1, L=10800, N=40, P=8, cuts=[r * 1350 for r in range(9)], seed=808)
