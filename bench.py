@@ -92,8 +92,9 @@ def parse_args(argv=None):
                          "of a smaller case; 0 = the whole step)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads measured after the default 720P headline "
-                         "(480P chunk, whole 480P vs 8 slices, long horizon, FP8 and NVFP4 "
-                         "caches, 8-rank sequence-parallel step, QKV projection)")
+                         "(480P chunk and its 4-rank slices, whole 480P vs 8 slices, long "
+                         "horizon, FP8 and NVFP4 caches, 8-rank sequence-parallel step and "
+                         "the exchange after attention, QKV projection)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -587,11 +588,12 @@ def graph_launch_us(torch, step, n_launch, stream, budget_ms=250.0):
 
 def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
     """The other workloads of the step, each measured like the headline (graph replay of
-    one step, device time per launch, clocks of its own window): the 480P chunk loop, the
-    whole 480P sequence against its 8 slices (with a bit-identity check), the batch-2
-    long-horizon rollout with table and on-the-fly cos/sin, the 720P step with FP8 and
-    NVFP4 caches (on the headline's inputs), and the QKV projection on the tensor cores
-    with cuBLAS on the same GEMM beside it.  Inputs of the extra workloads are drawn on
+    one step, device time per launch, clocks of its own window): the 480P chunk loop and
+    its 4-rank sequence-parallel slices, the whole 480P sequence against its 8 slices
+    (with a bit-identity check), the batch-2 long-horizon rollout with table and
+    on-the-fly cos/sin, the 720P step with FP8 and NVFP4 caches (on the headline's
+    inputs), its 8-rank sequence-parallel slices and the exchange after attention, and
+    the QKV projection on the tensor cores with cuBLAS on the same GEMM beside it.  Inputs of the extra workloads are drawn on
     the device (torch.randn with a fixed seed, rounded to bf16; norm weights U(0.5, 1.5))."""
     hbm = peaks["hbm_gbs"]
     out = {}
@@ -644,7 +646,34 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
           launches_per_step=len(w.chunks),
           note="7 chunk calls (start frames 0..18) into a 32760-token cache, graph replay; "
                "inputs 604 MB per step, above L2")
-    del ins, q_out
+
+    # the 4-rank sequence-parallel step at 480P emulated on this GPU: each chunk's 4 token
+    # slices (1170 tokens, all 12 heads) store each head's q, K and V at the rank that owns
+    # it (3 heads each)
+    P4 = 4
+    hl4, sl4 = w.N // P4, n // P4
+    sp_q = [torch.empty((w.B, n, hl4, wl.HEAD_DIM), dtype=torch.bfloat16, device=device)
+            for _ in range(P4)]
+    sp_k = [torch.zeros((w.B, w.cache_tokens, hl4, wl.HEAD_DIM), dtype=torch.bfloat16,
+                        device=device) for _ in range(P4)]
+    sp_v = [torch.zeros_like(sp_k[0]) for _ in range(P4)]
+    sp_in = [[tuple(x[:, r * sl4:(r + 1) * sl4].contiguous() for x in c) for r in range(P4)]
+             for c in ins]
+
+    def sp4_step():
+        for j, c in enumerate(w.chunks):
+            for r in range(P4):
+                q, k, v = sp_in[j][r]
+                a = c.token_begin + r * sl4
+                rope3d.rope3d_qk_norm_rope_append_sp(
+                    q, k, v, a, a + sl4, c.frame_offset, w.T, w.H, w.W, ins_w[0], ins_w[1],
+                    w.eps, sp_q, sp_k, sp_v, c.slot, tables, q_row0=c.token_begin)
+    us, win = graph_launch_us(torch, sp4_step, P4 * len(w.chunks), stream)
+    entry("chunk480p_3x30x52_h12_bf16/sp4", us, w.algorithmic_bytes(sl4), win,
+          launches_per_step=P4 * len(w.chunks),
+          note="4 ranks emulated as 4 launches per chunk over 1170-token slices; every head "
+               "stored to its owner's buffers (3 heads each, all on this GPU)")
+    del sp_q, sp_k, sp_v, sp_in, ins, q_out
 
     # whole 480P sequence (one call of 32760 tokens) against 8 slices of 4095 tokens
     w = wl.full_480p()
