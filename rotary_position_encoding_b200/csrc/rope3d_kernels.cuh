@@ -390,6 +390,70 @@ __device__ __forceinline__ void pair_trig(const Params& p, const PairInfo<PPV>& 
     }
 }
 
+// The same table in a lean form for the register kernel, where registers decide how many
+// blocks fit an SM: per pair only its column in its axis table and its axis (two bits),
+// the three axis rows found once per row.  Same cos and sin as above.  Measured on B200:
+// 8 registers fewer at 720P, the FP8 step 3% and the register path 1% faster; the ring
+// kernel, which has registers to spare, keeps the per-pair pointers (0.8% faster).
+template <int PPV>
+struct PairCols {
+    float inv[PPV];   // angle per unit position (on-the-fly trig only)
+    int col[PPV];     // the pair's column in its axis table
+    uint32_t axes;    // two bits per pair: 0 = t, 1 = h, 2 = w
+};
+
+template <int PPV>
+__device__ __forceinline__ PairCols<PPV> pair_cols(const Params& p, int pair0) {
+    PairCols<PPV> pc;
+    pc.axes = 0;
+#pragma unroll
+    for (int m = 0; m < PPV; ++m) {
+        const int j = pair0 + m;
+        pc.inv[m] = p.inv_freq[j];
+        const uint32_t a = j < p.n_t ? 0u : (j < p.n_t + p.n_h ? 1u : 2u);
+        pc.col[m] = a == 0 ? j : (a == 1 ? j - p.n_t : j - p.n_t - p.n_h);
+        pc.axes |= a << (2 * m);
+    }
+    return pc;
+}
+
+template <int TRIG, int PPV>
+__device__ __forceinline__ void pair_trig(const Params& p, const PairCols<PPV>& pc,
+                                          const RowPos& pos, float (&cs)[PPV],
+                                          float (&sn)[PPV]) {
+    if constexpr (TRIG == kTrigTable) {
+        const float2* rt = p.tab_t + pos.t_g * p.n_t;
+        const float2* rh = p.tab_h + (int64_t)pos.h * p.n_h;
+        const float2* rw = p.tab_w + (int64_t)pos.w * p.n_w;
+#pragma unroll
+        for (int m = 0; m < PPV; ++m) {
+            const uint32_t a = (pc.axes >> (2 * m)) & 3u;
+            if (kDeviceChecks) {
+                const int64_t x = a == 0 ? pos.t_g : (a == 1 ? (int64_t)pos.h : (int64_t)pos.w);
+                const int64_t rows = a == 0 ? p.tab_rows_t
+                                            : (a == 1 ? p.tab_rows_h : p.tab_rows_w);
+                if (x < 0 || x >= rows) {
+                    record_index_error(p);
+                    cs[m] = 1.0f;
+                    sn[m] = 0.0f;
+                    continue;
+                }
+            }
+            const float2 e = __ldg((a == 0 ? rt : (a == 1 ? rh : rw)) + pc.col[m]);
+            cs[m] = e.x;
+            sn[m] = e.y;
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < PPV; ++m) {
+            const uint32_t a = (pc.axes >> (2 * m)) & 3u;
+            const int64_t x = a == 0 ? pos.t_g : (a == 1 ? (int64_t)pos.h : (int64_t)pos.w);
+            const float phi = (float)x * pc.inv[m];
+            sincosf(phi, &sn[m], &cs[m]);
+        }
+    }
+}
+
 // acc + lo^2 + hi^2 for the two bf16 halves of a 32-bit word (lo, the element at the lower
 // address, first), without widening them: fma.rn.f32.bf16 multiplies two bf16 operands
 // (the product of two 8-bit significands is exact in fp32) and adds an fp32 operand with
@@ -1183,7 +1247,7 @@ qk_norm_rope_kernel(const Params p) {
         stage_weights(p, s_wq, s_wk);
         __syncthreads();
     }
-    const PairInfo<NP> pi = pair_info<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
+    const PairCols<NP> pi = pair_cols<NP>(p, first_pair<T, PAIR>(t % Tr::kVecsPerHead));
     int dst[VPT];
     if constexpr (SP) {
 #pragma unroll

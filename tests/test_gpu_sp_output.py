@@ -62,7 +62,7 @@ def test_buffers_aligned_to_16_bytes_only(dtype):
         n = int(np.prod(shape))
         buf = torch.full((n + pad,), fill, dtype=td, device="cuda")
         t = buf[pad:].view(shape)
-        assert t.data_ptr() % 32 == 16
+        assert n == 0 or t.data_ptr() % 32 == 16  # an empty slice has no address
         return t
 
     o = []
