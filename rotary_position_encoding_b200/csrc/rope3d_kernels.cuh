@@ -707,24 +707,30 @@ __device__ __forceinline__ void fp8_scale_pair(uint32_t k0, uint32_t k1, int lan
     s1 = fp8_scale_from_key(w >> 16);
 }
 
-// Key of the largest magnitude in a vector of input elements.  For bf16 the magnitudes
-// are compared as 16-bit integers (ordered like the values), and the key of a bf16 value
-// with bits b is (b + 0x1F) >> 7, fp8_key of its fp32 widening b << 16.
+// Key of the largest magnitude in a vector of input elements.  For bf16 three
+// `max.xorsign.abs.bf16x2` reduce the four words to two magnitudes (the sign bits, an
+// xor of the inputs', are masked off; a NaN element is passed over, as the definition's
+// "greater than" test passes it over), compared as 16-bit integers; the key of a bf16
+// value with bits b is (b + 0x1F) >> 7, fp8_key of its fp32 widening b << 16.
 __device__ __forceinline__ uint32_t vec_key(const uint4& v) {
-    uint32_t m = max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-    m = max_u16x2(m, v.z & 0x7FFF7FFFu);
-    m = max_u16x2(m, v.w & 0x7FFF7FFFu);
+    uint32_t a, b, m;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(v.z), "r"(v.w));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
+    m &= 0x7FFF7FFFu;
     return (max(m & 0xFFFFu, m >> 16) + 0x1Fu) >> 7;
 }
 __device__ __forceinline__ uint32_t vec_key(const float4& v) {
     return fp8_key(fmaxf(max3f(fabsf(v.x), fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
 }
-// Largest magnitude of a vector of input elements (exact; bf16 magnitudes compare as
-// 16-bit integers).
+// Largest magnitude of a vector of input elements (exact; for bf16 the same reduction
+// as vec_key, then the larger of the two magnitudes widened to fp32).
 __device__ __forceinline__ float vec_abs_max(const uint4& v) {
-    uint32_t m = max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
-    m = max_u16x2(m, v.z & 0x7FFF7FFFu);
-    m = max_u16x2(m, v.w & 0x7FFF7FFFu);
+    uint32_t a, b, m;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(v.z), "r"(v.w));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
+    m &= 0x7FFF7FFFu;
     return __uint_as_float(max(m & 0xFFFFu, m >> 16) << 16);
 }
 __device__ __forceinline__ float vec_abs_max(const float4& v) {
@@ -814,11 +820,25 @@ __device__ __forceinline__ float block_max(float x, int lanes) {
 
 // Store E codes of one vector at vector index vi of an FP8 cache (E bytes per vector);
 // the values are scaled two at a time (packed fp32x2 multiplies).
+// E4M3 codes of four values in one 32-bit word, a in the low byte: two conversions into
+// the halves of one register.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    uint32_t r;
+    asm("{\n"
+        "  .reg .b16 lo, hi;\n"
+        "  cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n"
+        "  cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n"
+        "  mov.b32 %0, {lo, hi};\n"
+        "}"
+        : "=r"(r)
+        : "f"(a), "f"(b), "f"(c), "f"(d));
+    return r;
+}
 __device__ __forceinline__ uint32_t e4m3x4_scaled(float a, float b, float c, float d,
                                                   float2 inv2) {
     const float2 x = __fmul2_rn(make_float2(a, b), inv2);
     const float2 y = __fmul2_rn(make_float2(c, d), inv2);
-    return e4m3x2(x.x, x.y) | (e4m3x2(y.x, y.y) << 16);
+    return e4m3x4(x.x, x.y, y.x, y.y);
 }
 __device__ __forceinline__ void store_fp8(void* cache, int64_t vi, const float (&v)[8],
                                           float inv) {
@@ -887,8 +907,8 @@ __device__ __forceinline__ void store_v_fp8(void* vc, int64_t vi,
         const float2 a = bf16x2_times_pow2(x.x, s), b = bf16x2_times_pow2(x.y, s);
         const float2 c = bf16x2_times_pow2(x.z, s), d = bf16x2_times_pow2(x.w, s);
         uint2 w;
-        w.x = e4m3x2(a.x, a.y) | (e4m3x2(b.x, b.y) << 16);
-        w.y = e4m3x2(c.x, c.y) | (e4m3x2(d.x, d.y) << 16);
+        w.x = e4m3x4(a.x, a.y, b.x, b.y);
+        w.y = e4m3x4(c.x, c.y, d.x, d.y);
         __stcs(reinterpret_cast<uint2*>(vc) + vi, w);
     } else {
         float v[Tr::kElems];
