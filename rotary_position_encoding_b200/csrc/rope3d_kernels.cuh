@@ -707,11 +707,11 @@ __device__ __forceinline__ void fp8_scale_pair(uint32_t k0, uint32_t k1, int lan
     s1 = fp8_scale_from_key(w >> 16);
 }
 
-// Key of the largest magnitude in a vector of input elements.  For bf16 three
-// `max.xorsign.abs.bf16x2` reduce the four words to two magnitudes (the sign bits, an
-// xor of the inputs', are masked off; a NaN element is passed over, as the definition's
-// "greater than" test passes it over), compared as 16-bit integers; the key of a bf16
-// value with bits b is (b + 0x1F) >> 7, fp8_key of its fp32 widening b << 16.
+// Key of the largest magnitude in a vector of finite input elements (the quantizer's
+// domain).  For bf16 three `max.xorsign.abs.bf16x2` reduce the four words to two
+// magnitudes (the sign bits, an xor of the inputs', are masked off), compared as 16-bit
+// integers; the key of a bf16 value with bits b is (b + 0x1F) >> 7, fp8_key of its fp32
+// widening b << 16.
 __device__ __forceinline__ uint32_t vec_key(const uint4& v) {
     uint32_t a, b, m;
     asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
