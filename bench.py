@@ -94,7 +94,8 @@ def parse_args(argv=None):
                     help="skip the other workloads measured after the default 720P headline "
                          "(480P chunk and its 4-rank slices, whole 480P vs 8 slices, long "
                          "horizon, FP8 and NVFP4 caches, 8-rank sequence-parallel step and "
-                         "the exchange after attention, QKV projection)")
+                         "the exchange after attention, the rotation alone, QKV projection "
+                         "and the step it feeds)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -592,8 +593,9 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
     its 4-rank sequence-parallel slices, the whole 480P sequence against its 8 slices
     (with a bit-identity check), the batch-2 long-horizon rollout with table and
     on-the-fly cos/sin, the 720P step with FP8 and NVFP4 caches (on the headline's
-    inputs), its 8-rank sequence-parallel slices and the exchange after attention, and
-    the QKV projection on the tensor cores with cuBLAS on the same GEMM beside it.  Inputs of the extra workloads are drawn on
+    inputs), its 8-rank sequence-parallel slices and the exchange after attention, the
+    rotation alone, the QKV projection on the tensor cores with cuBLAS on the same GEMM
+    beside it, and the step fed by the projection.  Inputs of the extra workloads are drawn on
     the device (torch.randn with a fixed seed, rounded to bf16; norm weights U(0.5, 1.5))."""
     hbm = peaks["hbm_gbs"]
     out = {}
@@ -813,6 +815,17 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
                "13.8 MB of o (every token, 5 heads) to the 8 ranks' token slices")
     del o_sets, o_out
 
+    # RoPE alone (rope3d_apply) on the headline's q rows: read x, write the rotated rows
+    def apply_step():
+        for j, c in enumerate(w.chunks):
+            rope3d.rope3d_apply(ins[j][0], q_out[j], c.token_begin, c.token_end,
+                                c.frame_offset, w.T, w.H, w.W, tables)
+    us, win = graph_launch_us(torch, apply_step, len(w.chunks), stream)
+    entry(f"{w.name}/apply_rotation_only", us, 2 * w.B * n * w.dim * 2, win,
+          launches_per_step=len(w.chunks),
+          note="rope3d_apply: the 3D rotation alone (no norm, no cache), x read and the "
+               "rotated rows written, 221 MB per call")
+
     # the QKV projection on the tensor cores (timed alone: the burst peak applies)
     K = w.dim
     xs = [randn_bf16((w.B * n, K), 400 + j) for j in range(3)]
@@ -846,7 +859,38 @@ def run_configs(torch, rope3d, device, stream, clocks, peaks, headline):
         "clocks": {"window": win, "name": "projection"},
         "note": "x [10800, 5120] bf16 times W^T, W [15360, 5120] bf16, fp32 accumulate, bf16 "
                 "out; 3 input sets, graph replay"}
-    del xs, wt, outs, y
+    del outs, y
+
+    # the step fed by the projection (rope3d_qkv_norm_rope_append): the 7 chunk calls of
+    # the 720P step from hidden states, 3 input sets cycled
+    xs3 = [x.view(w.B, n, K) for x in xs]
+    ws = torch.zeros(rope3d.rope3d_qkv_workspace_bytes(w.B, n, w.N), dtype=torch.uint8,
+                     device=device)
+    kcf = torch.zeros((w.B, w.cache_tokens, w.N, wl.HEAD_DIM), dtype=torch.bfloat16,
+                      device=device)
+    vcf = torch.zeros_like(kcf)
+
+    def fused():
+        for j, c in enumerate(w.chunks):
+            rope3d.rope3d_qkv_norm_rope_append(
+                xs3[j % 3], wt, bt, q_out[j], ws, c.token_begin, c.token_end, c.frame_offset,
+                w.T, w.H, w.W, wq_d, wk_d, w.eps, kcf, vcf, c.slot, tables)
+    us, win = graph_launch_us(torch, fused, len(w.chunks), stream)
+    tf = flops / (us * 1e-6) / 1e12
+    out[f"{w.name}/qkv_fused_step"] = {
+        "bound": "tensor", "avg_call_us": round(us, 2), "algorithmic_flops_per_call": flops,
+        "achieved_tflops": round(tf, 1), "peak_tflops": burst,
+        "peak_source": "MEASURED_PEAKS.json bf16_tflops (burst, as for the projection alone)",
+        "frac": round(tf / burst, 4), "tokens_per_s": round(w.B * n / (us * 1e-6), 1),
+        "kernel": "rope3d::qkv_proj_kernel<2> (norm-weight, RoPE and V-append epilogue) + "
+                  "rope3d::qk_row_scale_kernel",
+        "projection_alone_us": out[f"{w.name}/qkv_projection"]["avg_launch_us"],
+        "clocks": {"window": win, "name": "projection-fed step"},
+        "note": "7 chunk calls of rope3d_qkv_norm_rope_append from x [1, 10800, 5120] bf16 "
+                "(3 input sets cycled): the projection GEMM with its epilogue, then the "
+                "per-row RMSNorm scale of q and K; graph replay, time per call"}
+    del xs, xs3, wt, ws, kcf, vcf
+
     torch.cuda.empty_cache()
     return out
 
