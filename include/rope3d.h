@@ -428,10 +428,10 @@ ROPE3D_API int rope3d_check_device_status(const rope3d_tables* tables, void* cud
  *
  * Every call shares the array and it keeps the last call's contents; calls that overlap
  * on the GPU (on different streams or from different host threads) race on it and must
- * be serialised by the caller.  The status word of the bounded waits is not reported
- * back.  The first call on a device looks up the array's device address (one-time set-up
- * with that device current); make that first call before any stream capture.  Other
- * arguments, layouts and errors are those of rope3d_qk_norm_rope_append.
+ * be serialised by the caller.  The status word of the bounded waits is read back by
+ * rope3d_noalloc_check_status.  The first call on a device looks up the array's device
+ * address (one-time set-up with that device current).  Other arguments, layouts and
+ * errors are those of rope3d_qk_norm_rope_append.
  */
 ROPE3D_API int rope3d_qk_norm_rope_append_noalloc(
     const void* q, const void* k, const void* v, void* q_out, int64_t B, int64_t N, int D,
@@ -439,6 +439,18 @@ ROPE3D_API int rope3d_qk_norm_rope_append_noalloc(
     const float* q_norm_w, const float* k_norm_w, float eps, void* k_cache, void* v_cache,
     int64_t cache_tokens, int64_t slot, int n_t, int n_h, int n_w, double theta, int schedule,
     int trig, void* cuda_stream);
+
+/*
+ * The status word of rope3d_qk_norm_rope_append_noalloc on the current device, read and
+ * cleared as rope3d_check_device_status does for a tables object: synchronises
+ * cuda_stream, copies the word (a 4-byte device-to-host copy into the caller's stack; no
+ * allocation), clears it when it is set, and returns ROPE3D_OK, ROPE3D_ETIMEOUT (a
+ * bounded wait of the last no-allocation call gave up; its outputs are incomplete) or
+ * ROPE3D_EINDEX (checked build only).  The word is the one every no-allocation call
+ * clears first, so it reports the calls since the last read or the last call, whichever
+ * came later.  ROPE3D_ECUDA if the copy fails.
+ */
+ROPE3D_API int rope3d_noalloc_check_status(void* cuda_stream);
 
 /* Fixed text for a status code (never NULL). */
 ROPE3D_API const char* rope3d_strerror(int status);

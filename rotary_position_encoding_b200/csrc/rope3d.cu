@@ -854,20 +854,15 @@ void rope3d_tables_destroy(rope3d_tables* tables) {
     delete tables;
 }
 
-int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream) {
-    if (tables == nullptr) return fail(ROPE3D_EINVAL, "tables is NULL");
-    int cur = 0;
-    cudaError_t e = cudaGetDevice(&cur);
-    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (cur != tables->device)
-        return fail(ROPE3D_EDEVICE, "tables were built on device %d, current device is %d",
-                    tables->device, cur);
-    cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+namespace {
+
+// Reads the device status word at d_status in stream order, clears it when set, and maps
+// it to a status code.
+int read_status_word(int* d_status, cudaStream_t stream) {
     int word = 0;
-    e = cudaMemcpyAsync(&word, tables->d_status, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    cudaError_t e = cudaMemcpyAsync(&word, d_status, sizeof(int), cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e == cudaSuccess && word != 0)
-        e = cudaMemsetAsync(tables->d_status, 0, sizeof(int), stream);
+    if (e == cudaSuccess && word != 0) e = cudaMemsetAsync(d_status, 0, sizeof(int), stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "status read: %s", cudaGetErrorString(e));
     if (word & rope3d::kStatusWaitTimeout)
@@ -876,6 +871,19 @@ int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream) {
         return fail(ROPE3D_EINDEX, "a kernel of the checked build derived a cache, table or "
                                    "destination row outside its extent and skipped it");
     return ok();
+}
+
+}  // namespace
+
+int rope3d_check_device_status(const rope3d_tables* tables, void* cuda_stream) {
+    if (tables == nullptr) return fail(ROPE3D_EINVAL, "tables is NULL");
+    int cur = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (cur != tables->device)
+        return fail(ROPE3D_EDEVICE, "tables were built on device %d, current device is %d",
+                    tables->device, cur);
+    return read_status_word(tables->d_status, static_cast<cudaStream_t>(cuda_stream));
 }
 
 void rope3d_testing_set_waits(uint64_t wait_limit_ns, uint32_t tx_extra_bytes) {
@@ -1650,4 +1658,16 @@ extern "C" int rope3d_qk_norm_rope_append_noalloc(
     return rope3d_qk_norm_rope_append(q, k, v, q_out, B, N, D, dtype, token_begin, token_end,
                                       frame_offset, T, H, W, q_norm_w, k_norm_w, eps, k_cache,
                                       v_cache, cache_tokens, slot, &tb, trig, cuda_stream);
+}
+
+extern "C" int rope3d_noalloc_check_status(void* cuda_stream) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ROPE3D_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    unsigned char* scratch = nullptr;
+    const int rc = noalloc_scratch_address(dev, &scratch);
+    if (rc != ROPE3D_OK) return rc;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    return read_status_word(reinterpret_cast<int*>(scratch),
+                            static_cast<cudaStream_t>(cuda_stream));
 }

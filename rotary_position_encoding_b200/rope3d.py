@@ -109,6 +109,7 @@ SIGNATURES = {
                          _VP, _INT, ctypes.POINTER(rope3d_options), _VP], _INT),
     "rope3d_decode_positions": ([_I64, _I64, _I64, _INT, _INT, _INT, _I64, _I64, _VP, _VP], _INT),
     "rope3d_check_device_status": ([_VP, _VP], _INT),
+    "rope3d_noalloc_check_status": ([_VP], _INT),
     "rope3d_qk_norm_rope_append_noalloc": ([_VP, _VP, _VP, _VP, _I64, _I64, _INT, _INT, _I64,
                                             _I64, _I64, _INT, _INT, _INT, _VP, _VP,
                                             ctypes.c_float, _VP, _VP, _I64, _I64, _INT, _INT,
@@ -541,6 +542,14 @@ def rope3d_check_device_status(tables: Tables, stream=None) -> int:
     with these tables: ROPE3D_OK, ROPE3D_ETIMEOUT, or (checked build) ROPE3D_EINDEX.
     Raises on a failure to read it."""
     status = load_library().rope3d_check_device_status(tables.handle, _stream(stream))
+    if status not in (ROPE3D_OK, ROPE3D_ETIMEOUT, ROPE3D_EINDEX):
+        _check(status)
+    return status
+
+
+def rope3d_noalloc_check_status(stream=None) -> int:
+    """The same for the no-allocation entry point's status word on the current device."""
+    status = load_library().rope3d_noalloc_check_status(_stream(stream))
     if status not in (ROPE3D_OK, ROPE3D_ETIMEOUT, ROPE3D_EINDEX):
         _check(status)
     return status

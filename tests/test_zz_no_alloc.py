@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_support import assert_close, to_device, to_f64
+from gpu_support import assert_close, kernel_path, to_device, to_f64
 from rotary_position_encoding_b200 import rope3d, workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -107,3 +107,48 @@ def test_noalloc_wrapper_checks_tensors_before_the_call():
         rope3d.rope3d_qk_norm_rope_append_noalloc(q, q, q, q.clone(), token_begin=0,
                                                   token_end=4, k_cache=kc, v_cache=kc.clone(),
                                                   **dict(args, q_norm_w=wq[:8]))
+
+
+def test_noalloc_status_reports_a_wait_that_timed_out():
+    """The status word of the no-allocation entry point: a bounded wait of the ring kernel
+    that never fills (a test setting makes every stage wait for 16 bytes its copies never
+    deliver; every copy lands, only the wait runs out) is reported by
+    rope3d_noalloc_check_status; the read clears it, and the next call is bit-identical to
+    the ordinary entry point."""
+    w = wl.chunk_480p()
+    wq_np, wk_np = wl.norm_weights(w.seed, w.dim)
+    wq, wk = torch.from_numpy(wq_np).cuda(), torch.from_numpy(wk_np).cuda()
+    shape = (w.B, w.cache_tokens, w.N, wl.HEAD_DIM)
+    kc, vc = (torch.zeros(shape, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    chunk = w.chunks[1]
+    q, k, v = (to_device(x, w.dtype) for x in wl.chunk_inputs(w, 1))
+    q_new = torch.empty_like(q)
+    args = dict(frame_offset=chunk.frame_offset, T=w.T, H=w.H, W=w.W, q_norm_w=wq,
+                k_norm_w=wk, eps=w.eps, slot=chunk.slot)
+    assert rope3d.rope3d_noalloc_check_status() == rope3d.ROPE3D_OK
+    rope3d.rope3d_testing_set_waits(20_000_000, 16)  # 20 ms, 16 bytes never delivered
+    try:
+        with kernel_path(rope3d.ROPE3D_PATH_TMA):
+            rope3d.rope3d_qk_norm_rope_append_noalloc(
+                q, k, v, q_new, chunk.token_begin, chunk.token_end, k_cache=kc, v_cache=vc,
+                **args)
+        status = rope3d.rope3d_noalloc_check_status()
+    finally:
+        rope3d.rope3d_testing_set_waits(0, 0)
+    assert status == rope3d.ROPE3D_ETIMEOUT
+    assert rope3d.rope3d_noalloc_check_status() == rope3d.ROPE3D_OK  # cleared by the read
+    with kernel_path(rope3d.ROPE3D_PATH_TMA):
+        rope3d.rope3d_qk_norm_rope_append_noalloc(
+            q, k, v, q_new, chunk.token_begin, chunk.token_end, k_cache=kc, v_cache=vc, **args)
+    assert rope3d.rope3d_noalloc_check_status() == rope3d.ROPE3D_OK
+    tables = rope3d.rope3d_tables_init(max_t=21, max_h=w.H, max_w=w.W)
+    kr, vr = (torch.zeros_like(kc) for _ in range(2))
+    q_ref = torch.empty_like(q)
+    rope3d.rope3d_qk_norm_rope_append(q, k, v, q_ref, chunk.token_begin, chunk.token_end,
+                                      chunk.frame_offset, w.T, w.H, w.W, wq, wk, w.eps, kr, vr,
+                                      chunk.slot, tables)
+    torch.cuda.synchronize()
+    assert torch.equal(q_new.view(torch.int16), q_ref.view(torch.int16))
+    assert torch.equal(kc.view(torch.int16), kr.view(torch.int16))
+    assert torch.equal(vc.view(torch.int16), vr.view(torch.int16))
+    tables.close()
